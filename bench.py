@@ -1,0 +1,468 @@
+"""Benchmark of the PowerSGD compression step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1] [--impl ours|reference]
+
+One step = the whole hot path over one batch of synthetic gradients held in
+HBM: psgd_step (error-feedback add, P = MQ, worker mean, orthogonalisation,
+Q = M^T P_hat, worker mean, residual), the uncompressed mean of the 1-D
+tensors and the post-compression momentum update, all through the C ABI.
+Metric: gradient elements compressed per second (W * sum(m*n) per step),
+whole job; with N GPUs each rank runs an independent replica (the method's
+workers are simulated on one GPU) and value = N * elements / max-over-ranks
+time.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from synth import GradientSource, get as get_workload, pack_offsets  # noqa: E402
+
+METRIC = "gradient elements compressed/sec"
+UNIT = "elements/s"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def _kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "rank_gradient_compression_02_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_record(workload: str, mode: str):
+    """DRAM bytes per launch of the first pass from a committed ncu summary,
+    valid only for the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    key = f"{workload}/{mode}"
+    r = rec.get(key)
+    if not r or r.get("kernel_hash") != _kernel_source_hash():
+        return None
+    return r.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            out_dir = os.path.join(ROOT, "gpurun_out") if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else "/tmp"
+            self.path = os.path.join(out_dir, f"clocks_bench_{os.getpid()}.csv")
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() in ("active", "1", "yes"):
+                        reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """Max of a per-rank time over all ranks (the job's time)."""
+    if world <= 1:
+        return ms
+    import torch.distributed as dist
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(elements_per_replica: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank runs one replica of the workload."""
+    return elements_per_replica * world / (ms_per_step * 1e-3)
+
+
+# --------------------------------------------------------------------------
+# workload buffers
+
+class Buffers:
+    def __init__(self, wl, rank, device, seed=1234):
+        self.wl = wl
+        self.rank = rank
+        W, L = wl.workers, len(wl.layers)
+        gdt = torch.bfloat16 if wl.grad_dtype == "bf16" else torch.float32
+        align = 64  # elements: 256 B for fp32, 128 B for bf16
+        self.offs = pack_offsets(wl.layers, align)
+        total = self.offs[-1]
+        self.G_flat = [torch.empty(total, dtype=gdt, device=device) for _ in range(W)]
+        self.E_flat = [torch.zeros(total, dtype=torch.float32, device=device) for _ in range(W)]
+        self.G = [[self.G_flat[w][self.offs[l]:self.offs[l] + m * n].view(m, n) for l, (m, n) in enumerate(wl.layers)]
+                  for w in range(W)]
+        self.E = [[self.E_flat[w][self.offs[l]:self.offs[l] + m * n].view(m, n) for l, (m, n) in enumerate(wl.layers)]
+                  for w in range(W)]
+        src = GradientSource(wl, seed)
+        self.src = src
+        src.fill(0, self.G)
+        self.Q = [src.initial_q(l, rank).to(device) for l in range(L)]
+        self.P = [torch.empty(m, rank, device=device) for (m, _) in wl.layers]
+        self.params = self.mom = None
+        if wl.momentum:
+            self.params = [torch.zeros(m, n, device=device) for (m, n) in wl.layers]
+            self.mom = [torch.zeros(m, n, device=device) for (m, n) in wl.layers]
+        self.vecs = self.vout = self.vx = self.vmom = None
+        if wl.vectors:
+            self.vecs = [[t.to(device) for t in src.vector_grads(0, w)] for w in range(W)]
+            self.vout = [torch.empty(k, device=device) for k in wl.vectors]
+            self.vx = [torch.zeros(k, device=device) for k in wl.vectors]
+            self.vmom = [torch.zeros(k, device=device) for k in wl.vectors]
+
+
+def device_bytes_needed(wl, rank):
+    W = wl.workers
+    gsz = 2 if wl.grad_dtype == "bf16" else 4
+    e = wl.elements_per_worker
+    b = W * e * (gsz + 4)
+    if wl.momentum:
+        b += 2 * e * 4
+    return b
+
+
+def run_step(lib, B, wl):
+    lib.step(B.G, B.E, B.Q, B.P, None)
+    if B.vecs is not None:
+        beta, lr = wl.momentum if wl.momentum else (0.0, 0.0)
+        lib.vec_mean(B.vecs, B.vout, B.vx, B.vmom, lr=lr, beta=beta)
+    if B.params is not None:
+        beta, lr = wl.momentum
+        lib.momentum_step(B.params, B.mom, lr, beta)
+
+
+def launches_per_step(lib, B):
+    n = lib.step_launches
+    if B.vecs is not None:
+        n += 1
+    if B.params is not None:
+        n += 1
+    return n
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timing (bounded sample)
+
+def oracle_sample(wl, rank, budget_s=15.0, seed=1234, max_layers=None):
+    """Time the float64 oracle on a bounded sample of the workload: whole
+    layers (all workers) in list order until the oracle time passes
+    budget_s.  Returns (elements/s, elements, seconds, threads, text)."""
+    import oracle.powersgd64 as ora
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    src = GradientSource(wl, seed)
+    done_el, spent, layers_done = 0, 0.0, 0
+    order = list(range(len(wl.layers)))
+    for l in order:
+        if max_layers is not None and layers_done >= max_layers:
+            break
+        m, n = wl.layers[l]
+        G = [src.layer_grad(0, w, l).to(torch.float64).numpy() for w in range(wl.workers)]
+        E = [np.zeros((m, n)) for _ in range(wl.workers)]
+        Q = src.initial_q(l, rank).to(torch.float64).numpy()
+        t0 = time.perf_counter()
+        ora.step(G, E, Q)
+        spent += time.perf_counter() - t0
+        done_el += wl.workers * m * n
+        layers_done += 1
+        del G, E
+        if spent >= budget_s:
+            break
+    text = (f"{layers_done} of {len(wl.layers)} layers (all {wl.workers} workers, one step, float64 NumPy; "
+            f"BLAS threads {threads}, elementwise ops single-threaded)")
+    return done_el / spent, done_el, spent, threads, text
+
+
+# --------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="1", help="workload: 0, 1, 2, 3, 4a, 4b or a name")
+    ap.add_argument("--rank", type=int, default=None, help="rank r (default: the workload's)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--lazy", action="store_true", help="lazy error representation")
+    ap.add_argument("--sum-first", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--oracle-budget", type=float, default=15.0)
+    args = ap.parse_args()
+
+    wl = get_workload(args.config)
+    r = args.rank if args.rank is not None else wl.rank
+    wl = wl.with_rank(r)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank_id = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    mode = ("lazy" if args.lazy else "eager") + ("+sumfirst" if args.sum_first else "")
+    config = {"workload": wl.name, "layers": len(wl.layers), "elements_per_worker": wl.elements_per_worker,
+              "workers": wl.workers, "rank": r, "grad_dtype": wl.grad_dtype, "mode": mode,
+              "l2": "inputs larger than L2 (no flush needed)" if wl.elements * 4 > 4 * 126e6 else "inputs fit L2",
+              "parallelism": f"replicas{world}"}
+
+    if args.impl == "reference":
+        if rank_id != 0:
+            return
+        run_reference(args, wl, r, config, world)
+        return
+
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    device = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(device)
+
+    from rank_gradient_compression_02_b200 import PowerSGD
+    free, _ = torch.cuda.mem_get_info()
+    need = device_bytes_needed(wl, r)
+    if need > free * 0.95:
+        raise SystemExit(f"workload needs {need/1e9:.1f} GB, {free/1e9:.1f} GB free")
+    B = Buffers(wl, r, device)
+    lib = PowerSGD(wl.layers, r, wl.workers, grad_dtype=wl.grad_dtype, lazy_errors=args.lazy,
+                   sum_first=args.sum_first)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        run_step(lib, B, wl)
+    lib.status()
+    barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local if world > 1 else 0)
+    clocks.start()
+    lib.profile(True)
+    stream = torch.cuda.current_stream()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        run_step(lib, B, wl)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    kern_ms, kern_steps = lib.profile_read()
+    lib.profile(False)
+    clk = clocks.stop()
+    lib.status()
+    ms = max_over_ranks(ms, world, device)
+    ms_per_step = ms / args.steps
+    value = job_value(wl.elements, world, ms_per_step)
+
+    # roofline of the dominant kernel (first pass unless measured otherwise)
+    peak, peak_kind = _peaks()
+    gsz = 2 if wl.grad_dtype == "bf16" else 4
+    per_launch_ms = [k / max(1, kern_steps) for k in kern_ms]
+    # algorithmic bytes per launch: pass A reads G and E (or M) and writes M;
+    # pass B reads M; pass C reads M and writes E'
+    alg = [wl.elements * (gsz + 8), wl.elements * 4, 0 if args.lazy else wl.elements * 8]
+    names = ["pass_a", "pass_b", "pass_c"]
+    dom = max(range(3), key=lambda i: per_launch_ms[i])
+    achieved = alg[dom] / (per_launch_ms[dom] * 1e-3) / 1e9 if per_launch_ms[dom] > 0 else 0.0
+    traffic = _traffic_record(wl.name, mode) if dom == 0 else None
+    step_min_bytes = wl.elements * (gsz + 8)
+    roofline = {"bound": "hbm", "kernel": names[dom], "achieved": round(achieved, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_kind": f"{peak_kind} hbm_gbs",
+                "per_kernel_ms": {n: round(t, 4) for n, t in zip(names, per_launch_ms)},
+                "step_algorithmic_frac": round(step_min_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 4)}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(lib, B, wl, r, args, world, device)
+
+    cpu = None
+    if rank_id == 0 and world == 1 and not args.no_cpu_baseline:
+        v, el, sec, threads, text = oracle_sample(wl, r, budget_s=args.oracle_budget)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": text,
+               "seconds": round(sec, 2)}
+
+    out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f32" if wl.grad_dtype == "f32" else "bf16-in/f32",
+           "data": "synthetic (seeded low-rank + noise gradients, resident in HBM)",
+           "config": config, "gpu_launches": args.steps * launches_per_step(lib, B),
+           "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+           "hbm_gbs_step": round(step_min_bytes / (ms_per_step * 1e-3) / 1e9, 1)}
+    if rank_id == 0:
+        print(json.dumps(out), flush=True)
+    lib.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_e2e(lib, B, wl, r, args, world, device):
+    """The same metric through psgd_step_host: pinned host gradients copied
+    in every step, P_hat and Q_bar (and the 1-D means) read back."""
+    gsz = 2 if wl.grad_dtype == "bf16" else 4
+    host_bytes = wl.elements * gsz
+    if host_bytes > 16e9:
+        return {"value": None, "unit": UNIT, "skipped": "host copy of the gradients exceeds 16 GB"}
+    import torch.distributed as dist
+    W, L = wl.workers, len(wl.layers)
+    Gh = [torch.empty(B.offs[-1], dtype=B.G_flat[0].dtype).pin_memory() for _ in range(W)]
+    for w in range(W):
+        Gh[w].copy_(B.G_flat[w])
+    Gh_views = [[Gh[w][B.offs[l]:B.offs[l] + m * n] for l, (m, n) in enumerate(wl.layers)] for w in range(W)]
+    Ph = [torch.empty(m, r).pin_memory() for (m, _) in wl.layers]
+    Qh = [torch.empty(n, r).pin_memory() for (_, n) in wl.layers]
+    vh = vout_h = None
+    if B.vecs is not None:
+        vh = [[t.cpu().pin_memory() for t in B.vecs[w]] for w in range(W)]
+        vout_h = [torch.empty(k).pin_memory() for k in wl.vectors]
+    stream = torch.cuda.current_stream()
+
+    def one():
+        lib.step_host(Gh_views, B.E, B.Q, Ph, Qh)
+        if vh is not None:
+            for w in range(W):
+                for k in range(len(wl.vectors)):
+                    B.vecs[w][k].copy_(vh[w][k], non_blocking=True)
+            beta, lr = wl.momentum if wl.momentum else (0.0, 0.0)
+            lib.vec_mean(B.vecs, B.vout, B.vx, B.vmom, lr=lr, beta=beta)
+            for k in range(len(wl.vectors)):
+                vout_h[k].copy_(B.vout[k], non_blocking=True)
+        if B.params is not None:
+            beta, lr = wl.momentum
+            lib.momentum_step(B.params, B.mom, lr, beta)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    per = ms / args.e2e_steps
+    h2d = host_bytes + (sum(wl.vectors) * 4 * W if vh is not None else 0)
+    d2h = sum((m + n) * r * 4 for (m, n) in wl.layers) + (sum(wl.vectors) * 4 if vh is not None else 0)
+    return {"value": wl.elements * world / (per * 1e-3), "unit": UNIT, "ms_per_step": per,
+            "steps": args.e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def run_reference(args, wl, r, config, world):
+    """The float64 oracle on the host cores, each step a bounded sample of
+    the workload (one layer, all workers, in turn), same metric and unit."""
+    import oracle.powersgd64 as ora
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    src = GradientSource(wl, 1234)
+    # smallest layers first so that K steps stay within minutes
+    order = sorted(range(len(wl.layers)), key=lambda l: wl.layers[l][0] * wl.layers[l][1])
+    cache = {}
+
+    def inputs(l):
+        if l not in cache:
+            m, n = wl.layers[l]
+            G = [src.layer_grad(0, w, l).to(torch.float64).numpy() for w in range(wl.workers)]
+            cache.clear()
+            cache[l] = (G, [np.zeros((m, n)) for _ in range(wl.workers)], src.initial_q(l, r).double().numpy())
+        return cache[l]
+
+    def one(i):
+        l = order[i % len(order)]
+        G, E, Q = inputs(l)
+        t0 = time.perf_counter()
+        ora.step(G, E, Q)
+        return time.perf_counter() - t0, wl.workers * wl.layers[l][0] * wl.layers[l][1]
+
+    for i in range(args.warmup):
+        one(i)
+    spent, el = 0.0, 0
+    for i in range(args.steps):
+        s, e = one(i)
+        spent += s
+        el += e
+    value = el / spent
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": spent / args.steps * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded low-rank + noise gradients)", "config": config,
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                            "sample": "each step: one layer of the workload (all workers), smallest layers first, "
+                                      "float64 NumPy oracle"},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

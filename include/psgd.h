@@ -1,0 +1,190 @@
+/*
+ * psgd.h - C ABI of the B200 PowerSGD compression-step library (libpsgd.so).
+ *
+ * What it computes.  For every gradient matrix M (m x n, row-major, leading
+ * dimension n; convolution weights are passed already viewed as
+ * out x (in*k*k), "anthology-of-the-sota" note-152 on PowerSGD, section
+ * "Method", per-layer approximation with reshaped conv tensors) and W
+ * workers, one call of psgd_step performs one PowerSGD compression step in
+ * the order the same section gives:
+ *
+ *   M_w   = G_w + E_w                         error feedback ("Concepts")
+ *   P_bar = (1/W) sum_w M_w Q                 right multiply + all-reduce
+ *   P_hat = P_bar R^-1  (Gram-Schmidt QR)     orthogonalisation of P
+ *   Q_bar = (1/W) sum_w M_w^T P_hat           left multiply + all-reduce
+ *   E'_w  = M_w - P_hat Q_bar^T               new error memory
+ *   G_hat = P_hat Q_bar^T                     decompressed mean gradient
+ *
+ * and Q (the warm start, "Concepts", warm-start subspace iteration) is
+ * replaced by Q_bar.  The W workers are replica buffers in this GPU's memory;
+ * the "all-reduce" is an on-device mean, computed in a fixed order so that
+ * results are bitwise reproducible run to run.
+ *
+ * Orthogonalisation: P_hat is the Q factor of the thin QR of P_bar with a
+ * positive diagonal (what Gram-Schmidt produces).  The library computes it
+ * as a Cholesky QR: the r x r Gram matrix of P_bar is accumulated in
+ * float64, factored (Cholesky, float64), and P_hat = P_bar T with T the
+ * inverse of the factor.  A column whose squared norm after projection on
+ * the previous ones is <= 1e-12 * max_k ||pbar_k||^2 becomes zero (the
+ * pages say nothing about rank deficiency; this is the rule the float64
+ * oracle uses too).  NaN inputs propagate; they are not trapped.
+ *
+ * Precision: G is float32 or bfloat16; E, Q, P_hat, Q_bar, G_hat and all
+ * accumulation are float32, Gram and Cholesky float64.
+ *
+ * Ownership: the caller owns every tensor passed in (device memory, e.g.
+ * PyTorch tensors).  The library owns its workspace and pointer tables,
+ * allocated in psgd_create and released in psgd_destroy.  E and Q are
+ * updated in place.
+ *
+ * Alignment: every device pointer passed must be 16-byte aligned
+ * (PSGD_ERR_ALIGN otherwise).  Rows need not be: n may be odd.
+ *
+ * Streams and ordering: every call enqueues work on `stream` (a
+ * cudaStream_t passed as void*, NULL = legacy default stream) and returns
+ * without synchronising.  Calls on one context must be ordered (one stream,
+ * or synchronised by the caller): they share workspace and counters.
+ * Pointer tables are re-uploaded (on `stream`) only when the pointers
+ * passed differ from the previous call's.
+ *
+ * Errors: argument checks are synchronous and return a code; a failed CUDA
+ * call returns PSGD_ERR_CUDA.  psgd_last_error gives a message.  Device-side
+ * problems are reported through psgd_status.  No call spins on the device.
+ */
+#ifndef PSGD_H
+#define PSGD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PSGD_API __attribute__((visibility("default")))
+#else
+#define PSGD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    PSGD_OK = 0,
+    PSGD_ERR_ARG = 1,    /* null pointer, bad shape, rank or worker count */
+    PSGD_ERR_ALIGN = 2,  /* a device pointer is not 16-byte aligned */
+    PSGD_ERR_CUDA = 3,   /* a CUDA runtime call failed */
+    PSGD_ERR_OOM = 4,    /* workspace allocation failed */
+    PSGD_ERR_STATE = 5,  /* call not valid in this context's mode */
+    PSGD_ERR_DEVICE = 6  /* the device status word is set (psgd_status) */
+};
+
+typedef enum { PSGD_F32 = 0, PSGD_BF16 = 1 } psgd_dtype; /* dtype of G only */
+
+enum {
+    /* Keep M_w (not E'_w) in the error buffers between steps and rebuild
+     * E'_w = M_w - P_hat Q_bar^T on the fly in the next step's first pass
+     * (saves one read and one write of every worker element per step).  The
+     * error buffers then hold M_w after psgd_step; psgd_materialize_errors
+     * turns them into E'_w. */
+    PSGD_FLAG_LAZY_ERRORS = 1u,
+    /* Sum the W workers' M_w element-wise before multiplying by Q or P_hat
+     * (one product per matrix element instead of one per worker element).
+     * Same result up to rounding, by linearity (note-152, "Concepts"). */
+    PSGD_FLAG_SUM_FIRST = 2u
+};
+
+typedef struct { int64_t m, n; } psgd_layer;   /* one gradient matrix */
+typedef struct psgd_ctx psgd_ctx;              /* opaque */
+
+/* Create a context on the current CUDA device.
+ * layers[num_layers]: matrix shapes, m >= 1, n >= 1 (num_layers may be 0:
+ *   every step is then a no-op).
+ * rank: 1 <= rank <= 32 and rank <= min(m, n) for every layer.
+ * workers: 1 <= workers <= 256.
+ * seed: key of the initial-Q draw (psgd_init_q).
+ * grad_dtype: PSGD_F32 or PSGD_BF16.  flags: PSGD_FLAG_*.
+ * Allocates the workspace (see psgd_workspace_bytes).  On error *out is
+ * NULL. */
+PSGD_API int psgd_create(psgd_ctx **out, const psgd_layer *layers, int num_layers, int rank, int workers,
+                uint64_t seed, int grad_dtype, unsigned flags);
+
+PSGD_API void psgd_destroy(psgd_ctx *ctx);
+
+/* Draw Q0 ~ N(0, 1) for every layer into q[l] (device, n x rank float32,
+ * row-major).  Philox4x64-10 (Salmon et al., SC'11) keyed by (seed, l),
+ * counter (b, 0, 0, 0) for element block b = e / 4 (e = j*rank + k), then
+ * Box-Muller on the word pairs (0,1), (2,3) in float64, rounded to float32.
+ * The initial Q is not orthogonalised and is shared by all workers. */
+PSGD_API int psgd_init_q(psgd_ctx *ctx, float *const *q, void *stream);
+
+/* One compression step for all layers and workers.
+ * grads[w*L + l]:  device, m x n, grad dtype, read only.
+ * errors[w*L + l]: device, m x n float32, E_w in, E'_w out (in place).  With
+ *                  PSGD_FLAG_LAZY_ERRORS: M_w out (see the flag).
+ * q[l]:            device, n x rank float32, warm start in, Q_bar out.
+ * p_hat[l]:        device, m x rank float32 out, or p_hat == NULL, or an
+ *                  entry NULL to skip that layer's copy.
+ * recon[l]:        device, m x n float32 out (G_hat), or NULL / NULL entry.
+ * The last P_hat and Q_bar are also kept inside the context (for
+ * psgd_momentum_step and the lazy representation). */
+PSGD_API int psgd_step(psgd_ctx *ctx, const void *const *grads, float *const *errors, float *const *q,
+              float *const *p_hat, float *const *recon, void *stream);
+
+/* The same step with HOST gradients: grads_host[w*L + l] are host pointers
+ * (pinned for asynchronous copies; pageable works but serialises).  The
+ * library copies them into a device staging area it owns (allocated on
+ * first use), runs psgd_step, and copies P_hat and Q_bar back to
+ * p_hat_host[l] (m x rank) and q_host[l] (n x rank) if those are non-NULL.
+ * errors and q stay device pointers (they are state). */
+PSGD_API int psgd_step_host(psgd_ctx *ctx, const void *const *grads_host, float *const *errors, float *const *q,
+                   float *const *p_hat_host, float *const *q_host, void *stream);
+
+/* PSGD_FLAG_LAZY_ERRORS only: write E'_w = M_w - P_hat Q_bar^T (from the
+ * last step) into errors[w*L + l] in place.  The next step then starts from
+ * E'_w as in the eager mode. */
+PSGD_API int psgd_materialize_errors(psgd_ctx *ctx, float *const *errors, void *stream);
+
+/* Post-compression momentum (note-152, "Concepts"): for every layer, with
+ * G_hat = P_hat Q_bar^T of the last step (recomputed on the fly, never read
+ * from memory): mom = beta*mom + G_hat; params = params - lr*mom.
+ * params[l], mom[l]: device m x n float32, updated in place. */
+PSGD_API int psgd_momentum_step(psgd_ctx *ctx, float *const *params, float *const *mom, float lr, float beta,
+                       void *stream);
+
+/* Small tensors travel uncompressed (note-152, "Method"): out[k] = mean over
+ * the ctx's W workers of vecs[w*count + k] (len[k] float32 elements each,
+ * summed in worker order).  If params and mom are non-NULL, also applies
+ * the momentum update above with out[k] as the gradient. */
+PSGD_API int psgd_vec_mean(psgd_ctx *ctx, const float *const *vecs, float *const *out, const int64_t *len, int count,
+                  float *const *params, float *const *mom, float lr, float beta, void *stream);
+
+/* Synchronise the last stream used and read the device status word:
+ * PSGD_OK, or PSGD_ERR_DEVICE if a kernel flagged an inconsistency (e.g.
+ * overlapping steps on one context), or PSGD_ERR_CUDA if a launch failed. */
+PSGD_API int psgd_status(psgd_ctx *ctx);
+
+/* Bytes of device workspace the context holds (excluding host staging). */
+PSGD_API int psgd_workspace_bytes(const psgd_ctx *ctx, size_t *bytes);
+
+/* Number of kernel launches one psgd_step makes for this context (for
+ * launch accounting). */
+PSGD_API int psgd_step_launches(const psgd_ctx *ctx);
+
+/* Per-kernel timing of psgd_step, for measurement: with enable != 0 every
+ * later psgd_step records CUDA events (on its stream) around each of its
+ * kernel launches.  psgd_profile_read synchronises on those events, writes
+ * the summed device milliseconds of the first pass (error feedback + P),
+ * the second pass (Q) and the third pass (residual / decompression, 0 in
+ * lazy mode) to ms[0..2] and the number of recorded steps to *steps, and
+ * clears the record.  Recording adds three event records per step. */
+PSGD_API int psgd_profile_enable(psgd_ctx *ctx, int enable);
+PSGD_API int psgd_profile_read(psgd_ctx *ctx, double *ms, int *steps);
+
+/* Last error message of the context ("" if none); ctx may be NULL for
+ * errors of psgd_create. */
+PSGD_API const char *psgd_last_error(const psgd_ctx *ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PSGD_H */

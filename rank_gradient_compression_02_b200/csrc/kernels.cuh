@@ -1,0 +1,754 @@
+// The streaming kernels of one PowerSGD step (grouped over all layers).
+//
+//   pass A: M_w = G_w + E_w (stored over E_w), partial P = sum_w M_w Q per
+//           (row, column chunk); the last CTA of a row block sums the chunk
+//           partials into P_bar and a float64 Gram partial; the last row
+//           block of a layer factors the Gram matrix (Cholesky QR) into T.
+//   pass B: P_hat = P_bar T for the tile's rows; partial Q = sum_w M_w^T P_hat
+//           per (row block, column); the last CTA of a column chunk sums the
+//           row-block partials into Q_bar.
+//   pass C: rec = P_hat Q_bar^T per element; E'_w = M_w - rec, optional
+//           G_hat = rec, optional momentum.
+//
+// Step order from "anthology-of-the-sota" note-152 on PowerSGD, "Method".
+// Every cross-CTA sum runs in a fixed order, so results are bitwise
+// reproducible.  No CTA waits on another: the last CTA to arrive at a
+// counter does the reduction.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace psgd {
+
+// ---------------------------------------------------------------------------
+// tile decode
+struct TileCoord {
+    int l, rb, c;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const Params& p, const LayerDesc& d, int l) {
+    const int local = static_cast<int>(blockIdx.x - d.tile_begin);
+    TileCoord tc;
+    tc.l = l;
+    tc.rb = local / d.nchunk;
+    tc.c = local - tc.rb * d.nchunk;
+    return tc;
+}
+
+// ---------------------------------------------------------------------------
+// orthogonalisation: factor the r x r Gram matrix (float64) with one warp.
+// Cholesky G = R^T R column by column; column j is dropped (row j of R and
+// column j of T set to zero) if its pivot, the squared norm of p_bar_j after
+// projection on the kept columns before it, is <= drop_tol * max_k G_kk.
+// T = R^-1 on the kept columns, so P_hat = P_bar T.
+template <int R>
+__device__ void factor_gram_warp(const double* Gs, double* Rs, double* Ts, int* drop, int r, double drop_tol,
+                                 int lane) {
+    for (int idx = lane; idx < R * R; idx += 32) {
+        Rs[idx] = 0.0;
+        Ts[idx] = 0.0;
+    }
+    __syncwarp();
+    double maxd = 0.0;
+    for (int k = 0; k < r; ++k) maxd = fmax(maxd, Gs[k * R + k]);
+    const double tau = drop_tol * maxd;
+    for (int j = 0; j < r; ++j) {
+        double d = Gs[j * R + j];
+        for (int k = 0; k < j; ++k) d -= Rs[k * R + j] * Rs[k * R + j];
+        const bool dropped = (d <= tau);
+        const double rjj = dropped ? 0.0 : sqrt(d);
+        const int i = lane;
+        if (i > j && i < r) {
+            double s = Gs[j * R + i];
+            for (int k = 0; k < j; ++k) s -= Rs[k * R + j] * Rs[k * R + i];
+            Rs[j * R + i] = dropped ? 0.0 : s / rjj;
+        }
+        __syncwarp();
+        if (lane == 0) {
+            Rs[j * R + j] = rjj;
+            drop[j] = dropped ? 1 : 0;
+        }
+        __syncwarp();
+    }
+    for (int j = 0; j < r; ++j) {
+        const int l = lane;
+        if (l <= j) {
+            double t;
+            if (drop[j]) {
+                t = 0.0;
+            } else if (l == j) {
+                t = 1.0 / Rs[j * R + j];
+            } else {
+                double s = 0.0;
+                for (int k = l; k < j; ++k) s += Ts[l * R + k] * Rs[k * R + j];
+                t = -s / Rs[j * R + j];
+            }
+            Ts[l * R + j] = t;
+        }
+        __syncwarp();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// pass A
+
+template <int R>
+struct SmemA {
+    // layout inside dynamic shared memory (bytes)
+    static __host__ __device__ size_t ptr_bytes(int W) { return static_cast<size_t>(2 * W) * sizeof(void*); }
+    static __host__ __device__ size_t rows_bytes(int tm) { return static_cast<size_t>(tm) * R * sizeof(double); }
+    static __host__ __device__ size_t fac_bytes() { return 3 * R * R * sizeof(double) + 2 * R * sizeof(int) + 64; }
+    static __host__ __device__ size_t total(int W, int tm) {
+        return ((ptr_bytes(W) + 15) & ~size_t(15)) + ((rows_bytes(tm) + 15) & ~size_t(15)) + fac_bytes();
+    }
+};
+
+template <int R, int VEC, typename GT, bool LAZY, bool SF>
+__device__ __forceinline__ void pass_a_rows(const Params& p, const LayerDesc& d, const TileCoord& tc,
+                                            const GT* const* gp, float* const* ep, const float* ph_prev) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int r = p.r;
+    const int W = p.workers;
+    const int64_t n = d.n, m = d.m;
+    const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
+    const int64_t i1 = min(i0 + d.tm, m);
+    const int s0 = tc.c * d.slots;
+    const int ns = min(d.slots, d.nvec - s0);
+    const bool active = lane < ns;
+    const int64_t j = static_cast<int64_t>(s0 + (active ? lane : 0)) * VEC;
+
+    // warm-start Q rows of this lane's columns, zero-padded to R
+    float qv[VEC][R];
+    {
+        const float* Q = p.t.q[tc.l];
+#pragma unroll
+        for (int v = 0; v < VEC; ++v)
+#pragma unroll
+            for (int k = 0; k < R; ++k) qv[v][k] = (active && k < r) ? Q[(j + v) * r + k] : 0.f;
+    }
+    // previous Q_bar for rebuilding E' (lazy representation)
+    float qp[LAZY ? VEC : 1][LAZY ? R : 1];
+    if constexpr (LAZY) {
+        const float* Qb = p.ws.qbar + d.qrow_off;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v)
+#pragma unroll
+            for (int k = 0; k < R; ++k) qp[v][k] = (active && p.use_prev) ? Qb[(j + v) * R + k] : 0.f;
+    }
+
+    double* ppart = p.ws.ppart + d.ppart_off;
+    constexpr int U = (VEC == 4) ? 4 : 8;
+    constexpr int LG = Log2<R>::value;
+
+    for (int64_t i = i0 + warp; i < i1; i += kWarps) {
+        double acc[R];
+#pragma unroll
+        for (int k = 0; k < R; ++k) acc[k] = 0.0;
+        if (active) {
+            const int64_t base = i * n + j;
+            float rec[VEC];
+            if constexpr (LAZY) {
+                float ph[R];
+#pragma unroll
+                for (int k = 0; k < R; ++k) ph[k] = ph_prev[(i - i0) * R + k];
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) rec[v] = recon_dot<R>(ph, qp[v]);
+            }
+            float msum[VEC];
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) msum[v] = 0.f;
+            int w = 0;
+            for (; w + U <= W; w += U) {
+                float g[U][VEC], e[U][VEC];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    ld_grad<GT, VEC>(gp[w + u] + base, g[u]);
+                    ld_f32<VEC>(ep[w + u] + base, e[u]);
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) {
+                        float ev = e[u][v];
+                        if constexpr (LAZY) ev = ev - rec[v];
+                        e[u][v] = g[u][v] + ev;
+                    }
+                    st_f32<VEC>(ep[w + u] + base, e[u]);
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    if constexpr (SF) {
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) msum[v] += e[u][v];
+                    } else {
+                        // one worker's product over this lane's VEC columns
+                        // in float32, then accumulated in float64
+                        float pw[R];
+#pragma unroll
+                        for (int k = 0; k < R; ++k) pw[k] = 0.f;
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v)
+#pragma unroll
+                            for (int k = 0; k < R; ++k) pw[k] = fmaf(e[u][v], qv[v][k], pw[k]);
+#pragma unroll
+                        for (int k = 0; k < R; ++k) acc[k] += static_cast<double>(pw[k]);
+                    }
+                }
+            }
+            for (; w < W; ++w) {
+                float g[VEC], e[VEC];
+                ld_grad<GT, VEC>(gp[w] + base, g);
+                ld_f32<VEC>(ep[w] + base, e);
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) {
+                    float ev = e[v];
+                    if constexpr (LAZY) ev = ev - rec[v];
+                    e[v] = g[v] + ev;
+                }
+                st_f32<VEC>(ep[w] + base, e);
+                if constexpr (SF) {
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) msum[v] += e[v];
+                } else {
+                    float pw[R];
+#pragma unroll
+                    for (int k = 0; k < R; ++k) pw[k] = 0.f;
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v)
+#pragma unroll
+                        for (int k = 0; k < R; ++k) pw[k] = fmaf(e[v], qv[v][k], pw[k]);
+#pragma unroll
+                    for (int k = 0; k < R; ++k) acc[k] += static_cast<double>(pw[k]);
+                }
+            }
+            if constexpr (SF) {
+                float pw[R];
+#pragma unroll
+                for (int k = 0; k < R; ++k) pw[k] = 0.f;
+#pragma unroll
+                for (int v = 0; v < VEC; ++v)
+#pragma unroll
+                    for (int k = 0; k < R; ++k) pw[k] = fmaf(msum[v], qv[v][k], pw[k]);
+#pragma unroll
+                for (int k = 0; k < R; ++k) acc[k] = static_cast<double>(pw[k]);
+            }
+        }
+        TransposeReduce<double, R, 16>::run(acc, lane);
+        if ((lane & ((32 >> LG) - 1)) == 0) {
+            const int k = lane >> (5 - LG);
+            ppart[(static_cast<int64_t>(tc.c) * m + i) * R + k] = acc[0];
+        }
+    }
+}
+
+// Last CTA of a row block: P_bar rows and the Gram partial.  Last row block
+// of a layer: Gram sum and factorisation.
+template <int R>
+__device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileCoord& tc, double* pb_s,
+                                unsigned char* fac) {
+    __shared__ int s_flag;
+    constexpr int NG = R * (R + 1) / 2;
+    const int tid = threadIdx.x;
+    unsigned* cnt = p.ws.cnt + d.cnt_off;
+
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(&cnt[tc.rb], 1u);
+        if (prev >= static_cast<unsigned>(d.nchunk)) atomicOr(p.ws.status, kStatusCounter);
+        s_flag = (prev == static_cast<unsigned>(d.nchunk - 1));
+    }
+    __syncthreads();
+    if (!s_flag) return;
+    __threadfence();
+
+    const int64_t m = d.m;
+    const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
+    const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), m - i0));
+    const double* ppart = p.ws.ppart + d.ppart_off;
+    double* pbar = p.ws.pbar + d.prow_off;
+    const double inv_w = 1.0 / static_cast<double>(p.workers);
+    for (int idx = tid; idx < rows * R; idx += kThreads) {
+        const int64_t i = i0 + idx / R;
+        const int k = idx % R;
+        double s = 0.0;
+        for (int c = 0; c < d.nchunk; ++c) s += __ldcg(&ppart[(static_cast<int64_t>(c) * m + i) * R + k]);
+        const double v = s * inv_w;
+        pb_s[idx] = v;
+        pbar[i * R + k] = v;
+    }
+    if (tid == 0) cnt[tc.rb] = 0u;
+    __syncthreads();
+
+    // Gram partial of this row block, float64
+    double* gram = p.ws.gram + d.gram_off + static_cast<int64_t>(tc.rb) * NG;
+    for (int pidx = tid; pidx < NG; pidx += kThreads) {
+        int a = 0, rem = pidx;
+        while (rem >= R - a) {
+            rem -= R - a;
+            ++a;
+        }
+        const int b = a + rem;
+        double s = 0.0;
+        for (int ii = 0; ii < rows; ++ii) s += pb_s[ii * R + a] * pb_s[ii * R + b];
+        gram[pidx] = s;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(&cnt[d.nrb], 1u);
+        if (prev >= static_cast<unsigned>(d.nrb)) atomicOr(p.ws.status, kStatusCounter);
+        s_flag = (prev == static_cast<unsigned>(d.nrb - 1));
+    }
+    __syncthreads();
+    if (!s_flag) return;
+    __threadfence();
+
+    double* Gs = reinterpret_cast<double*>(fac);
+    double* Rs = Gs + R * R;
+    double* Ts = Rs + R * R;
+    int* drop = reinterpret_cast<int*>(Ts + R * R);
+    const double* gall = p.ws.gram + d.gram_off;
+    for (int pidx = tid; pidx < NG; pidx += kThreads) {
+        int a = 0, rem = pidx;
+        while (rem >= R - a) {
+            rem -= R - a;
+            ++a;
+        }
+        const int b = a + rem;
+        double s = 0.0;
+        for (int rb = 0; rb < d.nrb; ++rb) s += __ldcg(&gall[static_cast<int64_t>(rb) * NG + pidx]);
+        Gs[a * R + b] = s;
+        Gs[b * R + a] = s;
+    }
+    __syncthreads();
+    if (tid < 32) {
+        factor_gram_warp<R>(Gs, Rs, Ts, drop, p.r, p.drop_tol, tid);
+        double* T = p.ws.T + d.t_off;
+        for (int idx = tid; idx < R * R; idx += 32) T[idx] = Ts[idx];
+    }
+    if (tid == 0) cnt[d.nrb] = 0u;
+}
+
+template <int R, typename GT, bool LAZY, bool SF>
+__global__ void __launch_bounds__(kThreads, (R >= 32) ? 1 : 2) k_pass_a(Params p) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int l = p.t.tile_layer[blockIdx.x];
+    const LayerDesc d = p.t.layers[l];
+    const TileCoord tc = decode_tile(p, d, l);
+    const int W = p.workers;
+    const int L = p.num_layers;
+
+    const GT** gp = reinterpret_cast<const GT**>(smem);
+    float** ep = reinterpret_cast<float**>(smem + static_cast<size_t>(W) * sizeof(void*));
+    double* rows_d = reinterpret_cast<double*>(smem + ((SmemA<R>::ptr_bytes(W) + 15) & ~size_t(15)));
+    float* rows_s = reinterpret_cast<float*>(rows_d);
+    unsigned char* fac = reinterpret_cast<unsigned char*>(rows_d) + ((SmemA<R>::rows_bytes(d.tm) + 15) & ~size_t(15));
+
+    for (int w = threadIdx.x; w < W; w += kThreads) {
+        gp[w] = static_cast<const GT*>(p.t.grads[w * L + l]);
+        ep[w] = p.t.errors[w * L + l];
+    }
+    if constexpr (LAZY) {
+        const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
+        const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), d.m - i0));
+        const float* ph = p.ws.phat + d.prow_off + i0 * R;
+        for (int idx = threadIdx.x; idx < rows * R; idx += kThreads) rows_s[idx] = p.use_prev ? ph[idx] : 0.f;
+    }
+    __syncthreads();
+
+    if (d.vec == 4) {
+        if constexpr (R <= 8) pass_a_rows<R, 4, GT, LAZY, SF>(p, d, tc, gp, ep, rows_s);
+    } else if (d.vec == 2) {
+        if constexpr (R <= 16) pass_a_rows<R, 2, GT, LAZY, SF>(p, d, tc, gp, ep, rows_s);
+    } else {
+        pass_a_rows<R, 1, GT, LAZY, SF>(p, d, tc, gp, ep, rows_s);
+    }
+    pass_a_epilogue<R>(p, d, tc, rows_d, fac);
+}
+
+// ---------------------------------------------------------------------------
+// pass B
+
+template <int R>
+struct SmemB {
+    static __host__ __device__ size_t ptr_bytes(int W) { return static_cast<size_t>(W) * sizeof(void*); }
+    static __host__ __device__ size_t rows_bytes(int tm) { return static_cast<size_t>(tm) * R * sizeof(float); }
+    static __host__ __device__ size_t t_bytes() { return R * R * sizeof(double); }
+    static __host__ __device__ size_t red_bytes(int vec) {
+        return static_cast<size_t>(kWarps) * R * vec * 32 * sizeof(float);
+    }
+    static __host__ __device__ size_t total(int W, int tm, int vec) {
+        return ((ptr_bytes(W) + 15) & ~size_t(15)) + ((rows_bytes(tm) + 15) & ~size_t(15)) + t_bytes() +
+               red_bytes(vec);
+    }
+};
+
+// P_hat rows [i0, i0+rows) of a layer into shared memory: P_bar T, float64
+// accumulation in column order.  Chunk 0 also writes them out.
+template <int R>
+__device__ __forceinline__ void load_phat_rows(const Params& p, const LayerDesc& d, const TileCoord& tc,
+                                               float* ph_s, double* T_s, bool write_out) {
+    const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
+    const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), d.m - i0));
+    const double* T = p.ws.T + d.t_off;
+    for (int idx = threadIdx.x; idx < R * R; idx += kThreads) T_s[idx] = T[idx];
+    __syncthreads();
+    const double* pbar = p.ws.pbar + d.prow_off + i0 * R;
+    float* phat_ws = p.ws.phat + d.prow_off + i0 * R;
+    float* out = (p.t.p_hat_out != nullptr) ? p.t.p_hat_out[tc.l] : nullptr;
+    const int r = p.r;
+    for (int idx = threadIdx.x; idx < rows * R; idx += kThreads) {
+        const int ii = idx / R;
+        const int k = idx % R;
+        double s = 0.0;
+        for (int a = 0; a <= k; ++a) s += pbar[ii * R + a] * T_s[a * R + k];
+        const float v = static_cast<float>(s);
+        ph_s[idx] = v;
+        if (write_out) {
+            phat_ws[idx] = v;
+            if (out != nullptr && k < r) out[(i0 + ii) * r + k] = v;
+        }
+    }
+    __syncthreads();
+}
+
+template <int R, int VEC, bool SF>
+__device__ __forceinline__ void pass_b_rows(const Params& p, const LayerDesc& d, const TileCoord& tc,
+                                            float* const* ep, const float* ph_s, float* red_s) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int W = p.workers;
+    const int64_t n = d.n, m = d.m;
+    const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
+    const int64_t i1 = min(i0 + d.tm, m);
+    const int s0 = tc.c * d.slots;
+    const int ns = min(d.slots, d.nvec - s0);
+    const bool active = lane < ns;
+    const int64_t j = static_cast<int64_t>(s0 + (active ? lane : 0)) * VEC;
+    constexpr int U = (VEC == 4) ? 4 : 8;
+
+    float qacc[VEC][R];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v)
+#pragma unroll
+        for (int k = 0; k < R; ++k) qacc[v][k] = 0.f;
+
+    if (active) {
+        for (int64_t i = i0 + warp; i < i1; i += kWarps) {
+            float ph[R];
+#pragma unroll
+            for (int k = 0; k < R; ++k) ph[k] = ph_s[(i - i0) * R + k];
+            const int64_t base = i * n + j;
+            float msum[VEC];
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) msum[v] = 0.f;
+            int w = 0;
+            for (; w + U <= W; w += U) {
+                float e[U][VEC];
+#pragma unroll
+                for (int u = 0; u < U; ++u) ld_f32<VEC>(ep[w + u] + base, e[u]);
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    if constexpr (SF) {
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) msum[v] += e[u][v];
+                    } else {
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v)
+#pragma unroll
+                            for (int k = 0; k < R; ++k) qacc[v][k] = fmaf(e[u][v], ph[k], qacc[v][k]);
+                    }
+                }
+            }
+            for (; w < W; ++w) {
+                float e[VEC];
+                ld_f32<VEC>(ep[w] + base, e);
+                if constexpr (SF) {
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) msum[v] += e[v];
+                } else {
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v)
+#pragma unroll
+                        for (int k = 0; k < R; ++k) qacc[v][k] = fmaf(e[v], ph[k], qacc[v][k]);
+                }
+            }
+            if constexpr (SF) {
+#pragma unroll
+                for (int v = 0; v < VEC; ++v)
+#pragma unroll
+                    for (int k = 0; k < R; ++k) qacc[v][k] = fmaf(msum[v], ph[k], qacc[v][k]);
+            }
+        }
+    }
+    // this warp's partial, laid out [warp][k][v][lane] (conflict-free)
+#pragma unroll
+    for (int k = 0; k < R; ++k)
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) red_s[((warp * R + k) * VEC + v) * 32 + lane] = qacc[v][k];
+    __syncthreads();
+    // sum over warps in order; write the row block's partial Q rows
+    double* qpart = p.ws.qpart + d.qpart_off;
+    const int cols = ns * VEC;
+    for (int idx = threadIdx.x; idx < cols * R; idx += kThreads) {
+        const int cc = idx / R;        // local column
+        const int k = idx % R;
+        const int ln = cc / VEC, v = cc % VEC;
+        double s = 0.0;
+#pragma unroll
+        for (int wp = 0; wp < kWarps; ++wp) s += static_cast<double>(red_s[((wp * R + k) * VEC + v) * 32 + ln]);
+        qpart[(static_cast<int64_t>(tc.rb) * n + static_cast<int64_t>(s0) * VEC + cc) * R + k] = s;
+    }
+}
+
+template <int R>
+__device__ void pass_b_epilogue(const Params& p, const LayerDesc& d, const TileCoord& tc) {
+    __shared__ int s_flag;
+    const int tid = threadIdx.x;
+    unsigned* cnt = p.ws.cnt + d.cnt_off + d.nrb + 1;
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(&cnt[tc.c], 1u);
+        if (prev >= static_cast<unsigned>(d.nrb)) atomicOr(p.ws.status, kStatusCounter);
+        s_flag = (prev == static_cast<unsigned>(d.nrb - 1));
+    }
+    __syncthreads();
+    if (!s_flag) return;
+    __threadfence();
+    const int64_t n = d.n;
+    const int s0 = tc.c * d.slots;
+    const int ns = min(d.slots, d.nvec - s0);
+    const int64_t col0 = static_cast<int64_t>(s0) * d.vec;
+    const int cols = ns * d.vec;
+    const double* qpart = p.ws.qpart + d.qpart_off;
+    float* qbar = p.ws.qbar + d.qrow_off;
+    float* qout = p.t.q[tc.l];
+    const int r = p.r;
+    const double inv_w = 1.0 / static_cast<double>(p.workers);
+    for (int idx = tid; idx < cols * R; idx += kThreads) {
+        const int64_t col = col0 + idx / R;
+        const int k = idx % R;
+        double s = 0.0;
+        for (int rb = 0; rb < d.nrb; ++rb) s += __ldcg(&qpart[(static_cast<int64_t>(rb) * n + col) * R + k]);
+        const float v = static_cast<float>(s * inv_w);
+        qbar[col * R + k] = v;
+        if (k < r) qout[col * r + k] = v;
+    }
+    if (tid == 0) cnt[tc.c] = 0u;
+}
+
+template <int R, bool SF>
+__global__ void __launch_bounds__(kThreads, 2) k_pass_b(Params p) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int l = p.t.tile_layer[blockIdx.x];
+    const LayerDesc d = p.t.layers[l];
+    const TileCoord tc = decode_tile(p, d, l);
+    const int W = p.workers;
+    const int L = p.num_layers;
+
+    float** ep = reinterpret_cast<float**>(smem);
+    float* ph_s = reinterpret_cast<float*>(smem + ((SmemB<R>::ptr_bytes(W) + 15) & ~size_t(15)));
+    double* T_s = reinterpret_cast<double*>(reinterpret_cast<unsigned char*>(ph_s) +
+                                            ((SmemB<R>::rows_bytes(d.tm) + 15) & ~size_t(15)));
+    float* red_s = reinterpret_cast<float*>(T_s + R * R);
+
+    for (int w = threadIdx.x; w < W; w += kThreads) ep[w] = p.t.errors[w * L + l];
+    load_phat_rows<R>(p, d, tc, ph_s, T_s, tc.c == 0);
+
+    if (d.vec == 4) {
+        if constexpr (R <= 8) pass_b_rows<R, 4, SF>(p, d, tc, ep, ph_s, red_s);
+    } else if (d.vec == 2) {
+        if constexpr (R <= 16) pass_b_rows<R, 2, SF>(p, d, tc, ep, ph_s, red_s);
+    } else {
+        pass_b_rows<R, 1, SF>(p, d, tc, ep, ph_s, red_s);
+    }
+    pass_b_epilogue<R>(p, d, tc);
+}
+
+// ---------------------------------------------------------------------------
+// pass C: residual / decompression / momentum
+
+template <int R>
+struct SmemC {
+    static __host__ __device__ size_t ptr_bytes(int W) { return static_cast<size_t>(W < 1 ? 1 : W) * sizeof(void*); }
+    static __host__ __device__ size_t rows_bytes(int tm) { return static_cast<size_t>(tm) * R * sizeof(float); }
+    static __host__ __device__ size_t total(int W, int tm) {
+        return ((ptr_bytes(W) + 15) & ~size_t(15)) + rows_bytes(tm);
+    }
+};
+
+template <int R, int VEC>
+__device__ __forceinline__ void pass_c_rows(const Params& p, const LayerDesc& d, const TileCoord& tc,
+                                            float* const* ep, const float* ph_s) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int W = p.do_resid ? p.workers : 0;
+    const int64_t n = d.n, m = d.m;
+    const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
+    const int64_t i1 = min(i0 + d.tm, m);
+    const int s0 = tc.c * d.slots;
+    const int ns = min(d.slots, d.nvec - s0);
+    if (lane >= ns) return;
+    const int64_t j = static_cast<int64_t>(s0 + lane) * VEC;
+    constexpr int U = (VEC == 4) ? 4 : 8;
+
+    float qb[VEC][R];
+    {
+        const float* Qb = p.ws.qbar + d.qrow_off;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v)
+#pragma unroll
+            for (int k = 0; k < R; ++k) qb[v][k] = Qb[(j + v) * R + k];
+    }
+    float* recon = (p.do_recon && p.t.recon_out != nullptr) ? p.t.recon_out[tc.l] : nullptr;
+    float* xs = p.do_mom ? p.t.params[tc.l] : nullptr;
+    float* ms = p.do_mom ? p.t.mom[tc.l] : nullptr;
+
+    for (int64_t i = i0 + warp; i < i1; i += kWarps) {
+        float ph[R];
+#pragma unroll
+        for (int k = 0; k < R; ++k) ph[k] = ph_s[(i - i0) * R + k];
+        float rec[VEC];
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) rec[v] = recon_dot<R>(ph, qb[v]);
+        const int64_t base = i * n + j;
+        if (recon != nullptr) st_f32<VEC>(recon + base, rec);
+        if (xs != nullptr) {
+            float x[VEC], mo[VEC];
+            ld_f32<VEC>(xs + base, x);
+            ld_f32<VEC>(ms + base, mo);
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) {
+                mo[v] = fmaf(p.beta, mo[v], rec[v]);
+                x[v] = fmaf(-p.lr, mo[v], x[v]);
+            }
+            st_f32<VEC>(ms + base, mo);
+            st_f32<VEC>(xs + base, x);
+        }
+        int w = 0;
+        for (; w + U <= W; w += U) {
+            float e[U][VEC];
+#pragma unroll
+            for (int u = 0; u < U; ++u) ld_f32<VEC>(ep[w + u] + base, e[u]);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) e[u][v] = e[u][v] - rec[v];
+                st_f32<VEC>(ep[w + u] + base, e[u]);
+            }
+        }
+        for (; w < W; ++w) {
+            float e[VEC];
+            ld_f32<VEC>(ep[w] + base, e);
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) e[v] = e[v] - rec[v];
+            st_f32<VEC>(ep[w] + base, e);
+        }
+    }
+}
+
+template <int R>
+__global__ void __launch_bounds__(kThreads, 2) k_pass_c(Params p) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int l = p.t.tile_layer[blockIdx.x];
+    const LayerDesc d = p.t.layers[l];
+    const TileCoord tc = decode_tile(p, d, l);
+    const int W = p.workers;
+    const int L = p.num_layers;
+    float** ep = reinterpret_cast<float**>(smem);
+    float* ph_s = reinterpret_cast<float*>(smem + ((SmemC<R>::ptr_bytes(W) + 15) & ~size_t(15)));
+    if (p.do_resid)
+        for (int w = threadIdx.x; w < W; w += kThreads) ep[w] = p.t.errors[w * L + l];
+    {
+        const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
+        const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), d.m - i0));
+        const float* ph = p.ws.phat + d.prow_off + i0 * R;
+        for (int idx = threadIdx.x; idx < rows * R; idx += kThreads) ph_s[idx] = ph[idx];
+    }
+    __syncthreads();
+    if (d.vec == 4) {
+        if constexpr (R <= 8) pass_c_rows<R, 4>(p, d, tc, ep, ph_s);
+    } else if (d.vec == 2) {
+        if constexpr (R <= 16) pass_c_rows<R, 2>(p, d, tc, ep, ph_s);
+    } else {
+        pass_c_rows<R, 1>(p, d, tc, ep, ph_s);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// small tensors: mean over workers (+ optional momentum)
+__global__ void k_vec_mean(const float* const* vecs, float* const* out, const int64_t* len, int count, int W,
+                           float inv_w, float* const* params, float* const* mom, float lr, float beta) {
+    const int k = blockIdx.y;
+    const int64_t nk = len[k];
+    float* o = out[k];
+    float* x = (params != nullptr) ? params[k] : nullptr;
+    float* mo = (mom != nullptr) ? mom[k] : nullptr;
+    for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < nk;
+         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float s = 0.f;
+        for (int w = 0; w < W; ++w) s += vecs[w * count + k][e];
+        const float g = s * inv_w;
+        o[e] = g;
+        if (x != nullptr && mo != nullptr) {
+            const float mv = fmaf(beta, mo[e], g);
+            mo[e] = mv;
+            x[e] = fmaf(-lr, mv, x[e]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// initial Q: Philox4x64-10 (Salmon et al., SC'11) + Box-Muller (1958)
+struct Philox4x64 {
+    static constexpr uint64_t M0 = 0xD2E7470EE14C6C93ull;
+    static constexpr uint64_t M1 = 0xCA5A826395121157ull;
+    static constexpr uint64_t W0 = 0x9E3779B97F4A7C15ull;
+    static constexpr uint64_t W1 = 0xBB67AE8584CAA73Bull;
+    __device__ static void run(uint64_t (&x)[4], uint64_t k0, uint64_t k1) {
+#pragma unroll
+        for (int rnd = 0; rnd < 10; ++rnd) {
+            if (rnd) {
+                k0 += W0;
+                k1 += W1;
+            }
+            const uint64_t hi0 = __umul64hi(M0, x[0]), lo0 = M0 * x[0];
+            const uint64_t hi1 = __umul64hi(M1, x[2]), lo1 = M1 * x[2];
+            const uint64_t y0 = hi1 ^ x[1] ^ k0;
+            const uint64_t y2 = hi0 ^ x[3] ^ k1;
+            x[0] = y0;
+            x[1] = lo1;
+            x[2] = y2;
+            x[3] = lo0;
+        }
+    }
+};
+
+__global__ void k_init_q(float* const* q, const LayerDesc* layers, int r, uint64_t seed) {
+    const int l = blockIdx.y;
+    const int64_t total = layers[l].n * r;
+    const int64_t nb = (total + 3) / 4;
+    float* out = q[l];
+    constexpr double kTwoPi = 2.0 * 3.141592653589793;
+    for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nb;
+         b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        uint64_t x[4] = {static_cast<uint64_t>(b), 0ull, 0ull, 0ull};
+        Philox4x64::run(x, seed, static_cast<uint64_t>(l));
+        double z[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const double u0 = (static_cast<double>(x[2 * h] >> 11) + 0.5) * (1.0 / 9007199254740992.0);
+            const double u1 = (static_cast<double>(x[2 * h + 1] >> 11) + 0.5) * (1.0 / 9007199254740992.0);
+            const double rho = sqrt(-2.0 * log(u0));
+            z[2 * h] = rho * cos(kTwoPi * u1);
+            z[2 * h + 1] = rho * sin(kTwoPi * u1);
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int64_t e = 4 * b + t;
+            if (e < total) out[e] = static_cast<float>(z[t]);
+        }
+    }
+}
+
+}  // namespace psgd

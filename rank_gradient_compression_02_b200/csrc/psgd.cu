@@ -1,0 +1,767 @@
+// Host side of libpsgd: the C ABI declared in include/psgd.h.
+//
+// One context = one set of layer shapes, a rank, a worker count.  It owns
+// the descriptor table, the tile map, the workspace (P partials, P_bar,
+// P_hat, Gram partials, T, Q partials, Q_bar, counters, status word) and
+// the device copies of the caller's pointer tables.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <array>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "psgd.h"
+#include "kernels.cuh"
+
+using psgd::LayerDesc;
+
+namespace {
+
+constexpr double kDropTol = 1e-12;
+constexpr int64_t kTileTargetElems = 65536;  // worker elements per tile (all W workers)
+constexpr int kRowsFloatsMax = 2048;         // TM * R bound (shared-memory rows buffer)
+
+int pad_rank(int r) {
+    int R = 1;
+    while (R < r) R <<= 1;
+    return R;
+}
+
+int max_vec_for_rank(int R) { return R <= 8 ? 4 : (R <= 16 ? 2 : 1); }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Device copy of a host pointer table.  Re-uploaded only when the contents
+// change; uploads go through a small ring of pinned buffers so that an
+// upload never overwrites a host buffer a previous async copy still reads.
+class DevTable {
+public:
+    ~DevTable() { release(); }
+    void release() {
+        if (dev_) cudaFree(dev_);
+        for (int i = 0; i < kRing; ++i) {
+            if (ring_[i]) cudaFreeHost(ring_[i]);
+            if (ev_[i]) cudaEventDestroy(ev_[i]);
+            ring_[i] = nullptr;
+            ev_[i] = nullptr;
+        }
+        dev_ = nullptr;
+        cap_ = 0;
+        cache_.clear();
+        valid_ = false;
+    }
+    cudaError_t reserve(size_t words) {
+        if (dev_ && words <= cap_) return cudaSuccess;
+        release();
+        cudaError_t e = cudaMalloc(&dev_, std::max<size_t>(words, 1) * 8);
+        if (e != cudaSuccess) return e;
+        for (int i = 0; i < kRing; ++i) {
+            e = cudaMallocHost(&ring_[i], std::max<size_t>(words, 1) * 8);
+            if (e != cudaSuccess) return e;
+            e = cudaEventCreateWithFlags(&ev_[i], cudaEventDisableTiming);
+            if (e != cudaSuccess) return e;
+        }
+        cap_ = words;
+        return cudaSuccess;
+    }
+    // Returns cudaSuccess and uploads (on stream) when vals differ.
+    cudaError_t update(const std::vector<uint64_t>& vals, cudaStream_t stream) {
+        cudaError_t e = reserve(vals.size());
+        if (e != cudaSuccess) return e;
+        if (valid_ && vals == cache_) return cudaSuccess;
+        const int slot = next_;
+        next_ = (next_ + 1) % kRing;
+        e = cudaEventSynchronize(ev_[slot]);  // normally long complete
+        if (e != cudaSuccess) return e;
+        if (!vals.empty()) std::memcpy(ring_[slot], vals.data(), vals.size() * 8);
+        if (!vals.empty()) {
+            e = cudaMemcpyAsync(dev_, ring_[slot], vals.size() * 8, cudaMemcpyHostToDevice, stream);
+            if (e != cudaSuccess) return e;
+        }
+        e = cudaEventRecord(ev_[slot], stream);
+        if (e != cudaSuccess) return e;
+        cache_ = vals;
+        valid_ = true;
+        return cudaSuccess;
+    }
+    void* dev() const { return dev_; }
+
+private:
+    static constexpr int kRing = 4;
+    void* dev_ = nullptr;
+    void* ring_[kRing] = {nullptr, nullptr, nullptr, nullptr};
+    cudaEvent_t ev_[kRing] = {nullptr, nullptr, nullptr, nullptr};
+    int next_ = 0;
+    size_t cap_ = 0;
+    std::vector<uint64_t> cache_;
+    bool valid_ = false;
+};
+
+thread_local std::string g_create_error;
+
+}  // namespace
+
+struct psgd_ctx {
+    int device = 0;
+    int L = 0, W = 0, r = 0, R = 0;
+    int dtype = PSGD_F32;
+    unsigned flags = 0;
+    uint64_t seed = 0;
+    std::vector<psgd_layer> shapes;
+    std::vector<LayerDesc> desc;
+    int64_t ntiles = 0;
+    size_t smem_a = 0, smem_b = 0, smem_c = 0;
+
+    // device allocations
+    void* ws = nullptr;
+    size_t ws_bytes = 0;
+    LayerDesc* desc_d = nullptr;
+    int* tile_layer_d = nullptr;
+    psgd::Work work{};
+
+    DevTable tab_w;    // grads[W*L], errors[W*L]
+    DevTable tab_l;    // q[L], p_hat[L], recon[L]
+    DevTable tab_m;    // params[L], mom[L]
+    DevTable tab_e;    // errors[W*L] for materialisation
+    DevTable tab_v;    // vector tables
+    DevTable tab_q;    // q[L] for the initial draw
+
+    void* stage = nullptr;  // device staging of host gradients
+    size_t stage_bytes = 0;
+
+    // optional per-kernel timing (psgd_profile_*)
+    bool profiling = false;
+    std::vector<std::array<cudaEvent_t, 4>> prof_ev;
+    size_t prof_used = 0;
+
+    bool have_step = false;
+    bool errors_hold_m = false;
+    cudaStream_t last_stream = nullptr;
+    std::string err;
+};
+
+namespace {
+
+int fail(psgd_ctx* ctx, int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    if (ctx)
+        ctx->err = buf;
+    else
+        g_create_error = buf;
+    return code;
+}
+
+int cuda_fail(psgd_ctx* ctx, cudaError_t e, const char* what) {
+    return fail(ctx, PSGD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Keeps the caller's current device: switches to the context's device for
+// the duration of a call.
+struct DeviceGuard {
+    int prev = -1;
+    bool switched = false;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) {
+            switched = (cudaSetDevice(dev) == cudaSuccess);
+        }
+    }
+    ~DeviceGuard() {
+        if (switched) cudaSetDevice(prev);
+    }
+};
+
+// ---- kernel dispatch over the padded rank ---------------------------------
+
+template <int R>
+struct Launch {
+    static void* pass_a(int dtype, bool lazy, bool sf) {
+        if (dtype == PSGD_BF16) {
+            if (lazy) return sf ? (void*)psgd::k_pass_a<R, uint16_t, true, true> : (void*)psgd::k_pass_a<R, uint16_t, true, false>;
+            return sf ? (void*)psgd::k_pass_a<R, uint16_t, false, true> : (void*)psgd::k_pass_a<R, uint16_t, false, false>;
+        }
+        if (lazy) return sf ? (void*)psgd::k_pass_a<R, float, true, true> : (void*)psgd::k_pass_a<R, float, true, false>;
+        return sf ? (void*)psgd::k_pass_a<R, float, false, true> : (void*)psgd::k_pass_a<R, float, false, false>;
+    }
+    static void* pass_b(bool sf) { return sf ? (void*)psgd::k_pass_b<R, true> : (void*)psgd::k_pass_b<R, false>; }
+    static void* pass_c() { return (void*)psgd::k_pass_c<R>; }
+};
+
+void* kernel_ptr(int which, int R, int dtype, bool lazy, bool sf) {
+#define PSGD_CASE(RR)                                        \
+    case RR:                                                 \
+        if (which == 0) return Launch<RR>::pass_a(dtype, lazy, sf); \
+        if (which == 1) return Launch<RR>::pass_b(sf);       \
+        return Launch<RR>::pass_c();
+    switch (R) {
+        PSGD_CASE(1)
+        PSGD_CASE(2)
+        PSGD_CASE(4)
+        PSGD_CASE(8)
+        PSGD_CASE(16)
+        PSGD_CASE(32)
+        default:
+            return nullptr;
+    }
+#undef PSGD_CASE
+}
+
+size_t smem_need(int which, int R, int W, int tm, int vec) {
+#define PSGD_CASE(RR)                                                         \
+    case RR:                                                                  \
+        if (which == 0) return psgd::SmemA<RR>::total(W, tm);                 \
+        if (which == 1) return psgd::SmemB<RR>::total(W, tm, vec);            \
+        return psgd::SmemC<RR>::total(W, tm);
+    switch (R) {
+        PSGD_CASE(1)
+        PSGD_CASE(2)
+        PSGD_CASE(4)
+        PSGD_CASE(8)
+        PSGD_CASE(16)
+        PSGD_CASE(32)
+        default:
+            return 0;
+    }
+#undef PSGD_CASE
+}
+
+psgd::Params base_params(psgd_ctx* ctx) {
+    psgd::Params p{};
+    p.t.layers = ctx->desc_d;
+    p.t.tile_layer = ctx->tile_layer_d;
+    p.ws = ctx->work;
+    p.num_layers = ctx->L;
+    p.workers = ctx->W;
+    p.r = ctx->r;
+    p.inv_w = 1.0f / static_cast<float>(ctx->W);
+    p.drop_tol = kDropTol;
+    return p;
+}
+
+int launch(psgd_ctx* ctx, int which, bool lazy, const psgd::Params& p, size_t smem, cudaStream_t stream) {
+    if (ctx->ntiles == 0) return PSGD_OK;
+    void* fn = kernel_ptr(which, ctx->R, ctx->dtype, lazy, (ctx->flags & PSGD_FLAG_SUM_FIRST) != 0);
+    if (!fn) return fail(ctx, PSGD_ERR_ARG, "no kernel for rank %d", ctx->r);
+    void* args[] = {const_cast<psgd::Params*>(&p)};
+    cudaError_t e = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(ctx->ntiles)), dim3(psgd::kThreads), args, smem,
+                                     stream);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "kernel launch");
+    return PSGD_OK;
+}
+
+int check_ptr_array(psgd_ctx* ctx, const void* const* a, size_t count, bool allow_null_entries, const char* name) {
+    if (count && !a) return fail(ctx, PSGD_ERR_ARG, "%s: null pointer array", name);
+    for (size_t i = 0; i < count; ++i) {
+        if (!a[i]) {
+            if (allow_null_entries) continue;
+            return fail(ctx, PSGD_ERR_ARG, "%s[%zu] is null", name, i);
+        }
+        if (!aligned16(a[i])) return fail(ctx, PSGD_ERR_ALIGN, "%s[%zu] is not 16-byte aligned", name, i);
+    }
+    return PSGD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* psgd_last_error(const psgd_ctx* ctx) { return ctx ? ctx->err.c_str() : g_create_error.c_str(); }
+
+int psgd_create(psgd_ctx** out, const psgd_layer* layers, int num_layers, int rank, int workers, uint64_t seed,
+                int grad_dtype, unsigned flags) {
+    g_create_error.clear();
+    if (!out) return fail(nullptr, PSGD_ERR_ARG, "out is null");
+    *out = nullptr;
+    if (num_layers < 0 || (num_layers > 0 && !layers)) return fail(nullptr, PSGD_ERR_ARG, "bad layer list");
+    if (rank < 1 || rank > psgd::kMaxRank) return fail(nullptr, PSGD_ERR_ARG, "rank %d not in [1, 32]", rank);
+    if (workers < 1 || workers > psgd::kMaxWorkers)
+        return fail(nullptr, PSGD_ERR_ARG, "workers %d not in [1, %d]", workers, psgd::kMaxWorkers);
+    if (grad_dtype != PSGD_F32 && grad_dtype != PSGD_BF16) return fail(nullptr, PSGD_ERR_ARG, "bad grad dtype");
+    if (flags & ~(PSGD_FLAG_LAZY_ERRORS | PSGD_FLAG_SUM_FIRST)) return fail(nullptr, PSGD_ERR_ARG, "unknown flags");
+    for (int l = 0; l < num_layers; ++l) {
+        const int64_t m = layers[l].m, n = layers[l].n;
+        if (m < 1 || n < 1) return fail(nullptr, PSGD_ERR_ARG, "layer %d: shape %lld x %lld", l, (long long)m, (long long)n);
+        if (rank > m || rank > n)
+            return fail(nullptr, PSGD_ERR_ARG, "layer %d: rank %d > min(%lld, %lld)", l, rank, (long long)m, (long long)n);
+        if (m > (int64_t(1) << 31) || n > (int64_t(1) << 31) || m * n > (int64_t(1) << 40))
+            return fail(nullptr, PSGD_ERR_ARG, "layer %d too large", l);
+    }
+
+    psgd_ctx* ctx = new psgd_ctx();
+    cudaGetDevice(&ctx->device);
+    ctx->L = num_layers;
+    ctx->W = workers;
+    ctx->r = rank;
+    ctx->R = pad_rank(rank);
+    ctx->dtype = grad_dtype;
+    ctx->flags = flags;
+    ctx->seed = seed;
+    ctx->shapes.assign(layers, layers + num_layers);
+
+    const int R = ctx->R;
+    const int NG = R * (R + 1) / 2;
+    const int vmax = max_vec_for_rank(R);
+    const int tm_cap = std::min(512, kRowsFloatsMax / R);
+    int64_t tiles = 0, prow = 0, qrow = 0, ppart = 0, qpart = 0, gram = 0, tt = 0, cnt = 0;
+    std::vector<int> tile_layer;
+    for (int l = 0; l < num_layers; ++l) {
+        LayerDesc d{};
+        d.m = layers[l].m;
+        d.n = layers[l].n;
+        int vec = 1;
+        for (int v : {4, 2, 1})
+            if (v <= vmax && d.n % v == 0) {
+                vec = v;
+                break;
+            }
+        d.vec = vec;
+        d.nvec = static_cast<int>(d.n / vec);
+        d.nchunk = (d.nvec + 31) / 32;
+        d.slots = (d.nvec + d.nchunk - 1) / d.nchunk;
+        const int64_t cols = static_cast<int64_t>(d.slots) * vec;
+        int64_t tm = (kTileTargetElems + cols * workers - 1) / (cols * workers);
+        tm = (tm + 7) / 8 * 8;
+        tm = std::max<int64_t>(8, std::min<int64_t>(tm, tm_cap));
+        tm = std::min<int64_t>(tm, (d.m + 7) / 8 * 8);
+        d.tm = static_cast<int>(tm);
+        d.nrb = static_cast<int>((d.m + tm - 1) / tm);
+        d.tile_begin = tiles;
+        d.prow_off = prow;
+        d.qrow_off = qrow;
+        d.ppart_off = ppart;
+        d.qpart_off = qpart;
+        d.gram_off = gram;
+        d.t_off = tt;
+        d.cnt_off = cnt;
+        const int64_t nt = static_cast<int64_t>(d.nrb) * d.nchunk;
+        tiles += nt;
+        prow += d.m * R;
+        qrow += d.n * R;
+        ppart += static_cast<int64_t>(d.nchunk) * d.m * R;
+        qpart += static_cast<int64_t>(d.nrb) * d.n * R;
+        gram += static_cast<int64_t>(d.nrb) * NG;
+        tt += R * R;
+        cnt += d.nrb + 1 + d.nchunk;
+        for (int64_t t = 0; t < nt; ++t) tile_layer.push_back(l);
+        ctx->desc.push_back(d);
+        ctx->smem_a = std::max(ctx->smem_a, smem_need(0, R, workers, d.tm, d.vec));
+        ctx->smem_b = std::max(ctx->smem_b, smem_need(1, R, workers, d.tm, d.vec));
+        ctx->smem_c = std::max(ctx->smem_c, smem_need(2, R, workers, d.tm, d.vec));
+    }
+    if (tiles > 0x7fffffff) {
+        delete ctx;
+        return fail(nullptr, PSGD_ERR_ARG, "too many tiles");
+    }
+    ctx->ntiles = tiles;
+
+    // one workspace allocation, carved into 256-byte aligned pieces
+    size_t off = 0;
+    auto carve = [&](size_t bytes) {
+        const size_t o = off;
+        off = align_up(off + std::max<size_t>(bytes, 1), 256);
+        return o;
+    };
+    const size_t o_desc = carve(sizeof(LayerDesc) * std::max(1, num_layers));
+    const size_t o_tile = carve(sizeof(int) * std::max<int64_t>(1, tiles));
+    const size_t o_pbar = carve(sizeof(double) * prow);
+    const size_t o_phat = carve(sizeof(float) * prow);
+    const size_t o_qbar = carve(sizeof(float) * qrow);
+    const size_t o_ppart = carve(sizeof(double) * ppart);
+    const size_t o_qpart = carve(sizeof(double) * qpart);
+    const size_t o_gram = carve(sizeof(double) * gram);
+    const size_t o_T = carve(sizeof(double) * tt);
+    const size_t o_cnt = carve(sizeof(unsigned) * cnt);
+    const size_t o_status = carve(sizeof(int));
+    ctx->ws_bytes = off;
+    cudaError_t e = cudaMalloc(&ctx->ws, ctx->ws_bytes);
+    if (e != cudaSuccess) {
+        fail(nullptr, PSGD_ERR_OOM, "workspace of %zu bytes: %s", ctx->ws_bytes, cudaGetErrorString(e));
+        delete ctx;
+        return PSGD_ERR_OOM;
+    }
+    unsigned char* base = static_cast<unsigned char*>(ctx->ws);
+    ctx->desc_d = reinterpret_cast<LayerDesc*>(base + o_desc);
+    ctx->tile_layer_d = reinterpret_cast<int*>(base + o_tile);
+    ctx->work.pbar = reinterpret_cast<double*>(base + o_pbar);
+    ctx->work.phat = reinterpret_cast<float*>(base + o_phat);
+    ctx->work.qbar = reinterpret_cast<float*>(base + o_qbar);
+    ctx->work.ppart = reinterpret_cast<double*>(base + o_ppart);
+    ctx->work.qpart = reinterpret_cast<double*>(base + o_qpart);
+    ctx->work.gram = reinterpret_cast<double*>(base + o_gram);
+    ctx->work.T = reinterpret_cast<double*>(base + o_T);
+    ctx->work.cnt = reinterpret_cast<unsigned*>(base + o_cnt);
+    ctx->work.status = reinterpret_cast<int*>(base + o_status);
+
+    e = cudaMemset(ctx->ws, 0, ctx->ws_bytes);
+    if (e == cudaSuccess && num_layers > 0)
+        e = cudaMemcpy(ctx->desc_d, ctx->desc.data(), sizeof(LayerDesc) * num_layers, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && tiles > 0)
+        e = cudaMemcpy(ctx->tile_layer_d, tile_layer.data(), sizeof(int) * tiles, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        fail(nullptr, PSGD_ERR_CUDA, "workspace init: %s", cudaGetErrorString(e));
+        cudaFree(ctx->ws);
+        delete ctx;
+        return PSGD_ERR_CUDA;
+    }
+    // opt in to the dynamic shared memory each kernel of this context needs
+    for (int lazy = 0; lazy < 2; ++lazy) {
+        const bool sf = (flags & PSGD_FLAG_SUM_FIRST) != 0;
+        const void* fa = kernel_ptr(0, R, grad_dtype, lazy != 0, sf);
+        const void* fb = kernel_ptr(1, R, grad_dtype, lazy != 0, sf);
+        const void* fc = kernel_ptr(2, R, grad_dtype, lazy != 0, sf);
+        e = cudaFuncSetAttribute(fa, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->smem_a));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fb, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->smem_b));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fc, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->smem_c));
+        if (e != cudaSuccess) {
+            fail(nullptr, PSGD_ERR_CUDA, "shared-memory opt-in: %s", cudaGetErrorString(e));
+            cudaFree(ctx->ws);
+            delete ctx;
+            return PSGD_ERR_CUDA;
+        }
+    }
+    *out = ctx;
+    return PSGD_OK;
+}
+
+void psgd_destroy(psgd_ctx* ctx) {
+    if (!ctx) return;
+    DeviceGuard g(ctx->device);
+    cudaDeviceSynchronize();
+    if (ctx->ws) cudaFree(ctx->ws);
+    if (ctx->stage) cudaFree(ctx->stage);
+    ctx->tab_w.release();
+    ctx->tab_l.release();
+    ctx->tab_m.release();
+    ctx->tab_e.release();
+    ctx->tab_v.release();
+    ctx->tab_q.release();
+    for (auto& a : ctx->prof_ev)
+        for (auto& x : a) cudaEventDestroy(x);
+    delete ctx;
+}
+
+int psgd_workspace_bytes(const psgd_ctx* ctx, size_t* bytes) {
+    if (!ctx || !bytes) return PSGD_ERR_ARG;
+    *bytes = ctx->ws_bytes;
+    return PSGD_OK;
+}
+
+int psgd_step_launches(const psgd_ctx* ctx) {
+    if (!ctx) return -1;
+    if (ctx->ntiles == 0) return 0;
+    return (ctx->flags & PSGD_FLAG_LAZY_ERRORS) ? 2 : 3;
+}
+
+int psgd_init_q(psgd_ctx* ctx, float* const* q, void* stream) {
+    if (!ctx) return PSGD_ERR_ARG;
+    ctx->err.clear();
+    int rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(q), ctx->L, false, "q");
+    if (rc) return rc;
+    if (ctx->L == 0) return PSGD_OK;
+    DeviceGuard g(ctx->device);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    std::vector<uint64_t> tab(ctx->L, 0);
+    for (int l = 0; l < ctx->L; ++l) tab[l] = reinterpret_cast<uint64_t>(q[l]);
+    cudaError_t e = ctx->tab_q.update(tab, s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "table upload");
+    int64_t maxn = 0;
+    for (auto& d : ctx->desc) maxn = std::max(maxn, d.n);
+    const int64_t blocks4 = (maxn * ctx->r + 3) / 4;
+    const unsigned gx = static_cast<unsigned>(std::min<int64_t>(1024, (blocks4 + 255) / 256));
+    psgd::k_init_q<<<dim3(std::max(1u, gx), ctx->L), 256, 0, s>>>(static_cast<float* const*>(ctx->tab_q.dev()),
+                                                                  ctx->desc_d, ctx->r, ctx->seed);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "init_q launch");
+    ctx->last_stream = s;
+    return PSGD_OK;
+}
+
+static int step_impl(psgd_ctx* ctx, const void* const* grads, float* const* errors, float* const* q,
+                     float* const* p_hat, float* const* recon, cudaStream_t s) {
+    const size_t WL = static_cast<size_t>(ctx->W) * ctx->L;
+    std::vector<uint64_t> tw(2 * WL);
+    for (size_t i = 0; i < WL; ++i) {
+        tw[i] = reinterpret_cast<uint64_t>(grads[i]);
+        tw[WL + i] = reinterpret_cast<uint64_t>(errors[i]);
+    }
+    std::vector<uint64_t> tl(3 * ctx->L, 0);
+    for (int l = 0; l < ctx->L; ++l) {
+        tl[l] = reinterpret_cast<uint64_t>(q[l]);
+        tl[ctx->L + l] = p_hat ? reinterpret_cast<uint64_t>(p_hat[l]) : 0;
+        tl[2 * ctx->L + l] = recon ? reinterpret_cast<uint64_t>(recon[l]) : 0;
+    }
+    cudaError_t e = ctx->tab_w.update(tw, s);
+    if (e == cudaSuccess) e = ctx->tab_l.update(tl, s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "table upload");
+
+    const bool lazy = (ctx->flags & PSGD_FLAG_LAZY_ERRORS) != 0;
+    psgd::Params p = base_params(ctx);
+    void* const* wt = static_cast<void* const*>(ctx->tab_w.dev());
+    void* const* lt = static_cast<void* const*>(ctx->tab_l.dev());
+    p.t.grads = reinterpret_cast<const void* const*>(wt);
+    p.t.errors = reinterpret_cast<float* const*>(wt + WL);
+    p.t.q = reinterpret_cast<float* const*>(lt);
+    p.t.p_hat_out = reinterpret_cast<float* const*>(lt + ctx->L);
+    p.t.recon_out = reinterpret_cast<float* const*>(lt + 2 * ctx->L);
+    p.use_prev = (lazy && ctx->errors_hold_m) ? 1 : 0;
+
+    cudaEvent_t* ev = nullptr;
+    if (ctx->profiling) {
+        if (ctx->prof_used == ctx->prof_ev.size()) {
+            std::array<cudaEvent_t, 4> a{};
+            for (auto& x : a) {
+                e = cudaEventCreate(&x);
+                if (e != cudaSuccess) return cuda_fail(ctx, e, "profiling event");
+            }
+            ctx->prof_ev.push_back(a);
+        }
+        ev = ctx->prof_ev[ctx->prof_used++].data();
+        cudaEventRecord(ev[0], s);
+    }
+    int rc = launch(ctx, 0, lazy, p, ctx->smem_a, s);
+    if (ev) cudaEventRecord(ev[1], s);
+    if (!rc) rc = launch(ctx, 1, lazy, p, ctx->smem_b, s);
+    if (ev) cudaEventRecord(ev[2], s);
+    if (!rc && (!lazy || recon)) {
+        psgd::Params pc = p;
+        pc.do_resid = lazy ? 0 : 1;
+        pc.do_recon = recon ? 1 : 0;
+        rc = launch(ctx, 2, lazy, pc, ctx->smem_c, s);
+    }
+    if (ev) cudaEventRecord(ev[3], s);
+    if (rc) return rc;
+    ctx->have_step = true;
+    ctx->errors_hold_m = lazy;
+    ctx->last_stream = s;
+    return PSGD_OK;
+}
+
+int psgd_step(psgd_ctx* ctx, const void* const* grads, float* const* errors, float* const* q, float* const* p_hat,
+              float* const* recon, void* stream) {
+    if (!ctx) return PSGD_ERR_ARG;
+    ctx->err.clear();
+    if (ctx->L == 0) return PSGD_OK;
+    const size_t WL = static_cast<size_t>(ctx->W) * ctx->L;
+    int rc = check_ptr_array(ctx, grads, WL, false, "grads");
+    if (!rc) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(errors), WL, false, "errors");
+    if (!rc) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(q), ctx->L, false, "q");
+    if (!rc && p_hat) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(p_hat), ctx->L, true, "p_hat");
+    if (!rc && recon) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(recon), ctx->L, true, "recon");
+    if (rc) return rc;
+    DeviceGuard g(ctx->device);
+    return step_impl(ctx, grads, errors, q, p_hat, recon, static_cast<cudaStream_t>(stream));
+}
+
+int psgd_step_host(psgd_ctx* ctx, const void* const* grads_host, float* const* errors, float* const* q,
+                   float* const* p_hat_host, float* const* q_host, void* stream) {
+    if (!ctx) return PSGD_ERR_ARG;
+    ctx->err.clear();
+    if (ctx->L == 0) return PSGD_OK;
+    const size_t WL = static_cast<size_t>(ctx->W) * ctx->L;
+    if (!grads_host) return fail(ctx, PSGD_ERR_ARG, "grads_host is null");
+    for (size_t i = 0; i < WL; ++i)
+        if (!grads_host[i]) return fail(ctx, PSGD_ERR_ARG, "grads_host[%zu] is null", i);
+    int rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(errors), WL, false, "errors");
+    if (!rc) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(q), ctx->L, false, "q");
+    if (rc) return rc;
+    DeviceGuard g(ctx->device);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t esz = ctx->dtype == PSGD_BF16 ? 2 : 4;
+    // staging layout: worker-major, every matrix 256-byte aligned
+    std::vector<size_t> offs(ctx->L);
+    size_t per_worker = 0;
+    for (int l = 0; l < ctx->L; ++l) {
+        offs[l] = per_worker;
+        per_worker = align_up(per_worker + static_cast<size_t>(ctx->desc[l].m * ctx->desc[l].n) * esz, 256);
+    }
+    const size_t need = per_worker * ctx->W;
+    if (need > ctx->stage_bytes) {
+        if (ctx->stage) cudaFree(ctx->stage);
+        ctx->stage = nullptr;
+        ctx->stage_bytes = 0;
+        cudaError_t e = cudaMalloc(&ctx->stage, need);
+        if (e != cudaSuccess) return fail(ctx, PSGD_ERR_OOM, "staging of %zu bytes: %s", need, cudaGetErrorString(e));
+        ctx->stage_bytes = need;
+    }
+    std::vector<const void*> dev_grads(WL);
+    for (int w = 0; w < ctx->W; ++w)
+        for (int l = 0; l < ctx->L; ++l) {
+            unsigned char* dst = static_cast<unsigned char*>(ctx->stage) + per_worker * w + offs[l];
+            const size_t bytes = static_cast<size_t>(ctx->desc[l].m * ctx->desc[l].n) * esz;
+            cudaError_t e = cudaMemcpyAsync(dst, grads_host[w * ctx->L + l], bytes, cudaMemcpyHostToDevice, s);
+            if (e != cudaSuccess) return cuda_fail(ctx, e, "gradient upload");
+            dev_grads[w * ctx->L + l] = dst;
+        }
+    rc = step_impl(ctx, dev_grads.data(), errors, q, nullptr, nullptr, s);
+    if (rc) return rc;
+    for (int l = 0; l < ctx->L; ++l) {
+        const LayerDesc& d = ctx->desc[l];
+        if (p_hat_host && p_hat_host[l]) {
+            // P_hat lives in the workspace with a padded row stride R
+            cudaError_t e = cudaMemcpy2DAsync(p_hat_host[l], sizeof(float) * ctx->r, ctx->work.phat + d.prow_off,
+                                              sizeof(float) * ctx->R, sizeof(float) * ctx->r, d.m,
+                                              cudaMemcpyDeviceToHost, s);
+            if (e != cudaSuccess) return cuda_fail(ctx, e, "P_hat download");
+        }
+        if (q_host && q_host[l]) {
+            cudaError_t e = cudaMemcpyAsync(q_host[l], q[l], sizeof(float) * d.n * ctx->r, cudaMemcpyDeviceToHost, s);
+            if (e != cudaSuccess) return cuda_fail(ctx, e, "Q download");
+        }
+    }
+    return PSGD_OK;
+}
+
+int psgd_materialize_errors(psgd_ctx* ctx, float* const* errors, void* stream) {
+    if (!ctx) return PSGD_ERR_ARG;
+    ctx->err.clear();
+    if (!(ctx->flags & PSGD_FLAG_LAZY_ERRORS)) return fail(ctx, PSGD_ERR_STATE, "context is not in lazy-error mode");
+    if (ctx->L == 0 || !ctx->errors_hold_m) return PSGD_OK;
+    const size_t WL = static_cast<size_t>(ctx->W) * ctx->L;
+    int rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(errors), WL, false, "errors");
+    if (rc) return rc;
+    DeviceGuard g(ctx->device);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    std::vector<uint64_t> te(WL);
+    for (size_t i = 0; i < WL; ++i) te[i] = reinterpret_cast<uint64_t>(errors[i]);
+    cudaError_t e = ctx->tab_e.update(te, s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "table upload");
+    psgd::Params p = base_params(ctx);
+    p.t.errors = static_cast<float* const*>(ctx->tab_e.dev());
+    p.do_resid = 1;
+    rc = launch(ctx, 2, true, p, ctx->smem_c, s);
+    if (rc) return rc;
+    ctx->errors_hold_m = false;
+    ctx->last_stream = s;
+    return PSGD_OK;
+}
+
+int psgd_momentum_step(psgd_ctx* ctx, float* const* params, float* const* mom, float lr, float beta, void* stream) {
+    if (!ctx) return PSGD_ERR_ARG;
+    ctx->err.clear();
+    if (ctx->L == 0) return PSGD_OK;
+    if (!ctx->have_step) return fail(ctx, PSGD_ERR_STATE, "no step has run yet");
+    int rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(params), ctx->L, false, "params");
+    if (!rc) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(mom), ctx->L, false, "mom");
+    if (rc) return rc;
+    DeviceGuard g(ctx->device);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    std::vector<uint64_t> tm(2 * ctx->L);
+    for (int l = 0; l < ctx->L; ++l) {
+        tm[l] = reinterpret_cast<uint64_t>(params[l]);
+        tm[ctx->L + l] = reinterpret_cast<uint64_t>(mom[l]);
+    }
+    cudaError_t e = ctx->tab_m.update(tm, s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "table upload");
+    psgd::Params p = base_params(ctx);
+    void* const* mt = static_cast<void* const*>(ctx->tab_m.dev());
+    p.t.params = reinterpret_cast<float* const*>(mt);
+    p.t.mom = reinterpret_cast<float* const*>(mt + ctx->L);
+    p.do_mom = 1;
+    p.lr = lr;
+    p.beta = beta;
+    rc = launch(ctx, 2, (ctx->flags & PSGD_FLAG_LAZY_ERRORS) != 0, p, ctx->smem_c, s);
+    if (rc) return rc;
+    ctx->last_stream = s;
+    return PSGD_OK;
+}
+
+int psgd_vec_mean(psgd_ctx* ctx, const float* const* vecs, float* const* out, const int64_t* len, int count,
+                  float* const* params, float* const* mom, float lr, float beta, void* stream) {
+    if (!ctx) return PSGD_ERR_ARG;
+    ctx->err.clear();
+    if (count < 0) return fail(ctx, PSGD_ERR_ARG, "count < 0");
+    if (count == 0) return PSGD_OK;
+    if (!len) return fail(ctx, PSGD_ERR_ARG, "len is null");
+    if (count > 65535) return fail(ctx, PSGD_ERR_ARG, "too many vectors");
+    if ((params == nullptr) != (mom == nullptr)) return fail(ctx, PSGD_ERR_ARG, "params and mom go together");
+    const size_t WK = static_cast<size_t>(ctx->W) * count;
+    int rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(vecs), WK, false, "vecs");
+    if (!rc) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(out), count, false, "out");
+    if (!rc && params) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(params), count, false, "params");
+    if (!rc && mom) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(mom), count, false, "mom");
+    if (rc) return rc;
+    int64_t maxlen = 0;
+    for (int k = 0; k < count; ++k) {
+        if (len[k] < 0) return fail(ctx, PSGD_ERR_ARG, "len[%d] < 0", k);
+        maxlen = std::max(maxlen, len[k]);
+    }
+    if (maxlen == 0) return PSGD_OK;
+    DeviceGuard g(ctx->device);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // table: vecs[W*K] | out[K] | params[K] | mom[K] | len[K]
+    std::vector<uint64_t> tv(WK + 4 * static_cast<size_t>(count), 0);
+    for (size_t i = 0; i < WK; ++i) tv[i] = reinterpret_cast<uint64_t>(vecs[i]);
+    for (int k = 0; k < count; ++k) {
+        tv[WK + k] = reinterpret_cast<uint64_t>(out[k]);
+        tv[WK + count + k] = params ? reinterpret_cast<uint64_t>(params[k]) : 0;
+        tv[WK + 2 * count + k] = mom ? reinterpret_cast<uint64_t>(mom[k]) : 0;
+        tv[WK + 3 * count + k] = static_cast<uint64_t>(len[k]);
+    }
+    cudaError_t e = ctx->tab_v.update(tv, s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "table upload");
+    uint64_t* t = static_cast<uint64_t*>(ctx->tab_v.dev());
+    const unsigned gx = static_cast<unsigned>(std::min<int64_t>(256, (maxlen + 255) / 256));
+    psgd::k_vec_mean<<<dim3(gx, count), 256, 0, s>>>(
+        reinterpret_cast<const float* const*>(t), reinterpret_cast<float* const*>(t + WK),
+        reinterpret_cast<const int64_t*>(t + WK + 3 * count), count, ctx->W, 1.0f / static_cast<float>(ctx->W),
+        params ? reinterpret_cast<float* const*>(t + WK + count) : nullptr,
+        mom ? reinterpret_cast<float* const*>(t + WK + 2 * count) : nullptr, lr, beta);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "vec_mean launch");
+    ctx->last_stream = s;
+    return PSGD_OK;
+}
+
+int psgd_profile_enable(psgd_ctx* ctx, int enable) {
+    if (!ctx) return PSGD_ERR_ARG;
+    ctx->profiling = enable != 0;
+    return PSGD_OK;
+}
+
+int psgd_profile_read(psgd_ctx* ctx, double* ms, int* steps) {
+    if (!ctx || !ms || !steps) return PSGD_ERR_ARG;
+    DeviceGuard g(ctx->device);
+    ms[0] = ms[1] = ms[2] = 0.0;
+    for (size_t i = 0; i < ctx->prof_used; ++i) {
+        auto& a = ctx->prof_ev[i];
+        cudaError_t e = cudaEventSynchronize(a[3]);
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "profile sync");
+        for (int k = 0; k < 3; ++k) {
+            float t = 0.f;
+            e = cudaEventElapsedTime(&t, a[k], a[k + 1]);
+            if (e != cudaSuccess) return cuda_fail(ctx, e, "profile elapsed");
+            ms[k] += t;
+        }
+    }
+    *steps = static_cast<int>(ctx->prof_used);
+    ctx->prof_used = 0;
+    return PSGD_OK;
+}
+
+int psgd_status(psgd_ctx* ctx) {
+    if (!ctx) return PSGD_ERR_ARG;
+    DeviceGuard g(ctx->device);
+    cudaError_t e = cudaStreamSynchronize(ctx->last_stream);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "synchronise");
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "pending error");
+    int st = 0;
+    e = cudaMemcpy(&st, ctx->work.status, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "status read");
+    if (st) return fail(ctx, PSGD_ERR_DEVICE, "device status word 0x%x", st);
+    return PSGD_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,275 @@
+"""GPU parity: the CUDA library (through its C ABI) against the float64
+oracle on the same seeded inputs, element by element (relative Frobenius
+norms), at sizes that span several tiles and ragged tails."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.powersgd64 as ora
+from oracle import philox64
+from synth import C0, GradientSource
+
+from . import _harness as H
+
+pytestmark = pytest.mark.gpu
+
+# shapes with every vector width (n % 4 == 0, n % 2 == 0, n odd), tall and
+# wide, chunks with ragged tails, and min(m, n) = 33 so every rank fits
+MIXED = [(300, 650), (64, 576), (40, 130), (256, 128), (33, 37), (700, 33), (129, 1000)]
+
+
+@pytest.mark.parametrize("rank", [1, 2, 3, 4, 8, 16, 32])
+@pytest.mark.parametrize("workers", [1, 3])
+def test_mixed_shapes_f32(rank, workers):
+    wl = H.small_workload(MIXED, rank, workers)
+    _, _, hist = H.run_free(wl, steps=3)
+    for t, e in enumerate(hist):
+        H.assert_close(e, H.TOL["f32"], f"step {t}")
+
+
+@pytest.mark.parametrize("rank", [1, 4, 16])
+def test_mixed_shapes_bf16(rank):
+    wl = H.small_workload(MIXED, rank, 4, dtype="bf16")
+    _, _, hist = H.run_free(wl, steps=3)
+    for t, e in enumerate(hist):
+        # the oracle reads the same bf16 values widened exactly, so the
+        # error stays at float32 level although the bar is 2e-2
+        H.assert_close(e, H.TOL["bf16"], f"step {t}")
+        H.assert_close(e, 1e-4, f"step {t} (fp32-level)")
+
+
+@pytest.mark.parametrize("rank", [2, 8])
+def test_sixteen_workers(rank):
+    wl = H.small_workload(MIXED[:4], rank, 16)
+    _, _, hist = H.run_free(wl, steps=2)
+    for t, e in enumerate(hist):
+        H.assert_close(e, H.TOL["f32"], f"step {t}")
+
+
+@pytest.mark.parametrize("lazy,sum_first", [(True, False), (False, True), (True, True)])
+def test_modes(lazy, sum_first):
+    wl = H.small_workload(MIXED, 4, 3)
+    _, _, hist = H.run_free(wl, steps=4, lazy=lazy, sum_first=sum_first)
+    for t, e in enumerate(hist):
+        H.assert_close(e, H.TOL["f32"], f"step {t}")
+
+
+def test_from_random_state():
+    wl = H.small_workload(MIXED, 4, 3)
+    _, _, hist = H.run_free(wl, steps=2, random_state=0.05)
+    for t, e in enumerate(hist):
+        H.assert_close(e, H.TOL["f32"], f"step {t}")
+
+
+def test_single_matrix_workload_all_steps():
+    # 256 x 128, r = 2, W = 1, 10 warm-started steps, absolute noise 0.01
+    _, _, hist = H.run_free(C0, steps=C0.steps)
+    for t, e in enumerate(hist):
+        H.assert_close(e, H.TOL["f32"], f"step {t}")
+
+
+def _run_steps(wl, steps, lazy=False, seed=1234):
+    run = H.LibRun(wl, seed=seed, lazy=lazy)
+    for t in range(steps):
+        run.fill_grads_host(t)
+        run.run_step()
+    if lazy:
+        run.lib.materialize_errors(run.E)
+    torch.cuda.synchronize()
+    return run
+
+
+def test_bitwise_deterministic():
+    wl = H.small_workload(MIXED, 4, 3)
+    a = _run_steps(wl, 3)
+    b = _run_steps(wl, 3)
+    for l in range(len(wl.layers)):
+        assert torch.equal(a.Q[l], b.Q[l])
+        assert torch.equal(a.P[l], b.P[l])
+        for w in range(wl.workers):
+            assert torch.equal(a.E[w][l], b.E[w][l])
+
+
+def test_lazy_equals_eager_bitwise():
+    # E' = M - P_hat Q_bar^T rebuilt in the next step's first pass is the
+    # same float32 arithmetic as the eager residual, so the runs agree bit
+    # for bit
+    wl = H.small_workload(MIXED, 4, 3)
+    a = _run_steps(wl, 4, lazy=False)
+    b = _run_steps(wl, 4, lazy=True)
+    for l in range(len(wl.layers)):
+        assert torch.equal(a.Q[l], b.Q[l])
+        assert torch.equal(a.P[l], b.P[l])
+        for w in range(wl.workers):
+            assert torch.equal(a.E[w][l], b.E[w][l])
+
+
+def test_resume_bitwise():
+    # 3 steps, hand the state (E, Q) to a fresh context, 3 more steps ==
+    # 6 straight steps
+    wl = H.small_workload(MIXED, 4, 3)
+    straight = _run_steps(wl, 6)
+    first = _run_steps(wl, 3)
+    second = H.LibRun(wl)
+    second.set_state(first.E, first.Q)
+    # the gradient source must be at the same step
+    for t in range(3, 6):
+        host = [[first.src.layer_grad(t, w, l) for l in range(len(wl.layers))] for w in range(wl.workers)]
+        for w in range(wl.workers):
+            for l in range(len(wl.layers)):
+                second.G[w][l].copy_(host[w][l])
+        second.run_step()
+    torch.cuda.synchronize()
+    for l in range(len(wl.layers)):
+        assert torch.equal(straight.Q[l], second.Q[l])
+        for w in range(wl.workers):
+            assert torch.equal(straight.E[w][l], second.E[w][l])
+
+
+def test_zero_input_gives_zero_factors():
+    wl = H.small_workload([(64, 48), (33, 7)], 3, 2)
+    run = H.LibRun(wl)
+    for w in range(2):
+        for l in range(2):
+            run.G[w][l].zero_()
+    run.run_step()
+    run.lib.status()
+    for l in range(2):
+        assert torch.count_nonzero(run.P[l]) == 0
+        assert torch.count_nonzero(run.Q[l]) == 0
+        assert torch.count_nonzero(run.Rc[l]) == 0
+        for w in range(2):
+            assert torch.count_nonzero(run.E[w][l]) == 0
+
+
+def test_nan_propagates():
+    wl = H.small_workload([(64, 48)], 2, 2)
+    run = H.LibRun(wl)
+    run.fill_grads_host(0)
+    run.G[1][0][5, 7] = float("nan")
+    run.run_step()
+    run.lib.status()
+    assert torch.isnan(run.P[0]).any()
+    assert torch.isnan(run.Q[0]).any()
+    assert torch.isnan(run.E[0][0]).any()
+
+
+def test_exact_low_rank_reproduced():
+    # noiseless rank-3 gradient, one worker: E' = 0 up to float32 rounding
+    m, n, r = 300, 650, 3
+    g = torch.Generator().manual_seed(5)
+    U = torch.linalg.qr(torch.randn(m, r, generator=g, dtype=torch.float64))[0]
+    M = (U @ torch.randn(r, n, generator=g, dtype=torch.float64)).float()
+    wl = H.small_workload([(m, n)], r, 1)
+    run = H.LibRun(wl)
+    run.G[0][0].copy_(M)
+    run.run_step()
+    run.lib.status()
+    rel = (run.E[0][0].double().norm() / M.double().norm()).item()
+    assert rel < 1e-5, rel
+
+
+def test_init_q_matches_oracle_draw():
+    layers = [(64, 48), (33, 7), (10, 130)]
+    from rank_gradient_compression_02_b200 import PowerSGD
+    lib = PowerSGD(layers, 3, 2, seed=987654321)
+    q = [torch.empty(n, 3, device="cuda") for (_, n) in layers]
+    lib.init_q(q)
+    lib.status()
+    for l, (_, n) in enumerate(layers):
+        want = philox64.initial_q(987654321, l, n, 3)
+        got = q[l].cpu().numpy()
+        np.testing.assert_allclose(got, want, rtol=2e-7, atol=1e-7)
+
+
+def test_vec_mean_and_momentum():
+    from rank_gradient_compression_02_b200 import PowerSGD
+    W = 5
+    lens = [64, 64, 128, 10, 1, 1000]
+    lib = PowerSGD([(8, 8)], 2, W)
+    g = torch.Generator().manual_seed(3)
+    host = [[torch.randn(k, generator=g) for k in lens] for _ in range(W)]
+    vecs = [[t.cuda() for t in hw] for hw in host]
+    out = [torch.empty(k, device="cuda") for k in lens]
+    x = [torch.zeros(k, device="cuda") for k in lens]
+    mo = [torch.zeros(k, device="cuda") for k in lens]
+    x_ref = [np.zeros(k) for k in lens]
+    m_ref = [np.zeros(k) for k in lens]
+    for it in range(3):
+        lib.vec_mean(vecs, out, x, mo, lr=0.1, beta=0.9)
+        for i in range(len(lens)):
+            mean = ora.vec_mean([host[w][i].double().numpy() for w in range(W)])
+            x_ref[i], m_ref[i] = ora.momentum_update(x_ref[i], m_ref[i], mean, 0.1, 0.9)
+            np.testing.assert_allclose(out[i].cpu().numpy(), mean, rtol=1e-6, atol=1e-6)
+    lib.status()
+    for i in range(len(lens)):
+        np.testing.assert_allclose(x[i].cpu().numpy(), x_ref[i], rtol=1e-5, atol=1e-6)
+
+
+def test_momentum_step_matches_oracle():
+    wl = H.small_workload(MIXED[:4], 2, 3)
+    run = H.LibRun(wl)
+    L = len(wl.layers)
+    params = [torch.zeros(m, n, device="cuda") for (m, n) in wl.layers]
+    mom = [torch.zeros(m, n, device="cuda") for (m, n) in wl.layers]
+    Q0 = [run.src.initial_q(l) for l in range(L)]
+    E0 = [[torch.zeros(m, n) for (m, n) in wl.layers] for _ in range(wl.workers)]
+    run.set_state(E0, Q0)
+    orc = H.OracleRun(range(L), {l: [e[l].double().numpy() for e in E0] for l in range(L)},
+                      {l: Q0[l].double().numpy() for l in range(L)})
+    xr = [np.zeros((m, n)) for (m, n) in wl.layers]
+    mr = [np.zeros((m, n)) for (m, n) in wl.layers]
+    for t in range(3):
+        host = run.fill_grads_host(t)
+        run.run_step()
+        run.lib.momentum_step(params, mom, 0.1, 0.9)
+        orc.step({l: [host[w][l].double().numpy() for w in range(wl.workers)] for l in range(L)})
+        for l in range(L):
+            xr[l], mr[l] = ora.momentum_update(xr[l], mr[l], orc.last[l]["G_hat"], 0.1, 0.9)
+    run.lib.status()
+    for l in range(L):
+        assert H.rel_fro(H.to64(params[l]), xr[l]) < 1e-4
+        assert H.rel_fro(H.to64(mom[l]), mr[l]) < 1e-4
+
+
+def test_step_host_matches_device_step():
+    wl = H.small_workload(MIXED, 4, 3)
+    a = H.LibRun(wl)
+    b = H.LibRun(wl)
+    L = len(wl.layers)
+    for t in range(2):
+        host = a.fill_grads_host(t)
+        a.run_step()
+        pinned = [[host[w][l].pin_memory() for l in range(L)] for w in range(wl.workers)]
+        ph = [torch.empty(m, wl.rank).pin_memory() for (m, _) in wl.layers]
+        qh = [torch.empty(n, wl.rank).pin_memory() for (_, n) in wl.layers]
+        b.lib.step_host(pinned, b.E, b.Q, ph, qh)
+        torch.cuda.synchronize()
+        for l in range(L):
+            assert torch.equal(a.Q[l].cpu(), qh[l])
+            assert torch.equal(a.P[l].cpu(), ph[l])
+            for w in range(wl.workers):
+                assert torch.equal(a.E[w][l], b.E[w][l])
+
+
+def test_bad_arguments_rejected():
+    from rank_gradient_compression_02_b200 import PowerSGD, PsgdError
+    wl = H.small_workload([(64, 48)], 2, 2)
+    run = H.LibRun(wl)
+    base = torch.zeros(64 * 48 + 4, device="cuda")
+    odd = base[1:1 + 64 * 48].view(64, 48)          # 4-byte offset: misaligned
+    E_bad = [[odd], [run.E[1][0]]]
+    with pytest.raises(PsgdError) as ei:
+        run.lib.step(run.G, E_bad, run.Q, run.P, None)
+    assert ei.value.code == 2
+    with pytest.raises(PsgdError) as ei:
+        run.lib.step(run.G, [[0], [run.E[1][0]]], run.Q, run.P, None)
+    assert ei.value.code == 1
+    with pytest.raises(PsgdError) as ei:
+        run.lib.materialize_errors(run.E)   # not a lazy context
+    assert ei.value.code == 5
+    with pytest.raises(PsgdError):
+        PowerSGD([(4, 3)], 4, 1)             # rank > min(m, n)
+    run.lib.status()
