@@ -413,17 +413,24 @@ int psgd_create(psgd_ctx** out, const psgd_layer* layers, int num_layers, int ra
         delete ctx;
         return PSGD_ERR_CUDA;
     }
-    // opt in to the dynamic shared memory each kernel of this context needs
+    // opt in to the dynamic shared memory each kernel of this context needs.
+    // The attribute is per kernel, shared by every context: only ever raise
+    // it, so that a context with smaller tiles never breaks an existing one.
+    auto raise_smem = [](const void* fn, size_t need) -> cudaError_t {
+        cudaFuncAttributes fa{};
+        cudaError_t err = cudaFuncGetAttributes(&fa, fn);
+        if (err != cudaSuccess) return err;
+        if (static_cast<size_t>(fa.maxDynamicSharedSizeBytes) >= need) return cudaSuccess;
+        return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(need));
+    };
     for (int lazy = 0; lazy < 2; ++lazy) {
         const bool sf = (flags & PSGD_FLAG_SUM_FIRST) != 0;
         const void* fa = kernel_ptr(0, R, grad_dtype, lazy != 0, sf);
         const void* fb = kernel_ptr(1, R, grad_dtype, lazy != 0, sf);
         const void* fc = kernel_ptr(2, R, grad_dtype, lazy != 0, sf);
-        e = cudaFuncSetAttribute(fa, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->smem_a));
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(fb, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->smem_b));
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(fc, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ctx->smem_c));
+        e = raise_smem(fa, ctx->smem_a);
+        if (e == cudaSuccess) e = raise_smem(fb, ctx->smem_b);
+        if (e == cudaSuccess) e = raise_smem(fc, ctx->smem_c);
         if (e != cudaSuccess) {
             fail(nullptr, PSGD_ERR_CUDA, "shared-memory opt-in: %s", cudaGetErrorString(e));
             cudaFree(ctx->ws);
