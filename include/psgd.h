@@ -169,6 +169,42 @@ PSGD_API int psgd_workspace_bytes(const psgd_ctx *ctx, size_t *bytes);
  * launch accounting). */
 PSGD_API int psgd_step_launches(const psgd_ctx *ctx);
 
+/* Allocation-free step for one layer.  No counterpart in the pages: this
+ * entry point exists for callers that cannot allocate device memory, for
+ * example code whose device memory is owned by another allocator (a
+ * framework's caching pool that must account for every byte), code that
+ * must not pay for cudaMalloc's implicit device synchronisation inside a
+ * training loop, or code running where allocation is not permitted.
+ *
+ * It runs the same kernels and computes the same eager step as psgd_step
+ * for a single m x n layer, with no context: every piece of scratch (layer
+ * descriptor, pointer table, P and Q partials, P_bar, P_hat, Q_bar, Gram
+ * partials, T, counters) lives in one file-scope static device array of
+ * PSGD_STATIC_SCRATCH_BYTES (16 MiB).  Every GPU that loads the library
+ * holds that array until the process exits.  The call allocates no device
+ * memory and calls no allocating routine (the descriptor and pointer table
+ * are staged from the stack); only a failed call stores its message in
+ * thread-local host memory for psgd_last_error(NULL).
+ *
+ * grads[w], errors[w]: HOST arrays of W device pointers (m x n, grad dtype
+ * and float32); q: device n x rank (warm start in, Q_bar out); p_hat:
+ * device m x rank or NULL; recon: device m x n or NULL.  Same argument
+ * rules as psgd_create / psgd_step (1 <= rank <= min(m, n, 32),
+ * 1 <= workers <= 256, 16-byte aligned pointers).  A layer whose scratch
+ * does not fit in the static array is rejected with PSGD_ERR_ARG before
+ * any device work (psgd_last_error(NULL) says how much it needs).
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) once for that device; make that first call before
+ * any stream capture.  All calls share the one array and it keeps the last
+ * call's contents (the counters are cleared at the start of every call):
+ * calls that overlap on the GPU - on two streams, or from two threads -
+ * race and corrupt each other; order them. */
+#define PSGD_STATIC_SCRATCH_BYTES (16u << 20)
+PSGD_API int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int grad_dtype,
+                              const void *const *grads, float *const *errors, float *q, float *p_hat,
+                              float *recon, void *stream);
+
 /* Per-kernel timing of psgd_step, for measurement: with enable != 0 every
  * later psgd_step records CUDA events (on its stream) around each of its
  * kernel launches.  psgd_profile_read synchronises on those events, writes

@@ -53,6 +53,8 @@ _SIGS = {
     "psgd_workspace_bytes": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_size_t)]),
     "psgd_step_launches": (ctypes.c_int, [_P]),
     "psgd_last_error": (ctypes.c_char_p, [_P]),
+    "psgd_step_static": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        _PP, _PP, _P, _P, _P, _P]),
     "psgd_profile_enable": (ctypes.c_int, [_P, ctypes.c_int]),
     "psgd_profile_read": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
 }
@@ -97,6 +99,21 @@ def _stream_handle(stream) -> int:
     if isinstance(stream, int):
         return stream
     return stream.cuda_stream
+
+
+def step_static(m: int, n: int, rank: int, grads, errors, q, p_hat=None, recon=None, grad_dtype: str = "f32",
+                stream=None):
+    """Allocation-free one-layer step (psgd_step_static): grads[w], errors[w]
+    per worker; every scratch buffer lives in the library's static device
+    array.  For callers that cannot allocate device memory."""
+    lib = load()
+    W = len(grads)
+    rc = lib.psgd_step_static(int(m), int(n), int(rank), W, PSGD_BF16 if grad_dtype == "bf16" else PSGD_F32,
+                              _ptrs(grads), _ptrs(errors), q.data_ptr(),
+                              p_hat.data_ptr() if p_hat is not None else None,
+                              recon.data_ptr() if recon is not None else None, _stream_handle(stream))
+    if rc:
+        raise PsgdError(rc, lib.psgd_last_error(None).decode())
 
 
 class PowerSGD:

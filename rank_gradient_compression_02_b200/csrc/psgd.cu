@@ -9,6 +9,7 @@
 #include <algorithm>
 #include <array>
 #include <cstdarg>
+#include <mutex>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -728,6 +729,176 @@ int psgd_vec_mean(psgd_ctx* ctx, const float* const* vecs, float* const* out, co
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "vec_mean launch");
     ctx->last_stream = s;
+    return PSGD_OK;
+}
+
+// ---- allocation-free single-layer step ------------------------------------
+// All scratch of psgd_step_static lives in this array; host code never uses
+// its name as an address: the device address comes from
+// cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) unsigned char g_psgd_static_scratch[PSGD_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_addr[kMaxDevices] = {};
+
+cudaError_t static_scratch_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_psgd_static_scratch);
+        if (e != cudaSuccess) return e;
+        g_static_addr[dev] = p;
+    }
+    *out = g_static_addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int grad_dtype, const void* const* grads,
+                     float* const* errors, float* q, float* p_hat, float* recon, void* stream) {
+    g_create_error.clear();
+    if (rank < 1 || rank > psgd::kMaxRank) return fail(nullptr, PSGD_ERR_ARG, "rank %d not in [1, 32]", rank);
+    if (workers < 1 || workers > psgd::kMaxWorkers)
+        return fail(nullptr, PSGD_ERR_ARG, "workers %d not in [1, %d]", workers, psgd::kMaxWorkers);
+    if (grad_dtype != PSGD_F32 && grad_dtype != PSGD_BF16) return fail(nullptr, PSGD_ERR_ARG, "bad grad dtype");
+    if (m < 1 || n < 1 || rank > m || rank > n || m > (int64_t(1) << 31) || n > (int64_t(1) << 31))
+        return fail(nullptr, PSGD_ERR_ARG, "bad shape %lld x %lld for rank %d", (long long)m, (long long)n, rank);
+    if (!grads || !errors || !q) return fail(nullptr, PSGD_ERR_ARG, "null pointer argument");
+    for (int w = 0; w < workers; ++w) {
+        if (!grads[w] || !errors[w]) return fail(nullptr, PSGD_ERR_ARG, "null pointer for worker %d", w);
+        if (!aligned16(grads[w]) || !aligned16(errors[w]))
+            return fail(nullptr, PSGD_ERR_ALIGN, "pointer of worker %d is not 16-byte aligned", w);
+    }
+    if (!aligned16(q) || (p_hat && !aligned16(p_hat)) || (recon && !aligned16(recon)))
+        return fail(nullptr, PSGD_ERR_ALIGN, "q, p_hat or recon is not 16-byte aligned");
+
+    // tile geometry of the one layer (same rules as a context's)
+    const int R = pad_rank(rank);
+    const int NG = R * (R + 1) / 2;
+    LayerDesc d{};
+    d.m = m;
+    d.n = n;
+    d.vec = 1;
+    for (int v : {4, 2, 1})
+        if (v <= max_vec_for_rank(R) && n % v == 0) {
+            d.vec = v;
+            break;
+        }
+    d.nvec = static_cast<int>(n / d.vec);
+    d.nchunk = (d.nvec + 31) / 32;
+    d.slots = (d.nvec + d.nchunk - 1) / d.nchunk;
+    {
+        const int64_t cols = static_cast<int64_t>(d.slots) * d.vec;
+        int64_t tm = (kTileTargetElems + cols * workers - 1) / (cols * workers);
+        tm = (tm + 7) / 8 * 8;
+        tm = std::max<int64_t>(8, std::min<int64_t>(tm, std::min(512, kRowsFloatsMax / R)));
+        tm = std::min<int64_t>(tm, (m + 7) / 8 * 8);
+        d.tm = static_cast<int>(tm);
+        d.nrb = static_cast<int>((m + tm - 1) / tm);
+    }
+    const int64_t ntiles = static_cast<int64_t>(d.nrb) * d.nchunk;
+
+    // scratch layout inside the static array
+    size_t off = 0;
+    auto carve = [&](size_t bytes) {
+        const size_t o = off;
+        off = align_up(off + std::max<size_t>(bytes, 1), 256);
+        return o;
+    };
+    const int ntab = 2 * workers + 3;
+    const size_t o_desc = carve(sizeof(LayerDesc));
+    const size_t o_tab = carve(sizeof(uint64_t) * ntab);
+    const size_t o_tile = carve(sizeof(int) * ntiles);
+    const size_t o_pbar = carve(sizeof(double) * m * R);
+    const size_t o_phat = carve(sizeof(float) * m * R);
+    const size_t o_qbar = carve(sizeof(float) * n * R);
+    const size_t o_ppart = carve(sizeof(double) * d.nchunk * m * R);
+    const size_t o_qpart = carve(sizeof(double) * d.nrb * n * R);
+    const size_t o_gram = carve(sizeof(double) * d.nrb * NG);
+    const size_t o_T = carve(sizeof(double) * R * R);
+    const size_t o_cnt = carve(sizeof(unsigned) * (d.nrb + 1 + d.nchunk));
+    const size_t o_status = carve(sizeof(int));
+    if (off > PSGD_STATIC_SCRATCH_BYTES)
+        return fail(nullptr, PSGD_ERR_ARG, "layer %lld x %lld at rank %d with %d workers needs %zu bytes of scratch; "
+                    "the static scratch holds %u", (long long)m, (long long)n, rank, workers, off,
+                    PSGD_STATIC_SCRATCH_BYTES);
+    // o_desc .. o_tab are the first pieces; the descriptor's own offsets are relative to the work arrays
+    d.tile_begin = 0;
+    d.prow_off = d.qrow_off = d.ppart_off = d.qpart_off = d.gram_off = d.t_off = d.cnt_off = 0;
+
+    void* base_v = nullptr;
+    cudaError_t e = static_scratch_address(&base_v);
+    if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "static scratch address: %s", cudaGetErrorString(e));
+    unsigned char* base = static_cast<unsigned char*>(base_v);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    // descriptor and pointer table from host stack memory (no allocation)
+    uint64_t tab[2 * psgd::kMaxWorkers + 3];
+    for (int w = 0; w < workers; ++w) {
+        tab[w] = reinterpret_cast<uint64_t>(grads[w]);
+        tab[workers + w] = reinterpret_cast<uint64_t>(errors[w]);
+    }
+    tab[2 * workers] = reinterpret_cast<uint64_t>(q);
+    tab[2 * workers + 1] = reinterpret_cast<uint64_t>(p_hat);
+    tab[2 * workers + 2] = reinterpret_cast<uint64_t>(recon);
+    e = cudaMemcpyAsync(base + o_desc, &d, sizeof(LayerDesc), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(base + o_tab, tab, sizeof(uint64_t) * ntab, cudaMemcpyHostToDevice, s);
+    // tile -> layer map is all zeros (one layer); counters and status start at zero
+    if (e == cudaSuccess) e = cudaMemsetAsync(base + o_tile, 0, sizeof(int) * ntiles, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(base + o_cnt, 0, o_status + sizeof(int) - o_cnt, s);
+    if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "scratch set-up: %s", cudaGetErrorString(e));
+
+    psgd::Params p{};
+    uint64_t* tab_d = reinterpret_cast<uint64_t*>(base + o_tab);
+    p.t.layers = reinterpret_cast<const LayerDesc*>(base + o_desc);
+    p.t.tile_layer = reinterpret_cast<const int*>(base + o_tile);
+    p.t.grads = reinterpret_cast<const void* const*>(tab_d);
+    p.t.errors = reinterpret_cast<float* const*>(tab_d + workers);
+    p.t.q = reinterpret_cast<float* const*>(tab_d + 2 * workers);
+    p.t.p_hat_out = reinterpret_cast<float* const*>(tab_d + 2 * workers + 1);
+    p.t.recon_out = reinterpret_cast<float* const*>(tab_d + 2 * workers + 2);
+    p.ws.pbar = reinterpret_cast<double*>(base + o_pbar);
+    p.ws.phat = reinterpret_cast<float*>(base + o_phat);
+    p.ws.qbar = reinterpret_cast<float*>(base + o_qbar);
+    p.ws.ppart = reinterpret_cast<double*>(base + o_ppart);
+    p.ws.qpart = reinterpret_cast<double*>(base + o_qpart);
+    p.ws.gram = reinterpret_cast<double*>(base + o_gram);
+    p.ws.T = reinterpret_cast<double*>(base + o_T);
+    p.ws.cnt = reinterpret_cast<unsigned*>(base + o_cnt);
+    p.ws.status = reinterpret_cast<int*>(base + o_status);
+    p.num_layers = 1;
+    p.workers = workers;
+    p.r = rank;
+    p.inv_w = 1.0f / static_cast<float>(workers);
+    p.drop_tol = kDropTol;
+
+    const size_t smem[3] = {smem_need(0, R, workers, d.tm, d.vec), smem_need(1, R, workers, d.tm, d.vec),
+                            smem_need(2, R, workers, d.tm, d.vec)};
+    for (int which = 0; which < 3; ++which) {
+        void* fn = kernel_ptr(which, R, grad_dtype, false, false);
+        cudaFuncAttributes fa{};
+        e = cudaFuncGetAttributes(&fa, fn);
+        if (e == cudaSuccess && static_cast<size_t>(fa.maxDynamicSharedSizeBytes) < smem[which])
+            e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem[which]));
+        if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "shared-memory opt-in: %s", cudaGetErrorString(e));
+        psgd::Params pw = p;
+        if (which == 2) {
+            pw.do_resid = 1;
+            pw.do_recon = recon ? 1 : 0;
+        }
+        void* args[] = {&pw};
+        e = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(ntiles)), dim3(psgd::kThreads), args, smem[which], s);
+        if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
+    }
     return PSGD_OK;
 }
 
