@@ -252,15 +252,26 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--oracle-budget", type=float, default=15.0)
+    ap.add_argument("--layers", default=None, help="comma-separated layer indices (a subset, for small captures)")
+    ap.add_argument("--workers", type=int, default=None, help="override the worker count (small captures)")
+    ap.add_argument("--iters", type=int, default=1, help="power iterations per step")
     args = ap.parse_args()
 
+    from dataclasses import replace
     wl = get_workload(args.config)
     r = args.rank if args.rank is not None else wl.rank
     wl = wl.with_rank(r)
+    if args.layers:
+        idx = [int(x) for x in args.layers.split(",")]
+        wl = replace(wl, name=f"{wl.name}[layers {args.layers}]", layers=tuple(wl.layers[i] for i in idx),
+                     vectors=())
+    if args.workers:
+        wl = replace(wl, name=f"{wl.name}[W={args.workers}]", workers=args.workers)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank_id = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    mode = ("lazy" if args.lazy else "eager") + ("+sumfirst" if args.sum_first else "")
+    mode = ("lazy" if args.lazy else "eager") + ("+sumfirst" if args.sum_first else "") + \
+        (f"+iters{args.iters}" if args.iters != 1 else "")
     config = {"workload": wl.name, "layers": len(wl.layers), "elements_per_worker": wl.elements_per_worker,
               "workers": wl.workers, "rank": r, "grad_dtype": wl.grad_dtype, "mode": mode,
               "l2": "inputs larger than L2 (no flush needed)" if wl.elements * 4 > 4 * 126e6 else "inputs fit L2",
@@ -286,7 +297,7 @@ def main():
         raise SystemExit(f"workload needs {need/1e9:.1f} GB, {free/1e9:.1f} GB free")
     B = Buffers(wl, r, device)
     lib = PowerSGD(wl.layers, r, wl.workers, grad_dtype=wl.grad_dtype, lazy_errors=args.lazy,
-                   sum_first=args.sum_first)
+                   sum_first=args.sum_first, power_iters=args.iters)
     torch.cuda.synchronize()
 
     def barrier():

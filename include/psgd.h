@@ -89,7 +89,12 @@ enum {
     /* Sum the W workers' M_w element-wise before multiplying by Q or P_hat
      * (one product per matrix element instead of one per worker element).
      * Same result up to rounding, by linearity (note-152, "Concepts"). */
-    PSGD_FLAG_SUM_FIRST = 2u
+    PSGD_FLAG_SUM_FIRST = 2u,
+    /* No warm start (the ablation of note-152, "Claims" C4): every step
+     * first overwrites q[l] with a fresh N(0, 1) draw, the psgd_init_q
+     * generator with draw index = step number (1, 2, ...; psgd_init_q is
+     * draw 0).  One extra launch per step. */
+    PSGD_FLAG_NO_WARM_START = 4u
 };
 
 typedef struct { int64_t m, n; } psgd_layer;   /* one gradient matrix */
@@ -165,8 +170,9 @@ PSGD_API int psgd_status(psgd_ctx *ctx);
 /* Bytes of device workspace the context holds (excluding host staging). */
 PSGD_API int psgd_workspace_bytes(const psgd_ctx *ctx, size_t *bytes);
 
-/* Number of kernel launches one psgd_step makes for this context (for
- * launch accounting). */
+/* Number of kernel launches one regular psgd_step makes for this context
+ * (for launch accounting; an SVD-refresh step adds the launches stated at
+ * psgd_set_svd_refresh). */
 PSGD_API int psgd_step_launches(const psgd_ctx *ctx);
 
 /* Allocation-free step for one layer.  No counterpart in the pages: this
@@ -205,12 +211,35 @@ PSGD_API int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int g
                               const void *const *grads, float *const *errors, float *q, float *p_hat,
                               float *recon, void *stream);
 
+/* Power (subspace) iterations per step, 1 <= iters <= 8 (default 1; the
+ * "PowerSGD" glossary page: one or two suffice).  Every iteration repeats
+ * P = M Q, mean, orthogonalisation, Q = M^T P_hat, mean, the next one
+ * starting from the Q_bar just formed; the residual uses the last
+ * iteration's factors.  Later iterations read M (already formed) instead of
+ * G and E, so each costs one more read of M for P and one for Q. */
+PSGD_API int psgd_set_power_iters(psgd_ctx *ctx, int iters);
+
+/* PowerSGD+ periodic SVD refresh ("From PowerSGD to PowerSGD+", Abstract:
+ * the projection subspace is periodically re-aligned with the optimal one
+ * through a singular value decomposition).  With every > 0, every step
+ * whose number (1, 2, ...) is a multiple of `every` runs `iters` subspace
+ * iterations (1 <= iters <= 64) from the warm start and then a
+ * Rayleigh-Ritz rotation: C = Q_bar^T Q_bar = W Lambda W^T (Jacobi,
+ * float64, eigenvalues descending, each column of W signed so that its
+ * largest-magnitude entry is positive), P_hat <- P_hat W, Q_bar <- Q_bar W.
+ * Once the iterations have converged, P_hat = U_r and Q_bar = V_r Sigma_r
+ * (singular vectors up to sign) of the worker-mean matrix, and the
+ * residual is taken against that truncated SVD.  every = 0 turns it off
+ * (the default).  Adds 2 * (iters - power_iters) + 1 launches on refresh
+ * steps. */
+PSGD_API int psgd_set_svd_refresh(psgd_ctx *ctx, int every, int iters);
+
 /* Per-kernel timing of psgd_step, for measurement: with enable != 0 every
  * later psgd_step records CUDA events (on its stream) around each of its
  * kernel launches.  psgd_profile_read synchronises on those events, writes
  * the summed device milliseconds of the first pass (error feedback + P),
- * the second pass (Q) and the third pass (residual / decompression, 0 in
- * lazy mode) to ms[0..2] and the number of recorded steps to *steps, and
+ * the second pass (Q, plus every later power iteration) and the third pass
+ * (residual / decompression, 0 in lazy mode) to ms[0..2] and the number of recorded steps to *steps, and
  * clears the record.  Recording adds three event records per step. */
 PSGD_API int psgd_profile_enable(psgd_ctx *ctx, int enable);
 PSGD_API int psgd_profile_read(psgd_ctx *ctx, double *ms, int *steps);

@@ -15,7 +15,9 @@ two published definitions:
     deviates", Ann. Math. Stat. 29 (1958).
 
 Mapping (a convention of this repository, stated in the C header too):
-key = (seed, layer), counter = (b, 0, 0, 0) for block b = e // 4, where e =
+key = (seed, layer), counter = (b, s, 0, 0) for block b = e // 4 and draw
+index s (0 for the initial Q; step number s >= 1 for the fresh Q of a step
+without warm start), where e =
 j*r + k indexes Q0 (n x r, row-major); word t = e % 4 of the block feeds
 normal t.  Each 64-bit word x becomes u = ((x >> 11) + 0.5) * 2^-53 in (0, 1);
 words (0, 1) and (2, 3) are Box-Muller pairs: z_even = rho*cos(2*pi*u_odd),
@@ -72,12 +74,13 @@ def box_muller_block(words):
     return out
 
 
-def initial_q(seed: int, layer: int, n: int, r: int) -> np.ndarray:
-    """Q0 for one layer (n x r float32) under the mapping above."""
+def initial_q(seed: int, layer: int, n: int, r: int, draw: int = 0) -> np.ndarray:
+    """Q for one layer (n x r float32) under the mapping above; draw 0 is
+    the initial Q, draw s >= 1 the fresh Q of step s without warm start."""
     total = n * r
     vals = np.empty(total, dtype=np.float64)
     for b in range((total + 3) // 4):
-        z = box_muller_block(philox4x64_10((b, 0, 0, 0), (seed, layer)))
+        z = box_muller_block(philox4x64_10((b, draw, 0, 0), (seed, layer)))
         for t in range(4):
             e = 4 * b + t
             if e < total:

@@ -127,25 +127,54 @@ def vec_mean(vecs: Sequence[np.ndarray]) -> np.ndarray:
     return worker_mean(vecs)
 
 
-def step(G: Sequence[np.ndarray], E: Sequence[np.ndarray], Q, drop_tol: float = DROP_TOL) -> dict:
+def step(G: Sequence[np.ndarray], E: Sequence[np.ndarray], Q, drop_tol: float = DROP_TOL, iters: int = 1) -> dict:
     """One PowerSGD compression step for one layer and W workers, in the
     order of [N152] "Method".
 
     G, E: length-W lists of m x n arrays (gradient and error memory of each
     worker).  Q: n x r warm start shared by all workers.
+    iters: power (subspace) iterations in the step ([GLOS] warm-start
+    paragraph: one or two suffice).  Reading: every iteration repeats the
+    right multiply, mean, orthogonalisation, left multiply and mean, the next
+    iteration starting from the Q_bar just formed; the residual uses the
+    last iteration's factors.
     Returns M, P (per worker), P_bar, P_hat, Qw (per worker), Q_bar,
-    E_new (per worker) and G_hat.
+    E_new (per worker) and G_hat (of the last iteration).
     """
     W = len(G)
     M = [error_feedback_add(G[w], E[w]) for w in range(W)]
-    P = [right_multiply(M[w], Q) for w in range(W)]
-    P_bar = worker_mean(P)
-    P_hat = gram_schmidt(P_bar, drop_tol)
-    Qw = [left_multiply(M[w], P_hat) for w in range(W)]
-    Q_bar = worker_mean(Qw)
+    Q_cur = _f64(Q)
+    for _ in range(iters):
+        P = [right_multiply(M[w], Q_cur) for w in range(W)]
+        P_bar = worker_mean(P)
+        P_hat = gram_schmidt(P_bar, drop_tol)
+        Qw = [left_multiply(M[w], P_hat) for w in range(W)]
+        Q_bar = worker_mean(Qw)
+        Q_cur = Q_bar
     E_new = [residual(M[w], P_hat, Q_bar) for w in range(W)]
     G_hat = decompress(P_hat, Q_bar)
     return dict(M=M, P=P, P_bar=P_bar, P_hat=P_hat, Qw=Qw, Q_bar=Q_bar, E_new=E_new, G_hat=G_hat)
+
+
+def svd_refresh_step(G: Sequence[np.ndarray], E: Sequence[np.ndarray], rank: int) -> dict:
+    """A PowerSGD+ refresh step ([PLUS] Abstract: the projection subspace is
+    periodically re-aligned with the optimal one by a singular value
+    decomposition).  Reading: on a refresh step the compressed form of the
+    aggregate M_bar = mean_w(G_w + E_w) is its rank-r truncated SVD,
+    P_hat = U_r, Q_bar = V_r Sigma_r (so the warm start of the next step is
+    V_r Sigma_r), and the error memory is E'_w = M_w - U_r Sigma_r V_r^T.
+    The SVD is a library primitive here (LAPACK through NumPy); singular
+    vectors are unique only up to sign, so callers compare them up to
+    column sign."""
+    W = len(G)
+    M = [error_feedback_add(G[w], E[w]) for w in range(W)]
+    M_bar = worker_mean(M)
+    U, s, Vt = np.linalg.svd(M_bar, full_matrices=False)
+    P_hat = U[:, :rank].copy()
+    Q_bar = Vt[:rank, :].T * s[None, :rank]
+    E_new = [residual(M[w], P_hat, Q_bar) for w in range(W)]
+    G_hat = decompress(P_hat, Q_bar)
+    return dict(M=M, M_bar=M_bar, P_hat=P_hat, Q_bar=Q_bar, E_new=E_new, G_hat=G_hat, sigma=s)
 
 
 def run(layers_G, E0, Q0, drop_tol: float = DROP_TOL):

@@ -20,6 +20,7 @@ PSGD_OK, PSGD_ERR_ARG, PSGD_ERR_ALIGN, PSGD_ERR_CUDA, PSGD_ERR_OOM, PSGD_ERR_STA
 PSGD_F32, PSGD_BF16 = 0, 1
 FLAG_LAZY_ERRORS = 1
 FLAG_SUM_FIRST = 2
+FLAG_NO_WARM_START = 4
 
 _ERR_NAMES = {1: "PSGD_ERR_ARG", 2: "PSGD_ERR_ALIGN", 3: "PSGD_ERR_CUDA", 4: "PSGD_ERR_OOM",
               5: "PSGD_ERR_STATE", 6: "PSGD_ERR_DEVICE"}
@@ -55,6 +56,8 @@ _SIGS = {
     "psgd_last_error": (ctypes.c_char_p, [_P]),
     "psgd_step_static": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         _PP, _PP, _P, _P, _P, _P]),
+    "psgd_set_power_iters": (ctypes.c_int, [_P, ctypes.c_int]),
+    "psgd_set_svd_refresh": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int]),
     "psgd_profile_enable": (ctypes.c_int, [_P, ctypes.c_int]),
     "psgd_profile_read": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
 }
@@ -124,14 +127,16 @@ class PowerSGD:
     """
 
     def __init__(self, layers: Sequence[Sequence[int]], rank: int, workers: int, seed: int = 1234,
-                 grad_dtype: str = "f32", lazy_errors: bool = False, sum_first: bool = False):
+                 grad_dtype: str = "f32", lazy_errors: bool = False, sum_first: bool = False,
+                 power_iters: int = 1, warm_start: bool = True, svd_every: int = 0, svd_iters: int = 8):
         self.lib = load()
         self.layers = [(int(m), int(n)) for m, n in layers]
         self.rank = int(rank)
         self.workers = int(workers)
         self.grad_dtype = grad_dtype
         arr = (_Layer * max(1, len(self.layers)))(*[_Layer(m, n) for m, n in self.layers])
-        flags = (FLAG_LAZY_ERRORS if lazy_errors else 0) | (FLAG_SUM_FIRST if sum_first else 0)
+        flags = (FLAG_LAZY_ERRORS if lazy_errors else 0) | (FLAG_SUM_FIRST if sum_first else 0) | \
+            (0 if warm_start else FLAG_NO_WARM_START)
         h = _P()
         rc = self.lib.psgd_create(ctypes.byref(h), arr, len(self.layers), self.rank, self.workers,
                                   ctypes.c_uint64(seed & (2**64 - 1)),
@@ -139,6 +144,10 @@ class PowerSGD:
         if rc:
             raise PsgdError(rc, self.lib.psgd_last_error(None).decode())
         self._h = h
+        if power_iters != 1:
+            self._check(self.lib.psgd_set_power_iters(self._h, int(power_iters)))
+        if svd_every:
+            self._check(self.lib.psgd_set_svd_refresh(self._h, int(svd_every), int(svd_iters)))
 
     # -- helpers
     def _check(self, rc: int):

@@ -23,15 +23,39 @@ struct LayerDesc {
     int slots;      // vector slots per chunk (<= 32); chunks are balanced
     int tm;         // rows per tile (multiple of 8)
     int nrb;        // row blocks = ceil(m / tm)
+    int nsup;       // super-blocks of kSuper row blocks (two-level reductions)
+    int pad_;
     int64_t tile_begin;  // index of this layer's first tile in the grouped grid
     int64_t prow_off;    // P_bar (double) / P_hat (float) rows, stride R
     int64_t qrow_off;    // Q_bar rows (stride R floats)
     int64_t ppart_off;   // P partials [nchunk][m][R] doubles
     int64_t qpart_off;   // Q partials [nrb][n][R] doubles
     int64_t gram_off;    // Gram partials [nrb][R(R+1)/2] doubles
+    int64_t gsup_off;    // Gram super-block partials [nsup][R(R+1)/2] doubles
+    int64_t qsup_off;    // Q super-block partials [nsup][n][R] doubles
     int64_t t_off;       // T = R^-1, R x R doubles
-    int64_t cnt_off;     // counters: [nrb] row blocks of pass A, [1] layer, [nchunk] chunks of pass B
+    int64_t cnt_off;     // counters, see counter_layout()
 };
+
+// Row-block partials are summed in two levels: every kSuper row blocks into
+// a super-block partial (by the last of them to finish), then the
+// super-blocks (by the last super-block).  Both levels sum in index order.
+constexpr int kSuper = 32;
+
+// Counter offsets inside a layer's counter block.
+struct CounterLayout {
+    int64_t a_rb, a_sup, a_layer, b_sup, b_chunk, total;
+};
+__host__ __device__ inline CounterLayout counter_layout(int nrb, int nsup, int nchunk) {
+    CounterLayout c;
+    c.a_rb = 0;                                   // [nrb]  chunk tiles done per row block (pass A)
+    c.a_sup = nrb;                                // [nsup] row blocks done per super-block (pass A)
+    c.a_layer = nrb + nsup;                       // [1]    super-blocks done (pass A)
+    c.b_sup = c.a_layer + 1;                      // [nchunk][nsup] row-block tiles done (pass B)
+    c.b_chunk = c.b_sup + static_cast<int64_t>(nchunk) * nsup;  // [nchunk] super-blocks done (pass B)
+    c.total = c.b_chunk + nchunk;
+    return c;
+}
 
 struct Tables {
     const LayerDesc* layers;
@@ -57,6 +81,8 @@ struct Work {
     double* ppart;
     double* qpart;
     double* gram;
+    double* gsup;
+    double* qsup;
     double* T;
     unsigned* cnt;
     int* status;

@@ -103,7 +103,7 @@ struct SmemA {
     }
 };
 
-template <int R, int VEC, typename GT, bool LAZY, bool SF>
+template <int R, int VEC, typename GT, bool LAZY, bool SF, bool READM>
 __device__ __forceinline__ void pass_a_rows(const Params& p, const LayerDesc& d, const TileCoord& tc,
                                             const GT* const* gp, float* const* ep, const float* ph_prev) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -138,6 +138,10 @@ __device__ __forceinline__ void pass_a_rows(const Params& p, const LayerDesc& d,
 
     double* ppart = p.ws.ppart + d.ppart_off;
     constexpr int U = (VEC == 4) ? 4 : 8;
+    // products are summed in float32 over runs of 8 terms (F workers x VEC
+    // columns), then added to the float64 row accumulator
+    constexpr int F = 8 / VEC;
+    static_assert(U % F == 0, "flush interval must divide the unroll");
     constexpr int LG = Log2<R>::value;
 
     for (int64_t i = i0 + warp; i < i1; i += kWarps) {
@@ -162,50 +166,59 @@ __device__ __forceinline__ void pass_a_rows(const Params& p, const LayerDesc& d,
                 float g[U][VEC], e[U][VEC];
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    ld_grad<GT, VEC>(gp[w + u] + base, g[u]);
+                    if constexpr (!READM) ld_grad<GT, VEC>(gp[w + u] + base, g[u]);
                     ld_f32<VEC>(ep[w + u] + base, e[u]);
                 }
+                if constexpr (!READM) {
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
+                    for (int u = 0; u < U; ++u) {
 #pragma unroll
-                    for (int v = 0; v < VEC; ++v) {
-                        float ev = e[u][v];
-                        if constexpr (LAZY) ev = ev - rec[v];
-                        e[u][v] = g[u][v] + ev;
+                        for (int v = 0; v < VEC; ++v) {
+                            float ev = e[u][v];
+                            if constexpr (LAZY) ev = ev - rec[v];
+                            e[u][v] = g[u][v] + ev;
+                        }
+                        st_f32<VEC>(ep[w + u] + base, e[u]);
                     }
-                    st_f32<VEC>(ep[w + u] + base, e[u]);
                 }
+                if constexpr (SF) {
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    if constexpr (SF) {
+                    for (int u = 0; u < U; ++u)
 #pragma unroll
                         for (int v = 0; v < VEC; ++v) msum[v] += e[u][v];
-                    } else {
-                        // one worker's product over this lane's VEC columns
-                        // in float32, then accumulated in float64
-                        float pw[R];
+                } else {
+                    float pw[R];
 #pragma unroll
-                        for (int k = 0; k < R; ++k) pw[k] = 0.f;
+                    for (int k = 0; k < R; ++k) pw[k] = 0.f;
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
 #pragma unroll
                         for (int v = 0; v < VEC; ++v)
 #pragma unroll
                             for (int k = 0; k < R; ++k) pw[k] = fmaf(e[u][v], qv[v][k], pw[k]);
+                        if ((u + 1) % F == 0) {
 #pragma unroll
-                        for (int k = 0; k < R; ++k) acc[k] += static_cast<double>(pw[k]);
+                            for (int k = 0; k < R; ++k) {
+                                acc[k] += static_cast<double>(pw[k]);
+                                pw[k] = 0.f;
+                            }
+                        }
                     }
                 }
             }
             for (; w < W; ++w) {
                 float g[VEC], e[VEC];
-                ld_grad<GT, VEC>(gp[w] + base, g);
                 ld_f32<VEC>(ep[w] + base, e);
+                if constexpr (!READM) {
+                    ld_grad<GT, VEC>(gp[w] + base, g);
 #pragma unroll
-                for (int v = 0; v < VEC; ++v) {
-                    float ev = e[v];
-                    if constexpr (LAZY) ev = ev - rec[v];
-                    e[v] = g[v] + ev;
+                    for (int v = 0; v < VEC; ++v) {
+                        float ev = e[v];
+                        if constexpr (LAZY) ev = ev - rec[v];
+                        e[v] = g[v] + ev;
+                    }
+                    st_f32<VEC>(ep[w] + base, e);
                 }
-                st_f32<VEC>(ep[w] + base, e);
                 if constexpr (SF) {
 #pragma unroll
                     for (int v = 0; v < VEC; ++v) msum[v] += e[v];
@@ -249,12 +262,14 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
     __shared__ int s_flag;
     constexpr int NG = R * (R + 1) / 2;
     const int tid = threadIdx.x;
+    const CounterLayout cl = counter_layout(d.nrb, d.nsup, d.nchunk);
     unsigned* cnt = p.ws.cnt + d.cnt_off;
 
+    // 1) the last chunk tile of a row block: P_bar rows and the Gram partial
     __syncthreads();
     if (tid == 0) {
         __threadfence();
-        const unsigned prev = atomicAdd(&cnt[tc.rb], 1u);
+        const unsigned prev = atomicAdd(&cnt[cl.a_rb + tc.rb], 1u);
         if (prev >= static_cast<unsigned>(d.nchunk)) atomicOr(p.ws.status, kStatusCounter);
         s_flag = (prev == static_cast<unsigned>(d.nchunk - 1));
     }
@@ -277,11 +292,10 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
         pb_s[idx] = v;
         pbar[i * R + k] = v;
     }
-    if (tid == 0) cnt[tc.rb] = 0u;
+    if (tid == 0) cnt[cl.a_rb + tc.rb] = 0u;
     __syncthreads();
 
-    // Gram partial of this row block, float64
-    double* gram = p.ws.gram + d.gram_off + static_cast<int64_t>(tc.rb) * NG;
+    double* gram = p.ws.gram + d.gram_off;
     for (int pidx = tid; pidx < NG; pidx += kThreads) {
         int a = 0, rem = pidx;
         while (rem >= R - a) {
@@ -291,14 +305,38 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
         const int b = a + rem;
         double s = 0.0;
         for (int ii = 0; ii < rows; ++ii) s += pb_s[ii * R + a] * pb_s[ii * R + b];
-        gram[pidx] = s;
+        gram[static_cast<int64_t>(tc.rb) * NG + pidx] = s;
     }
+
+    // 2) the last row block of a super-block: sum its Gram partials
+    const int sup = tc.rb / kSuper;
+    const int rb0 = sup * kSuper;
+    const int nin = min(kSuper, d.nrb - rb0);
     __syncthreads();
     if (tid == 0) {
         __threadfence();
-        const unsigned prev = atomicAdd(&cnt[d.nrb], 1u);
-        if (prev >= static_cast<unsigned>(d.nrb)) atomicOr(p.ws.status, kStatusCounter);
-        s_flag = (prev == static_cast<unsigned>(d.nrb - 1));
+        const unsigned prev = atomicAdd(&cnt[cl.a_sup + sup], 1u);
+        if (prev >= static_cast<unsigned>(nin)) atomicOr(p.ws.status, kStatusCounter);
+        s_flag = (prev == static_cast<unsigned>(nin - 1));
+    }
+    __syncthreads();
+    if (!s_flag) return;
+    __threadfence();
+    double* gsup = p.ws.gsup + d.gsup_off;
+    for (int pidx = tid; pidx < NG; pidx += kThreads) {
+        double s = 0.0;
+        for (int k = 0; k < nin; ++k) s += __ldcg(&gram[static_cast<int64_t>(rb0 + k) * NG + pidx]);
+        gsup[static_cast<int64_t>(sup) * NG + pidx] = s;
+    }
+    if (tid == 0) cnt[cl.a_sup + sup] = 0u;
+
+    // 3) the last super-block of the layer: Gram sum and factorisation
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(&cnt[cl.a_layer], 1u);
+        if (prev >= static_cast<unsigned>(d.nsup)) atomicOr(p.ws.status, kStatusCounter);
+        s_flag = (prev == static_cast<unsigned>(d.nsup - 1));
     }
     __syncthreads();
     if (!s_flag) return;
@@ -308,7 +346,6 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
     double* Rs = Gs + R * R;
     double* Ts = Rs + R * R;
     int* drop = reinterpret_cast<int*>(Ts + R * R);
-    const double* gall = p.ws.gram + d.gram_off;
     for (int pidx = tid; pidx < NG; pidx += kThreads) {
         int a = 0, rem = pidx;
         while (rem >= R - a) {
@@ -317,7 +354,7 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
         }
         const int b = a + rem;
         double s = 0.0;
-        for (int rb = 0; rb < d.nrb; ++rb) s += __ldcg(&gall[static_cast<int64_t>(rb) * NG + pidx]);
+        for (int k = 0; k < d.nsup; ++k) s += __ldcg(&gsup[static_cast<int64_t>(k) * NG + pidx]);
         Gs[a * R + b] = s;
         Gs[b * R + a] = s;
     }
@@ -327,11 +364,13 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
         double* T = p.ws.T + d.t_off;
         for (int idx = tid; idx < R * R; idx += 32) T[idx] = Ts[idx];
     }
-    if (tid == 0) cnt[d.nrb] = 0u;
+    if (tid == 0) cnt[cl.a_layer] = 0u;
 }
 
-template <int R, typename GT, bool LAZY, bool SF>
-__global__ void __launch_bounds__(kThreads, (R >= 32) ? 1 : 2) k_pass_a(Params p) {
+// READM: a later power iteration of the same step; M is already in the
+// error buffers, so only M is read (no gradient, no store).
+template <int R, typename GT, bool LAZY, bool SF, bool READM>
+__global__ void __launch_bounds__(kThreads, (R >= 32) ? 1 : (R <= 4 ? 3 : 2)) k_pass_a(Params p) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int l = p.t.tile_layer[blockIdx.x];
     const LayerDesc d = p.t.layers[l];
@@ -358,11 +397,11 @@ __global__ void __launch_bounds__(kThreads, (R >= 32) ? 1 : 2) k_pass_a(Params p
     __syncthreads();
 
     if (d.vec == 4) {
-        if constexpr (R <= 8) pass_a_rows<R, 4, GT, LAZY, SF>(p, d, tc, gp, ep, rows_s);
+        if constexpr (R <= 8) pass_a_rows<R, 4, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
     } else if (d.vec == 2) {
-        if constexpr (R <= 16) pass_a_rows<R, 2, GT, LAZY, SF>(p, d, tc, gp, ep, rows_s);
+        if constexpr (R <= 16) pass_a_rows<R, 2, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
     } else {
-        pass_a_rows<R, 1, GT, LAZY, SF>(p, d, tc, gp, ep, rows_s);
+        pass_a_rows<R, 1, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
     }
     pass_a_epilogue<R>(p, d, tc, rows_d, fac);
 }
@@ -505,23 +544,51 @@ template <int R>
 __device__ void pass_b_epilogue(const Params& p, const LayerDesc& d, const TileCoord& tc) {
     __shared__ int s_flag;
     const int tid = threadIdx.x;
-    unsigned* cnt = p.ws.cnt + d.cnt_off + d.nrb + 1;
-    __syncthreads();
-    if (tid == 0) {
-        __threadfence();
-        const unsigned prev = atomicAdd(&cnt[tc.c], 1u);
-        if (prev >= static_cast<unsigned>(d.nrb)) atomicOr(p.ws.status, kStatusCounter);
-        s_flag = (prev == static_cast<unsigned>(d.nrb - 1));
-    }
-    __syncthreads();
-    if (!s_flag) return;
-    __threadfence();
+    const CounterLayout cl = counter_layout(d.nrb, d.nsup, d.nchunk);
+    unsigned* cnt = p.ws.cnt + d.cnt_off;
     const int64_t n = d.n;
     const int s0 = tc.c * d.slots;
     const int ns = min(d.slots, d.nvec - s0);
     const int64_t col0 = static_cast<int64_t>(s0) * d.vec;
     const int cols = ns * d.vec;
+
+    // 1) the last row block of a super-block (for this chunk): sum its partials
+    const int sup = tc.rb / kSuper;
+    const int rb0 = sup * kSuper;
+    const int nin = min(kSuper, d.nrb - rb0);
+    unsigned* c1 = &cnt[cl.b_sup + static_cast<int64_t>(tc.c) * d.nsup + sup];
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(c1, 1u);
+        if (prev >= static_cast<unsigned>(nin)) atomicOr(p.ws.status, kStatusCounter);
+        s_flag = (prev == static_cast<unsigned>(nin - 1));
+    }
+    __syncthreads();
+    if (!s_flag) return;
+    __threadfence();
     const double* qpart = p.ws.qpart + d.qpart_off;
+    double* qsup = p.ws.qsup + d.qsup_off;
+    for (int idx = tid; idx < cols * R; idx += kThreads) {
+        const int64_t col = col0 + idx / R;
+        const int k = idx % R;
+        double s = 0.0;
+        for (int j = 0; j < nin; ++j) s += __ldcg(&qpart[(static_cast<int64_t>(rb0 + j) * n + col) * R + k]);
+        qsup[(static_cast<int64_t>(sup) * n + col) * R + k] = s;
+    }
+    if (tid == 0) *c1 = 0u;
+
+    // 2) the last super-block of the chunk: Q_bar for the chunk's columns
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(&cnt[cl.b_chunk + tc.c], 1u);
+        if (prev >= static_cast<unsigned>(d.nsup)) atomicOr(p.ws.status, kStatusCounter);
+        s_flag = (prev == static_cast<unsigned>(d.nsup - 1));
+    }
+    __syncthreads();
+    if (!s_flag) return;
+    __threadfence();
     float* qbar = p.ws.qbar + d.qrow_off;
     float* qout = p.t.q[tc.l];
     const int r = p.r;
@@ -530,16 +597,16 @@ __device__ void pass_b_epilogue(const Params& p, const LayerDesc& d, const TileC
         const int64_t col = col0 + idx / R;
         const int k = idx % R;
         double s = 0.0;
-        for (int rb = 0; rb < d.nrb; ++rb) s += __ldcg(&qpart[(static_cast<int64_t>(rb) * n + col) * R + k]);
+        for (int j = 0; j < d.nsup; ++j) s += __ldcg(&qsup[(static_cast<int64_t>(j) * n + col) * R + k]);
         const float v = static_cast<float>(s * inv_w);
         qbar[col * R + k] = v;
         if (k < r) qout[col * r + k] = v;
     }
-    if (tid == 0) cnt[tc.c] = 0u;
+    if (tid == 0) cnt[cl.b_chunk + tc.c] = 0u;
 }
 
 template <int R, bool SF>
-__global__ void __launch_bounds__(kThreads, 2) k_pass_b(Params p) {
+__global__ void __launch_bounds__(kThreads, (R <= 4 ? 3 : 2)) k_pass_b(Params p) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int l = p.t.tile_layer[blockIdx.x];
     const LayerDesc d = p.t.layers[l];
@@ -676,6 +743,155 @@ __global__ void __launch_bounds__(kThreads, 2) k_pass_c(Params p) {
 }
 
 // ---------------------------------------------------------------------------
+// Rayleigh-Ritz rotation after converged subspace iterations (SVD refresh):
+// C = Q_bar^T Q_bar = W diag(lambda) W^T (cyclic Jacobi, float64, one warp,
+// eigenvalues sorted descending, every column of W signed so that its
+// largest-magnitude entry is positive), then P_hat <- P_hat W and
+// Q_bar <- Q_bar W.  When span(P_hat) is the top-r left singular subspace of
+// the worker mean, this makes P_hat = U_r and Q_bar = V_r Sigma_r; P_hat Q_bar^T
+// is unchanged.  One CTA per layer.
+template <int R>
+__global__ void __launch_bounds__(kThreads) k_rayleigh_ritz(Params p) {
+    __shared__ double C[R * R];
+    __shared__ double V[R * R];
+    __shared__ double Wm[R * R];
+    __shared__ double lam[R];
+    __shared__ int order[R];
+    const int l = blockIdx.x;
+    const LayerDesc d = p.t.layers[l];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int r = p.r;
+    constexpr int NG = R * (R + 1) / 2;
+    float* qbar = p.ws.qbar + d.qrow_off;
+    float* phat = p.ws.phat + d.prow_off;
+
+    // 1) C = Q_bar^T Q_bar (pairs over warps, rows over lanes, fixed order)
+    for (int pidx = warp; pidx < NG; pidx += kWarps) {
+        int a = 0, rem = pidx;
+        while (rem >= R - a) {
+            rem -= R - a;
+            ++a;
+        }
+        const int b = a + rem;
+        double s = 0.0;
+        for (int64_t j = lane; j < d.n; j += 32)
+            s += static_cast<double>(qbar[j * R + a]) * static_cast<double>(qbar[j * R + b]);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) {
+            C[a * R + b] = s;
+            C[b * R + a] = s;
+        }
+    }
+    __syncthreads();
+
+    // 2) eigen-decomposition of the r x r block by cyclic Jacobi (warp 0)
+    if (warp == 0) {
+        for (int idx = lane; idx < R * R; idx += 32) V[idx] = (idx / R == idx % R) ? 1.0 : 0.0;
+        __syncwarp();
+        double scale = 0.0;
+        for (int k = 0; k < r; ++k) scale += C[k * R + k] * C[k * R + k];
+        for (int sweep = 0; sweep < 40; ++sweep) {
+            double off = 0.0;
+            for (int a = 0; a < r; ++a)
+                for (int b = a + 1; b < r; ++b) off += C[a * R + b] * C[a * R + b];
+            if (!(off > 1e-30 * scale)) break;   // converged (also stops on NaN)
+            for (int a = 0; a < r - 1; ++a) {
+                for (int b = a + 1; b < r; ++b) {
+                    const double apq = C[a * R + b];
+                    if (apq == 0.0) continue;
+                    const double theta = (C[b * R + b] - C[a * R + a]) / (2.0 * apq);
+                    const double t = (theta == 0.0) ? 1.0
+                                                    : copysign(1.0, theta) / (fabs(theta) + sqrt(theta * theta + 1.0));
+                    const double c = 1.0 / sqrt(t * t + 1.0);
+                    const double sn = t * c;
+                    const int k = lane;
+                    if (k < r) {
+                        const double cp = C[k * R + a], cq = C[k * R + b];
+                        C[k * R + a] = c * cp - sn * cq;
+                        C[k * R + b] = sn * cp + c * cq;
+                    }
+                    __syncwarp();
+                    if (k < r) {
+                        const double rp = C[a * R + k], rq = C[b * R + k];
+                        C[a * R + k] = c * rp - sn * rq;
+                        C[b * R + k] = sn * rp + c * rq;
+                        const double vp = V[k * R + a], vq = V[k * R + b];
+                        V[k * R + a] = c * vp - sn * vq;
+                        V[k * R + b] = sn * vp + c * vq;
+                    }
+                    __syncwarp();
+                }
+            }
+        }
+        if (lane == 0) {
+            for (int k = 0; k < R; ++k) {
+                lam[k] = (k < r) ? C[k * R + k] : 0.0;
+                order[k] = k;
+            }
+            for (int a = 0; a < r; ++a) {   // selection sort, descending, stable
+                int best = a;
+                for (int b = a + 1; b < r; ++b)
+                    if (lam[order[b]] > lam[order[best]]) best = b;
+                const int tmp = order[a];
+                for (int b = best; b > a; --b) order[b] = order[b - 1];
+                order[a] = tmp;
+            }
+        }
+        __syncwarp();
+        for (int idx = lane; idx < R * R; idx += 32) Wm[idx] = 0.0;
+        __syncwarp();
+        if (lane < r) {
+            const int src = order[lane];
+            int arg = 0;
+            double best = -1.0;
+            for (int k = 0; k < r; ++k) {
+                const double v = fabs(V[k * R + src]);
+                if (v > best) {
+                    best = v;
+                    arg = k;
+                }
+            }
+            const double sg = (V[arg * R + src] < 0.0) ? -1.0 : 1.0;
+            for (int k = 0; k < r; ++k) Wm[k * R + lane] = sg * V[k * R + src];
+        }
+    }
+    __syncthreads();
+
+    // 3) rotate Q_bar and P_hat in place (one row per thread)
+    float* qout = p.t.q[l];
+    float* pout = (p.t.p_hat_out != nullptr) ? p.t.p_hat_out[l] : nullptr;
+    for (int64_t j = tid; j < d.n; j += kThreads) {
+        double row[R];
+#pragma unroll
+        for (int k = 0; k < R; ++k) row[k] = qbar[j * R + k];
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            double v = 0.0;
+#pragma unroll
+            for (int a = 0; a < R; ++a) v += row[a] * Wm[a * R + k];
+            const float f = static_cast<float>(v);
+            qbar[j * R + k] = f;
+            if (k < r) qout[j * r + k] = f;
+        }
+    }
+    for (int64_t i = tid; i < d.m; i += kThreads) {
+        double row[R];
+#pragma unroll
+        for (int k = 0; k < R; ++k) row[k] = phat[i * R + k];
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            double v = 0.0;
+#pragma unroll
+            for (int a = 0; a < R; ++a) v += row[a] * Wm[a * R + k];
+            const float f = static_cast<float>(v);
+            phat[i * R + k] = f;
+            if (pout != nullptr && k < r) pout[i * r + k] = f;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // small tensors: mean over workers (+ optional momentum)
 __global__ void k_vec_mean(const float* const* vecs, float* const* out, const int64_t* len, int count, int W,
                            float inv_w, float* const* params, float* const* mom, float lr, float beta) {
@@ -724,7 +940,7 @@ struct Philox4x64 {
     }
 };
 
-__global__ void k_init_q(float* const* q, const LayerDesc* layers, int r, uint64_t seed) {
+__global__ void k_init_q(float* const* q, const LayerDesc* layers, int r, uint64_t seed, uint64_t draw) {
     const int l = blockIdx.y;
     const int64_t total = layers[l].n * r;
     const int64_t nb = (total + 3) / 4;
@@ -732,7 +948,7 @@ __global__ void k_init_q(float* const* q, const LayerDesc* layers, int r, uint64
     constexpr double kTwoPi = 2.0 * 3.141592653589793;
     for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nb;
          b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        uint64_t x[4] = {static_cast<uint64_t>(b), 0ull, 0ull, 0ull};
+        uint64_t x[4] = {static_cast<uint64_t>(b), draw, 0ull, 0ull};
         Philox4x64::run(x, seed, static_cast<uint64_t>(l));
         double z[4];
 #pragma unroll

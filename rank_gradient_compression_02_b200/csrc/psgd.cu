@@ -25,7 +25,7 @@ namespace {
 
 constexpr double kDropTol = 1e-12;
 constexpr int64_t kTileTargetElems = 65536;  // worker elements per tile (all W workers)
-constexpr int kRowsFloatsMax = 2048;         // TM * R bound (shared-memory rows buffer)
+constexpr int kRowsFloatsMax = 4096;         // TM * R bound (shared-memory rows buffer)
 
 int pad_rank(int r) {
     int R = 1;
@@ -38,6 +38,49 @@ int max_vec_for_rank(int R) { return R <= 8 ? 4 : (R <= 16 ? 2 : 1); }
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Element counts of one layer's share of the workspace.
+struct LayerSizes {
+    int64_t prow, qrow, ppart, qpart, gram, gsup, qsup, t, cnt, tiles;
+};
+
+// Tile geometry of one m x n layer at padded rank R with W workers: lane
+// vector width, balanced column chunks, rows per tile for ~64K worker
+// elements per tile, super-blocks for the two-level reductions.
+LayerDesc layer_geometry(int64_t m, int64_t n, int R, int workers, LayerSizes* sz) {
+    LayerDesc d{};
+    d.m = m;
+    d.n = n;
+    d.vec = 1;
+    for (int v : {4, 2, 1})
+        if (v <= max_vec_for_rank(R) && n % v == 0) {
+            d.vec = v;
+            break;
+        }
+    d.nvec = static_cast<int>(n / d.vec);
+    d.nchunk = (d.nvec + 31) / 32;
+    d.slots = (d.nvec + d.nchunk - 1) / d.nchunk;
+    const int64_t cols = static_cast<int64_t>(d.slots) * d.vec;
+    int64_t tm = (kTileTargetElems + cols * workers - 1) / (cols * workers);
+    tm = (tm + 7) / 8 * 8;
+    tm = std::max<int64_t>(8, std::min<int64_t>(tm, std::min(512, kRowsFloatsMax / R)));
+    tm = std::min<int64_t>(tm, (m + 7) / 8 * 8);
+    d.tm = static_cast<int>(tm);
+    d.nrb = static_cast<int>((m + tm - 1) / tm);
+    d.nsup = (d.nrb + psgd::kSuper - 1) / psgd::kSuper;
+    const int NG = R * (R + 1) / 2;
+    sz->prow = m * R;
+    sz->qrow = n * R;
+    sz->ppart = static_cast<int64_t>(d.nchunk) * m * R;
+    sz->qpart = static_cast<int64_t>(d.nrb) * n * R;
+    sz->gram = static_cast<int64_t>(d.nrb) * NG;
+    sz->gsup = static_cast<int64_t>(d.nsup) * NG;
+    sz->qsup = static_cast<int64_t>(d.nsup) * n * R;
+    sz->t = static_cast<int64_t>(R) * R;
+    sz->cnt = psgd::counter_layout(d.nrb, d.nsup, d.nchunk).total;
+    sz->tiles = static_cast<int64_t>(d.nrb) * d.nchunk;
+    return d;
+}
 
 // Device copy of a host pointer table.  Re-uploaded only when the contents
 // change; uploads go through a small ring of pinned buffers so that an
@@ -142,6 +185,11 @@ struct psgd_ctx {
     std::vector<std::array<cudaEvent_t, 4>> prof_ev;
     size_t prof_used = 0;
 
+    int iters = 1;          // power iterations per step
+    int svd_every = 0;      // SVD refresh period in steps (0: off)
+    int svd_iters = 0;      // subspace iterations on a refresh step
+    uint64_t steps_done = 0;
+
     bool have_step = false;
     bool errors_hold_m = false;
     cudaStream_t last_stream = nullptr;
@@ -188,14 +236,19 @@ template <int R>
 struct Launch {
     static void* pass_a(int dtype, bool lazy, bool sf) {
         if (dtype == PSGD_BF16) {
-            if (lazy) return sf ? (void*)psgd::k_pass_a<R, uint16_t, true, true> : (void*)psgd::k_pass_a<R, uint16_t, true, false>;
-            return sf ? (void*)psgd::k_pass_a<R, uint16_t, false, true> : (void*)psgd::k_pass_a<R, uint16_t, false, false>;
+            if (lazy) return sf ? (void*)psgd::k_pass_a<R, uint16_t, true, true, false> : (void*)psgd::k_pass_a<R, uint16_t, true, false, false>;
+            return sf ? (void*)psgd::k_pass_a<R, uint16_t, false, true, false> : (void*)psgd::k_pass_a<R, uint16_t, false, false, false>;
         }
-        if (lazy) return sf ? (void*)psgd::k_pass_a<R, float, true, true> : (void*)psgd::k_pass_a<R, float, true, false>;
-        return sf ? (void*)psgd::k_pass_a<R, float, false, true> : (void*)psgd::k_pass_a<R, float, false, false>;
+        if (lazy) return sf ? (void*)psgd::k_pass_a<R, float, true, true, false> : (void*)psgd::k_pass_a<R, float, true, false, false>;
+        return sf ? (void*)psgd::k_pass_a<R, float, false, true, false> : (void*)psgd::k_pass_a<R, float, false, false, false>;
+    }
+    // later power iterations: M already formed in the error buffers
+    static void* pass_a_m(bool sf) {
+        return sf ? (void*)psgd::k_pass_a<R, float, false, true, true> : (void*)psgd::k_pass_a<R, float, false, false, true>;
     }
     static void* pass_b(bool sf) { return sf ? (void*)psgd::k_pass_b<R, true> : (void*)psgd::k_pass_b<R, false>; }
     static void* pass_c() { return (void*)psgd::k_pass_c<R>; }
+    static void* rayleigh_ritz() { return (void*)psgd::k_rayleigh_ritz<R>; }
 };
 
 void* kernel_ptr(int which, int R, int dtype, bool lazy, bool sf) {
@@ -203,6 +256,8 @@ void* kernel_ptr(int which, int R, int dtype, bool lazy, bool sf) {
     case RR:                                                 \
         if (which == 0) return Launch<RR>::pass_a(dtype, lazy, sf); \
         if (which == 1) return Launch<RR>::pass_b(sf);       \
+        if (which == 3) return Launch<RR>::pass_a_m(sf);     \
+        if (which == 4) return Launch<RR>::rayleigh_ritz();  \
         return Launch<RR>::pass_c();
     switch (R) {
         PSGD_CASE(1)
@@ -220,7 +275,7 @@ void* kernel_ptr(int which, int R, int dtype, bool lazy, bool sf) {
 size_t smem_need(int which, int R, int W, int tm, int vec) {
 #define PSGD_CASE(RR)                                                         \
     case RR:                                                                  \
-        if (which == 0) return psgd::SmemA<RR>::total(W, tm);                 \
+        if (which == 0 || which == 3) return psgd::SmemA<RR>::total(W, tm);   \
         if (which == 1) return psgd::SmemB<RR>::total(W, tm, vec);            \
         return psgd::SmemC<RR>::total(W, tm);
     switch (R) {
@@ -288,7 +343,8 @@ int psgd_create(psgd_ctx** out, const psgd_layer* layers, int num_layers, int ra
     if (workers < 1 || workers > psgd::kMaxWorkers)
         return fail(nullptr, PSGD_ERR_ARG, "workers %d not in [1, %d]", workers, psgd::kMaxWorkers);
     if (grad_dtype != PSGD_F32 && grad_dtype != PSGD_BF16) return fail(nullptr, PSGD_ERR_ARG, "bad grad dtype");
-    if (flags & ~(PSGD_FLAG_LAZY_ERRORS | PSGD_FLAG_SUM_FIRST)) return fail(nullptr, PSGD_ERR_ARG, "unknown flags");
+    if (flags & ~(PSGD_FLAG_LAZY_ERRORS | PSGD_FLAG_SUM_FIRST | PSGD_FLAG_NO_WARM_START))
+        return fail(nullptr, PSGD_ERR_ARG, "unknown flags");
     for (int l = 0; l < num_layers; ++l) {
         const int64_t m = layers[l].m, n = layers[l].n;
         if (m < 1 || n < 1) return fail(nullptr, PSGD_ERR_ARG, "layer %d: shape %lld x %lld", l, (long long)m, (long long)n);
@@ -310,50 +366,32 @@ int psgd_create(psgd_ctx** out, const psgd_layer* layers, int num_layers, int ra
     ctx->shapes.assign(layers, layers + num_layers);
 
     const int R = ctx->R;
-    const int NG = R * (R + 1) / 2;
-    const int vmax = max_vec_for_rank(R);
-    const int tm_cap = std::min(512, kRowsFloatsMax / R);
-    int64_t tiles = 0, prow = 0, qrow = 0, ppart = 0, qpart = 0, gram = 0, tt = 0, cnt = 0;
+    int64_t tiles = 0, prow = 0, qrow = 0, ppart = 0, qpart = 0, gram = 0, gsup = 0, qsup = 0, tt = 0, cnt = 0;
     std::vector<int> tile_layer;
     for (int l = 0; l < num_layers; ++l) {
-        LayerDesc d{};
-        d.m = layers[l].m;
-        d.n = layers[l].n;
-        int vec = 1;
-        for (int v : {4, 2, 1})
-            if (v <= vmax && d.n % v == 0) {
-                vec = v;
-                break;
-            }
-        d.vec = vec;
-        d.nvec = static_cast<int>(d.n / vec);
-        d.nchunk = (d.nvec + 31) / 32;
-        d.slots = (d.nvec + d.nchunk - 1) / d.nchunk;
-        const int64_t cols = static_cast<int64_t>(d.slots) * vec;
-        int64_t tm = (kTileTargetElems + cols * workers - 1) / (cols * workers);
-        tm = (tm + 7) / 8 * 8;
-        tm = std::max<int64_t>(8, std::min<int64_t>(tm, tm_cap));
-        tm = std::min<int64_t>(tm, (d.m + 7) / 8 * 8);
-        d.tm = static_cast<int>(tm);
-        d.nrb = static_cast<int>((d.m + tm - 1) / tm);
+        LayerSizes sz{};
+        LayerDesc d = layer_geometry(layers[l].m, layers[l].n, R, workers, &sz);
         d.tile_begin = tiles;
         d.prow_off = prow;
         d.qrow_off = qrow;
         d.ppart_off = ppart;
         d.qpart_off = qpart;
         d.gram_off = gram;
+        d.gsup_off = gsup;
+        d.qsup_off = qsup;
         d.t_off = tt;
         d.cnt_off = cnt;
-        const int64_t nt = static_cast<int64_t>(d.nrb) * d.nchunk;
-        tiles += nt;
-        prow += d.m * R;
-        qrow += d.n * R;
-        ppart += static_cast<int64_t>(d.nchunk) * d.m * R;
-        qpart += static_cast<int64_t>(d.nrb) * d.n * R;
-        gram += static_cast<int64_t>(d.nrb) * NG;
-        tt += R * R;
-        cnt += d.nrb + 1 + d.nchunk;
-        for (int64_t t = 0; t < nt; ++t) tile_layer.push_back(l);
+        tiles += sz.tiles;
+        prow += sz.prow;
+        qrow += sz.qrow;
+        ppart += sz.ppart;
+        qpart += sz.qpart;
+        gram += sz.gram;
+        gsup += sz.gsup;
+        qsup += sz.qsup;
+        tt += sz.t;
+        cnt += sz.cnt;
+        for (int64_t t = 0; t < sz.tiles; ++t) tile_layer.push_back(l);
         ctx->desc.push_back(d);
         ctx->smem_a = std::max(ctx->smem_a, smem_need(0, R, workers, d.tm, d.vec));
         ctx->smem_b = std::max(ctx->smem_b, smem_need(1, R, workers, d.tm, d.vec));
@@ -380,6 +418,8 @@ int psgd_create(psgd_ctx** out, const psgd_layer* layers, int num_layers, int ra
     const size_t o_ppart = carve(sizeof(double) * ppart);
     const size_t o_qpart = carve(sizeof(double) * qpart);
     const size_t o_gram = carve(sizeof(double) * gram);
+    const size_t o_gsup = carve(sizeof(double) * gsup);
+    const size_t o_qsup = carve(sizeof(double) * qsup);
     const size_t o_T = carve(sizeof(double) * tt);
     const size_t o_cnt = carve(sizeof(unsigned) * cnt);
     const size_t o_status = carve(sizeof(int));
@@ -399,6 +439,8 @@ int psgd_create(psgd_ctx** out, const psgd_layer* layers, int num_layers, int ra
     ctx->work.ppart = reinterpret_cast<double*>(base + o_ppart);
     ctx->work.qpart = reinterpret_cast<double*>(base + o_qpart);
     ctx->work.gram = reinterpret_cast<double*>(base + o_gram);
+    ctx->work.gsup = reinterpret_cast<double*>(base + o_gsup);
+    ctx->work.qsup = reinterpret_cast<double*>(base + o_qsup);
     ctx->work.T = reinterpret_cast<double*>(base + o_T);
     ctx->work.cnt = reinterpret_cast<unsigned*>(base + o_cnt);
     ctx->work.status = reinterpret_cast<int*>(base + o_status);
@@ -429,7 +471,9 @@ int psgd_create(psgd_ctx** out, const psgd_layer* layers, int num_layers, int ra
         const void* fa = kernel_ptr(0, R, grad_dtype, lazy != 0, sf);
         const void* fb = kernel_ptr(1, R, grad_dtype, lazy != 0, sf);
         const void* fc = kernel_ptr(2, R, grad_dtype, lazy != 0, sf);
+        const void* fam = kernel_ptr(3, R, grad_dtype, false, sf);
         e = raise_smem(fa, ctx->smem_a);
+        if (e == cudaSuccess) e = raise_smem(fam, ctx->smem_a);
         if (e == cudaSuccess) e = raise_smem(fb, ctx->smem_b);
         if (e == cudaSuccess) e = raise_smem(fc, ctx->smem_c);
         if (e != cudaSuccess) {
@@ -469,7 +513,9 @@ int psgd_workspace_bytes(const psgd_ctx* ctx, size_t* bytes) {
 int psgd_step_launches(const psgd_ctx* ctx) {
     if (!ctx) return -1;
     if (ctx->ntiles == 0) return 0;
-    return (ctx->flags & PSGD_FLAG_LAZY_ERRORS) ? 2 : 3;
+    int n = 2 * ctx->iters + ((ctx->flags & PSGD_FLAG_LAZY_ERRORS) ? 0 : 1);
+    if (ctx->flags & PSGD_FLAG_NO_WARM_START) n += 1;
+    return n;
 }
 
 int psgd_init_q(psgd_ctx* ctx, float* const* q, void* stream) {
@@ -489,7 +535,7 @@ int psgd_init_q(psgd_ctx* ctx, float* const* q, void* stream) {
     const int64_t blocks4 = (maxn * ctx->r + 3) / 4;
     const unsigned gx = static_cast<unsigned>(std::min<int64_t>(1024, (blocks4 + 255) / 256));
     psgd::k_init_q<<<dim3(std::max(1u, gx), ctx->L), 256, 0, s>>>(static_cast<float* const*>(ctx->tab_q.dev()),
-                                                                  ctx->desc_d, ctx->r, ctx->seed);
+                                                                  ctx->desc_d, ctx->r, ctx->seed, 0ull);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "init_q launch");
     ctx->last_stream = s;
@@ -538,9 +584,36 @@ static int step_impl(psgd_ctx* ctx, const void* const* grads, float* const* erro
         ev = ctx->prof_ev[ctx->prof_used++].data();
         cudaEventRecord(ev[0], s);
     }
-    int rc = launch(ctx, 0, lazy, p, ctx->smem_a, s);
+    int rc = PSGD_OK;
+    if (ctx->flags & PSGD_FLAG_NO_WARM_START) {
+        // no warm start: a fresh Q for this step (draw index = step number)
+        int64_t maxn = 0;
+        for (auto& d : ctx->desc) maxn = std::max(maxn, d.n);
+        const int64_t blocks4 = (maxn * ctx->r + 3) / 4;
+        const unsigned gx = static_cast<unsigned>(std::min<int64_t>(1024, (blocks4 + 255) / 256));
+        psgd::k_init_q<<<dim3(std::max(1u, gx), ctx->L), 256, 0, s>>>(p.t.q, ctx->desc_d, ctx->r, ctx->seed,
+                                                                      ctx->steps_done + 1);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "fresh Q launch");
+    }
+    rc = launch(ctx, 0, lazy, p, ctx->smem_a, s);
     if (ev) cudaEventRecord(ev[1], s);
     if (!rc) rc = launch(ctx, 1, lazy, p, ctx->smem_b, s);
+    const bool refresh = ctx->svd_every > 0 && (ctx->steps_done + 1) % ctx->svd_every == 0;
+    const int iters = refresh ? ctx->svd_iters : ctx->iters;
+    for (int it = 1; it < iters && !rc; ++it) {
+        psgd::Params pi = p;
+        pi.use_prev = 0;
+        rc = launch(ctx, 3, false, pi, ctx->smem_a, s);
+        if (!rc) rc = launch(ctx, 1, lazy, pi, ctx->smem_b, s);
+    }
+    if (refresh && !rc) {
+        // Rayleigh-Ritz: one CTA per layer
+        void* fn = kernel_ptr(4, ctx->R, ctx->dtype, false, false);
+        void* args[] = {&p};
+        e = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(ctx->L)), dim3(psgd::kThreads), args, 0, s);
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "Rayleigh-Ritz launch");
+    }
     if (ev) cudaEventRecord(ev[2], s);
     if (!rc && (!lazy || recon)) {
         psgd::Params pc = p;
@@ -552,6 +625,7 @@ static int step_impl(psgd_ctx* ctx, const void* const* grads, float* const* erro
     if (rc) return rc;
     ctx->have_step = true;
     ctx->errors_hold_m = lazy;
+    ctx->steps_done += 1;
     ctx->last_stream = s;
     return PSGD_OK;
 }
@@ -782,29 +856,9 @@ int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int grad_dtype
 
     // tile geometry of the one layer (same rules as a context's)
     const int R = pad_rank(rank);
-    const int NG = R * (R + 1) / 2;
-    LayerDesc d{};
-    d.m = m;
-    d.n = n;
-    d.vec = 1;
-    for (int v : {4, 2, 1})
-        if (v <= max_vec_for_rank(R) && n % v == 0) {
-            d.vec = v;
-            break;
-        }
-    d.nvec = static_cast<int>(n / d.vec);
-    d.nchunk = (d.nvec + 31) / 32;
-    d.slots = (d.nvec + d.nchunk - 1) / d.nchunk;
-    {
-        const int64_t cols = static_cast<int64_t>(d.slots) * d.vec;
-        int64_t tm = (kTileTargetElems + cols * workers - 1) / (cols * workers);
-        tm = (tm + 7) / 8 * 8;
-        tm = std::max<int64_t>(8, std::min<int64_t>(tm, std::min(512, kRowsFloatsMax / R)));
-        tm = std::min<int64_t>(tm, (m + 7) / 8 * 8);
-        d.tm = static_cast<int>(tm);
-        d.nrb = static_cast<int>((m + tm - 1) / tm);
-    }
-    const int64_t ntiles = static_cast<int64_t>(d.nrb) * d.nchunk;
+    LayerSizes sz{};
+    LayerDesc d = layer_geometry(m, n, R, workers, &sz);
+    const int64_t ntiles = sz.tiles;
 
     // scratch layout inside the static array
     size_t off = 0;
@@ -817,22 +871,25 @@ int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int grad_dtype
     const size_t o_desc = carve(sizeof(LayerDesc));
     const size_t o_tab = carve(sizeof(uint64_t) * ntab);
     const size_t o_tile = carve(sizeof(int) * ntiles);
-    const size_t o_pbar = carve(sizeof(double) * m * R);
-    const size_t o_phat = carve(sizeof(float) * m * R);
-    const size_t o_qbar = carve(sizeof(float) * n * R);
-    const size_t o_ppart = carve(sizeof(double) * d.nchunk * m * R);
-    const size_t o_qpart = carve(sizeof(double) * d.nrb * n * R);
-    const size_t o_gram = carve(sizeof(double) * d.nrb * NG);
-    const size_t o_T = carve(sizeof(double) * R * R);
-    const size_t o_cnt = carve(sizeof(unsigned) * (d.nrb + 1 + d.nchunk));
+    const size_t o_pbar = carve(sizeof(double) * sz.prow);
+    const size_t o_phat = carve(sizeof(float) * sz.prow);
+    const size_t o_qbar = carve(sizeof(float) * sz.qrow);
+    const size_t o_ppart = carve(sizeof(double) * sz.ppart);
+    const size_t o_qpart = carve(sizeof(double) * sz.qpart);
+    const size_t o_gram = carve(sizeof(double) * sz.gram);
+    const size_t o_gsup = carve(sizeof(double) * sz.gsup);
+    const size_t o_qsup = carve(sizeof(double) * sz.qsup);
+    const size_t o_T = carve(sizeof(double) * sz.t);
+    const size_t o_cnt = carve(sizeof(unsigned) * sz.cnt);
     const size_t o_status = carve(sizeof(int));
     if (off > PSGD_STATIC_SCRATCH_BYTES)
         return fail(nullptr, PSGD_ERR_ARG, "layer %lld x %lld at rank %d with %d workers needs %zu bytes of scratch; "
                     "the static scratch holds %u", (long long)m, (long long)n, rank, workers, off,
                     PSGD_STATIC_SCRATCH_BYTES);
-    // o_desc .. o_tab are the first pieces; the descriptor's own offsets are relative to the work arrays
+    // every array of the one layer starts at its own piece: offsets are 0
     d.tile_begin = 0;
-    d.prow_off = d.qrow_off = d.ppart_off = d.qpart_off = d.gram_off = d.t_off = d.cnt_off = 0;
+    d.prow_off = d.qrow_off = d.ppart_off = d.qpart_off = d.gram_off = d.gsup_off = d.qsup_off = d.t_off =
+        d.cnt_off = 0;
 
     void* base_v = nullptr;
     cudaError_t e = static_scratch_address(&base_v);
@@ -872,6 +929,8 @@ int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int grad_dtype
     p.ws.ppart = reinterpret_cast<double*>(base + o_ppart);
     p.ws.qpart = reinterpret_cast<double*>(base + o_qpart);
     p.ws.gram = reinterpret_cast<double*>(base + o_gram);
+    p.ws.gsup = reinterpret_cast<double*>(base + o_gsup);
+    p.ws.qsup = reinterpret_cast<double*>(base + o_qsup);
     p.ws.T = reinterpret_cast<double*>(base + o_T);
     p.ws.cnt = reinterpret_cast<unsigned*>(base + o_cnt);
     p.ws.status = reinterpret_cast<int*>(base + o_status);
@@ -899,6 +958,23 @@ int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int grad_dtype
         e = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(ntiles)), dim3(psgd::kThreads), args, smem[which], s);
         if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
     }
+    return PSGD_OK;
+}
+
+int psgd_set_power_iters(psgd_ctx* ctx, int iters) {
+    if (!ctx) return PSGD_ERR_ARG;
+    if (iters < 1 || iters > 8) return fail(ctx, PSGD_ERR_ARG, "power iterations %d not in [1, 8]", iters);
+    ctx->iters = iters;
+    return PSGD_OK;
+}
+
+int psgd_set_svd_refresh(psgd_ctx* ctx, int every, int iters) {
+    if (!ctx) return PSGD_ERR_ARG;
+    if (every < 0) return fail(ctx, PSGD_ERR_ARG, "refresh period %d < 0", every);
+    if (every > 0 && (iters < 1 || iters > 64))
+        return fail(ctx, PSGD_ERR_ARG, "refresh iterations %d not in [1, 64]", iters);
+    ctx->svd_every = every;
+    ctx->svd_iters = every > 0 ? iters : 0;
     return PSGD_OK;
 }
 

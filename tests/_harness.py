@@ -37,12 +37,15 @@ class LibRun:
     """Device state of one library context (per-layer tensors)."""
 
     def __init__(self, wl: Workload, seed: int = 1234, lazy: bool = False, sum_first: bool = False,
-                 recon: bool = True, device: str = "cuda"):
+                 recon: bool = True, device: str = "cuda", iters: int = 1, warm_start: bool = True,
+                 svd_every: int = 0, svd_iters: int = 8):
         from rank_gradient_compression_02_b200 import PowerSGD
         self.wl = wl
+        self.seed = seed
         self.src = GradientSource(wl, seed)
         self.lib = PowerSGD(wl.layers, wl.rank, wl.workers, seed=seed, grad_dtype=wl.grad_dtype,
-                            lazy_errors=lazy, sum_first=sum_first)
+                            lazy_errors=lazy, sum_first=sum_first, power_iters=iters, warm_start=warm_start,
+                            svd_every=svd_every, svd_iters=svd_iters)
         self.lazy = lazy
         gdt = torch.bfloat16 if wl.grad_dtype == "bf16" else torch.float32
         W, L = wl.workers, len(wl.layers)
@@ -79,15 +82,18 @@ class LibRun:
 class OracleRun:
     """Float64 oracle state for a subset of layers."""
 
-    def __init__(self, layers_idx: Sequence[int], E0, Q0):
+    def __init__(self, layers_idx: Sequence[int], E0, Q0, iters: int = 1):
         self.idx = list(layers_idx)
         self.E = {l: [np.asarray(e, dtype=np.float64) for e in E0[l]] for l in self.idx}
         self.Q = {l: np.asarray(Q0[l], dtype=np.float64) for l in self.idx}
+        self.iters = iters
         self.last: Dict[int, dict] = {}
 
-    def step(self, G: Dict[int, List[np.ndarray]]):
+    def step(self, G: Dict[int, List[np.ndarray]], Q_override: Optional[Dict[int, np.ndarray]] = None):
         for l in self.idx:
-            o = ora.step(G[l], self.E[l], self.Q[l])
+            if Q_override is not None:
+                self.Q[l] = np.asarray(Q_override[l], dtype=np.float64)
+            o = ora.step(G[l], self.E[l], self.Q[l], iters=self.iters)
             self.E[l] = o["E_new"]
             self.Q[l] = o["Q_bar"]
             self.last[l] = o
@@ -109,6 +115,14 @@ def compare_layer(run: LibRun, o: dict, l: int, tol: float, G_list=None, check_r
     return errs
 
 
+def sign_aligned(got: np.ndarray, want: np.ndarray) -> np.ndarray:
+    """got with every column's sign flipped to agree with want's column
+    (singular vectors are unique only up to sign)."""
+    s = np.sign(np.einsum("ij,ij->j", got, want))
+    s[s == 0] = 1.0
+    return got * s[None, :]
+
+
 def assert_close(errs: Dict[str, float], tol: float, what: str = ""):
     bad = {k: v for k, v in errs.items() if not (v <= tol)}
     assert not bad, f"{what}: errors above {tol}: {bad} (all: {errs})"
@@ -120,12 +134,12 @@ def small_workload(layers, rank, workers, dtype="f32", noise=("rel", 0.1), name=
 
 
 def run_free(wl: Workload, steps: int, lazy=False, sum_first=False, seed=1234, random_state: float = 0.0,
-             layers_idx: Optional[Sequence[int]] = None):
+             layers_idx: Optional[Sequence[int]] = None, iters: int = 1, warm_start: bool = True):
     """Run `steps` free-running steps on small inputs generated on the host.
     Returns (run, oracle, per-step max errors over the checked layers).  In
     lazy-error mode the error buffers hold M_w between steps; E' is
     compared only after the last step, once materialised."""
-    run = LibRun(wl, seed=seed, lazy=lazy, sum_first=sum_first)
+    run = LibRun(wl, seed=seed, lazy=lazy, sum_first=sum_first, iters=iters, warm_start=warm_start)
     L = len(wl.layers)
     idx = list(range(L)) if layers_idx is None else list(layers_idx)
     # initial state from synth on the host; the device gets a copy
@@ -137,7 +151,7 @@ def run_free(wl: Workload, steps: int, lazy=False, sum_first=False, seed=1234, r
     run.set_state(E0, Q0)
     E0_np = {l: [E0[w][l].to(torch.float64).numpy() for w in range(wl.workers)] for l in idx}
     Q0_np = {l: Q0[l].to(torch.float64).numpy() for l in idx}
-    orc = OracleRun(idx, E0_np, Q0_np)
+    orc = OracleRun(idx, E0_np, Q0_np, iters=iters)
     history = []
     for t in range(steps):
         host = run.fill_grads_host(t)
@@ -146,7 +160,12 @@ def run_free(wl: Workload, steps: int, lazy=False, sum_first=False, seed=1234, r
         if lazy and last:
             run.lib.materialize_errors(run.E)
         torch.cuda.synchronize()
-        orc.step({l: [host[w][l].to(torch.float64).numpy() for w in range(wl.workers)] for l in idx})
+        qo = None
+        if not warm_start:
+            # the step's fresh Q: the oracle's own Philox draw (draw = step number)
+            from oracle import philox64
+            qo = {l: philox64.initial_q(seed, l, wl.layers[l][1], wl.rank, draw=t + 1) for l in idx}
+        orc.step({l: [host[w][l].to(torch.float64).numpy() for w in range(wl.workers)] for l in idx}, qo)
         step_errs = {}
         for l in idx:
             e = compare_layer(run, orc.last[l], l, TOL[wl.grad_dtype])

@@ -218,9 +218,64 @@ def check_vec_mean(ora):
     np.testing.assert_allclose(ora.vec_mean(vs), [2.0, 3.0, 1.0], atol=1e-15)
 
 
+def check_power_iterations(ora):
+    """k power iterations in one step equal k warm-started single steps on the
+    same M without error feedback (each iteration is one step of subspace
+    iteration, [GLOS] warm-start paragraph), and converge twice as fast."""
+    rng = _rng(11)
+    m, n, r = 40, 30, 2
+    U = np.linalg.qr(rng.standard_normal((m, 4)))[0]
+    V = np.linalg.qr(rng.standard_normal((n, 4)))[0]
+    M = U @ np.diag([5.0, 2.5, 1.25, 0.625]) @ V.T + 1e-3 * rng.standard_normal((m, n))
+    Q = rng.standard_normal((n, r))
+    Z = np.zeros_like(M)
+    two = ora.step([M], [Z], Q, iters=2)
+    one = ora.step([M], [Z], ora.step([M], [Z], Q)["Q_bar"])
+    for key in ("P_hat", "Q_bar", "G_hat"):
+        np.testing.assert_allclose(two[key], one[key], atol=1e-12, err_msg=key)
+    np.testing.assert_allclose(two["E_new"][0], M - one["G_hat"], atol=1e-12)
+    # residual uses the last iteration's factors: P_hat^T E' = 0
+    np.testing.assert_allclose(two["P_hat"].T @ two["E_new"][0], 0.0, atol=1e-12)
+    Ur, _, _ = ora.jacobi_svd(M)
+    e1 = ora.subspace_sin_max(Ur[:, :r], ora.step([M], [Z], Q, iters=3)["P_hat"])
+    q = Q
+    for _ in range(3):
+        o = ora.step([M], [Z], q)
+        q = o["Q_bar"]
+    assert abs(e1 - ora.subspace_sin_max(Ur[:, :r], o["P_hat"])) < 1e-12
+
+
+def check_svd_refresh(ora):
+    """The refresh step's reconstruction is the best rank-r approximation of
+    the worker mean (Eckart-Young: its error is the tail of the singular
+    values), its factors are orthonormal / orthogonal with descending norms,
+    it agrees with the hand-written Jacobi SVD, and converged warm-started
+    power iterations reach the same reconstruction."""
+    rng = _rng(12)
+    m, n, r, W = 36, 28, 3, 3
+    U = np.linalg.qr(rng.standard_normal((m, 6)))[0]
+    V = np.linalg.qr(rng.standard_normal((n, 6)))[0]
+    base = U @ np.diag([6.0, 3.0, 1.5, 0.5, 0.2, 0.1]) @ V.T
+    G = [base + 0.01 * rng.standard_normal((m, n)) for _ in range(W)]
+    E = [0.01 * rng.standard_normal((m, n)) for _ in range(W)]
+    o = ora.svd_refresh_step(G, E, r)
+    Mbar = sum(g + e for g, e in zip(G, E)) / W
+    s = np.linalg.svd(Mbar, compute_uv=False)
+    assert abs(np.linalg.norm(Mbar - o["G_hat"]) ** 2 - np.sum(s[r:] ** 2)) < 1e-10
+    np.testing.assert_allclose(o["P_hat"].T @ o["P_hat"], np.eye(r), atol=1e-12)
+    QtQ = o["Q_bar"].T @ o["Q_bar"]
+    np.testing.assert_allclose(QtQ, np.diag(s[:r] ** 2), atol=1e-10)
+    Uj, sj, Vj = ora.jacobi_svd(Mbar)
+    np.testing.assert_allclose(Uj[:, :r] @ np.diag(sj[:r]) @ Vj[:, :r].T, o["G_hat"], atol=1e-10)
+    for w in range(W):
+        np.testing.assert_allclose(o["E_new"][w], G[w] + E[w] - o["G_hat"], atol=1e-12)
+    deep = ora.step(G, E, rng.standard_normal((n, r)), iters=40)
+    np.testing.assert_allclose(deep["G_hat"], o["G_hat"], atol=1e-9)
+
+
 ALL_CHECKS = [
     check_hand_cases, check_gram_schmidt_vs_householder, check_gram_schmidt_rank_deficient,
     check_rank1_closed_form, check_exact_low_rank, check_identities, check_linearity,
     check_jacobi_svd, check_warm_start_convergence, check_error_feedback_telescopes,
-    check_momentum_closed_form, check_vec_mean,
+    check_momentum_closed_form, check_vec_mean, check_power_iterations, check_svd_refresh,
 ]

@@ -76,7 +76,18 @@ def _momentum_dampened(x, mom, g_hat, lr, beta):
     return np.asarray(x) - lr * mom, mom
 
 
+def _step_restarts_iterations(G, E, Q, drop_tol=ora.DROP_TOL, iters=1):
+    # every iteration starts again from the warm start instead of the last Q_bar
+    out = None
+    for _ in range(iters):
+        out = _ORIG_STEP(G, E, Q, drop_tol, 1)
+    return out
+
+
+_ORIG_STEP = ora.step
+
 MUTANTS = {
+    "iterations_restart": {"step": _step_restarts_iterations},
     "ef_ignores_error": {"error_feedback_add": _ef_ignores_error},
     "residual_wrong_sign": {"residual": _residual_wrong_sign},
     "gs_no_normalise": {"gram_schmidt": _gs_no_normalise},

@@ -56,6 +56,66 @@ def test_modes(lazy, sum_first):
         H.assert_close(e, H.TOL["f32"], f"step {t}")
 
 
+@pytest.mark.parametrize("iters,lazy", [(2, False), (3, False), (2, True)])
+def test_power_iterations(iters, lazy):
+    wl = H.small_workload(MIXED, 4, 3)
+    run, _, hist = H.run_free(wl, steps=3, lazy=lazy, iters=iters)
+    assert run.lib.step_launches == 2 * iters + (0 if lazy else 1)
+    for t, e in enumerate(hist):
+        H.assert_close(e, H.TOL["f32"], f"step {t}")
+
+
+def test_no_warm_start():
+    # every step starts from a fresh Philox draw instead of the last Q_bar
+    wl = H.small_workload(MIXED, 2, 3)
+    _, _, hist = H.run_free(wl, steps=3, warm_start=False)
+    for t, e in enumerate(hist):
+        H.assert_close(e, H.TOL["f32"], f"step {t}")
+
+
+@pytest.mark.parametrize("rank,lazy", [(2, False), (4, False), (3, True)])
+def test_svd_refresh(rank, lazy):
+    # every second step is a PowerSGD+ refresh: 12 subspace iterations from
+    # the warm start + Rayleigh-Ritz, against the oracle's exact truncated
+    # SVD of the worker mean; singular vectors compared up to sign
+    wl = H.small_workload(MIXED[:5], rank, 3)
+    L, W = len(wl.layers), wl.workers
+    run = H.LibRun(wl, lazy=lazy, svd_every=2, svd_iters=12)
+    Q0 = [run.src.initial_q(l) for l in range(L)]
+    E0 = [[torch.zeros(m, n) for (m, n) in wl.layers] for _ in range(W)]
+    run.set_state(E0, Q0)
+    E = {l: [np.zeros(wl.layers[l]) for _ in range(W)] for l in range(L)}
+    Q = {l: Q0[l].double().numpy() for l in range(L)}
+    steps = 4
+    for t in range(steps):
+        host = run.fill_grads_host(t)
+        run.run_step()
+        last = t == steps - 1
+        if lazy and last:
+            run.lib.materialize_errors(run.E)
+        torch.cuda.synchronize()
+        refresh = (t + 1) % 2 == 0
+        for l in range(L):
+            G = [host[w][l].double().numpy() for w in range(W)]
+            o = ora.svd_refresh_step(G, E[l], rank) if refresh else ora.step(G, E[l], Q[l])
+            E[l], Q[l] = o["E_new"], o["Q_bar"]
+            errs = {"G_hat": H.rel_fro(H.to64(run.Rc[l]), o["G_hat"]),
+                    "P_hat": H.rel_fro(H.sign_aligned(H.to64(run.P[l]), o["P_hat"]), o["P_hat"]),
+                    "Q_bar": H.rel_fro(H.sign_aligned(H.to64(run.Q[l]), o["Q_bar"]), o["Q_bar"])}
+            if not lazy or last:
+                errs["E_new"] = max(H.rel_fro(H.to64(run.E[w][l]), o["E_new"][w],
+                                              denom=np.linalg.norm(o["M"][w])) for w in range(W))
+            H.assert_close(errs, H.TOL["f32"], f"step {t} layer {l} refresh={refresh}")
+            if refresh:
+                # singular-vector form: orthogonal Q_bar columns, descending norms
+                Qg = H.to64(run.Q[l])
+                C = Qg.T @ Qg
+                off = np.abs(C - np.diag(np.diag(C))).max() / np.abs(C).max()
+                assert off < 1e-5, off
+                assert np.all(np.diff(np.diag(C)) <= 1e-6 * C[0, 0])
+    run.lib.status()
+
+
 def test_from_random_state():
     wl = H.small_workload(MIXED, 4, 3)
     _, _, hist = H.run_free(wl, steps=2, random_state=0.05)
