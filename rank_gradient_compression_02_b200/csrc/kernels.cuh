@@ -92,14 +92,27 @@ __device__ void factor_gram_warp(const double* Gs, double* Rs, double* Ts, int* 
 // ---------------------------------------------------------------------------
 // pass A
 
+// Rank 32 uses the rank-lane kernels (one lane per rank index,
+// the tile's M rows staged in shared memory and read as broadcasts); they
+// walk a chunk (up to 32 * VEC columns) in sub-chunks of 32 columns.
+template <int R>
+struct IsWide { static constexpr bool value = R >= 32; };
+constexpr int kWideCols = 32;
+constexpr int kWideRows = 64;    // rows per tile cap for the rank-lane kernels
+
 template <int R>
 struct SmemA {
     // layout inside dynamic shared memory (bytes)
     static __host__ __device__ size_t ptr_bytes(int W) { return static_cast<size_t>(2 * W) * sizeof(void*); }
     static __host__ __device__ size_t rows_bytes(int tm) { return static_cast<size_t>(tm) * R * sizeof(double); }
     static __host__ __device__ size_t fac_bytes() { return 3 * R * R * sizeof(double) + 2 * R * sizeof(int) + 64; }
+    // rank-lane kernels: M tile, lazy reconstruction tile, previous Q_bar rows
+    static __host__ __device__ size_t wide_bytes(int tm) {
+        return IsWide<R>::value ? static_cast<size_t>(2 * tm * kWideCols + kWideCols * R) * sizeof(float) : 0;
+    }
     static __host__ __device__ size_t total(int W, int tm) {
-        return ((ptr_bytes(W) + 15) & ~size_t(15)) + ((rows_bytes(tm) + 15) & ~size_t(15)) + fac_bytes();
+        return ((ptr_bytes(W) + 15) & ~size_t(15)) + ((rows_bytes(tm) + 15) & ~size_t(15)) +
+               ((fac_bytes() + 15) & ~size_t(15)) + wide_bytes(tm);
     }
 };
 
@@ -254,6 +267,168 @@ __device__ __forceinline__ void pass_a_rows(const Params& p, const LayerDesc& d,
     }
 }
 
+// Rank-lane variant of the first pass (R = 16 or 32): lane k of a warp (of
+// a half-warp when R = 16) owns rank index k.  The tile's columns (up to
+// 32 * VEC) are walked in sub-chunks of 32: for every worker the CTA stages
+// the sub-chunk's M = G + E rows in shared memory (and stores M over E);
+// each lane then walks its rows, reading M as broadcasts and its slice of Q
+// from registers.  Products are summed in float32 over runs of 8 columns
+// and flushed to a float64 per-row accumulator; the row's partial over the
+// chunk needs no lane reduction.
+template <int R, typename GT, bool LAZY, bool SF, bool READM>
+__device__ __forceinline__ void pass_a_wide(const Params& p, const LayerDesc& d, const TileCoord& tc,
+                                            const GT* const* gp, float* const* ep, const float* ph_prev,
+                                            float* m_s, float* rec_s, float* qp_s) {
+    constexpr int HW = 32 / R;                       // rows side by side per warp
+    constexpr int RPL = kWideRows / (kWarps * HW);   // rows per lane, at most
+    constexpr int SPT = kWideRows / kWarps;          // staged rows per thread, at most
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int k = lane % R;
+    const int h = lane / R;
+    const int r = p.r;
+    const int W = p.workers;
+    const int64_t n = d.n, m = d.m;
+    const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
+    const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), m - i0));
+    const int64_t jc = static_cast<int64_t>(tc.c) * d.slots * d.vec;   // chunk's first column
+    const int width = static_cast<int>(min(static_cast<int64_t>(d.slots) * d.vec, n - jc));
+    const float* Q = p.t.q[tc.l];
+    const float* Qb = p.ws.qbar + d.qrow_off;
+
+    double acc[RPL];
+#pragma unroll
+    for (int t = 0; t < RPL; ++t) acc[t] = 0.0;
+
+    for (int sc = 0; sc * kWideCols < width; ++sc) {
+        const int64_t j0 = jc + sc * kWideCols;
+        const int ncols = min(kWideCols, width - sc * kWideCols);
+        float qreg[kWideCols];
+#pragma unroll
+        for (int jj = 0; jj < kWideCols; ++jj) qreg[jj] = (jj < ncols && k < r) ? Q[(j0 + jj) * r + k] : 0.f;
+        if constexpr (LAZY) {
+            // reconstruction of the previous step for this sub-chunk
+            __syncthreads();
+            for (int idx = tid; idx < kWideCols * R; idx += kThreads) {
+                const int jj = idx / R;
+                qp_s[idx] = (jj < ncols && p.use_prev) ? Qb[(j0 + jj) * R + (idx % R)] : 0.f;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int s2 = 0; s2 < SPT; ++s2) {
+                const int ii = warp + kWarps * s2;
+                if (ii < rows) {
+                    float ph[R];
+#pragma unroll
+                    for (int kk = 0; kk < R; ++kk) ph[kk] = ph_prev[ii * R + kk];
+                    rec_s[ii * kWideCols + lane] = recon_dot<R>(ph, qp_s + lane * R);
+                }
+            }
+        }
+        float msum[SPT];
+#pragma unroll
+        for (int s2 = 0; s2 < SPT; ++s2) msum[s2] = 0.f;
+
+        for (int w = 0; w < W; ++w) {
+            // stage worker w's sub-chunk rows: a warp per row, a lane per column
+            float gv[SPT], ev[SPT];
+#pragma unroll
+            for (int s2 = 0; s2 < SPT; ++s2) {
+                const int ii = warp + kWarps * s2;
+                gv[s2] = 0.f;
+                ev[s2] = 0.f;
+                if (ii < rows && lane < ncols) {
+                    const int64_t off = (i0 + ii) * n + j0 + lane;
+                    ev[s2] = ep[w][off];
+                    if constexpr (!READM) {
+                        float g1[1];
+                        ld_grad<GT, 1>(gp[w] + off, g1);
+                        gv[s2] = g1[0];
+                    }
+                }
+            }
+            if constexpr (!SF) __syncthreads();   // every lane is done with the previous tile
+#pragma unroll
+            for (int s2 = 0; s2 < SPT; ++s2) {
+                const int ii = warp + kWarps * s2;
+                if (ii < rows) {
+                    float mval = 0.f;
+                    if (lane < ncols) {
+                        mval = ev[s2];
+                        if constexpr (!READM) {
+                            float e2 = ev[s2];
+                            if constexpr (LAZY) e2 = e2 - rec_s[ii * kWideCols + lane];
+                            mval = gv[s2] + e2;
+                            ep[w][(i0 + ii) * n + j0 + lane] = mval;
+                        }
+                    }
+                    if constexpr (SF) {
+                        msum[s2] += mval;
+                    } else {
+                        m_s[ii * kWideCols + lane] = mval;
+                    }
+                }
+            }
+            if constexpr (SF) continue;
+            __syncthreads();
+#pragma unroll
+            for (int t = 0; t < RPL; ++t) {
+                const int ii = warp * HW + h + t * kWarps * HW;
+                if (ii < rows) {
+                    const float4* mrow = reinterpret_cast<const float4*>(m_s + ii * kWideCols);
+                    float run = 0.f;
+#pragma unroll
+                    for (int q4 = 0; q4 < kWideCols / 4; ++q4) {
+                        const float4 mv = mrow[q4];
+                        run = fmaf(mv.x, qreg[4 * q4 + 0], run);
+                        run = fmaf(mv.y, qreg[4 * q4 + 1], run);
+                        run = fmaf(mv.z, qreg[4 * q4 + 2], run);
+                        run = fmaf(mv.w, qreg[4 * q4 + 3], run);
+                        if (q4 & 1) {
+                            acc[t] += static_cast<double>(run);
+                            run = 0.f;
+                        }
+                    }
+                }
+            }
+        }
+        if constexpr (SF) {
+            __syncthreads();
+#pragma unroll
+            for (int s2 = 0; s2 < SPT; ++s2) {
+                const int ii = warp + kWarps * s2;
+                if (ii < rows) m_s[ii * kWideCols + lane] = msum[s2];
+            }
+            __syncthreads();
+#pragma unroll
+            for (int t = 0; t < RPL; ++t) {
+                const int ii = warp * HW + h + t * kWarps * HW;
+                if (ii < rows) {
+                    const float4* mrow = reinterpret_cast<const float4*>(m_s + ii * kWideCols);
+                    float run = 0.f;
+#pragma unroll
+                    for (int q4 = 0; q4 < kWideCols / 4; ++q4) {
+                        const float4 mv = mrow[q4];
+                        run = fmaf(mv.x, qreg[4 * q4 + 0], run);
+                        run = fmaf(mv.y, qreg[4 * q4 + 1], run);
+                        run = fmaf(mv.z, qreg[4 * q4 + 2], run);
+                        run = fmaf(mv.w, qreg[4 * q4 + 3], run);
+                        if (q4 & 1) {
+                            acc[t] += static_cast<double>(run);
+                            run = 0.f;
+                        }
+                    }
+                }
+            }
+        }
+    }
+    double* ppart = p.ws.ppart + d.ppart_off;
+#pragma unroll
+    for (int t = 0; t < RPL; ++t) {
+        const int ii = warp * HW + h + t * kWarps * HW;
+        if (ii < rows) ppart[(static_cast<int64_t>(tc.c) * m + i0 + ii) * R + k] = acc[t];
+    }
+}
+
 // Last CTA of a row block: P_bar rows and the Gram partial.  Last row block
 // of a layer: Gram sum and factorisation.
 template <int R>
@@ -370,7 +545,7 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
 // READM: a later power iteration of the same step; M is already in the
 // error buffers, so only M is read (no gradient, no store).
 template <int R, typename GT, bool LAZY, bool SF, bool READM>
-__global__ void __launch_bounds__(kThreads, (R >= 32) ? 1 : (R <= 4 ? 3 : 2)) k_pass_a(Params p) {
+__global__ void __launch_bounds__(kThreads, (R <= 4 ? 3 : 2)) k_pass_a(Params p) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int l = p.t.tile_layer[blockIdx.x];
     const LayerDesc d = p.t.layers[l];
@@ -383,6 +558,7 @@ __global__ void __launch_bounds__(kThreads, (R >= 32) ? 1 : (R <= 4 ? 3 : 2)) k_
     double* rows_d = reinterpret_cast<double*>(smem + ((SmemA<R>::ptr_bytes(W) + 15) & ~size_t(15)));
     float* rows_s = reinterpret_cast<float*>(rows_d);
     unsigned char* fac = reinterpret_cast<unsigned char*>(rows_d) + ((SmemA<R>::rows_bytes(d.tm) + 15) & ~size_t(15));
+    float* wide = reinterpret_cast<float*>(fac + ((SmemA<R>::fac_bytes() + 15) & ~size_t(15)));
 
     for (int w = threadIdx.x; w < W; w += kThreads) {
         gp[w] = static_cast<const GT*>(p.t.grads[w * L + l]);
@@ -396,12 +572,17 @@ __global__ void __launch_bounds__(kThreads, (R >= 32) ? 1 : (R <= 4 ? 3 : 2)) k_
     }
     __syncthreads();
 
-    if (d.vec == 4) {
-        if constexpr (R <= 8) pass_a_rows<R, 4, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
-    } else if (d.vec == 2) {
-        if constexpr (R <= 16) pass_a_rows<R, 2, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
+    if constexpr (IsWide<R>::value) {
+        pass_a_wide<R, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s, wide, wide + d.tm * kWideCols,
+                                            wide + 2 * d.tm * kWideCols);
     } else {
-        pass_a_rows<R, 1, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
+        if (d.vec == 4) {
+            pass_a_rows<R, 4, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
+        } else if (d.vec == 2) {
+            pass_a_rows<R, 2, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
+        } else {
+            pass_a_rows<R, 1, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
+        }
     }
     pass_a_epilogue<R>(p, d, tc, rows_d, fac);
 }
@@ -415,6 +596,12 @@ struct SmemB {
     static __host__ __device__ size_t rows_bytes(int tm) { return static_cast<size_t>(tm) * R * sizeof(float); }
     static __host__ __device__ size_t t_bytes() { return R * R * sizeof(double); }
     static __host__ __device__ size_t red_bytes(int vec) {
+        if (IsWide<R>::value) {
+            // rank-lane kernel: the M tile (tm x 128), reused for the row-group sums
+            const size_t tile = static_cast<size_t>(kWideRows) * 4 * kWideCols * sizeof(float);
+            const size_t red = static_cast<size_t>(2 * (32 / R)) * 4 * kWideCols * R * sizeof(float);
+            return tile > red ? tile : red;
+        }
         return static_cast<size_t>(kWarps) * R * vec * 32 * sizeof(float);
     }
     static __host__ __device__ size_t total(int W, int tm, int vec) {
@@ -540,6 +727,107 @@ __device__ __forceinline__ void pass_b_rows(const Params& p, const LayerDesc& d,
     }
 }
 
+// Stage worker w's M tile (rows x chunk width, zero beyond) into m_s
+// (row stride 4 * kWideCols floats); float4 accesses when VEC = 4.
+__device__ __forceinline__ void stage_m_tile(const float* src, int64_t n, int64_t i0, int64_t jc, int rows,
+                                             int width, int vec, float* m_s) {
+    constexpr int STR = 4 * kWideCols;
+    if (vec == 4) {
+        for (int idx = threadIdx.x; idx < kWideRows * kWideCols; idx += kThreads) {
+            const int ii = idx / kWideCols, q = idx % kWideCols;
+            if (ii >= rows) break;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (4 * q < width) v = *reinterpret_cast<const float4*>(src + (i0 + ii) * n + jc + 4 * q);
+            *reinterpret_cast<float4*>(m_s + ii * STR + 4 * q) = v;
+        }
+    } else {
+        for (int idx = threadIdx.x; idx < kWideRows * STR; idx += kThreads) {
+            const int ii = idx / STR, jj = idx % STR;
+            if (ii >= rows) break;
+            m_s[ii * STR + jj] = (jj < width) ? src[(i0 + ii) * n + jc + jj] : 0.f;
+        }
+    }
+}
+
+// Rank-lane variant of the second pass (R = 16 or 32): lane k owns rank
+// index k, warp w owns 32 columns of the chunk (w % 4) and a row group
+// (w / 4, split again between half-warps when R = 16).  Per worker the CTA
+// stages the M tile in shared memory; a lane accumulates, in float32, the
+// products of its 32 columns with P_hat[i][k] over its rows and all
+// workers; the row groups are summed in float64 at the end.
+template <int R, bool SF>
+__device__ __forceinline__ void pass_b_wide(const Params& p, const LayerDesc& d, const TileCoord& tc,
+                                            float* const* ep, const float* ph_s, float* m_s) {
+    constexpr int HW = 32 / R;
+    constexpr int NG = 2 * HW;                 // row groups
+    constexpr int STR = 4 * kWideCols;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int k = lane % R;
+    const int h = lane / R;
+    const int cg = warp & 3;
+    const int grp = (warp >> 2) * HW + h;
+    const int W = p.workers;
+    const int64_t n = d.n, m = d.m;
+    const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
+    const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), m - i0));
+    const int64_t jc = static_cast<int64_t>(tc.c) * d.slots * d.vec;
+    const int width = static_cast<int>(min(static_cast<int64_t>(d.slots) * d.vec, n - jc));
+
+    float acc[kWideCols];
+#pragma unroll
+    for (int c = 0; c < kWideCols; ++c) acc[c] = 0.f;
+    auto accumulate = [&]() {
+        for (int ii = grp; ii < rows; ii += NG) {
+            const float ph = ph_s[ii * R + k];
+            const float4* mrow = reinterpret_cast<const float4*>(m_s + ii * STR + cg * kWideCols);
+#pragma unroll
+            for (int c4 = 0; c4 < kWideCols / 4; ++c4) {
+                const float4 mv = mrow[c4];
+                acc[4 * c4 + 0] = fmaf(mv.x, ph, acc[4 * c4 + 0]);
+                acc[4 * c4 + 1] = fmaf(mv.y, ph, acc[4 * c4 + 1]);
+                acc[4 * c4 + 2] = fmaf(mv.z, ph, acc[4 * c4 + 2]);
+                acc[4 * c4 + 3] = fmaf(mv.w, ph, acc[4 * c4 + 3]);
+            }
+        }
+    };
+    if constexpr (SF) {
+        // sum of the workers' tiles, then one product
+        for (int w = 0; w < W; ++w) {
+            if (w == 0) {
+                stage_m_tile(ep[0], n, i0, jc, rows, width, d.vec, m_s);
+            } else {
+                for (int idx = tid; idx < rows * STR; idx += kThreads) {
+                    const int ii = idx / STR, jj = idx % STR;
+                    if (jj < width) m_s[idx] += ep[w][(i0 + ii) * n + jc + jj];
+                }
+            }
+            __syncthreads();
+        }
+        accumulate();
+    } else {
+        for (int w = 0; w < W; ++w) {
+            if (w) __syncthreads();
+            stage_m_tile(ep[w], n, i0, jc, rows, width, d.vec, m_s);
+            __syncthreads();
+            accumulate();
+        }
+    }
+    __syncthreads();
+    // row-group partials [grp][column][k], then fixed-order float64 sums
+    float* red_s = m_s;
+#pragma unroll
+    for (int c = 0; c < kWideCols; ++c) red_s[(grp * STR + cg * kWideCols + c) * R + k] = acc[c];
+    __syncthreads();
+    double* qpart = p.ws.qpart + d.qpart_off;
+    for (int idx = tid; idx < width * R; idx += kThreads) {
+        const int col = idx / R, kk = idx % R;
+        double s2 = 0.0;
+#pragma unroll
+        for (int g = 0; g < NG; ++g) s2 += static_cast<double>(red_s[(g * STR + col) * R + kk]);
+        qpart[(static_cast<int64_t>(tc.rb) * n + jc + col) * R + kk] = s2;
+    }
+}
+
 template <int R>
 __device__ void pass_b_epilogue(const Params& p, const LayerDesc& d, const TileCoord& tc) {
     __shared__ int s_flag;
@@ -623,12 +911,16 @@ __global__ void __launch_bounds__(kThreads, (R <= 4 ? 3 : 2)) k_pass_b(Params p)
     for (int w = threadIdx.x; w < W; w += kThreads) ep[w] = p.t.errors[w * L + l];
     load_phat_rows<R>(p, d, tc, ph_s, T_s, tc.c == 0);
 
-    if (d.vec == 4) {
-        if constexpr (R <= 8) pass_b_rows<R, 4, SF>(p, d, tc, ep, ph_s, red_s);
-    } else if (d.vec == 2) {
-        if constexpr (R <= 16) pass_b_rows<R, 2, SF>(p, d, tc, ep, ph_s, red_s);
+    if constexpr (IsWide<R>::value) {
+        pass_b_wide<R, SF>(p, d, tc, ep, ph_s, red_s);
     } else {
-        pass_b_rows<R, 1, SF>(p, d, tc, ep, ph_s, red_s);
+        if (d.vec == 4) {
+            pass_b_rows<R, 4, SF>(p, d, tc, ep, ph_s, red_s);
+        } else if (d.vec == 2) {
+            pass_b_rows<R, 2, SF>(p, d, tc, ep, ph_s, red_s);
+        } else {
+            pass_b_rows<R, 1, SF>(p, d, tc, ep, ph_s, red_s);
+        }
     }
     pass_b_epilogue<R>(p, d, tc);
 }
@@ -640,10 +932,98 @@ template <int R>
 struct SmemC {
     static __host__ __device__ size_t ptr_bytes(int W) { return static_cast<size_t>(W < 1 ? 1 : W) * sizeof(void*); }
     static __host__ __device__ size_t rows_bytes(int tm) { return static_cast<size_t>(tm) * R * sizeof(float); }
+    static __host__ __device__ size_t wide_bytes() {
+        return IsWide<R>::value ? static_cast<size_t>(R) * 4 * kWideCols * sizeof(float) : 0;
+    }
     static __host__ __device__ size_t total(int W, int tm) {
-        return ((ptr_bytes(W) + 15) & ~size_t(15)) + rows_bytes(tm);
+        return ((ptr_bytes(W) + 15) & ~size_t(15)) + ((rows_bytes(tm) + 15) & ~size_t(15)) + wide_bytes();
     }
 };
+
+// Rank-lane variant of the third pass (R = 16 or 32).  The tile's
+// reconstruction rec = P_hat Q_bar^T (rows x chunk width) is formed once
+// from shared memory (Q_bar transposed, float4 per lane) with the same
+// float32 operation order as recon_dot, then applied to every worker:
+// thread (warp w, lane q) owns rows w + 8 s and columns 4q .. 4q+3.
+template <int R>
+__device__ __forceinline__ void pass_c_wide(const Params& p, const LayerDesc& d, const TileCoord& tc,
+                                            float* const* ep, const float* ph_s, float* qt_s) {
+    constexpr int STR = 4 * kWideCols;
+    constexpr int SR = kWideRows / kWarps;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int W = p.do_resid ? p.workers : 0;
+    const int64_t n = d.n, m = d.m;
+    const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
+    const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), m - i0));
+    const int64_t jc = static_cast<int64_t>(tc.c) * d.slots * d.vec;
+    const int width = static_cast<int>(min(static_cast<int64_t>(d.slots) * d.vec, n - jc));
+    const float* Qb = p.ws.qbar + d.qrow_off;
+    for (int idx = tid; idx < R * STR; idx += kThreads) {
+        const int kk = idx / STR, jj = idx % STR;
+        qt_s[idx] = (jj < width) ? Qb[(jc + jj) * R + kk] : 0.f;
+    }
+    __syncthreads();
+    float rec[SR][4];
+#pragma unroll
+    for (int s2 = 0; s2 < SR; ++s2)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) rec[s2][v] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < R; ++kk) {
+        const float4 q = *reinterpret_cast<const float4*>(qt_s + kk * STR + 4 * lane);
+#pragma unroll
+        for (int s2 = 0; s2 < SR; ++s2) {
+            const int ii = warp + kWarps * s2;
+            const float ph = (ii < rows) ? ph_s[ii * R + kk] : 0.f;
+            rec[s2][0] = fmaf(ph, q.x, rec[s2][0]);
+            rec[s2][1] = fmaf(ph, q.y, rec[s2][1]);
+            rec[s2][2] = fmaf(ph, q.z, rec[s2][2]);
+            rec[s2][3] = fmaf(ph, q.w, rec[s2][3]);
+        }
+    }
+    float* recon = (p.do_recon && p.t.recon_out != nullptr) ? p.t.recon_out[tc.l] : nullptr;
+    float* xs = p.do_mom ? p.t.params[tc.l] : nullptr;
+    float* ms = p.do_mom ? p.t.mom[tc.l] : nullptr;
+    const int jq = 4 * lane;
+    if (jq >= width) return;
+    const bool full4 = (d.vec == 4);   // 4 columns, 16-byte aligned
+    const int nv = min(4, width - jq);
+#pragma unroll
+    for (int s2 = 0; s2 < SR; ++s2) {
+        const int ii = warp + kWarps * s2;
+        if (ii >= rows) break;
+        const int64_t base = (i0 + ii) * n + jc + jq;
+        auto apply = [&](float* ptr, auto&& op) {
+            if (full4) {
+                float4 v = *reinterpret_cast<float4*>(ptr + base);
+                op(v.x, 0); op(v.y, 1); op(v.z, 2); op(v.w, 3);
+                *reinterpret_cast<float4*>(ptr + base) = v;
+            } else {
+                for (int v = 0; v < nv; ++v) op(ptr[base + v], v);
+            }
+        };
+        if (recon != nullptr) apply(recon, [&](float& x, int v) { x = rec[s2][v]; });
+        if (xs != nullptr) {
+            if (full4) {
+                float4 mo = *reinterpret_cast<float4*>(ms + base);
+                float4 x = *reinterpret_cast<float4*>(xs + base);
+                mo.x = fmaf(p.beta, mo.x, rec[s2][0]); x.x = fmaf(-p.lr, mo.x, x.x);
+                mo.y = fmaf(p.beta, mo.y, rec[s2][1]); x.y = fmaf(-p.lr, mo.y, x.y);
+                mo.z = fmaf(p.beta, mo.z, rec[s2][2]); x.z = fmaf(-p.lr, mo.z, x.z);
+                mo.w = fmaf(p.beta, mo.w, rec[s2][3]); x.w = fmaf(-p.lr, mo.w, x.w);
+                *reinterpret_cast<float4*>(ms + base) = mo;
+                *reinterpret_cast<float4*>(xs + base) = x;
+            } else {
+                for (int v = 0; v < nv; ++v) {
+                    const float mo = fmaf(p.beta, ms[base + v], rec[s2][v]);
+                    ms[base + v] = mo;
+                    xs[base + v] = fmaf(-p.lr, mo, xs[base + v]);
+                }
+            }
+        }
+        for (int w = 0; w < W; ++w) apply(ep[w], [&](float& x, int v) { x = x - rec[s2][v]; });
+    }
+}
 
 template <int R, int VEC>
 __device__ __forceinline__ void pass_c_rows(const Params& p, const LayerDesc& d, const TileCoord& tc,
@@ -724,6 +1104,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_pass_c(Params p) {
     const int L = p.num_layers;
     float** ep = reinterpret_cast<float**>(smem);
     float* ph_s = reinterpret_cast<float*>(smem + ((SmemC<R>::ptr_bytes(W) + 15) & ~size_t(15)));
+    float* qt_s = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(ph_s) +
+                                           ((SmemC<R>::rows_bytes(d.tm) + 15) & ~size_t(15)));
     if (p.do_resid)
         for (int w = threadIdx.x; w < W; w += kThreads) ep[w] = p.t.errors[w * L + l];
     {
@@ -733,12 +1115,16 @@ __global__ void __launch_bounds__(kThreads, 2) k_pass_c(Params p) {
         for (int idx = threadIdx.x; idx < rows * R; idx += kThreads) ph_s[idx] = ph[idx];
     }
     __syncthreads();
-    if (d.vec == 4) {
-        if constexpr (R <= 8) pass_c_rows<R, 4>(p, d, tc, ep, ph_s);
-    } else if (d.vec == 2) {
-        if constexpr (R <= 16) pass_c_rows<R, 2>(p, d, tc, ep, ph_s);
+    if constexpr (IsWide<R>::value) {
+        pass_c_wide<R>(p, d, tc, ep, ph_s, qt_s);
     } else {
-        pass_c_rows<R, 1>(p, d, tc, ep, ph_s);
+        if (d.vec == 4) {
+            pass_c_rows<R, 4>(p, d, tc, ep, ph_s);
+        } else if (d.vec == 2) {
+            pass_c_rows<R, 2>(p, d, tc, ep, ph_s);
+        } else {
+            pass_c_rows<R, 1>(p, d, tc, ep, ph_s);
+        }
     }
 }
 

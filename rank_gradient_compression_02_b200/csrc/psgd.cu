@@ -33,7 +33,9 @@ int pad_rank(int r) {
     return R;
 }
 
-int max_vec_for_rank(int R) { return R <= 8 ? 4 : (R <= 16 ? 2 : 1); }
+// lanes load VEC adjacent columns (a chunk is up to 32 * VEC columns); the
+// lane-per-column kernels keep VEC x R values of Q per lane in registers
+int max_vec_for_rank(int R) { return R <= 8 ? 4 : (R <= 16 ? 2 : 4); }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -63,7 +65,7 @@ LayerDesc layer_geometry(int64_t m, int64_t n, int R, int workers, LayerSizes* s
     const int64_t cols = static_cast<int64_t>(d.slots) * d.vec;
     int64_t tm = (kTileTargetElems + cols * workers - 1) / (cols * workers);
     tm = (tm + 7) / 8 * 8;
-    tm = std::max<int64_t>(8, std::min<int64_t>(tm, std::min(512, kRowsFloatsMax / R)));
+    tm = std::max<int64_t>(8, std::min<int64_t>(tm, std::min(R >= 32 ? psgd::kWideRows : 512, kRowsFloatsMax / R)));
     tm = std::min<int64_t>(tm, (m + 7) / 8 * 8);
     d.tm = static_cast<int>(tm);
     d.nrb = static_cast<int>((m + tm - 1) / tm);
