@@ -576,10 +576,11 @@ __global__ void __launch_bounds__(kThreads, (R <= 4 ? 3 : 2)) k_pass_a(Params p)
         pass_a_wide<R, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s, wide, wide + d.tm * kWideCols,
                                             wide + 2 * d.tm * kWideCols);
     } else {
+        // VEC x R values of Q live in registers: VEC = 4 up to R = 8, 2 up to 16
         if (d.vec == 4) {
-            pass_a_rows<R, 4, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
+            if constexpr (R <= 8) pass_a_rows<R, 4, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
         } else if (d.vec == 2) {
-            pass_a_rows<R, 2, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
+            if constexpr (R <= 16) pass_a_rows<R, 2, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
         } else {
             pass_a_rows<R, 1, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
         }
@@ -915,9 +916,9 @@ __global__ void __launch_bounds__(kThreads, (R <= 4 ? 3 : 2)) k_pass_b(Params p)
         pass_b_wide<R, SF>(p, d, tc, ep, ph_s, red_s);
     } else {
         if (d.vec == 4) {
-            pass_b_rows<R, 4, SF>(p, d, tc, ep, ph_s, red_s);
+            if constexpr (R <= 8) pass_b_rows<R, 4, SF>(p, d, tc, ep, ph_s, red_s);
         } else if (d.vec == 2) {
-            pass_b_rows<R, 2, SF>(p, d, tc, ep, ph_s, red_s);
+            if constexpr (R <= 16) pass_b_rows<R, 2, SF>(p, d, tc, ep, ph_s, red_s);
         } else {
             pass_b_rows<R, 1, SF>(p, d, tc, ep, ph_s, red_s);
         }
@@ -1119,9 +1120,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_pass_c(Params p) {
         pass_c_wide<R>(p, d, tc, ep, ph_s, qt_s);
     } else {
         if (d.vec == 4) {
-            pass_c_rows<R, 4>(p, d, tc, ep, ph_s);
+            if constexpr (R <= 8) pass_c_rows<R, 4>(p, d, tc, ep, ph_s);
         } else if (d.vec == 2) {
-            pass_c_rows<R, 2>(p, d, tc, ep, ph_s);
+            if constexpr (R <= 16) pass_c_rows<R, 2>(p, d, tc, ep, ph_s);
         } else {
             pass_c_rows<R, 1>(p, d, tc, ep, ph_s);
         }
