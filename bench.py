@@ -255,6 +255,7 @@ def main():
     ap.add_argument("--layers", default=None, help="comma-separated layer indices (a subset, for small captures)")
     ap.add_argument("--workers", type=int, default=None, help="override the worker count (small captures)")
     ap.add_argument("--iters", type=int, default=1, help="power iterations per step")
+    ap.add_argument("--no-variants", action="store_true", help="skip timing the lazy-error variant")
     args = ap.parse_args()
 
     from dataclasses import replace
@@ -348,6 +349,32 @@ def main():
                 "per_kernel_ms": {n: round(t, 4) for n, t in zip(names, per_launch_ms)},
                 "step_algorithmic_frac": round(step_min_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 4)}
 
+    # the lazy-error representation of the same step (E' rebuilt inside the
+    # next step's first pass; bit-identical results), timed the same way
+    variants = {}
+    if not args.lazy and not args.no_variants:
+        lazy_lib = PowerSGD(wl.layers, r, wl.workers, grad_dtype=wl.grad_dtype, lazy_errors=True,
+                            sum_first=args.sum_first, power_iters=args.iters)
+        for _ in range(args.warmup):
+            run_step(lazy_lib, B, wl)
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            run_step(lazy_lib, B, wl)
+        lazy_lib.materialize_errors(B.E)    # the last step's E' written out, inside the timed region
+        e1.record(stream)
+        torch.cuda.synchronize()
+        lazy_lib.status()
+        lms = max_over_ranks(e0.elapsed_time(e1), world, device) / args.steps
+        variants["lazy_errors"] = {"ms_per_step": lms, "value": job_value(wl.elements, world, lms),
+                                   "step_algorithmic_frac": round(step_min_bytes / (lms * 1e-3) / 1e9 / peak, 4),
+                                   "note": "error buffers hold M between steps; E' materialised once at the end "
+                                           "of the timed region"}
+        lazy_lib.close()
+
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(lib, B, wl, r, args, world, device)
@@ -363,7 +390,7 @@ def main():
            "vs_baseline": None, "dtype": "f32" if wl.grad_dtype == "f32" else "bf16-in/f32",
            "data": "synthetic (seeded low-rank + noise gradients, resident in HBM)",
            "config": config, "gpu_launches": args.steps * launches_per_step(lib, B),
-           "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+           "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "variants": variants,
            "hbm_gbs_step": round(step_min_bytes / (ms_per_step * 1e-3) / 1e9, 1)}
     if rank_id == 0:
         print(json.dumps(out), flush=True)

@@ -92,9 +92,9 @@ __device__ void factor_gram_warp(const double* Gs, double* Rs, double* Ts, int* 
 // ---------------------------------------------------------------------------
 // pass A
 
-// Rank 32 uses the rank-lane kernels (one lane per rank index,
-// the tile's M rows staged in shared memory and read as broadcasts); they
-// walk a chunk (up to 32 * VEC columns) in sub-chunks of 32 columns.
+// Rank 32 uses the rank-lane kernels (one lane per rank index, M rows
+// parked in shared memory and read as broadcasts); they walk a chunk (up to
+// 32 * VEC columns) in sub-chunks of 32 columns.
 template <int R>
 struct IsWide { static constexpr bool value = R >= 32; };
 constexpr int kWideCols = 32;
@@ -106,9 +106,10 @@ struct SmemA {
     static __host__ __device__ size_t ptr_bytes(int W) { return static_cast<size_t>(2 * W) * sizeof(void*); }
     static __host__ __device__ size_t rows_bytes(int tm) { return static_cast<size_t>(tm) * R * sizeof(double); }
     static __host__ __device__ size_t fac_bytes() { return 3 * R * R * sizeof(double) + 2 * R * sizeof(int) + 64; }
-    // rank-lane kernels: M tile, lazy reconstruction tile, previous Q_bar rows
+    // rank-lane kernel: every warp's parked rows (tm x 32 floats in all)
     static __host__ __device__ size_t wide_bytes(int tm) {
-        return IsWide<R>::value ? static_cast<size_t>(2 * tm * kWideCols + kWideCols * R) * sizeof(float) : 0;
+        (void)tm;
+        return IsWide<R>::value ? static_cast<size_t>(kWideRows * kWideCols) * sizeof(float) : 0;
     }
     static __host__ __device__ size_t total(int W, int tm) {
         return ((ptr_bytes(W) + 15) & ~size_t(15)) + ((rows_bytes(tm) + 15) & ~size_t(15)) +
@@ -267,164 +268,158 @@ __device__ __forceinline__ void pass_a_rows(const Params& p, const LayerDesc& d,
     }
 }
 
-// Rank-lane variant of the first pass (R = 16 or 32): lane k of a warp (of
-// a half-warp when R = 16) owns rank index k.  The tile's columns (up to
-// 32 * VEC) are walked in sub-chunks of 32: for every worker the CTA stages
-// the sub-chunk's M = G + E rows in shared memory (and stores M over E);
-// each lane then walks its rows, reading M as broadcasts and its slice of Q
-// from registers.  Products are summed in float32 over runs of 8 columns
-// and flushed to a float64 per-row accumulator; the row's partial over the
-// chunk needs no lane reduction.
+// Rank-lane variant of the first pass (R = 32): lane k owns rank index k.
+// Warp w owns rows w, w + 8, ... of the tile and stages them itself: for
+// every (sub-chunk of 32 columns, worker) it forms M = G + E for its rows
+// (a lane per column; M is stored over E), parks them in its own slice of
+// shared memory, prefetches the next (sub-chunk, worker) into registers and
+// then walks the parked rows, reading M as broadcasts against its slice of
+// Q held in registers.  No CTA-wide barrier in the loop.  Products are
+// summed in float32 over runs of 8 columns and flushed to a float64 per-row
+// accumulator; the row's partial over the chunk needs no lane reduction.
 template <int R, typename GT, bool LAZY, bool SF, bool READM>
 __device__ __forceinline__ void pass_a_wide(const Params& p, const LayerDesc& d, const TileCoord& tc,
                                             const GT* const* gp, float* const* ep, const float* ph_prev,
-                                            float* m_s, float* rec_s, float* qp_s) {
-    constexpr int HW = 32 / R;                       // rows side by side per warp
-    constexpr int RPL = kWideRows / (kWarps * HW);   // rows per lane, at most
-    constexpr int SPT = kWideRows / kWarps;          // staged rows per thread, at most
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int k = lane % R;
-    const int h = lane / R;
+                                            float* m_s) {
+    static_assert(R == 32, "rank-lane kernels map one lane per rank index");
+    constexpr int RPL = kWideRows / kWarps;   // rows per warp, at most
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int k = lane;
     const int r = p.r;
     const int W = p.workers;
     const int64_t n = d.n, m = d.m;
     const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
     const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), m - i0));
-    const int64_t jc = static_cast<int64_t>(tc.c) * d.slots * d.vec;   // chunk's first column
+    const int64_t jc = static_cast<int64_t>(tc.c) * d.slots * d.vec;
     const int width = static_cast<int>(min(static_cast<int64_t>(d.slots) * d.vec, n - jc));
+    const int nsc = (width + kWideCols - 1) / kWideCols;
+    const int total = nsc * W;
     const float* Q = p.t.q[tc.l];
     const float* Qb = p.ws.qbar + d.qrow_off;
+    float* ms_w = m_s + warp * RPL * kWideCols;
+
+    float gv[RPL], ev[RPL];
+    auto load = [&](int it) {
+        const int sc = it / W, w = it - sc * W;
+        const int64_t j0 = jc + sc * kWideCols;
+        const int ncols = min(kWideCols, width - sc * kWideCols);
+#pragma unroll
+        for (int t = 0; t < RPL; ++t) {
+            const int ii = warp + kWarps * t;
+            gv[t] = 0.f;
+            ev[t] = 0.f;
+            if (ii < rows && lane < ncols) {
+                const int64_t off = (i0 + ii) * n + j0 + lane;
+                ev[t] = ep[w][off];
+                if constexpr (!READM) {
+                    float g1[1];
+                    ld_grad<GT, 1>(gp[w] + off, g1);
+                    gv[t] = g1[0];
+                }
+            }
+        }
+    };
 
     double acc[RPL];
 #pragma unroll
     for (int t = 0; t < RPL; ++t) acc[t] = 0.0;
+    float qreg[kWideCols];
+    float rec[LAZY ? RPL : 1];
+    float msum[SF ? RPL : 1];
 
-    for (int sc = 0; sc * kWideCols < width; ++sc) {
+    auto walk_rows = [&]() {
+#pragma unroll
+        for (int t = 0; t < RPL; ++t) {
+            const int ii = warp + kWarps * t;
+            if (ii < rows) {
+                const float4* mrow = reinterpret_cast<const float4*>(ms_w + t * kWideCols);
+                float run = 0.f;
+#pragma unroll
+                for (int q4 = 0; q4 < kWideCols / 4; ++q4) {
+                    const float4 mv = mrow[q4];
+                    run = fmaf(mv.x, qreg[4 * q4 + 0], run);
+                    run = fmaf(mv.y, qreg[4 * q4 + 1], run);
+                    run = fmaf(mv.z, qreg[4 * q4 + 2], run);
+                    run = fmaf(mv.w, qreg[4 * q4 + 3], run);
+                    if (q4 & 1) {
+                        acc[t] += static_cast<double>(run);
+                        run = 0.f;
+                    }
+                }
+            }
+        }
+    };
+
+    load(0);
+    for (int it = 0; it < total; ++it) {
+        const int sc = it / W, w = it - sc * W;
         const int64_t j0 = jc + sc * kWideCols;
         const int ncols = min(kWideCols, width - sc * kWideCols);
-        float qreg[kWideCols];
+        if (w == 0) {
+            // this lane's slice of Q for the sub-chunk: Q[j0 + jj][k]
 #pragma unroll
-        for (int jj = 0; jj < kWideCols; ++jj) qreg[jj] = (jj < ncols && k < r) ? Q[(j0 + jj) * r + k] : 0.f;
-        if constexpr (LAZY) {
-            // reconstruction of the previous step for this sub-chunk
-            __syncthreads();
-            for (int idx = tid; idx < kWideCols * R; idx += kThreads) {
-                const int jj = idx / R;
-                qp_s[idx] = (jj < ncols && p.use_prev) ? Qb[(j0 + jj) * R + (idx % R)] : 0.f;
-            }
-            __syncthreads();
+            for (int jj = 0; jj < kWideCols; ++jj) qreg[jj] = (jj < ncols && k < r) ? Q[(j0 + jj) * r + k] : 0.f;
+            if constexpr (LAZY) {
+                // the previous step's reconstruction of (row, this lane's column)
+                float qp[R];
 #pragma unroll
-            for (int s2 = 0; s2 < SPT; ++s2) {
-                const int ii = warp + kWarps * s2;
-                if (ii < rows) {
-                    float ph[R];
+                for (int kk = 0; kk < R; ++kk)
+                    qp[kk] = (lane < ncols && p.use_prev) ? Qb[(j0 + lane) * R + kk] : 0.f;
 #pragma unroll
-                    for (int kk = 0; kk < R; ++kk) ph[kk] = ph_prev[ii * R + kk];
-                    rec_s[ii * kWideCols + lane] = recon_dot<R>(ph, qp_s + lane * R);
+                for (int t = 0; t < RPL; ++t) {
+                    // recon_dot's operation order, P_hat row read from shared memory
+                    const int ii = min(warp + kWarps * t, rows - 1);
+                    float s2 = 0.f;
+#pragma unroll
+                    for (int kk = 0; kk < R; ++kk) s2 = fmaf(ph_prev[ii * R + kk], qp[kk], s2);
+                    rec[t] = s2;
                 }
+            }
+            if constexpr (SF) {
+#pragma unroll
+                for (int t = 0; t < RPL; ++t) msum[t] = 0.f;
             }
         }
-        float msum[SPT];
+        // M for this worker's rows
 #pragma unroll
-        for (int s2 = 0; s2 < SPT; ++s2) msum[s2] = 0.f;
-
-        for (int w = 0; w < W; ++w) {
-            // stage worker w's sub-chunk rows: a warp per row, a lane per column
-            float gv[SPT], ev[SPT];
-#pragma unroll
-            for (int s2 = 0; s2 < SPT; ++s2) {
-                const int ii = warp + kWarps * s2;
-                gv[s2] = 0.f;
-                ev[s2] = 0.f;
-                if (ii < rows && lane < ncols) {
-                    const int64_t off = (i0 + ii) * n + j0 + lane;
-                    ev[s2] = ep[w][off];
-                    if constexpr (!READM) {
-                        float g1[1];
-                        ld_grad<GT, 1>(gp[w] + off, g1);
-                        gv[s2] = g1[0];
-                    }
+        for (int t = 0; t < RPL; ++t) {
+            const int ii = warp + kWarps * t;
+            float mval = ev[t];
+            if (ii < rows && lane < ncols) {
+                if constexpr (!READM) {
+                    float e2 = ev[t];
+                    if constexpr (LAZY) e2 = e2 - rec[t];
+                    mval = gv[t] + e2;
+                    ep[w][(i0 + ii) * n + j0 + lane] = mval;
                 }
+            } else {
+                mval = 0.f;
             }
-            if constexpr (!SF) __syncthreads();   // every lane is done with the previous tile
-#pragma unroll
-            for (int s2 = 0; s2 < SPT; ++s2) {
-                const int ii = warp + kWarps * s2;
-                if (ii < rows) {
-                    float mval = 0.f;
-                    if (lane < ncols) {
-                        mval = ev[s2];
-                        if constexpr (!READM) {
-                            float e2 = ev[s2];
-                            if constexpr (LAZY) e2 = e2 - rec_s[ii * kWideCols + lane];
-                            mval = gv[s2] + e2;
-                            ep[w][(i0 + ii) * n + j0 + lane] = mval;
-                        }
-                    }
-                    if constexpr (SF) {
-                        msum[s2] += mval;
-                    } else {
-                        m_s[ii * kWideCols + lane] = mval;
-                    }
-                }
-            }
-            if constexpr (SF) continue;
-            __syncthreads();
-#pragma unroll
-            for (int t = 0; t < RPL; ++t) {
-                const int ii = warp * HW + h + t * kWarps * HW;
-                if (ii < rows) {
-                    const float4* mrow = reinterpret_cast<const float4*>(m_s + ii * kWideCols);
-                    float run = 0.f;
-#pragma unroll
-                    for (int q4 = 0; q4 < kWideCols / 4; ++q4) {
-                        const float4 mv = mrow[q4];
-                        run = fmaf(mv.x, qreg[4 * q4 + 0], run);
-                        run = fmaf(mv.y, qreg[4 * q4 + 1], run);
-                        run = fmaf(mv.z, qreg[4 * q4 + 2], run);
-                        run = fmaf(mv.w, qreg[4 * q4 + 3], run);
-                        if (q4 & 1) {
-                            acc[t] += static_cast<double>(run);
-                            run = 0.f;
-                        }
-                    }
-                }
+            if constexpr (SF) {
+                msum[t] += mval;
+            } else {
+                ms_w[t * kWideCols + lane] = mval;
             }
         }
+        if (it + 1 < total) load(it + 1);   // in flight while the rows are walked
         if constexpr (SF) {
-            __syncthreads();
+            if (w == W - 1) {
 #pragma unroll
-            for (int s2 = 0; s2 < SPT; ++s2) {
-                const int ii = warp + kWarps * s2;
-                if (ii < rows) m_s[ii * kWideCols + lane] = msum[s2];
+                for (int t = 0; t < RPL; ++t) ms_w[t * kWideCols + lane] = msum[t];
+                __syncwarp();
+                walk_rows();
+                __syncwarp();
             }
-            __syncthreads();
-#pragma unroll
-            for (int t = 0; t < RPL; ++t) {
-                const int ii = warp * HW + h + t * kWarps * HW;
-                if (ii < rows) {
-                    const float4* mrow = reinterpret_cast<const float4*>(m_s + ii * kWideCols);
-                    float run = 0.f;
-#pragma unroll
-                    for (int q4 = 0; q4 < kWideCols / 4; ++q4) {
-                        const float4 mv = mrow[q4];
-                        run = fmaf(mv.x, qreg[4 * q4 + 0], run);
-                        run = fmaf(mv.y, qreg[4 * q4 + 1], run);
-                        run = fmaf(mv.z, qreg[4 * q4 + 2], run);
-                        run = fmaf(mv.w, qreg[4 * q4 + 3], run);
-                        if (q4 & 1) {
-                            acc[t] += static_cast<double>(run);
-                            run = 0.f;
-                        }
-                    }
-                }
-            }
+        } else {
+            __syncwarp();
+            walk_rows();
+            __syncwarp();
         }
     }
     double* ppart = p.ws.ppart + d.ppart_off;
 #pragma unroll
     for (int t = 0; t < RPL; ++t) {
-        const int ii = warp * HW + h + t * kWarps * HW;
+        const int ii = warp + kWarps * t;
         if (ii < rows) ppart[(static_cast<int64_t>(tc.c) * m + i0 + ii) * R + k] = acc[t];
     }
 }
@@ -573,8 +568,7 @@ __global__ void __launch_bounds__(kThreads, (R <= 4 ? 3 : 2)) k_pass_a(Params p)
     __syncthreads();
 
     if constexpr (IsWide<R>::value) {
-        pass_a_wide<R, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s, wide, wide + d.tm * kWideCols,
-                                            wide + 2 * d.tm * kWideCols);
+        pass_a_wide<R, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s, wide);
     } else {
         // VEC x R values of Q live in registers: VEC = 4 up to R = 8, 2 up to 16
         if (d.vec == 4) {
@@ -598,10 +592,8 @@ struct SmemB {
     static __host__ __device__ size_t t_bytes() { return R * R * sizeof(double); }
     static __host__ __device__ size_t red_bytes(int vec) {
         if (IsWide<R>::value) {
-            // rank-lane kernel: the M tile (tm x 128), reused for the row-group sums
-            const size_t tile = static_cast<size_t>(kWideRows) * 4 * kWideCols * sizeof(float);
-            const size_t red = static_cast<size_t>(2 * (32 / R)) * 4 * kWideCols * R * sizeof(float);
-            return tile > red ? tile : red;
+            // rank-lane kernel: parked rows (tm x 32) + warp partials (8 x 32 x R)
+            return static_cast<size_t>(kWideRows * kWideCols + kWarps * kWideCols * R) * sizeof(float);
         }
         return static_cast<size_t>(kWarps) * R * vec * 32 * sizeof(float);
     }
@@ -728,104 +720,105 @@ __device__ __forceinline__ void pass_b_rows(const Params& p, const LayerDesc& d,
     }
 }
 
-// Stage worker w's M tile (rows x chunk width, zero beyond) into m_s
-// (row stride 4 * kWideCols floats); float4 accesses when VEC = 4.
-__device__ __forceinline__ void stage_m_tile(const float* src, int64_t n, int64_t i0, int64_t jc, int rows,
-                                             int width, int vec, float* m_s) {
-    constexpr int STR = 4 * kWideCols;
-    if (vec == 4) {
-        for (int idx = threadIdx.x; idx < kWideRows * kWideCols; idx += kThreads) {
-            const int ii = idx / kWideCols, q = idx % kWideCols;
-            if (ii >= rows) break;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (4 * q < width) v = *reinterpret_cast<const float4*>(src + (i0 + ii) * n + jc + 4 * q);
-            *reinterpret_cast<float4*>(m_s + ii * STR + 4 * q) = v;
-        }
-    } else {
-        for (int idx = threadIdx.x; idx < kWideRows * STR; idx += kThreads) {
-            const int ii = idx / STR, jj = idx % STR;
-            if (ii >= rows) break;
-            m_s[ii * STR + jj] = (jj < width) ? src[(i0 + ii) * n + jc + jj] : 0.f;
-        }
-    }
-}
-
-// Rank-lane variant of the second pass (R = 16 or 32): lane k owns rank
-// index k, warp w owns 32 columns of the chunk (w % 4) and a row group
-// (w / 4, split again between half-warps when R = 16).  Per worker the CTA
-// stages the M tile in shared memory; a lane accumulates, in float32, the
-// products of its 32 columns with P_hat[i][k] over its rows and all
-// workers; the row groups are summed in float64 at the end.
+// Rank-lane variant of the second pass (R = 32): lane k owns rank index k
+// and warp w rows w, w + 8, ... of the tile.  For every sub-chunk of 32
+// columns and every worker a warp parks its M rows in its own slice of
+// shared memory (prefetching the next ones into registers) and accumulates,
+// in float32, M[i][c] * P_hat[i][k] for its 32 columns; at the end of a
+// sub-chunk the 8 warps' partials are summed in float64 in warp order.
 template <int R, bool SF>
 __device__ __forceinline__ void pass_b_wide(const Params& p, const LayerDesc& d, const TileCoord& tc,
-                                            float* const* ep, const float* ph_s, float* m_s) {
-    constexpr int HW = 32 / R;
-    constexpr int NG = 2 * HW;                 // row groups
-    constexpr int STR = 4 * kWideCols;
+                                            float* const* ep, const float* ph_s, float* sm) {
+    static_assert(R == 32, "rank-lane kernels map one lane per rank index");
+    constexpr int RPL = kWideRows / kWarps;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int k = lane % R;
-    const int h = lane / R;
-    const int cg = warp & 3;
-    const int grp = (warp >> 2) * HW + h;
+    const int k = lane;
     const int W = p.workers;
     const int64_t n = d.n, m = d.m;
     const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
     const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), m - i0));
     const int64_t jc = static_cast<int64_t>(tc.c) * d.slots * d.vec;
     const int width = static_cast<int>(min(static_cast<int64_t>(d.slots) * d.vec, n - jc));
+    const int nsc = (width + kWideCols - 1) / kWideCols;
+    float* ms_w = sm + warp * RPL * kWideCols;               // parked rows
+    float* red_s = sm + kWideRows * kWideCols;               // [warp][column][k]
+    double* qpart = p.ws.qpart + d.qpart_off;
 
-    float acc[kWideCols];
+    float ph[RPL];
 #pragma unroll
-    for (int c = 0; c < kWideCols; ++c) acc[c] = 0.f;
-    auto accumulate = [&]() {
-        for (int ii = grp; ii < rows; ii += NG) {
-            const float ph = ph_s[ii * R + k];
-            const float4* mrow = reinterpret_cast<const float4*>(m_s + ii * STR + cg * kWideCols);
+    for (int t = 0; t < RPL; ++t) {
+        const int ii = warp + kWarps * t;
+        ph[t] = (ii < rows) ? ph_s[ii * R + k] : 0.f;
+    }
+    float mv_in[RPL];
+    auto load = [&](int it) {
+        const int sc = it / W, w = it - sc * W;
+        const int ncols = min(kWideCols, width - sc * kWideCols);
 #pragma unroll
-            for (int c4 = 0; c4 < kWideCols / 4; ++c4) {
-                const float4 mv = mrow[c4];
-                acc[4 * c4 + 0] = fmaf(mv.x, ph, acc[4 * c4 + 0]);
-                acc[4 * c4 + 1] = fmaf(mv.y, ph, acc[4 * c4 + 1]);
-                acc[4 * c4 + 2] = fmaf(mv.z, ph, acc[4 * c4 + 2]);
-                acc[4 * c4 + 3] = fmaf(mv.w, ph, acc[4 * c4 + 3]);
-            }
+        for (int t = 0; t < RPL; ++t) {
+            const int ii = warp + kWarps * t;
+            mv_in[t] = (ii < rows && lane < ncols) ? ep[w][(i0 + ii) * n + jc + sc * kWideCols + lane] : 0.f;
         }
     };
-    if constexpr (SF) {
-        // sum of the workers' tiles, then one product
-        for (int w = 0; w < W; ++w) {
-            if (w == 0) {
-                stage_m_tile(ep[0], n, i0, jc, rows, width, d.vec, m_s);
-            } else {
-                for (int idx = tid; idx < rows * STR; idx += kThreads) {
-                    const int ii = idx / STR, jj = idx % STR;
-                    if (jj < width) m_s[idx] += ep[w][(i0 + ii) * n + jc + jj];
+    const int total = nsc * W;
+    load(0);
+    float acc[kWideCols];
+    float msum[SF ? RPL : 1];
+    for (int it = 0; it < total; ++it) {
+        const int sc = it / W, w = it - sc * W;
+        if (w == 0) {
+#pragma unroll
+            for (int c = 0; c < kWideCols; ++c) acc[c] = 0.f;
+            if constexpr (SF) {
+#pragma unroll
+                for (int t = 0; t < RPL; ++t) msum[t] = 0.f;
+            }
+        }
+        bool walk = true;
+        if constexpr (SF) {
+#pragma unroll
+            for (int t = 0; t < RPL; ++t) msum[t] += mv_in[t];
+            walk = (w == W - 1);
+            if (walk) {
+#pragma unroll
+                for (int t = 0; t < RPL; ++t) ms_w[t * kWideCols + lane] = msum[t];
+            }
+        } else {
+#pragma unroll
+            for (int t = 0; t < RPL; ++t) ms_w[t * kWideCols + lane] = mv_in[t];
+        }
+        if (it + 1 < total) load(it + 1);
+        if (walk) {
+            __syncwarp();
+#pragma unroll
+            for (int t = 0; t < RPL; ++t) {
+                const float4* mrow = reinterpret_cast<const float4*>(ms_w + t * kWideCols);
+#pragma unroll
+                for (int c4 = 0; c4 < kWideCols / 4; ++c4) {
+                    const float4 mv = mrow[c4];
+                    acc[4 * c4 + 0] = fmaf(mv.x, ph[t], acc[4 * c4 + 0]);
+                    acc[4 * c4 + 1] = fmaf(mv.y, ph[t], acc[4 * c4 + 1]);
+                    acc[4 * c4 + 2] = fmaf(mv.z, ph[t], acc[4 * c4 + 2]);
+                    acc[4 * c4 + 3] = fmaf(mv.w, ph[t], acc[4 * c4 + 3]);
                 }
+            }
+            __syncwarp();
+        }
+        if (w == W - 1) {
+            // sub-chunk done: sum the warps' partials in warp order
+#pragma unroll
+            for (int c = 0; c < kWideCols; ++c) red_s[(warp * kWideCols + c) * R + k] = acc[c];
+            __syncthreads();
+            const int ncols = min(kWideCols, width - sc * kWideCols);
+            for (int idx = tid; idx < ncols * R; idx += kThreads) {
+                const int c = idx / R, kk = idx % R;
+                double s2 = 0.0;
+#pragma unroll
+                for (int wp = 0; wp < kWarps; ++wp) s2 += static_cast<double>(red_s[(wp * kWideCols + c) * R + kk]);
+                qpart[(static_cast<int64_t>(tc.rb) * n + jc + sc * kWideCols + c) * R + kk] = s2;
             }
             __syncthreads();
         }
-        accumulate();
-    } else {
-        for (int w = 0; w < W; ++w) {
-            if (w) __syncthreads();
-            stage_m_tile(ep[w], n, i0, jc, rows, width, d.vec, m_s);
-            __syncthreads();
-            accumulate();
-        }
-    }
-    __syncthreads();
-    // row-group partials [grp][column][k], then fixed-order float64 sums
-    float* red_s = m_s;
-#pragma unroll
-    for (int c = 0; c < kWideCols; ++c) red_s[(grp * STR + cg * kWideCols + c) * R + k] = acc[c];
-    __syncthreads();
-    double* qpart = p.ws.qpart + d.qpart_off;
-    for (int idx = tid; idx < width * R; idx += kThreads) {
-        const int col = idx / R, kk = idx % R;
-        double s2 = 0.0;
-#pragma unroll
-        for (int g = 0; g < NG; ++g) s2 += static_cast<double>(red_s[(g * STR + col) * R + kk]);
-        qpart[(static_cast<int64_t>(tc.rb) * n + jc + col) * R + kk] = s2;
     }
 }
 
