@@ -275,7 +275,7 @@ __device__ __forceinline__ void pass_a_rows(const Params& p, const LayerDesc& d,
 // shared memory, prefetches the next (sub-chunk, worker) into registers and
 // then walks the parked rows, reading M as broadcasts against its slice of
 // Q held in registers.  No CTA-wide barrier in the loop.  Products are
-// summed in float32 over runs of 8 columns and flushed to a float64 per-row
+// summed in float32 over runs of 8 terms and flushed to a float64 per-row
 // accumulator; the row's partial over the chunk needs no lane reduction.
 template <int R, typename GT, bool LAZY, bool SF, bool READM>
 __device__ __forceinline__ void pass_a_wide(const Params& p, const LayerDesc& d, const TileCoord& tc,
@@ -310,7 +310,7 @@ __device__ __forceinline__ void pass_a_wide(const Params& p, const LayerDesc& d,
             ev[t] = 0.f;
             if (ii < rows && lane < ncols) {
                 const int64_t off = (i0 + ii) * n + j0 + lane;
-                ev[t] = ep[w][off];
+                ev[t] = __ldcs(ep[w] + off);
                 if constexpr (!READM) {
                     float g1[1];
                     ld_grad<GT, 1>(gp[w] + off, g1);
@@ -327,23 +327,23 @@ __device__ __forceinline__ void pass_a_wide(const Params& p, const LayerDesc& d,
     float rec[LAZY ? RPL : 1];
     float msum[SF ? RPL : 1];
 
+    // two float32 runs (even and odd columns) in one packed fp32x2 FMA, each
+    // 8 terms long (16 columns), then both added to the float64 accumulator
     auto walk_rows = [&]() {
 #pragma unroll
         for (int t = 0; t < RPL; ++t) {
             const int ii = warp + kWarps * t;
             if (ii < rows) {
                 const float4* mrow = reinterpret_cast<const float4*>(ms_w + t * kWideCols);
-                float run = 0.f;
+                float2 run = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int q4 = 0; q4 < kWideCols / 4; ++q4) {
                     const float4 mv = mrow[q4];
-                    run = fmaf(mv.x, qreg[4 * q4 + 0], run);
-                    run = fmaf(mv.y, qreg[4 * q4 + 1], run);
-                    run = fmaf(mv.z, qreg[4 * q4 + 2], run);
-                    run = fmaf(mv.w, qreg[4 * q4 + 3], run);
-                    if (q4 & 1) {
-                        acc[t] += static_cast<double>(run);
-                        run = 0.f;
+                    run = __ffma2_rn(make_float2(mv.x, mv.y), make_float2(qreg[4 * q4 + 0], qreg[4 * q4 + 1]), run);
+                    run = __ffma2_rn(make_float2(mv.z, mv.w), make_float2(qreg[4 * q4 + 2], qreg[4 * q4 + 3]), run);
+                    if ((q4 & 3) == 3) {
+                        acc[t] += static_cast<double>(run.x) + static_cast<double>(run.y);
+                        run = make_float2(0.f, 0.f);
                     }
                 }
             }
@@ -540,7 +540,7 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
 // READM: a later power iteration of the same step; M is already in the
 // error buffers, so only M is read (no gradient, no store).
 template <int R, typename GT, bool LAZY, bool SF, bool READM>
-__global__ void __launch_bounds__(kThreads, (R <= 4 ? 3 : 2)) k_pass_a(Params p) {
+__global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_a(Params p) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int l = p.t.tile_layer[blockIdx.x];
     const LayerDesc d = p.t.layers[l];
@@ -570,9 +570,9 @@ __global__ void __launch_bounds__(kThreads, (R <= 4 ? 3 : 2)) k_pass_a(Params p)
     if constexpr (IsWide<R>::value) {
         pass_a_wide<R, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s, wide);
     } else {
-        // VEC x R values of Q live in registers: VEC = 4 up to R = 8, 2 up to 16
+        // VEC x R values of Q live in registers: VEC = 4 up to R = 4, 2 up to 16
         if (d.vec == 4) {
-            if constexpr (R <= 8) pass_a_rows<R, 4, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
+            if constexpr (R <= 4) pass_a_rows<R, 4, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
         } else if (d.vec == 2) {
             if constexpr (R <= 16) pass_a_rows<R, 2, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s);
         } else {
@@ -757,18 +757,18 @@ __device__ __forceinline__ void pass_b_wide(const Params& p, const LayerDesc& d,
 #pragma unroll
         for (int t = 0; t < RPL; ++t) {
             const int ii = warp + kWarps * t;
-            mv_in[t] = (ii < rows && lane < ncols) ? ep[w][(i0 + ii) * n + jc + sc * kWideCols + lane] : 0.f;
+            mv_in[t] = (ii < rows && lane < ncols) ? __ldcs(ep[w] + (i0 + ii) * n + jc + sc * kWideCols + lane) : 0.f;
         }
     };
     const int total = nsc * W;
     load(0);
-    float acc[kWideCols];
+    float2 acc[kWideCols / 2];   // columns (2c, 2c + 1)
     float msum[SF ? RPL : 1];
     for (int it = 0; it < total; ++it) {
         const int sc = it / W, w = it - sc * W;
         if (w == 0) {
 #pragma unroll
-            for (int c = 0; c < kWideCols; ++c) acc[c] = 0.f;
+            for (int c = 0; c < kWideCols / 2; ++c) acc[c] = make_float2(0.f, 0.f);
             if constexpr (SF) {
 #pragma unroll
                 for (int t = 0; t < RPL; ++t) msum[t] = 0.f;
@@ -793,13 +793,12 @@ __device__ __forceinline__ void pass_b_wide(const Params& p, const LayerDesc& d,
 #pragma unroll
             for (int t = 0; t < RPL; ++t) {
                 const float4* mrow = reinterpret_cast<const float4*>(ms_w + t * kWideCols);
+                const float2 pp = make_float2(ph[t], ph[t]);
 #pragma unroll
                 for (int c4 = 0; c4 < kWideCols / 4; ++c4) {
                     const float4 mv = mrow[c4];
-                    acc[4 * c4 + 0] = fmaf(mv.x, ph[t], acc[4 * c4 + 0]);
-                    acc[4 * c4 + 1] = fmaf(mv.y, ph[t], acc[4 * c4 + 1]);
-                    acc[4 * c4 + 2] = fmaf(mv.z, ph[t], acc[4 * c4 + 2]);
-                    acc[4 * c4 + 3] = fmaf(mv.w, ph[t], acc[4 * c4 + 3]);
+                    acc[2 * c4 + 0] = __ffma2_rn(make_float2(mv.x, mv.y), pp, acc[2 * c4 + 0]);
+                    acc[2 * c4 + 1] = __ffma2_rn(make_float2(mv.z, mv.w), pp, acc[2 * c4 + 1]);
                 }
             }
             __syncwarp();
@@ -807,7 +806,10 @@ __device__ __forceinline__ void pass_b_wide(const Params& p, const LayerDesc& d,
         if (w == W - 1) {
             // sub-chunk done: sum the warps' partials in warp order
 #pragma unroll
-            for (int c = 0; c < kWideCols; ++c) red_s[(warp * kWideCols + c) * R + k] = acc[c];
+            for (int c = 0; c < kWideCols / 2; ++c) {
+                red_s[(warp * kWideCols + 2 * c) * R + k] = acc[c].x;
+                red_s[(warp * kWideCols + 2 * c + 1) * R + k] = acc[c].y;
+            }
             __syncthreads();
             const int ncols = min(kWideCols, width - sc * kWideCols);
             for (int idx = tid; idx < ncols * R; idx += kThreads) {
@@ -888,7 +890,7 @@ __device__ void pass_b_epilogue(const Params& p, const LayerDesc& d, const TileC
 }
 
 template <int R, bool SF>
-__global__ void __launch_bounds__(kThreads, (R <= 4 ? 3 : 2)) k_pass_b(Params p) {
+__global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_b(Params p) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int l = p.t.tile_layer[blockIdx.x];
     const LayerDesc d = p.t.layers[l];
@@ -909,7 +911,7 @@ __global__ void __launch_bounds__(kThreads, (R <= 4 ? 3 : 2)) k_pass_b(Params p)
         pass_b_wide<R, SF>(p, d, tc, ep, ph_s, red_s);
     } else {
         if (d.vec == 4) {
-            if constexpr (R <= 8) pass_b_rows<R, 4, SF>(p, d, tc, ep, ph_s, red_s);
+            if constexpr (R <= 4) pass_b_rows<R, 4, SF>(p, d, tc, ep, ph_s, red_s);
         } else if (d.vec == 2) {
             if constexpr (R <= 16) pass_b_rows<R, 2, SF>(p, d, tc, ep, ph_s, red_s);
         } else {
@@ -1113,7 +1115,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_pass_c(Params p) {
         pass_c_wide<R>(p, d, tc, ep, ph_s, qt_s);
     } else {
         if (d.vec == 4) {
-            if constexpr (R <= 8) pass_c_rows<R, 4>(p, d, tc, ep, ph_s);
+            if constexpr (R <= 4) pass_c_rows<R, 4>(p, d, tc, ep, ph_s);
         } else if (d.vec == 2) {
             if constexpr (R <= 16) pass_c_rows<R, 2>(p, d, tc, ep, ph_s);
         } else {

@@ -35,7 +35,7 @@ int pad_rank(int r) {
 
 // lanes load VEC adjacent columns (a chunk is up to 32 * VEC columns); the
 // lane-per-column kernels keep VEC x R values of Q per lane in registers
-int max_vec_for_rank(int R) { return R <= 8 ? 4 : (R <= 16 ? 2 : 4); }
+int max_vec_for_rank(int R) { return R <= 4 ? 4 : (R <= 16 ? 2 : 4); }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
