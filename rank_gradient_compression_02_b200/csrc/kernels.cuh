@@ -644,7 +644,7 @@ __device__ __forceinline__ void pass_b_rows(const Params& p, const LayerDesc& d,
     const int ns = min(d.slots, d.nvec - s0);
     const bool active = lane < ns;
     const int64_t j = static_cast<int64_t>(s0 + (active ? lane : 0)) * VEC;
-    constexpr int U = (VEC == 4) ? 4 : 8;
+    constexpr int U = 8;   // 8 workers' loads in flight per lane (pass B only reads)
 
     float qacc[VEC][R];
 #pragma unroll

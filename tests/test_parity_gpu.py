@@ -340,3 +340,41 @@ def test_bad_arguments_rejected():
     with pytest.raises(PsgdError):
         PowerSGD([(4, 3)], 4, 1)             # rank > min(m, n)
     run.lib.status()
+
+
+def test_empty_layer_list_is_a_noop():
+    from rank_gradient_compression_02_b200 import PowerSGD
+    lib = PowerSGD([], 2, 3)
+    assert lib.step_launches == 0
+    lib.step([[], [], []], [[], [], []], [], [], None)
+    lib.momentum_step([], [], 0.1, 0.9)
+    lib.vec_mean([[], [], []], [])
+    lib.status()
+
+
+def test_many_workers():
+    # 64 workers on small ragged layers (the worker-pointer tables and the
+    # unrolled worker loops' remainders)
+    wl = H.small_workload([(40, 130), (33, 37)], 4, 64)
+    _, _, hist = H.run_free(wl, steps=2)
+    for t, e in enumerate(hist):
+        H.assert_close(e, H.TOL["f32"], f"step {t}")
+
+
+def test_max_workers_single_row():
+    # the largest worker count the library accepts, on a one-row layer and an
+    # odd-width layer
+    wl = H.small_workload([(1, 64), (9, 7)], 1, 256)
+    _, _, hist = H.run_free(wl, steps=1)
+    H.assert_close(hist[0], H.TOL["f32"], "step 0")
+
+
+def test_zero_length_vectors():
+    from rank_gradient_compression_02_b200 import PowerSGD
+    lib = PowerSGD([(8, 8)], 1, 2)
+    a = torch.zeros(0, device="cuda")
+    b = torch.zeros(16, device="cuda")
+    out = [torch.zeros(0, device="cuda"), torch.empty(16, device="cuda")]
+    lib.vec_mean([[a, b], [a, b + 2.0]], out)
+    lib.status()
+    assert torch.allclose(out[1], torch.ones(16, device="cuda"))
