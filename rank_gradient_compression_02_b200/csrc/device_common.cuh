@@ -199,12 +199,38 @@ struct Log2 { static constexpr int value = 1 + Log2<N / 2>::value; };
 template <>
 struct Log2<1> { static constexpr int value = 0; };
 
+// acc[k] = fma(a, x[k], acc[k]) for k < R, two k per packed fp32x2 FMA
+// (each component rounds exactly like fmaf)
+template <int R>
+__device__ __forceinline__ void axpy(float* acc, float a, const float* x) {
+    if constexpr (R >= 2) {
+        const float2 aa = make_float2(a, a);
+#pragma unroll
+        for (int k = 0; k < R; k += 2) {
+            const float2 r = __ffma2_rn(aa, make_float2(x[k], x[k + 1]), make_float2(acc[k], acc[k + 1]));
+            acc[k] = r.x;
+            acc[k + 1] = r.y;
+        }
+    } else {
+        acc[0] = fmaf(a, x[0], acc[0]);
+    }
+}
+
 // reconstruction of one element: sum_k ph[k] * qb[k], fixed order
 template <int R>
 __device__ __forceinline__ float recon_dot(const float (&ph)[R], const float* qb) {
     float s = 0.f;
 #pragma unroll
     for (int k = 0; k < R; ++k) s = fmaf(ph[k], qb[k], s);
+    return s;
+}
+
+// recon_dot for two elements at once (same per-element operation order)
+template <int R>
+__device__ __forceinline__ float2 recon_dot2(const float (&ph)[R], const float* qb0, const float* qb1) {
+    float2 s = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < R; ++k) s = __ffma2_rn(make_float2(ph[k], ph[k]), make_float2(qb0[k], qb1[k]), s);
     return s;
 }
 

@@ -209,7 +209,7 @@ __device__ __forceinline__ void pass_a_rows(const Params& p, const LayerDesc& d,
 #pragma unroll
                         for (int v = 0; v < VEC; ++v)
 #pragma unroll
-                            for (int k = 0; k < R; ++k) pw[k] = fmaf(e[u][v], qv[v][k], pw[k]);
+                            axpy<R>(pw, e[u][v], qv[v]);
                         if ((u + 1) % F == 0) {
 #pragma unroll
                             for (int k = 0; k < R; ++k) {
@@ -243,7 +243,7 @@ __device__ __forceinline__ void pass_a_rows(const Params& p, const LayerDesc& d,
 #pragma unroll
                     for (int v = 0; v < VEC; ++v)
 #pragma unroll
-                        for (int k = 0; k < R; ++k) pw[k] = fmaf(e[v], qv[v][k], pw[k]);
+                        axpy<R>(pw, e[v], qv[v]);
 #pragma unroll
                     for (int k = 0; k < R; ++k) acc[k] += static_cast<double>(pw[k]);
                 }
@@ -255,7 +255,7 @@ __device__ __forceinline__ void pass_a_rows(const Params& p, const LayerDesc& d,
 #pragma unroll
                 for (int v = 0; v < VEC; ++v)
 #pragma unroll
-                    for (int k = 0; k < R; ++k) pw[k] = fmaf(msum[v], qv[v][k], pw[k]);
+                    axpy<R>(pw, msum[v], qv[v]);
 #pragma unroll
                 for (int k = 0; k < R; ++k) acc[k] = static_cast<double>(pw[k]);
             }
@@ -675,7 +675,7 @@ __device__ __forceinline__ void pass_b_rows(const Params& p, const LayerDesc& d,
 #pragma unroll
                         for (int v = 0; v < VEC; ++v)
 #pragma unroll
-                            for (int k = 0; k < R; ++k) qacc[v][k] = fmaf(e[u][v], ph[k], qacc[v][k]);
+                            axpy<R>(qacc[v], e[u][v], ph);
                     }
                 }
             }
@@ -689,14 +689,14 @@ __device__ __forceinline__ void pass_b_rows(const Params& p, const LayerDesc& d,
 #pragma unroll
                     for (int v = 0; v < VEC; ++v)
 #pragma unroll
-                        for (int k = 0; k < R; ++k) qacc[v][k] = fmaf(e[v], ph[k], qacc[v][k]);
+                        axpy<R>(qacc[v], e[v], ph);
                 }
             }
             if constexpr (SF) {
 #pragma unroll
                 for (int v = 0; v < VEC; ++v)
 #pragma unroll
-                    for (int k = 0; k < R; ++k) qacc[v][k] = fmaf(msum[v], ph[k], qacc[v][k]);
+                    axpy<R>(qacc[v], msum[v], ph);
             }
         }
     }
@@ -1053,7 +1053,12 @@ __device__ __forceinline__ void pass_c_rows(const Params& p, const LayerDesc& d,
         for (int k = 0; k < R; ++k) ph[k] = ph_s[(i - i0) * R + k];
         float rec[VEC];
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) rec[v] = recon_dot<R>(ph, qb[v]);
+        for (int v = 0; v + 1 < VEC; v += 2) {
+            const float2 r2 = recon_dot2<R>(ph, qb[v], qb[v + 1]);
+            rec[v] = r2.x;
+            rec[v + 1] = r2.y;
+        }
+        if constexpr (VEC == 1) rec[0] = recon_dot<R>(ph, qb[0]);
         const int64_t base = i * n + j;
         if (recon != nullptr) st_f32<VEC>(recon + base, rec);
         if (xs != nullptr) {

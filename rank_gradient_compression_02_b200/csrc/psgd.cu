@@ -771,15 +771,24 @@ int psgd_vec_mean(psgd_ctx* ctx, const float* const* vecs, float* const* out, co
     if (count > 65535) return fail(ctx, PSGD_ERR_ARG, "too many vectors");
     if ((params == nullptr) != (mom == nullptr)) return fail(ctx, PSGD_ERR_ARG, "params and mom go together");
     const size_t WK = static_cast<size_t>(ctx->W) * count;
-    int rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(vecs), WK, false, "vecs");
-    if (!rc) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(out), count, false, "out");
-    if (!rc && params) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(params), count, false, "params");
-    if (!rc && mom) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(mom), count, false, "mom");
-    if (rc) return rc;
+    if (!vecs || !out) return fail(ctx, PSGD_ERR_ARG, "null pointer array");
     int64_t maxlen = 0;
     for (int k = 0; k < count; ++k) {
         if (len[k] < 0) return fail(ctx, PSGD_ERR_ARG, "len[%d] < 0", k);
         maxlen = std::max(maxlen, len[k]);
+        // an empty vector's pointers are never dereferenced (and may be null)
+        if (len[k] == 0) continue;
+        const void* ps[3] = {out[k], params ? params[k] : nullptr, mom ? mom[k] : nullptr};
+        for (int j = 0; j < 3; ++j) {
+            if (j > 0 && !params) break;
+            if (!ps[j]) return fail(ctx, PSGD_ERR_ARG, "null pointer for vector %d", k);
+            if (!aligned16(ps[j])) return fail(ctx, PSGD_ERR_ALIGN, "vector %d: pointer not 16-byte aligned", k);
+        }
+        for (int w = 0; w < ctx->W; ++w) {
+            const void* v = vecs[static_cast<size_t>(w) * count + k];
+            if (!v) return fail(ctx, PSGD_ERR_ARG, "vecs[%d][%d] is null", w, k);
+            if (!aligned16(v)) return fail(ctx, PSGD_ERR_ALIGN, "vecs[%d][%d] is not 16-byte aligned", w, k);
+        }
     }
     if (maxlen == 0) return PSGD_OK;
     DeviceGuard g(ctx->device);
