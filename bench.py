@@ -191,8 +191,60 @@ def run_step(lib, B, wl):
         lib.momentum_step(B.params, B.mom, lr, beta)
 
 
-def launches_per_step(lib, B):
-    n = lib.step_launches
+class DistBuffers:
+    """Send/receive buffers of the distributed step: the float64 P and Q
+    partials (all-reduced in place) and a flat copy of every local worker's
+    1-D gradients (all-reduced, then averaged over the global workers)."""
+
+    def __init__(self, lib, B, wl, device):
+        pe, qe = lib.dist_sizes()
+        self.p = torch.empty(pe, dtype=torch.float64, device=device)
+        self.q = torch.empty(qe, dtype=torch.float64, device=device)
+        self.vflat = self.vsum = self.vviews = None
+        if B.vecs is not None:
+            # every vector in a 16-byte aligned slot (the library's rule)
+            W = len(B.vecs)
+            self.slots = []
+            off = 0
+            for w in range(W):
+                for k in wl.vectors:
+                    self.slots.append((off, k))
+                    off += (k + 3) // 4 * 4
+            self.vflat = torch.zeros(max(off, 4), dtype=B.vecs[0][0].dtype, device=device)
+            self.pack(B.vecs)
+            self.vsum = torch.empty_like(self.vflat)
+            it = iter(self.slots)
+            self.vviews = [[self.vsum[o:o + k] for (o, k) in [next(it) for _ in wl.vectors]] for _ in range(W)]
+
+    def pack(self, vecs):
+        it = iter(self.slots)
+        for row in vecs:
+            for t in row:
+                o, k = next(it)
+                self.vflat[o:o + k].copy_(t)
+
+
+def dist_step(lib, B, wl, db, all_reduce):
+    """One data-parallel step across ranks: the library's three distributed
+    calls with the two all-reduces (SUM) of the P and Q partials between
+    them, then the 1-D means over all workers and the momentum update."""
+    lib.dist_p(B.G, B.E, B.Q, db.p, B.P, None)
+    all_reduce(db.p)
+    lib.dist_q(db.p, db.q)
+    all_reduce(db.q)
+    lib.dist_finish(db.q)
+    if db.vflat is not None:
+        db.vsum.copy_(db.vflat)
+        all_reduce(db.vsum)
+        beta, lr = wl.momentum if wl.momentum else (0.0, 0.0)
+        lib.vec_mean(db.vviews, B.vout, B.vx, B.vmom, lr=lr, beta=beta)
+    if B.params is not None:
+        beta, lr = wl.momentum
+        lib.momentum_step(B.params, B.mom, lr, beta)
+
+
+def launches_per_step(lib, B, dist: bool = False):
+    n = lib.step_launches + (2 if dist else 0)   # distributed: + orthogonalisation + Q_bar kernels
     if B.vecs is not None:
         n += 1
     if B.params is not None:
@@ -256,6 +308,8 @@ def main():
     ap.add_argument("--workers", type=int, default=None, help="override the worker count (small captures)")
     ap.add_argument("--iters", type=int, default=1, help="power iterations per step")
     ap.add_argument("--no-variants", action="store_true", help="skip timing the lazy-error variant")
+    ap.add_argument("--dist", action="store_true",
+                    help="use the distributed step with NCCL all-reduces even on one GPU")
     args = ap.parse_args()
 
     from dataclasses import replace
@@ -276,7 +330,8 @@ def main():
     config = {"workload": wl.name, "layers": len(wl.layers), "elements_per_worker": wl.elements_per_worker,
               "workers": wl.workers, "rank": r, "grad_dtype": wl.grad_dtype, "mode": mode,
               "l2": "inputs larger than L2 (no flush needed)" if wl.elements * 4 > 4 * 126e6 else "inputs fit L2",
-              "parallelism": f"replicas{world}"}
+              "parallelism": (f"dp{world} (P and Q all-reduced over NCCL; {wl.workers} simulated workers per GPU)"
+                              if world > 1 else "1 GPU")}
 
     if args.impl == "reference":
         if rank_id != 0:
@@ -285,8 +340,13 @@ def main():
         return
 
     import torch.distributed as dist
-    if world > 1:
+    if world > 1 or args.dist:
         torch.cuda.set_device(local)
+        if world == 1:
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", "29533")
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     device = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(device)
@@ -299,6 +359,20 @@ def main():
     B = Buffers(wl, r, device)
     lib = PowerSGD(wl.layers, r, wl.workers, grad_dtype=wl.grad_dtype, lazy_errors=args.lazy,
                    sum_first=args.sum_first, power_iters=args.iters)
+    dist_mode = world > 1 or args.dist
+    if dist_mode:
+        # every rank holds W local workers; P and Q are all-reduced over NCCL
+        lib.set_global_workers(wl.workers * world)
+        DB = DistBuffers(lib, B, wl, device)
+
+        def _all_reduce(t):
+            dist.all_reduce(t, op=dist.ReduceOp.SUM)
+
+        def step_fn():
+            dist_step(lib, B, wl, DB, _all_reduce)
+    else:
+        def step_fn():
+            run_step(lib, B, wl)
     torch.cuda.synchronize()
 
     def barrier():
@@ -306,7 +380,7 @@ def main():
             dist.barrier()
 
     for _ in range(args.warmup):
-        run_step(lib, B, wl)
+        step_fn()
     lib.status()
     barrier()
     torch.cuda.synchronize()
@@ -318,7 +392,7 @@ def main():
     ev1 = torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     for _ in range(args.steps):
-        run_step(lib, B, wl)
+        step_fn()
     ev1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -352,7 +426,7 @@ def main():
     # the lazy-error representation of the same step (E' rebuilt inside the
     # next step's first pass; bit-identical results), timed the same way
     variants = {}
-    if not args.lazy and not args.no_variants:
+    if not args.lazy and not args.no_variants and not dist_mode:
         lazy_lib = PowerSGD(wl.layers, r, wl.workers, grad_dtype=wl.grad_dtype, lazy_errors=True,
                             sum_first=args.sum_first, power_iters=args.iters)
         for _ in range(args.warmup):
@@ -377,7 +451,7 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(lib, B, wl, r, args, world, device)
+        e2e = run_e2e(lib, B, wl, r, args, world, device, DB if dist_mode else None)
 
     cpu = None
     if rank_id == 0 and world == 1 and not args.no_cpu_baseline:
@@ -389,19 +463,21 @@ def main():
            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f32" if wl.grad_dtype == "f32" else "bf16-in/f32",
            "data": "synthetic (seeded low-rank + noise gradients, resident in HBM)",
-           "config": config, "gpu_launches": args.steps * launches_per_step(lib, B),
+           "config": config, "gpu_launches": args.steps * launches_per_step(lib, B, dist_mode),
            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "variants": variants,
            "hbm_gbs_step": round(step_min_bytes / (ms_per_step * 1e-3) / 1e9, 1)}
     if rank_id == 0:
         print(json.dumps(out), flush=True)
     lib.close()
-    if world > 1:
+    if world > 1 or args.dist:
         dist.destroy_process_group()
 
 
-def run_e2e(lib, B, wl, r, args, world, device):
-    """The same metric through psgd_step_host: pinned host gradients copied
-    in every step, P_hat and Q_bar (and the 1-D means) read back."""
+def run_e2e(lib, B, wl, r, args, world, device, DB=None):
+    """The same metric through the public API with host buffers: pinned
+    host gradients copied in every step (psgd_step_host on one GPU; copies
+    into the device buffers before the distributed step on several), P_hat
+    and Q_bar (and the 1-D means) read back."""
     gsz = 2 if wl.grad_dtype == "bf16" else 4
     host_bytes = wl.elements * gsz
     if host_bytes > 16e9:
@@ -420,7 +496,26 @@ def run_e2e(lib, B, wl, r, args, world, device):
         vout_h = [torch.empty(k).pin_memory() for k in wl.vectors]
     stream = torch.cuda.current_stream()
 
+    def one_dist():
+        import torch.distributed as dist
+        for w in range(W):
+            B.G_flat[w].copy_(Gh[w], non_blocking=True)
+        if vh is not None:
+            for w in range(W):
+                for k in range(len(wl.vectors)):
+                    B.vecs[w][k].copy_(vh[w][k], non_blocking=True)
+            DB.pack(B.vecs)
+        dist_step(lib, B, wl, DB, lambda t: dist.all_reduce(t, op=dist.ReduceOp.SUM))
+        for l in range(L):
+            Ph[l].copy_(B.P[l], non_blocking=True)
+            Qh[l].copy_(B.Q[l], non_blocking=True)
+        if vh is not None:
+            for k in range(len(wl.vectors)):
+                vout_h[k].copy_(B.vout[k], non_blocking=True)
+
     def one():
+        if DB is not None:
+            return one_dist()
         lib.step_host(Gh_views, B.E, B.Q, Ph, Qh)
         if vh is not None:
             for w in range(W):

@@ -157,7 +157,10 @@ PSGD_API int psgd_momentum_step(psgd_ctx *ctx, float *const *params, float *cons
 
 /* Small tensors travel uncompressed (note-152, "Method"): out[k] = mean over
  * the ctx's W workers of vecs[w*count + k] (len[k] float32 elements each,
- * summed in worker order).  If params and mom are non-NULL, also applies
+ * summed in worker order).  After psgd_set_global_workers the sum is
+ * divided by the global worker count instead: pass vectors already summed
+ * over the ranks (an all-reduce of every local worker's vector) to get the
+ * global mean.  Vectors of length 0 may have null pointers.  If params and mom are non-NULL, also applies
  * the momentum update above with out[k] as the gradient. */
 PSGD_API int psgd_vec_mean(psgd_ctx *ctx, const float *const *vecs, float *const *out, const int64_t *len, int count,
                   float *const *params, float *const *mom, float lr, float beta, void *stream);
@@ -210,6 +213,37 @@ PSGD_API int psgd_step_launches(const psgd_ctx *ctx);
 PSGD_API int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int grad_dtype,
                               const void *const *grads, float *const *errors, float *q, float *p_hat,
                               float *recon, void *stream);
+
+/* Distributed step.  On a real data-parallel job every rank (GPU) holds
+ * its own workers (the context's `workers`, usually 1) and the two means of
+ * the step are all-reduces ("anthology-of-the-sota" note-152, "Method": P
+ * and then Q are all-reduced across workers).  The step is split at those
+ * two points so that the caller can run any all-reduce (e.g. NCCL, SUM over
+ * float64) between the calls:
+ *
+ *   psgd_dist_p:      M_w = G_w + E_w for the local workers; p_send =
+ *                     sum over local workers of M_w Q (per layer m x R rows,
+ *                     float64, R = rank rounded up to a power of two).
+ *   (caller)          p_sum = all-reduce(p_send, SUM)
+ *   psgd_dist_q:      P_bar = p_sum / W_global, Gram + Cholesky, P_hat;
+ *                     q_send = sum over local workers of M_w^T P_hat (n x R rows).
+ *   (caller)          q_sum = all-reduce(q_send, SUM)
+ *   psgd_dist_finish: Q_bar = q_sum / W_global into q; E'_w for the local
+ *                     workers (eager mode) and recon if it was given.
+ *
+ * psgd_dist_p takes the step's pointers (same meaning as psgd_step); the
+ * other two only the reduced buffers.  psgd_dist_sizes gives the float64
+ * element counts of p_send/p_sum and q_send/q_sum; psgd_set_global_workers
+ * sets W_global (default: the context's own worker count).  Calls out of
+ * order return PSGD_ERR_STATE; power iterations > 1 and SVD refresh are
+ * not available in the distributed step.  p_sum may alias p_send and q_sum
+ * q_send (in-place all-reduce). */
+PSGD_API int psgd_set_global_workers(psgd_ctx *ctx, int total_workers);
+PSGD_API int psgd_dist_sizes(const psgd_ctx *ctx, size_t *p_elems, size_t *q_elems);
+PSGD_API int psgd_dist_p(psgd_ctx *ctx, const void *const *grads, float *const *errors, float *const *q,
+                         float *const *p_hat, float *const *recon, double *p_send, void *stream);
+PSGD_API int psgd_dist_q(psgd_ctx *ctx, const double *p_sum, double *q_send, void *stream);
+PSGD_API int psgd_dist_finish(psgd_ctx *ctx, const double *q_sum, void *stream);
 
 /* Power (subspace) iterations per step, 1 <= iters <= 8 (default 1; the
  * "PowerSGD" glossary page: one or two suffice).  Every iteration repeats

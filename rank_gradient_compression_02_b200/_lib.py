@@ -57,6 +57,11 @@ _SIGS = {
     "psgd_step_static": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         _PP, _PP, _P, _P, _P, _P]),
     "psgd_set_power_iters": (ctypes.c_int, [_P, ctypes.c_int]),
+    "psgd_set_global_workers": (ctypes.c_int, [_P, ctypes.c_int]),
+    "psgd_dist_sizes": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]),
+    "psgd_dist_p": (ctypes.c_int, [_P, _PP, _PP, _PP, _PP, _PP, _P, _P]),
+    "psgd_dist_q": (ctypes.c_int, [_P, _P, _P, _P]),
+    "psgd_dist_finish": (ctypes.c_int, [_P, _P, _P]),
     "psgd_set_svd_refresh": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int]),
     "psgd_profile_enable": (ctypes.c_int, [_P, ctypes.c_int]),
     "psgd_profile_read": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
@@ -191,6 +196,27 @@ class PowerSGD:
                                            _ptrs(params) if params is not None else None,
                                            _ptrs(mom) if mom is not None else None, lr, beta,
                                            _stream_handle(stream)))
+
+    # -- distributed step (the caller all-reduces p_send and q_send, SUM)
+    def set_global_workers(self, total: int):
+        self._check(self.lib.psgd_set_global_workers(self._h, int(total)))
+
+    def dist_sizes(self):
+        pe, qe = ctypes.c_size_t(), ctypes.c_size_t()
+        self._check(self.lib.psgd_dist_sizes(self._h, ctypes.byref(pe), ctypes.byref(qe)))
+        return int(pe.value), int(qe.value)
+
+    def dist_p(self, grads, errors, q, p_send, p_hat=None, recon=None, stream=None):
+        self._check(self.lib.psgd_dist_p(self._h, self._wl(grads), self._wl(errors), _ptrs(q),
+                                         _ptrs(p_hat) if p_hat is not None else None,
+                                         _ptrs(recon) if recon is not None else None,
+                                         p_send.data_ptr(), _stream_handle(stream)))
+
+    def dist_q(self, p_sum, q_send, stream=None):
+        self._check(self.lib.psgd_dist_q(self._h, p_sum.data_ptr(), q_send.data_ptr(), _stream_handle(stream)))
+
+    def dist_finish(self, q_sum, stream=None):
+        self._check(self.lib.psgd_dist_finish(self._h, q_sum.data_ptr(), _stream_handle(stream)))
 
     def profile(self, enable: bool = True):
         self._check(self.lib.psgd_profile_enable(self._h, 1 if enable else 0))

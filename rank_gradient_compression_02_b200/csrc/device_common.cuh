@@ -97,6 +97,13 @@ struct Params {
     double drop_tol;
     int use_prev;   // lazy first pass: rebuild E' from the previous P_hat, Q_bar
     int do_recon, do_mom, do_resid;
+    // distributed step: the first two passes stop at this rank's partial
+    // sums (rows of P, rows of Q, not divided by the worker count), written
+    // to dist_out; the all-reduced sums come back through dist_in.
+    int dist;
+    double* dist_out;
+    const double* dist_in;
+    double inv_w_global;
 };
 
 enum : int { kStatusCounter = 1 };

@@ -458,11 +458,17 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
         const int k = idx % R;
         double s = 0.0;
         for (int c = 0; c < d.nchunk; ++c) s += __ldcg(&ppart[(static_cast<int64_t>(c) * m + i) * R + k]);
+        if (p.dist) {
+            // this rank's share of the all-reduce: the row's sum over its workers
+            p.dist_out[d.prow_off + i * R + k] = s;
+            continue;
+        }
         const double v = s * inv_w;
         pb_s[idx] = v;
         pbar[i * R + k] = v;
     }
     if (tid == 0) cnt[cl.a_rb + tc.rb] = 0u;
+    if (p.dist) return;
     __syncthreads();
 
     double* gram = p.ws.gram + d.gram_off;
@@ -882,6 +888,10 @@ __device__ void pass_b_epilogue(const Params& p, const LayerDesc& d, const TileC
         const int k = idx % R;
         double s = 0.0;
         for (int j = 0; j < d.nsup; ++j) s += __ldcg(&qsup[(static_cast<int64_t>(j) * n + col) * R + k]);
+        if (p.dist) {
+            p.dist_out[d.qrow_off + col * R + k] = s;   // this rank's share of the all-reduce
+            continue;
+        }
         const float v = static_cast<float>(s * inv_w);
         qbar[col * R + k] = v;
         if (k < r) qout[col * r + k] = v;
@@ -1126,6 +1136,68 @@ __global__ void __launch_bounds__(kThreads, 2) k_pass_c(Params p) {
         } else {
             pass_c_rows<R, 1>(p, d, tc, ep, ph_s);
         }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Distributed step, after the all-reduce of P: P_bar = (sum over all ranks'
+// workers) / W_global, its Gram matrix (float64, pairs over warps, rows over
+// lanes, fixed order) and the Cholesky factorisation into T.  One CTA per
+// layer.
+template <int R>
+__global__ void __launch_bounds__(kThreads) k_dist_orth(Params p) {
+    __shared__ double Gs[R * R];
+    __shared__ double Rs[R * R];
+    __shared__ double Ts[R * R];
+    __shared__ int drop[R];
+    const int l = blockIdx.x;
+    const LayerDesc d = p.t.layers[l];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int NG = R * (R + 1) / 2;
+    double* pbar = p.ws.pbar + d.prow_off;
+    const double* psum = p.dist_in + d.prow_off;
+    for (int64_t idx = tid; idx < d.m * R; idx += kThreads) pbar[idx] = psum[idx] * p.inv_w_global;
+    __syncthreads();
+    for (int pidx = warp; pidx < NG; pidx += kWarps) {
+        int a = 0, rem = pidx;
+        while (rem >= R - a) {
+            rem -= R - a;
+            ++a;
+        }
+        const int b = a + rem;
+        double s = 0.0;
+        for (int64_t i = lane; i < d.m; i += 32) s += pbar[i * R + a] * pbar[i * R + b];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) {
+            Gs[a * R + b] = s;
+            Gs[b * R + a] = s;
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        factor_gram_warp<R>(Gs, Rs, Ts, drop, p.r, p.drop_tol, lane);
+        double* T = p.ws.T + d.t_off;
+        for (int idx = lane; idx < R * R; idx += 32) T[idx] = Ts[idx];
+    }
+}
+
+// Distributed step, after the all-reduce of Q: Q_bar = sum / W_global into
+// the workspace (stride R) and the caller's Q (stride r).
+template <int R>
+__global__ void k_dist_qbar(Params p) {
+    const int l = blockIdx.y;
+    const LayerDesc d = p.t.layers[l];
+    float* qbar = p.ws.qbar + d.qrow_off;
+    float* qout = p.t.q[l];
+    const double* qsum = p.dist_in + d.qrow_off;
+    const int r = p.r;
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < d.n * R;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float v = static_cast<float>(qsum[idx] * p.inv_w_global);
+        qbar[idx] = v;
+        const int k = static_cast<int>(idx % R);
+        if (k < r) qout[(idx / R) * r + k] = v;
     }
 }
 

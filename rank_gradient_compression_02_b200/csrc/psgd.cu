@@ -188,6 +188,9 @@ struct psgd_ctx {
     size_t prof_used = 0;
 
     int iters = 1;          // power iterations per step
+    int w_global = 0;       // workers over all ranks (distributed step); 0 = W
+    int dist_phase = 0;     // distributed step: 0 idle, 1 after P, 2 after Q
+    bool tab_l_has_recon = false;
     int svd_every = 0;      // SVD refresh period in steps (0: off)
     int svd_iters = 0;      // subspace iterations on a refresh step
     uint64_t steps_done = 0;
@@ -251,6 +254,8 @@ struct Launch {
     static void* pass_b(bool sf) { return sf ? (void*)psgd::k_pass_b<R, true> : (void*)psgd::k_pass_b<R, false>; }
     static void* pass_c() { return (void*)psgd::k_pass_c<R>; }
     static void* rayleigh_ritz() { return (void*)psgd::k_rayleigh_ritz<R>; }
+    static void* dist_orth() { return (void*)psgd::k_dist_orth<R>; }
+    static void* dist_qbar() { return (void*)psgd::k_dist_qbar<R>; }
 };
 
 void* kernel_ptr(int which, int R, int dtype, bool lazy, bool sf) {
@@ -260,6 +265,8 @@ void* kernel_ptr(int which, int R, int dtype, bool lazy, bool sf) {
         if (which == 1) return Launch<RR>::pass_b(sf);       \
         if (which == 3) return Launch<RR>::pass_a_m(sf);     \
         if (which == 4) return Launch<RR>::rayleigh_ritz();  \
+        if (which == 5) return Launch<RR>::dist_orth();      \
+        if (which == 6) return Launch<RR>::dist_qbar();      \
         return Launch<RR>::pass_c();
     switch (R) {
         PSGD_CASE(1)
@@ -303,6 +310,7 @@ psgd::Params base_params(psgd_ctx* ctx) {
     p.r = ctx->r;
     p.inv_w = 1.0f / static_cast<float>(ctx->W);
     p.drop_tol = kDropTol;
+    p.inv_w_global = 1.0 / static_cast<double>(ctx->w_global > 0 ? ctx->w_global : ctx->W);
     return p;
 }
 
@@ -636,6 +644,7 @@ int psgd_step(psgd_ctx* ctx, const void* const* grads, float* const* errors, flo
               float* const* recon, void* stream) {
     if (!ctx) return PSGD_ERR_ARG;
     ctx->err.clear();
+    if (ctx->dist_phase != 0) return fail(ctx, PSGD_ERR_STATE, "a distributed step is in progress");
     if (ctx->L == 0) return PSGD_OK;
     const size_t WL = static_cast<size_t>(ctx->W) * ctx->L;
     int rc = check_ptr_array(ctx, grads, WL, false, "grads");
@@ -808,7 +817,8 @@ int psgd_vec_mean(psgd_ctx* ctx, const float* const* vecs, float* const* out, co
     const unsigned gx = static_cast<unsigned>(std::min<int64_t>(256, (maxlen + 255) / 256));
     psgd::k_vec_mean<<<dim3(gx, count), 256, 0, s>>>(
         reinterpret_cast<const float* const*>(t), reinterpret_cast<float* const*>(t + WK),
-        reinterpret_cast<const int64_t*>(t + WK + 3 * count), count, ctx->W, 1.0f / static_cast<float>(ctx->W),
+        reinterpret_cast<const int64_t*>(t + WK + 3 * count), count, ctx->W,
+        1.0f / static_cast<float>(ctx->w_global > 0 ? ctx->w_global : ctx->W),
         params ? reinterpret_cast<float* const*>(t + WK + count) : nullptr,
         mom ? reinterpret_cast<float* const*>(t + WK + 2 * count) : nullptr, lr, beta);
     e = cudaGetLastError();
@@ -969,6 +979,154 @@ int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int grad_dtype
         e = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(ntiles)), dim3(psgd::kThreads), args, smem[which], s);
         if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
     }
+    return PSGD_OK;
+}
+
+// ---- distributed step (the all-reduces between the calls are the caller's)
+
+int psgd_set_global_workers(psgd_ctx* ctx, int total) {
+    if (!ctx) return PSGD_ERR_ARG;
+    if (total < ctx->W) return fail(ctx, PSGD_ERR_ARG, "global workers %d < local workers %d", total, ctx->W);
+    ctx->w_global = total;
+    return PSGD_OK;
+}
+
+int psgd_dist_sizes(const psgd_ctx* ctx, size_t* p_elems, size_t* q_elems) {
+    if (!ctx || !p_elems || !q_elems) return PSGD_ERR_ARG;
+    size_t pe = 0, qe = 0;
+    for (auto& d : ctx->desc) {
+        pe += static_cast<size_t>(d.m) * ctx->R;
+        qe += static_cast<size_t>(d.n) * ctx->R;
+    }
+    *p_elems = pe;
+    *q_elems = qe;
+    return PSGD_OK;
+}
+
+static psgd::Params dist_params(psgd_ctx* ctx) {
+    psgd::Params p = base_params(ctx);
+    const size_t WL = static_cast<size_t>(ctx->W) * ctx->L;
+    void* const* wt = static_cast<void* const*>(ctx->tab_w.dev());
+    void* const* lt = static_cast<void* const*>(ctx->tab_l.dev());
+    p.t.grads = reinterpret_cast<const void* const*>(wt);
+    p.t.errors = reinterpret_cast<float* const*>(wt + WL);
+    p.t.q = reinterpret_cast<float* const*>(lt);
+    p.t.p_hat_out = reinterpret_cast<float* const*>(lt + ctx->L);
+    p.t.recon_out = reinterpret_cast<float* const*>(lt + 2 * ctx->L);
+    p.dist = 1;
+    return p;
+}
+
+int psgd_dist_p(psgd_ctx* ctx, const void* const* grads, float* const* errors, float* const* q, float* const* p_hat,
+                float* const* recon, double* p_send, void* stream) {
+    if (!ctx) return PSGD_ERR_ARG;
+    ctx->err.clear();
+    if (ctx->dist_phase != 0) return fail(ctx, PSGD_ERR_STATE, "psgd_dist_p called in the middle of a step");
+    if (ctx->iters != 1 || ctx->svd_every > 0)
+        return fail(ctx, PSGD_ERR_STATE, "the distributed step does one power iteration without SVD refresh");
+    if (ctx->L == 0) return PSGD_OK;
+    const size_t WL = static_cast<size_t>(ctx->W) * ctx->L;
+    int rc = check_ptr_array(ctx, grads, WL, false, "grads");
+    if (!rc) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(errors), WL, false, "errors");
+    if (!rc) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(q), ctx->L, false, "q");
+    if (!rc && p_hat) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(p_hat), ctx->L, true, "p_hat");
+    if (!rc && recon) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(recon), ctx->L, true, "recon");
+    if (!rc && (!p_send || !aligned16(p_send))) rc = fail(ctx, PSGD_ERR_ALIGN, "p_send null or not 16-byte aligned");
+    if (rc) return rc;
+    DeviceGuard g(ctx->device);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    std::vector<uint64_t> tw(2 * WL);
+    for (size_t i = 0; i < WL; ++i) {
+        tw[i] = reinterpret_cast<uint64_t>(grads[i]);
+        tw[WL + i] = reinterpret_cast<uint64_t>(errors[i]);
+    }
+    std::vector<uint64_t> tl(3 * ctx->L, 0);
+    for (int l = 0; l < ctx->L; ++l) {
+        tl[l] = reinterpret_cast<uint64_t>(q[l]);
+        tl[ctx->L + l] = p_hat ? reinterpret_cast<uint64_t>(p_hat[l]) : 0;
+        tl[2 * ctx->L + l] = recon ? reinterpret_cast<uint64_t>(recon[l]) : 0;
+    }
+    cudaError_t e = ctx->tab_w.update(tw, s);
+    if (e == cudaSuccess) e = ctx->tab_l.update(tl, s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "table upload");
+    const bool lazy = (ctx->flags & PSGD_FLAG_LAZY_ERRORS) != 0;
+    psgd::Params p = dist_params(ctx);
+    p.use_prev = (lazy && ctx->errors_hold_m) ? 1 : 0;
+    p.dist_out = p_send;
+    if (ctx->flags & PSGD_FLAG_NO_WARM_START) {
+        int64_t maxn = 0;
+        for (auto& d : ctx->desc) maxn = std::max(maxn, d.n);
+        const int64_t blocks4 = (maxn * ctx->r + 3) / 4;
+        const unsigned gx = static_cast<unsigned>(std::min<int64_t>(1024, (blocks4 + 255) / 256));
+        psgd::k_init_q<<<dim3(std::max(1u, gx), ctx->L), 256, 0, s>>>(p.t.q, ctx->desc_d, ctx->r, ctx->seed,
+                                                                      ctx->steps_done + 1);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "fresh Q launch");
+    }
+    rc = launch(ctx, 0, lazy, p, ctx->smem_a, s);
+    if (rc) return rc;
+    ctx->tab_l_has_recon = recon != nullptr;
+    ctx->dist_phase = 1;
+    ctx->last_stream = s;
+    return PSGD_OK;
+}
+
+int psgd_dist_q(psgd_ctx* ctx, const double* p_sum, double* q_send, void* stream) {
+    if (!ctx) return PSGD_ERR_ARG;
+    ctx->err.clear();
+    if (ctx->L == 0) return PSGD_OK;
+    if (ctx->dist_phase != 1) return fail(ctx, PSGD_ERR_STATE, "psgd_dist_q must follow psgd_dist_p");
+    if (!p_sum || !q_send || !aligned16(p_sum) || !aligned16(q_send))
+        return fail(ctx, PSGD_ERR_ALIGN, "p_sum / q_send null or not 16-byte aligned");
+    DeviceGuard g(ctx->device);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool lazy = (ctx->flags & PSGD_FLAG_LAZY_ERRORS) != 0;
+    psgd::Params p = dist_params(ctx);
+    p.dist_in = p_sum;
+    void* fn = kernel_ptr(5, ctx->R, ctx->dtype, false, false);
+    void* args[] = {&p};
+    cudaError_t e = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(ctx->L)), dim3(psgd::kThreads), args, 0, s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "distributed orthogonalisation launch");
+    p.dist_in = nullptr;
+    p.dist_out = q_send;
+    int rc = launch(ctx, 1, lazy, p, ctx->smem_b, s);
+    if (rc) return rc;
+    ctx->dist_phase = 2;
+    return PSGD_OK;
+}
+
+int psgd_dist_finish(psgd_ctx* ctx, const double* q_sum, void* stream) {
+    if (!ctx) return PSGD_ERR_ARG;
+    ctx->err.clear();
+    if (ctx->L == 0) return PSGD_OK;
+    if (ctx->dist_phase != 2) return fail(ctx, PSGD_ERR_STATE, "psgd_dist_finish must follow psgd_dist_q");
+    if (!q_sum || !aligned16(q_sum)) return fail(ctx, PSGD_ERR_ALIGN, "q_sum null or not 16-byte aligned");
+    DeviceGuard g(ctx->device);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool lazy = (ctx->flags & PSGD_FLAG_LAZY_ERRORS) != 0;
+    psgd::Params p = dist_params(ctx);
+    p.dist = 0;
+    p.dist_in = q_sum;
+    int64_t maxn = 0;
+    for (auto& d : ctx->desc) maxn = std::max(maxn, d.n);
+    const unsigned gx = static_cast<unsigned>(std::min<int64_t>(1024, (maxn * ctx->R + 255) / 256));
+    void* fn = kernel_ptr(6, ctx->R, ctx->dtype, false, false);
+    void* args[] = {&p};
+    cudaError_t e = cudaLaunchKernel(fn, dim3(std::max(1u, gx), static_cast<unsigned>(ctx->L)), dim3(256), args, 0, s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "distributed Q_bar launch");
+    const bool recon = ctx->tab_l_has_recon;
+    if (!lazy || recon) {
+        psgd::Params pc = p;
+        pc.dist_in = nullptr;
+        pc.do_resid = lazy ? 0 : 1;
+        pc.do_recon = recon ? 1 : 0;
+        int rc = launch(ctx, 2, lazy, pc, ctx->smem_c, s);
+        if (rc) return rc;
+    }
+    ctx->dist_phase = 0;
+    ctx->have_step = true;
+    ctx->errors_hold_m = lazy;
+    ctx->steps_done += 1;
     return PSGD_OK;
 }
 

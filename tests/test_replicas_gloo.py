@@ -1,8 +1,13 @@
-"""Host logic of the multi-GPU bench path (replicas, max-over-ranks timing)
-on CPU with gloo, world size 2."""
+"""Host logic of the multi-GPU bench path on CPU with gloo, world size 2:
+max-over-ranks timing, whole-job throughput, and the distributed step's
+orchestration (the two all-reduces of the P and Q partials, the global
+worker count, the 1-D means) driven through a float64 stand-in for the
+library built from the oracle's functions."""
 import os
 import socket
+import types
 
+import numpy as np
 import pytest
 import torch
 import torch.distributed as dist
@@ -17,10 +22,14 @@ def _free_port():
     return p
 
 
-def _worker(rank, world, port, q):
+def _init(rank, world, port):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
+
+
+def _worker_timing(rank, world, port, q):
+    _init(rank, world, port)
     import bench
     ms = 10.0 + 5.0 * rank        # rank 1 is the slow one
     got = bench.max_over_ranks(ms, world, torch.device("cpu"))
@@ -30,18 +39,22 @@ def _worker(rank, world, port, q):
     dist.destroy_process_group()
 
 
-def test_max_over_ranks_and_job_value():
+def _spawn(target, world, *args):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=target, args=(r, world, port, q) + args) for r in range(world)]
     for p in procs:
         p.start()
-    res = [q.get(timeout=120) for _ in procs]
+    res = [q.get(timeout=180) for _ in procs]
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, got, val in res:
+    return sorted(res, key=lambda x: x[0])
+
+
+def test_max_over_ranks_and_job_value():
+    for rank, got, val in _spawn(_worker_timing, 2):
         assert got == 15.0
         assert val == pytest.approx(1000 * 2 / 15e-3)
 
@@ -50,3 +63,133 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(3.0, 1, None) == 3.0
     assert bench.job_value(10, 1, 1.0) == pytest.approx(1e4)
+
+
+class FakeDistLib:
+    """float64 CPU stand-in with the library's distributed-call semantics
+    (oracle functions for the arithmetic)."""
+
+    def __init__(self, layers, rank, w_local):
+        import oracle.powersgd64 as ora
+        self.ora = ora
+        self.layers, self.r, self.W = layers, rank, w_local
+        self.Wg = w_local
+        self.Phat = [None] * len(layers)
+        self.Qbar = [None] * len(layers)
+
+    def set_global_workers(self, n):
+        self.Wg = n
+
+    def dist_sizes(self):
+        return sum(m for m, _ in self.layers) * self.r, sum(n for _, n in self.layers) * self.r
+
+    def dist_p(self, G, E, Q, p_send, P, recon):
+        self.E, self.Qv, self.P = E, Q, P
+        off = 0
+        for l, (m, n) in enumerate(self.layers):
+            acc = np.zeros((m, self.r))
+            for w in range(self.W):
+                E[w][l][...] = G[w][l] + E[w][l]          # M over E
+                acc += E[w][l].numpy() @ Q[l].numpy()
+            p_send[off:off + m * self.r] = torch.from_numpy(acc.ravel())
+            off += m * self.r
+
+    def dist_q(self, p_sum, q_send):
+        po = qo = 0
+        for l, (m, n) in enumerate(self.layers):
+            pbar = p_sum[po:po + m * self.r].numpy().reshape(m, self.r) / self.Wg
+            self.Phat[l] = self.ora.gram_schmidt(pbar)
+            self.P[l][...] = torch.from_numpy(self.Phat[l])
+            acc = sum(self.E[w][l].numpy().T @ self.Phat[l] for w in range(self.W))
+            q_send[qo:qo + n * self.r] = torch.from_numpy(acc.ravel())
+            po += m * self.r
+            qo += n * self.r
+
+    def dist_finish(self, q_sum):
+        qo = 0
+        for l, (m, n) in enumerate(self.layers):
+            self.Qbar[l] = q_sum[qo:qo + n * self.r].numpy().reshape(n, self.r) / self.Wg
+            self.Qv[l][...] = torch.from_numpy(self.Qbar[l])
+            for w in range(self.W):
+                self.E[w][l][...] = torch.from_numpy(self.E[w][l].numpy() - self.Phat[l] @ self.Qbar[l].T)
+            qo += n * self.r
+
+    def vec_mean(self, vecs, out, x, mom, lr=0.0, beta=0.0):
+        for k in range(len(out)):
+            g = sum(vecs[w][k] for w in range(self.W)) / self.Wg
+            out[k][...] = g
+            mom[k][...] = beta * mom[k] + g
+            x[k][...] = x[k] - lr * mom[k]
+
+    def momentum_step(self, params, mom, lr, beta):
+        for l in range(len(self.layers)):
+            ghat = torch.from_numpy(self.Phat[l] @ self.Qbar[l].T)
+            mom[l][...] = beta * mom[l] + ghat
+            params[l][...] = params[l] - lr * mom[l]
+
+
+LAYERS = [(12, 9), (7, 11)]
+R, WL = 2, 2
+
+
+def _grads(rank_id, w, l):
+    g = torch.Generator().manual_seed(1000 * rank_id + 10 * w + l)
+    m, n = LAYERS[l]
+    return torch.randn(m, n, generator=g, dtype=torch.float64)
+
+
+def _vecs(rank_id, w):
+    g = torch.Generator().manual_seed(777 + 10 * rank_id + w)
+    return [torch.randn(5, generator=g, dtype=torch.float64), torch.randn(3, generator=g, dtype=torch.float64)]
+
+
+def _worker_dist(rank, world, port, q):
+    _init(rank, world, port)
+    import bench
+    lib = FakeDistLib(LAYERS, R, WL)
+    lib.set_global_workers(WL * world)
+    B = types.SimpleNamespace()
+    B.G = [[_grads(rank, w, l) for l in range(len(LAYERS))] for w in range(WL)]
+    B.E = [[torch.zeros(m, n, dtype=torch.float64) for (m, n) in LAYERS] for _ in range(WL)]
+    g = torch.Generator().manual_seed(5)
+    B.Q = [torch.randn(n, R, generator=g, dtype=torch.float64) for (_, n) in LAYERS]
+    B.P = [torch.zeros(m, R, dtype=torch.float64) for (m, _) in LAYERS]
+    B.vecs = [_vecs(rank, w) for w in range(WL)]
+    B.vout = [torch.zeros(5, dtype=torch.float64), torch.zeros(3, dtype=torch.float64)]
+    B.vx = [torch.zeros(5, dtype=torch.float64), torch.zeros(3, dtype=torch.float64)]
+    B.vmom = [torch.zeros(5, dtype=torch.float64), torch.zeros(3, dtype=torch.float64)]
+    B.params = [torch.zeros(m, n, dtype=torch.float64) for (m, n) in LAYERS]
+    B.mom = [torch.zeros(m, n, dtype=torch.float64) for (m, n) in LAYERS]
+    wl = types.SimpleNamespace(vectors=(5, 3), momentum=(0.9, 0.1))
+    db = bench.DistBuffers(lib, B, wl, torch.device("cpu"))
+    db.p = db.p.double()
+    db.q = db.q.double()
+    bench.dist_step(lib, B, wl, db, lambda t: dist.all_reduce(t, op=dist.ReduceOp.SUM))
+    q.put((rank, [p.numpy().copy() for p in B.P], [x.numpy().copy() for x in B.Q],
+           [[e.numpy().copy() for e in Ew] for Ew in B.E], [v.numpy().copy() for v in B.vout],
+           [x.numpy().copy() for x in B.params]))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_distributed_step_orchestration_matches_oracle():
+    import oracle.powersgd64 as ora
+    world = 2
+    res = _spawn(_worker_dist, world)
+    g = torch.Generator().manual_seed(5)
+    Q0 = [torch.randn(n, R, generator=g, dtype=torch.float64).numpy() for (_, n) in LAYERS]
+    for l in range(len(LAYERS)):
+        G = [_grads(r, w, l).numpy() for r in range(world) for w in range(WL)]
+        o = ora.step(G, [np.zeros_like(x) for x in G], Q0[l])
+        ghat = o["G_hat"]
+        for r, P, Q, E, vout, params in res:
+            np.testing.assert_allclose(P[l], o["P_hat"], atol=1e-12)
+            np.testing.assert_allclose(Q[l], o["Q_bar"], atol=1e-12)
+            for w in range(WL):
+                np.testing.assert_allclose(E[w][l], o["E_new"][r * WL + w], atol=1e-12)
+            np.testing.assert_allclose(params[l], -0.1 * ghat, atol=1e-12)
+    vec_want = [sum(_vecs(r, w)[k] for r in range(world) for w in range(WL)).numpy() / (world * WL)
+                for k in range(2)]
+    for r, P, Q, E, vout, params in res:
+        for k in range(2):
+            np.testing.assert_allclose(vout[k], vec_want[k], atol=1e-12)
