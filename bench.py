@@ -331,7 +331,7 @@ def main():
               "workers": wl.workers, "rank": r, "grad_dtype": wl.grad_dtype, "mode": mode,
               "l2": "inputs larger than L2 (no flush needed)" if wl.elements * 4 > 4 * 126e6 else "inputs fit L2",
               "parallelism": (f"dp{world} (P and Q all-reduced over NCCL; {wl.workers} simulated workers per GPU)"
-                              if world > 1 else "1 GPU")}
+                              if (world > 1 or args.dist) else "1 GPU")}
 
     if args.impl == "reference":
         if rank_id != 0:

@@ -274,7 +274,10 @@ PSGD_API int psgd_set_svd_refresh(psgd_ctx *ctx, int every, int iters);
  * the summed device milliseconds of the first pass (error feedback + P),
  * the second pass (Q, plus every later power iteration) and the third pass
  * (residual / decompression, 0 in lazy mode) to ms[0..2] and the number of recorded steps to *steps, and
- * clears the record.  Recording adds three event records per step. */
+ * clears the record.  Recording adds six event records per step.  The
+ * distributed calls are recorded too (pass A in psgd_dist_p; the
+ * orthogonalisation and pass B in psgd_dist_q; Q_bar and pass C in
+ * psgd_dist_finish; the caller's all-reduces in between are not counted). */
 PSGD_API int psgd_profile_enable(psgd_ctx *ctx, int enable);
 PSGD_API int psgd_profile_read(psgd_ctx *ctx, double *ms, int *steps);
 

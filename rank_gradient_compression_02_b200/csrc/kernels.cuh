@@ -969,23 +969,37 @@ __device__ __forceinline__ void pass_c_wide(const Params& p, const LayerDesc& d,
         qt_s[idx] = (jj < width) ? Qb[(jc + jj) * R + kk] : 0.f;
     }
     __syncthreads();
-    float rec[SR][4];
+    // rec[s][v] = sum_k ph[row_s][k] * qbar[col_v][k], k ascending (recon_dot's
+    // order); four k at a time: Q_bar for them in registers, P_hat rows as
+    // float4 broadcasts, two columns per packed FMA
+    float2 rec2[SR][2];
 #pragma unroll
-    for (int s2 = 0; s2 < SR; ++s2)
+    for (int s2 = 0; s2 < SR; ++s2) rec2[s2][0] = rec2[s2][1] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int v = 0; v < 4; ++v) rec[s2][v] = 0.f;
+    for (int k4 = 0; k4 < R; k4 += 4) {
+        float4 q[4];
 #pragma unroll
-    for (int kk = 0; kk < R; ++kk) {
-        const float4 q = *reinterpret_cast<const float4*>(qt_s + kk * STR + 4 * lane);
+        for (int kk = 0; kk < 4; ++kk) q[kk] = *reinterpret_cast<const float4*>(qt_s + (k4 + kk) * STR + 4 * lane);
 #pragma unroll
         for (int s2 = 0; s2 < SR; ++s2) {
-            const int ii = warp + kWarps * s2;
-            const float ph = (ii < rows) ? ph_s[ii * R + kk] : 0.f;
-            rec[s2][0] = fmaf(ph, q.x, rec[s2][0]);
-            rec[s2][1] = fmaf(ph, q.y, rec[s2][1]);
-            rec[s2][2] = fmaf(ph, q.z, rec[s2][2]);
-            rec[s2][3] = fmaf(ph, q.w, rec[s2][3]);
+            const int ii = min(warp + kWarps * s2, rows - 1);
+            const float4 ph = *reinterpret_cast<const float4*>(ph_s + ii * R + k4);
+            const float phk[4] = {ph.x, ph.y, ph.z, ph.w};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const float2 pp = make_float2(phk[kk], phk[kk]);
+                rec2[s2][0] = __ffma2_rn(pp, make_float2(q[kk].x, q[kk].y), rec2[s2][0]);
+                rec2[s2][1] = __ffma2_rn(pp, make_float2(q[kk].z, q[kk].w), rec2[s2][1]);
+            }
         }
+    }
+    float rec[SR][4];
+#pragma unroll
+    for (int s2 = 0; s2 < SR; ++s2) {
+        rec[s2][0] = rec2[s2][0].x;
+        rec[s2][1] = rec2[s2][0].y;
+        rec[s2][2] = rec2[s2][1].x;
+        rec[s2][3] = rec2[s2][1].y;
     }
     float* recon = (p.do_recon && p.t.recon_out != nullptr) ? p.t.recon_out[tc.l] : nullptr;
     float* xs = p.do_mom ? p.t.params[tc.l] : nullptr;

@@ -184,13 +184,14 @@ struct psgd_ctx {
 
     // optional per-kernel timing (psgd_profile_*)
     bool profiling = false;
-    std::vector<std::array<cudaEvent_t, 4>> prof_ev;
+    std::vector<std::array<cudaEvent_t, 6>> prof_ev;   // begin/end of passes A, B, C
     size_t prof_used = 0;
 
     int iters = 1;          // power iterations per step
     int w_global = 0;       // workers over all ranks (distributed step); 0 = W
     int dist_phase = 0;     // distributed step: 0 idle, 1 after P, 2 after Q
     bool tab_l_has_recon = false;
+    cudaEvent_t* dist_ev = nullptr;   // profiling events of the step in progress
     int svd_every = 0;      // SVD refresh period in steps (0: off)
     int svd_iters = 0;      // subspace iterations on a refresh step
     uint64_t steps_done = 0;
@@ -552,6 +553,22 @@ int psgd_init_q(psgd_ctx* ctx, float* const* q, void* stream) {
     return PSGD_OK;
 }
 
+// Next set of profiling events (begin/end of passes A, B, C), or null when
+// profiling is off.
+static cudaEvent_t* profile_events(psgd_ctx* ctx, cudaError_t* err) {
+    *err = cudaSuccess;
+    if (!ctx->profiling) return nullptr;
+    if (ctx->prof_used == ctx->prof_ev.size()) {
+        std::array<cudaEvent_t, 6> a{};
+        for (auto& x : a) {
+            *err = cudaEventCreate(&x);
+            if (*err != cudaSuccess) return nullptr;
+        }
+        ctx->prof_ev.push_back(a);
+    }
+    return ctx->prof_ev[ctx->prof_used++].data();
+}
+
 static int step_impl(psgd_ctx* ctx, const void* const* grads, float* const* errors, float* const* q,
                      float* const* p_hat, float* const* recon, cudaStream_t s) {
     const size_t WL = static_cast<size_t>(ctx->W) * ctx->L;
@@ -581,19 +598,9 @@ static int step_impl(psgd_ctx* ctx, const void* const* grads, float* const* erro
     p.t.recon_out = reinterpret_cast<float* const*>(lt + 2 * ctx->L);
     p.use_prev = (lazy && ctx->errors_hold_m) ? 1 : 0;
 
-    cudaEvent_t* ev = nullptr;
-    if (ctx->profiling) {
-        if (ctx->prof_used == ctx->prof_ev.size()) {
-            std::array<cudaEvent_t, 4> a{};
-            for (auto& x : a) {
-                e = cudaEventCreate(&x);
-                if (e != cudaSuccess) return cuda_fail(ctx, e, "profiling event");
-            }
-            ctx->prof_ev.push_back(a);
-        }
-        ev = ctx->prof_ev[ctx->prof_used++].data();
-        cudaEventRecord(ev[0], s);
-    }
+    cudaEvent_t* ev = profile_events(ctx, &e);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "profiling event");
+    if (ev) cudaEventRecord(ev[0], s);
     int rc = PSGD_OK;
     if (ctx->flags & PSGD_FLAG_NO_WARM_START) {
         // no warm start: a fresh Q for this step (draw index = step number)
@@ -607,7 +614,10 @@ static int step_impl(psgd_ctx* ctx, const void* const* grads, float* const* erro
         if (e != cudaSuccess) return cuda_fail(ctx, e, "fresh Q launch");
     }
     rc = launch(ctx, 0, lazy, p, ctx->smem_a, s);
-    if (ev) cudaEventRecord(ev[1], s);
+    if (ev) {
+        cudaEventRecord(ev[1], s);
+        cudaEventRecord(ev[2], s);
+    }
     if (!rc) rc = launch(ctx, 1, lazy, p, ctx->smem_b, s);
     const bool refresh = ctx->svd_every > 0 && (ctx->steps_done + 1) % ctx->svd_every == 0;
     const int iters = refresh ? ctx->svd_iters : ctx->iters;
@@ -624,14 +634,17 @@ static int step_impl(psgd_ctx* ctx, const void* const* grads, float* const* erro
         e = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(ctx->L)), dim3(psgd::kThreads), args, 0, s);
         if (e != cudaSuccess) return cuda_fail(ctx, e, "Rayleigh-Ritz launch");
     }
-    if (ev) cudaEventRecord(ev[2], s);
+    if (ev) {
+        cudaEventRecord(ev[3], s);
+        cudaEventRecord(ev[4], s);
+    }
     if (!rc && (!lazy || recon)) {
         psgd::Params pc = p;
         pc.do_resid = lazy ? 0 : 1;
         pc.do_recon = recon ? 1 : 0;
         rc = launch(ctx, 2, lazy, pc, ctx->smem_c, s);
     }
-    if (ev) cudaEventRecord(ev[3], s);
+    if (ev) cudaEventRecord(ev[5], s);
     if (rc) return rc;
     ctx->have_step = true;
     ctx->errors_hold_m = lazy;
@@ -1063,7 +1076,12 @@ int psgd_dist_p(psgd_ctx* ctx, const void* const* grads, float* const* errors, f
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(ctx, e, "fresh Q launch");
     }
+    cudaEvent_t* ev = profile_events(ctx, &e);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "profiling event");
+    ctx->dist_ev = ev;
+    if (ev) cudaEventRecord(ev[0], s);
     rc = launch(ctx, 0, lazy, p, ctx->smem_a, s);
+    if (ev) cudaEventRecord(ev[1], s);
     if (rc) return rc;
     ctx->tab_l_has_recon = recon != nullptr;
     ctx->dist_phase = 1;
@@ -1085,11 +1103,14 @@ int psgd_dist_q(psgd_ctx* ctx, const double* p_sum, double* q_send, void* stream
     p.dist_in = p_sum;
     void* fn = kernel_ptr(5, ctx->R, ctx->dtype, false, false);
     void* args[] = {&p};
+    cudaEvent_t* ev = ctx->dist_ev;
+    if (ev) cudaEventRecord(ev[2], s);
     cudaError_t e = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(ctx->L)), dim3(psgd::kThreads), args, 0, s);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "distributed orthogonalisation launch");
     p.dist_in = nullptr;
     p.dist_out = q_send;
     int rc = launch(ctx, 1, lazy, p, ctx->smem_b, s);
+    if (ev) cudaEventRecord(ev[3], s);
     if (rc) return rc;
     ctx->dist_phase = 2;
     return PSGD_OK;
@@ -1112,6 +1133,8 @@ int psgd_dist_finish(psgd_ctx* ctx, const double* q_sum, void* stream) {
     const unsigned gx = static_cast<unsigned>(std::min<int64_t>(1024, (maxn * ctx->R + 255) / 256));
     void* fn = kernel_ptr(6, ctx->R, ctx->dtype, false, false);
     void* args[] = {&p};
+    cudaEvent_t* ev = ctx->dist_ev;
+    if (ev) cudaEventRecord(ev[4], s);
     cudaError_t e = cudaLaunchKernel(fn, dim3(std::max(1u, gx), static_cast<unsigned>(ctx->L)), dim3(256), args, 0, s);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "distributed Q_bar launch");
     const bool recon = ctx->tab_l_has_recon;
@@ -1123,6 +1146,8 @@ int psgd_dist_finish(psgd_ctx* ctx, const double* q_sum, void* stream) {
         int rc = launch(ctx, 2, lazy, pc, ctx->smem_c, s);
         if (rc) return rc;
     }
+    if (ev) cudaEventRecord(ev[5], s);
+    ctx->dist_ev = nullptr;
     ctx->dist_phase = 0;
     ctx->have_step = true;
     ctx->errors_hold_m = lazy;
@@ -1159,11 +1184,11 @@ int psgd_profile_read(psgd_ctx* ctx, double* ms, int* steps) {
     ms[0] = ms[1] = ms[2] = 0.0;
     for (size_t i = 0; i < ctx->prof_used; ++i) {
         auto& a = ctx->prof_ev[i];
-        cudaError_t e = cudaEventSynchronize(a[3]);
+        cudaError_t e = cudaEventSynchronize(a[5]);
         if (e != cudaSuccess) return cuda_fail(ctx, e, "profile sync");
         for (int k = 0; k < 3; ++k) {
             float t = 0.f;
-            e = cudaEventElapsedTime(&t, a[k], a[k + 1]);
+            e = cudaEventElapsedTime(&t, a[2 * k], a[2 * k + 1]);
             if (e != cudaSuccess) return cuda_fail(ctx, e, "profile elapsed");
             ms[k] += t;
         }
