@@ -26,8 +26,18 @@ struct TileCoord {
     int l, rb, c;
 };
 
-__device__ __forceinline__ TileCoord decode_tile(const Params& p, const LayerDesc& d, int l) {
-    const int local = static_cast<int>(blockIdx.x - d.tile_begin);
+// The Q pass (REVERSE) walks the tiles backwards, the other passes
+// forwards, so that each pass starts on the tiles the previous one touched
+// last, whose lines are still in L2.  The direction is a template argument:
+// a run-time select costs the first pass registers it does not have.
+template <bool REVERSE>
+__device__ __forceinline__ int tile_index() {
+    if constexpr (REVERSE) return static_cast<int>(gridDim.x - 1 - blockIdx.x);
+    else return static_cast<int>(blockIdx.x);
+}
+
+__device__ __forceinline__ TileCoord decode_tile(const LayerDesc& d, int t, int l) {
+    const int local = static_cast<int>(t - d.tile_begin);
     TileCoord tc;
     tc.l = l;
     tc.rb = local / d.nchunk;
@@ -175,29 +185,32 @@ __device__ __forceinline__ void pass_a_rows(const Params& p, const LayerDesc& d,
             float msum[VEC];
 #pragma unroll
             for (int v = 0; v < VEC; ++v) msum[v] = 0.f;
-            int w = 0;
-            for (; w + U <= W; w += U) {
-                float g[U][VEC], e[U][VEC];
+            // G workers' loads in flight, then M, the store and the products;
+            // float32 runs are flushed every F workers (<= 8 terms)
+            auto group = [&](auto GC, int w0) {
+                constexpr int G = decltype(GC)::value;
+                [[maybe_unused]] float g[G][VEC];
+                float e[G][VEC];
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    if constexpr (!READM) ld_grad<GT, VEC>(gp[w + u] + base, g[u]);
-                    ld_f32<VEC>(ep[w + u] + base, e[u]);
+                for (int u = 0; u < G; ++u) {
+                    if constexpr (!READM) ld_grad<GT, VEC>(gp[w0 + u] + base, g[u]);
+                    ld_f32<VEC>(ep[w0 + u] + base, e[u]);
                 }
                 if constexpr (!READM) {
 #pragma unroll
-                    for (int u = 0; u < U; ++u) {
+                    for (int u = 0; u < G; ++u) {
 #pragma unroll
                         for (int v = 0; v < VEC; ++v) {
                             float ev = e[u][v];
                             if constexpr (LAZY) ev = ev - rec[v];
                             e[u][v] = g[u][v] + ev;
                         }
-                        st_f32<VEC>(ep[w + u] + base, e[u]);
+                        st_f32<VEC>(ep[w0 + u] + base, e[u]);
                     }
                 }
                 if constexpr (SF) {
 #pragma unroll
-                    for (int u = 0; u < U; ++u)
+                    for (int u = 0; u < G; ++u)
 #pragma unroll
                         for (int v = 0; v < VEC; ++v) msum[v] += e[u][v];
                 } else {
@@ -205,12 +218,10 @@ __device__ __forceinline__ void pass_a_rows(const Params& p, const LayerDesc& d,
 #pragma unroll
                     for (int k = 0; k < R; ++k) pw[k] = 0.f;
 #pragma unroll
-                    for (int u = 0; u < U; ++u) {
+                    for (int u = 0; u < G; ++u) {
 #pragma unroll
-                        for (int v = 0; v < VEC; ++v)
-#pragma unroll
-                            axpy<R>(pw, e[u][v], qv[v]);
-                        if ((u + 1) % F == 0) {
+                        for (int v = 0; v < VEC; ++v) axpy<R>(pw, e[u][v], qv[v]);
+                        if ((u + 1) % F == 0 || u + 1 == G) {
 #pragma unroll
                             for (int k = 0; k < R; ++k) {
                                 acc[k] += static_cast<double>(pw[k]);
@@ -219,42 +230,28 @@ __device__ __forceinline__ void pass_a_rows(const Params& p, const LayerDesc& d,
                         }
                     }
                 }
-            }
-            for (; w < W; ++w) {
-                float g[VEC], e[VEC];
-                ld_f32<VEC>(ep[w] + base, e);
-                if constexpr (!READM) {
-                    ld_grad<GT, VEC>(gp[w] + base, g);
-#pragma unroll
-                    for (int v = 0; v < VEC; ++v) {
-                        float ev = e[v];
-                        if constexpr (LAZY) ev = ev - rec[v];
-                        e[v] = g[v] + ev;
-                    }
-                    st_f32<VEC>(ep[w] + base, e);
-                }
-                if constexpr (SF) {
-#pragma unroll
-                    for (int v = 0; v < VEC; ++v) msum[v] += e[v];
-                } else {
-                    float pw[R];
-#pragma unroll
-                    for (int k = 0; k < R; ++k) pw[k] = 0.f;
-#pragma unroll
-                    for (int v = 0; v < VEC; ++v)
-#pragma unroll
-                        axpy<R>(pw, e[v], qv[v]);
-#pragma unroll
-                    for (int k = 0; k < R; ++k) acc[k] += static_cast<double>(pw[k]);
+            };
+            int w = 0;
+            for (; w + U <= W; w += U) group(std::integral_constant<int, U>{}, w);
+            if constexpr (U > 4) {
+                if (w + 4 <= W) {
+                    group(std::integral_constant<int, 4>{}, w);
+                    w += 4;
                 }
             }
+            if constexpr (U > 2) {
+                if (w + 2 <= W) {
+                    group(std::integral_constant<int, 2>{}, w);
+                    w += 2;
+                }
+            }
+            if (w < W) group(std::integral_constant<int, 1>{}, w);
             if constexpr (SF) {
                 float pw[R];
 #pragma unroll
                 for (int k = 0; k < R; ++k) pw[k] = 0.f;
 #pragma unroll
                 for (int v = 0; v < VEC; ++v)
-#pragma unroll
                     axpy<R>(pw, msum[v], qv[v]);
 #pragma unroll
                 for (int k = 0; k < R; ++k) acc[k] = static_cast<double>(pw[k]);
@@ -548,9 +545,10 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
 template <int R, typename GT, bool LAZY, bool SF, bool READM>
 __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_a(Params p) {
     extern __shared__ __align__(16) unsigned char smem[];
-    const int l = p.t.tile_layer[blockIdx.x];
+    const int t = tile_index<false>();
+    const int l = p.t.tile_layer[t];
     const LayerDesc d = p.t.layers[l];
-    const TileCoord tc = decode_tile(p, d, l);
+    const TileCoord tc = decode_tile(d, t, l);
     const int W = p.workers;
     const int L = p.num_layers;
 
@@ -667,41 +665,37 @@ __device__ __forceinline__ void pass_b_rows(const Params& p, const LayerDesc& d,
             float msum[VEC];
 #pragma unroll
             for (int v = 0; v < VEC; ++v) msum[v] = 0.f;
-            int w = 0;
-            for (; w + U <= W; w += U) {
-                float e[U][VEC];
+            // G workers' loads in flight, then their products
+            auto group = [&](auto GC, int w0) {
+                constexpr int G = decltype(GC)::value;
+                float e[G][VEC];
 #pragma unroll
-                for (int u = 0; u < U; ++u) ld_f32<VEC>(ep[w + u] + base, e[u]);
+                for (int u = 0; u < G; ++u) ld_f32<VEC>(ep[w0 + u] + base, e[u]);
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
+                for (int u = 0; u < G; ++u) {
                     if constexpr (SF) {
 #pragma unroll
                         for (int v = 0; v < VEC; ++v) msum[v] += e[u][v];
                     } else {
 #pragma unroll
-                        for (int v = 0; v < VEC; ++v)
-#pragma unroll
-                            axpy<R>(qacc[v], e[u][v], ph);
+                        for (int v = 0; v < VEC; ++v) axpy<R>(qacc[v], e[u][v], ph);
                     }
                 }
+            };
+            int w = 0;
+            for (; w + U <= W; w += U) group(std::integral_constant<int, U>{}, w);
+            if (w + 4 <= W) {
+                group(std::integral_constant<int, 4>{}, w);
+                w += 4;
             }
-            for (; w < W; ++w) {
-                float e[VEC];
-                ld_f32<VEC>(ep[w] + base, e);
-                if constexpr (SF) {
-#pragma unroll
-                    for (int v = 0; v < VEC; ++v) msum[v] += e[v];
-                } else {
-#pragma unroll
-                    for (int v = 0; v < VEC; ++v)
-#pragma unroll
-                        axpy<R>(qacc[v], e[v], ph);
-                }
+            if (w + 2 <= W) {
+                group(std::integral_constant<int, 2>{}, w);
+                w += 2;
             }
+            if (w < W) group(std::integral_constant<int, 1>{}, w);
             if constexpr (SF) {
 #pragma unroll
                 for (int v = 0; v < VEC; ++v)
-#pragma unroll
                     axpy<R>(qacc[v], msum[v], ph);
             }
         }
@@ -902,9 +896,10 @@ __device__ void pass_b_epilogue(const Params& p, const LayerDesc& d, const TileC
 template <int R, bool SF>
 __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_b(Params p) {
     extern __shared__ __align__(16) unsigned char smem[];
-    const int l = p.t.tile_layer[blockIdx.x];
+    const int t = tile_index<true>();
+    const int l = p.t.tile_layer[t];
     const LayerDesc d = p.t.layers[l];
-    const TileCoord tc = decode_tile(p, d, l);
+    const TileCoord tc = decode_tile(d, t, l);
     const int W = p.workers;
     const int L = p.num_layers;
 
@@ -1097,34 +1092,41 @@ __device__ __forceinline__ void pass_c_rows(const Params& p, const LayerDesc& d,
             st_f32<VEC>(ms + base, mo);
             st_f32<VEC>(xs + base, x);
         }
-        int w = 0;
-        for (; w + U <= W; w += U) {
-            float e[U][VEC];
+        auto group = [&](auto GC, int w0) {
+            constexpr int G = decltype(GC)::value;
+            float e[G][VEC];
 #pragma unroll
-            for (int u = 0; u < U; ++u) ld_f32<VEC>(ep[w + u] + base, e[u]);
+            for (int u = 0; u < G; ++u) ld_f32<VEC>(ep[w0 + u] + base, e[u]);
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
+            for (int u = 0; u < G; ++u) {
 #pragma unroll
                 for (int v = 0; v < VEC; ++v) e[u][v] = e[u][v] - rec[v];
-                st_f32<VEC>(ep[w + u] + base, e[u]);
+                st_f32<VEC>(ep[w0 + u] + base, e[u]);
+            }
+        };
+        int w = 0;
+        for (; w + U <= W; w += U) group(std::integral_constant<int, U>{}, w);
+        if constexpr (U > 4) {
+            if (w + 4 <= W) {
+                group(std::integral_constant<int, 4>{}, w);
+                w += 4;
             }
         }
-        for (; w < W; ++w) {
-            float e[VEC];
-            ld_f32<VEC>(ep[w] + base, e);
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) e[v] = e[v] - rec[v];
-            st_f32<VEC>(ep[w] + base, e);
+        if (w + 2 <= W) {
+            group(std::integral_constant<int, 2>{}, w);
+            w += 2;
         }
+        if (w < W) group(std::integral_constant<int, 1>{}, w);
     }
 }
 
 template <int R>
 __global__ void __launch_bounds__(kThreads, 2) k_pass_c(Params p) {
     extern __shared__ __align__(16) unsigned char smem[];
-    const int l = p.t.tile_layer[blockIdx.x];
+    const int t = tile_index<false>();
+    const int l = p.t.tile_layer[t];
     const LayerDesc d = p.t.layers[l];
-    const TileCoord tc = decode_tile(p, d, l);
+    const TileCoord tc = decode_tile(d, t, l);
     const int W = p.workers;
     const int L = p.num_layers;
     float** ep = reinterpret_cast<float**>(smem);
