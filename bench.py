@@ -475,56 +475,77 @@ def main():
 
 def run_e2e(lib, B, wl, r, args, world, device, DB=None):
     """The same metric through the public API with host buffers: pinned
-    host gradients copied in every step (psgd_step_host on one GPU; copies
-    into the device buffers before the distributed step on several), P_hat
-    and Q_bar (and the 1-D means) read back."""
+    host gradients, one flat buffer per worker, copied in every step
+    (psgd_step_host_flat on one GPU; one copy per worker into the device
+    buffers before the distributed step on several), P_hat and Q_bar (and
+    the 1-D means) read back."""
     gsz = 2 if wl.grad_dtype == "bf16" else 4
     host_bytes = wl.elements * gsz
     if host_bytes > 16e9:
         return {"value": None, "unit": UNIT, "skipped": "host copy of the gradients exceeds 16 GB"}
     import torch.distributed as dist
     W, L = wl.workers, len(wl.layers)
+    # one pinned host buffer per worker holding every layer (a flat gradient
+    # bucket), uploaded with one copy per worker
     Gh = [torch.empty(B.offs[-1], dtype=B.G_flat[0].dtype).pin_memory() for _ in range(W)]
     for w in range(W):
         Gh[w].copy_(B.G_flat[w])
-    Gh_views = [[Gh[w][B.offs[l]:B.offs[l] + m * n] for l, (m, n) in enumerate(wl.layers)] for w in range(W)]
+    layer_offs = [B.offs[l] for l in range(L)]
+    span = max(B.offs[l] + m * n for l, (m, n) in enumerate(wl.layers))
     Ph = [torch.empty(m, r).pin_memory() for (m, _) in wl.layers]
     Qh = [torch.empty(n, r).pin_memory() for (_, n) in wl.layers]
-    vh = vout_h = None
+    vbytes = 0
     if B.vecs is not None:
-        vh = [[t.cpu().pin_memory() for t in B.vecs[w]] for w in range(W)]
-        vout_h = [torch.empty(k).pin_memory() for k in wl.vectors]
+        # the 1-D gradients of all workers in one pinned buffer, 16-byte
+        # aligned slots, one upload; the means come back in one download
+        slots, off = [], 0
+        for w in range(W):
+            for k in wl.vectors:
+                slots.append((off, k))
+                off += (k + 3) // 4 * 4
+        vflat_h = torch.zeros(max(off, 4)).pin_memory()
+        it = iter(slots)
+        for w in range(W):
+            for t in B.vecs[w]:
+                o, k = next(it)
+                vflat_h[o:o + k].copy_(t.cpu())
+        vflat_d = DB.vflat if DB is not None else torch.empty_like(vflat_h, device=device)
+        it = iter(slots)
+        vviews = [[vflat_d[o:o + k] for (o, k) in [next(it) for _ in wl.vectors]] for _ in range(W)]
+        oslots, ooff = [], 0
+        for k in wl.vectors:
+            oslots.append((ooff, k))
+            ooff += (k + 3) // 4 * 4
+        vout_d = torch.empty(max(ooff, 4), device=device)
+        vout_h = torch.empty(max(ooff, 4)).pin_memory()
+        vout_views = [vout_d[o:o + k] for (o, k) in oslots]
+        vbytes = vflat_h.numel() * 4
     stream = torch.cuda.current_stream()
 
     def one_dist():
         import torch.distributed as dist
         for w in range(W):
             B.G_flat[w].copy_(Gh[w], non_blocking=True)
-        if vh is not None:
-            for w in range(W):
-                for k in range(len(wl.vectors)):
-                    B.vecs[w][k].copy_(vh[w][k], non_blocking=True)
-            DB.pack(B.vecs)
+        if B.vecs is not None:
+            vflat_d.copy_(vflat_h, non_blocking=True)
         dist_step(lib, B, wl, DB, lambda t: dist.all_reduce(t, op=dist.ReduceOp.SUM))
         for l in range(L):
             Ph[l].copy_(B.P[l], non_blocking=True)
             Qh[l].copy_(B.Q[l], non_blocking=True)
-        if vh is not None:
-            for k in range(len(wl.vectors)):
-                vout_h[k].copy_(B.vout[k], non_blocking=True)
+        if B.vecs is not None:
+            for (o, k), v in zip(oslots, B.vout):
+                vout_d[o:o + k].copy_(v)
+            vout_h.copy_(vout_d, non_blocking=True)
 
     def one():
         if DB is not None:
             return one_dist()
-        lib.step_host(Gh_views, B.E, B.Q, Ph, Qh)
-        if vh is not None:
-            for w in range(W):
-                for k in range(len(wl.vectors)):
-                    B.vecs[w][k].copy_(vh[w][k], non_blocking=True)
+        lib.step_host_flat(Gh, layer_offs, B.E, B.Q, Ph, Qh)
+        if B.vecs is not None:
+            vflat_d.copy_(vflat_h, non_blocking=True)
             beta, lr = wl.momentum if wl.momentum else (0.0, 0.0)
-            lib.vec_mean(B.vecs, B.vout, B.vx, B.vmom, lr=lr, beta=beta)
-            for k in range(len(wl.vectors)):
-                vout_h[k].copy_(B.vout[k], non_blocking=True)
+            lib.vec_mean(vviews, vout_views, B.vx, B.vmom, lr=lr, beta=beta)
+            vout_h.copy_(vout_d, non_blocking=True)
         if B.params is not None:
             beta, lr = wl.momentum
             lib.momentum_step(B.params, B.mom, lr, beta)
@@ -543,8 +564,8 @@ def run_e2e(lib, B, wl, r, args, world, device, DB=None):
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world, device)
     per = ms / args.e2e_steps
-    h2d = host_bytes + (sum(wl.vectors) * 4 * W if vh is not None else 0)
-    d2h = sum((m + n) * r * 4 for (m, n) in wl.layers) + (sum(wl.vectors) * 4 if vh is not None else 0)
+    h2d = W * span * gsz + vbytes
+    d2h = sum((m + n) * r * 4 for (m, n) in wl.layers) + (vout_h.numel() * 4 if B.vecs is not None else 0)
     return {"value": wl.elements * world / (per * 1e-3), "unit": UNIT, "ms_per_step": per,
             "steps": args.e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 

@@ -143,6 +143,19 @@ PSGD_API int psgd_step(psgd_ctx *ctx, const void *const *grads, float *const *er
 PSGD_API int psgd_step_host(psgd_ctx *ctx, const void *const *grads_host, float *const *errors, float *const *q,
                    float *const *p_hat_host, float *const *q_host, void *stream);
 
+/* psgd_step_host for gradients packed into one host buffer per worker (a
+ * flat gradient bucket): layer l of worker w starts at element
+ * layer_offset[l] of grads_host[w] (grad dtype).  The library uploads each
+ * worker's buffer with ONE copy of elements [0, max_l(layer_offset[l] +
+ * m_l * n_l)), so the caller guarantees that span is one allocation
+ * (pinned for asynchronous copies); bytes between layers are copied and
+ * ignored.  layer_offset[l] * sizeof(grad dtype) must be a multiple of 16
+ * (PSGD_ERR_ALIGN otherwise), offsets must be >= 0.  Otherwise as
+ * psgd_step_host. */
+PSGD_API int psgd_step_host_flat(psgd_ctx *ctx, const void *const *grads_host, const int64_t *layer_offset,
+                                 float *const *errors, float *const *q, float *const *p_hat_host,
+                                 float *const *q_host, void *stream);
+
 /* PSGD_FLAG_LAZY_ERRORS only: write E'_w = M_w - P_hat Q_bar^T (from the
  * last step) into errors[w*L + l] in place.  The next step then starts from
  * E'_w as in the eager mode. */

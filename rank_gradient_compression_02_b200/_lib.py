@@ -46,6 +46,7 @@ _SIGS = {
     "psgd_init_q": (ctypes.c_int, [_P, _PP, _P]),
     "psgd_step": (ctypes.c_int, [_P, _PP, _PP, _PP, _PP, _PP, _P]),
     "psgd_step_host": (ctypes.c_int, [_P, _PP, _PP, _PP, _PP, _PP, _P]),
+    "psgd_step_host_flat": (ctypes.c_int, [_P, _PP, ctypes.POINTER(ctypes.c_int64), _PP, _PP, _PP, _PP, _P]),
     "psgd_materialize_errors": (ctypes.c_int, [_P, _PP, _P]),
     "psgd_momentum_step": (ctypes.c_int, [_P, _PP, _PP, ctypes.c_float, ctypes.c_float, _P]),
     "psgd_vec_mean": (ctypes.c_int, [_P, _PP, _PP, ctypes.POINTER(ctypes.c_int64), ctypes.c_int, _PP, _PP,
@@ -180,6 +181,15 @@ class PowerSGD:
                                             _ptrs(p_hat_host) if p_hat_host is not None else None,
                                             _ptrs(q_host) if q_host is not None else None,
                                             _stream_handle(stream)))
+
+    def step_host_flat(self, grads_host, layer_offsets, errors, q, p_hat_host=None, q_host=None, stream=None):
+        """grads_host[w]: one host buffer per worker holding every layer,
+        layer l starting at element layer_offsets[l]."""
+        offs = (ctypes.c_int64 * max(1, len(layer_offsets)))(*[int(o) for o in layer_offsets])
+        self._check(self.lib.psgd_step_host_flat(self._h, _ptrs(grads_host), offs, self._wl(errors), _ptrs(q),
+                                                 _ptrs(p_hat_host) if p_hat_host is not None else None,
+                                                 _ptrs(q_host) if q_host is not None else None,
+                                                 _stream_handle(stream)))
 
     def materialize_errors(self, errors, stream=None):
         self._check(self.lib.psgd_materialize_errors(self._h, self._wl(errors), _stream_handle(stream)))

@@ -670,10 +670,45 @@ int psgd_step(psgd_ctx* ctx, const void* const* grads, float* const* errors, flo
     return step_impl(ctx, grads, errors, q, p_hat, recon, static_cast<cudaStream_t>(stream));
 }
 
+// Staging area of at least `need` bytes for host gradients (grown on demand).
+static int ensure_stage(psgd_ctx* ctx, size_t need) {
+    if (need <= ctx->stage_bytes) return PSGD_OK;
+    if (ctx->stage) cudaFree(ctx->stage);
+    ctx->stage = nullptr;
+    ctx->stage_bytes = 0;
+    cudaError_t e = cudaMalloc(&ctx->stage, need);
+    if (e != cudaSuccess) return fail(ctx, PSGD_ERR_OOM, "staging of %zu bytes: %s", need, cudaGetErrorString(e));
+    ctx->stage_bytes = need;
+    return PSGD_OK;
+}
+
+// The step on staged gradients, then P_hat and Q_bar copied to the host.
+static int step_and_download(psgd_ctx* ctx, const void* const* dev_grads, float* const* errors, float* const* q,
+                             float* const* p_hat_host, float* const* q_host, cudaStream_t s) {
+    int rc = step_impl(ctx, dev_grads, errors, q, nullptr, nullptr, s);
+    if (rc) return rc;
+    for (int l = 0; l < ctx->L; ++l) {
+        const LayerDesc& d = ctx->desc[l];
+        if (p_hat_host && p_hat_host[l]) {
+            // P_hat lives in the workspace with a padded row stride R
+            cudaError_t e = cudaMemcpy2DAsync(p_hat_host[l], sizeof(float) * ctx->r, ctx->work.phat + d.prow_off,
+                                              sizeof(float) * ctx->R, sizeof(float) * ctx->r, d.m,
+                                              cudaMemcpyDeviceToHost, s);
+            if (e != cudaSuccess) return cuda_fail(ctx, e, "P_hat download");
+        }
+        if (q_host && q_host[l]) {
+            cudaError_t e = cudaMemcpyAsync(q_host[l], q[l], sizeof(float) * d.n * ctx->r, cudaMemcpyDeviceToHost, s);
+            if (e != cudaSuccess) return cuda_fail(ctx, e, "Q download");
+        }
+    }
+    return PSGD_OK;
+}
+
 int psgd_step_host(psgd_ctx* ctx, const void* const* grads_host, float* const* errors, float* const* q,
                    float* const* p_hat_host, float* const* q_host, void* stream) {
     if (!ctx) return PSGD_ERR_ARG;
     ctx->err.clear();
+    if (ctx->dist_phase != 0) return fail(ctx, PSGD_ERR_STATE, "a distributed step is in progress");
     if (ctx->L == 0) return PSGD_OK;
     const size_t WL = static_cast<size_t>(ctx->W) * ctx->L;
     if (!grads_host) return fail(ctx, PSGD_ERR_ARG, "grads_host is null");
@@ -692,15 +727,8 @@ int psgd_step_host(psgd_ctx* ctx, const void* const* grads_host, float* const* e
         offs[l] = per_worker;
         per_worker = align_up(per_worker + static_cast<size_t>(ctx->desc[l].m * ctx->desc[l].n) * esz, 256);
     }
-    const size_t need = per_worker * ctx->W;
-    if (need > ctx->stage_bytes) {
-        if (ctx->stage) cudaFree(ctx->stage);
-        ctx->stage = nullptr;
-        ctx->stage_bytes = 0;
-        cudaError_t e = cudaMalloc(&ctx->stage, need);
-        if (e != cudaSuccess) return fail(ctx, PSGD_ERR_OOM, "staging of %zu bytes: %s", need, cudaGetErrorString(e));
-        ctx->stage_bytes = need;
-    }
+    rc = ensure_stage(ctx, per_worker * ctx->W);
+    if (rc) return rc;
     std::vector<const void*> dev_grads(WL);
     for (int w = 0; w < ctx->W; ++w)
         for (int l = 0; l < ctx->L; ++l) {
@@ -710,23 +738,45 @@ int psgd_step_host(psgd_ctx* ctx, const void* const* grads_host, float* const* e
             if (e != cudaSuccess) return cuda_fail(ctx, e, "gradient upload");
             dev_grads[w * ctx->L + l] = dst;
         }
-    rc = step_impl(ctx, dev_grads.data(), errors, q, nullptr, nullptr, s);
-    if (rc) return rc;
+    return step_and_download(ctx, dev_grads.data(), errors, q, p_hat_host, q_host, s);
+}
+
+int psgd_step_host_flat(psgd_ctx* ctx, const void* const* grads_host, const int64_t* layer_offset,
+                        float* const* errors, float* const* q, float* const* p_hat_host, float* const* q_host,
+                        void* stream) {
+    if (!ctx) return PSGD_ERR_ARG;
+    ctx->err.clear();
+    if (ctx->dist_phase != 0) return fail(ctx, PSGD_ERR_STATE, "a distributed step is in progress");
+    if (ctx->L == 0) return PSGD_OK;
+    const size_t WL = static_cast<size_t>(ctx->W) * ctx->L;
+    if (!grads_host || !layer_offset) return fail(ctx, PSGD_ERR_ARG, "grads_host or layer_offset is null");
+    for (int w = 0; w < ctx->W; ++w)
+        if (!grads_host[w]) return fail(ctx, PSGD_ERR_ARG, "grads_host[%d] is null", w);
+    const size_t esz = ctx->dtype == PSGD_BF16 ? 2 : 4;
+    size_t span = 0;   // elements per worker buffer
     for (int l = 0; l < ctx->L; ++l) {
-        const LayerDesc& d = ctx->desc[l];
-        if (p_hat_host && p_hat_host[l]) {
-            // P_hat lives in the workspace with a padded row stride R
-            cudaError_t e = cudaMemcpy2DAsync(p_hat_host[l], sizeof(float) * ctx->r, ctx->work.phat + d.prow_off,
-                                              sizeof(float) * ctx->R, sizeof(float) * ctx->r, d.m,
-                                              cudaMemcpyDeviceToHost, s);
-            if (e != cudaSuccess) return cuda_fail(ctx, e, "P_hat download");
-        }
-        if (q_host && q_host[l]) {
-            cudaError_t e = cudaMemcpyAsync(q_host[l], q[l], sizeof(float) * d.n * ctx->r, cudaMemcpyDeviceToHost, s);
-            if (e != cudaSuccess) return cuda_fail(ctx, e, "Q download");
-        }
+        if (layer_offset[l] < 0) return fail(ctx, PSGD_ERR_ARG, "layer_offset[%d] < 0", l);
+        if ((static_cast<size_t>(layer_offset[l]) * esz) % 16 != 0)
+            return fail(ctx, PSGD_ERR_ALIGN, "layer_offset[%d] is not a multiple of 16 bytes", l);
+        span = std::max(span, static_cast<size_t>(layer_offset[l] + ctx->desc[l].m * ctx->desc[l].n));
     }
-    return PSGD_OK;
+    int rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(errors), WL, false, "errors");
+    if (!rc) rc = check_ptr_array(ctx, reinterpret_cast<const void* const*>(q), ctx->L, false, "q");
+    if (rc) return rc;
+    DeviceGuard g(ctx->device);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // staging layout: one 256-byte aligned slot per worker, the host layout inside
+    const size_t per_worker = align_up(span * esz, 256);
+    rc = ensure_stage(ctx, per_worker * ctx->W);
+    if (rc) return rc;
+    std::vector<const void*> dev_grads(WL);
+    for (int w = 0; w < ctx->W; ++w) {
+        unsigned char* dst = static_cast<unsigned char*>(ctx->stage) + per_worker * w;
+        cudaError_t e = cudaMemcpyAsync(dst, grads_host[w], span * esz, cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "gradient upload");
+        for (int l = 0; l < ctx->L; ++l) dev_grads[w * ctx->L + l] = dst + static_cast<size_t>(layer_offset[l]) * esz;
+    }
+    return step_and_download(ctx, dev_grads.data(), errors, q, p_hat_host, q_host, s);
 }
 
 int psgd_materialize_errors(psgd_ctx* ctx, float* const* errors, void* stream) {

@@ -321,6 +321,44 @@ def test_step_host_matches_device_step():
                 assert torch.equal(a.E[w][l], b.E[w][l])
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_step_host_flat_matches_device_step(dtype):
+    # one pinned buffer per worker, layers at 16-byte aligned offsets with
+    # gaps between them (the gap contents are uploaded and ignored)
+    from rank_gradient_compression_02_b200 import PsgdError
+    wl = H.small_workload(MIXED, 4, 3, dtype=dtype)
+    a = H.LibRun(wl)
+    b = H.LibRun(wl)
+    L = len(wl.layers)
+    esz = 2 if dtype == "bf16" else 4
+    per16 = 16 // esz
+    offs, o = [], 3 * per16
+    for (m, n) in wl.layers:
+        offs.append(o)
+        o = -(-(o + m * n + 5) // per16) * per16
+    hdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    flat = [torch.full((o,), float("nan"), dtype=hdt).pin_memory() for _ in range(wl.workers)]
+    for t in range(2):
+        host = a.fill_grads_host(t)
+        a.run_step()
+        for w in range(wl.workers):
+            for l, (m, n) in enumerate(wl.layers):
+                flat[w][offs[l]:offs[l] + m * n].copy_(host[w][l].reshape(-1))
+        ph = [torch.empty(m, wl.rank).pin_memory() for (m, _) in wl.layers]
+        qh = [torch.empty(n, wl.rank).pin_memory() for (_, n) in wl.layers]
+        b.lib.step_host_flat(flat, offs, b.E, b.Q, ph, qh)
+        torch.cuda.synchronize()
+        for l in range(L):
+            assert torch.equal(a.Q[l].cpu(), qh[l])
+            assert torch.equal(a.P[l].cpu(), ph[l])
+            for w in range(wl.workers):
+                assert torch.equal(a.E[w][l], b.E[w][l])
+    bad = list(offs)
+    bad[1] += 1    # not a multiple of 16 bytes
+    with pytest.raises(PsgdError):
+        b.lib.step_host_flat(flat, bad, b.E, b.Q)
+
+
 def test_bad_arguments_rejected():
     from rank_gradient_compression_02_b200 import PowerSGD, PsgdError
     wl = H.small_workload([(64, 48)], 2, 2)
