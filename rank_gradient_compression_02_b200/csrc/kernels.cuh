@@ -102,13 +102,58 @@ __device__ void factor_gram_warp(const double* Gs, double* Rs, double* Ts, int* 
 // ---------------------------------------------------------------------------
 // pass A
 
-// Rank 32 uses the rank-lane kernels (one lane per rank index, M rows
-// parked in shared memory and read as broadcasts); they walk a chunk (up to
-// 32 * VEC columns) in sub-chunks of 32 columns.
+// Rank 32 uses the wide kernels: a chunk (up to 32 * VEC columns) is walked
+// in sub-chunks of 32 columns.  Pass A forms M * Q on the tensor cores
+// (mma.sync m16n8k8 tf32, a warp per 16 rows); passes B and C map one lane
+// per rank index.  Tiles of the wide kernels have 16, 32 or 64 rows.
 template <int R>
 struct IsWide { static constexpr bool value = R >= 32; };
 constexpr int kWideCols = 32;
-constexpr int kWideRows = 64;    // rows per tile cap for the rank-lane kernels
+constexpr int kWideRows = 64;    // rows per tile cap for the wide kernels
+
+// ---- float32 products on the tf32 tensor cores ---------------------------
+// x = hi + lo with hi = x rounded to tf32 (10 mantissa bits, to nearest,
+// ties away) and lo = (x - hi) rounded to tf32; x - hi is exact.  A product
+// a * b is taken as a_hi b_hi + a_hi b_lo + a_lo b_hi: the dropped a_lo b_lo
+// and the rounding of the lo parts leave a relative error below 2^-21
+// (split-precision products on tensor cores: Markidis et al., "NVIDIA
+// Tensor Core Programmability, Performance & Precision", IPDPSW 2018).
+__device__ __forceinline__ uint32_t tf32_round(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void tf32_split(float x, uint32_t& hi, uint32_t& lo) {
+    hi = tf32_round(x);
+    lo = tf32_round(x - __uint_as_float(hi));
+}
+// c += A (16 x 8, row-major fragment) * B (8 x 8, column fragment), float32
+// accumulate.  Fragment of lane (g = lane / 4, t = lane % 4): a = A[g][t],
+// A[g + 8][t], A[g][t + 4], A[g + 8][t + 4]; b = B[t][g], B[t + 4][g];
+// c = C[g][2t], C[g][2t + 1], C[g + 8][2t], C[g + 8][2t + 1].
+__device__ __forceinline__ void mma_tf32(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// 3-term split product of one k-step: c = A B (c starts at zero)
+__device__ __forceinline__ void mma_tf32x3(float (&c)[4], const uint32_t (&ahi)[4], const uint32_t (&alo)[4],
+                                           const float4& b) {
+    // b = (b0 hi, b1 hi, b0 lo, b1 lo); small terms first
+    mma_tf32(c, alo, __float_as_uint(b.x), __float_as_uint(b.y));
+    mma_tf32(c, ahi, __float_as_uint(b.z), __float_as_uint(b.w));
+    mma_tf32(c, ahi, __float_as_uint(b.x), __float_as_uint(b.y));
+}
+
+constexpr int kMmaRows = 16;                  // rows per warp in the tensor-core pass A
+constexpr int kMaxKSteps = 32 * 4 / 8;        // k-steps of 8 columns in the widest chunk
+constexpr size_t kQfBytes = static_cast<size_t>(kMaxKSteps) * 4 * 32 * sizeof(float4);
+constexpr int kRedStride = 32 + 1;            // second pass: warp partial row stride (floats)
+constexpr size_t kPaBytes = static_cast<size_t>(kWarps) * 2 * 2 * 32 * 8 * sizeof(float);   // its A fragments
+constexpr int kRecStride = kWideCols + 1;     // lazy reconstruction tile row stride (floats)
+constexpr size_t kRecBytes = static_cast<size_t>(kWarps) * kMmaRows * kRecStride * sizeof(float);
 
 template <int R>
 struct SmemA {
@@ -116,10 +161,12 @@ struct SmemA {
     static __host__ __device__ size_t ptr_bytes(int W) { return static_cast<size_t>(2 * W) * sizeof(void*); }
     static __host__ __device__ size_t rows_bytes(int tm) { return static_cast<size_t>(tm) * R * sizeof(double); }
     static __host__ __device__ size_t fac_bytes() { return 3 * R * R * sizeof(double) + 2 * R * sizeof(int) + 64; }
-    // rank-lane kernel: every warp's parked rows (tm x 32 floats in all)
+    // tensor-core kernel: the chunk's split Q fragments (later the parts'
+    // P partials, kWarps x 16 x 32 doubles, the same 32 KB) and every warp's
+    // lazy reconstruction tile
     static __host__ __device__ size_t wide_bytes(int tm) {
         (void)tm;
-        return IsWide<R>::value ? static_cast<size_t>(kWideRows * kWideCols) * sizeof(float) : 0;
+        return IsWide<R>::value ? kQfBytes + kRecBytes : 0;
     }
     static __host__ __device__ size_t total(int W, int tm) {
         return ((ptr_bytes(W) + 15) & ~size_t(15)) + ((rows_bytes(tm) + 15) & ~size_t(15)) +
@@ -265,23 +312,142 @@ __device__ __forceinline__ void pass_a_rows(const Params& p, const LayerDesc& d,
     }
 }
 
-// Rank-lane variant of the first pass (R = 32): lane k owns rank index k.
-// Warp w owns rows w, w + 8, ... of the tile and stages them itself: for
-// every (sub-chunk of 32 columns, worker) it forms M = G + E for its rows
-// (a lane per column; M is stored over E), parks them in its own slice of
-// shared memory, prefetches the next (sub-chunk, worker) into registers and
-// then walks the parked rows, reading M as broadcasts against its slice of
-// Q held in registers.  No CTA-wide barrier in the loop.  Products are
-// summed in float32 over runs of 8 terms and flushed to a float64 per-row
-// accumulator; the row's partial over the chunk needs no lane reduction.
-template <int R, typename GT, bool LAZY, bool SF, bool READM>
-__device__ __forceinline__ void pass_a_wide(const Params& p, const LayerDesc& d, const TileCoord& tc,
-                                            const GT* const* gp, float* const* ep, const float* ph_prev,
-                                            float* m_s) {
-    static_assert(R == 32, "rank-lane kernels map one lane per rank index");
-    constexpr int RPL = kWideRows / kWarps;   // rows per warp, at most
+// Tensor-core variant of the first pass (R = 32).  The tile's rows split
+// into row groups of 16 (tm / 16 of them); each row group belongs to
+// kWarps / (tm / 16) warps ("parts") that deal the workers among
+// themselves.  For every (sub-chunk of 32 columns, worker) of its share a
+// warp loads G and E of its 16 x 32 block straight into the registers of
+// the mma A fragments (VEC-wide loads), forms M = G + E there, stores M
+// over E, prefetches the next block and multiplies: per k-step of 8
+// columns and 8 ranks, three tf32 products (mma_tf32x3) summed in float32,
+// then added to a float64 accumulator, i.e. float32 runs of 8 terms as in
+// the CUDA-core passes.  At the end the parts' partials are added in part
+// order and written per chunk.
+//
+// Fragment columns.  An mma k-step takes 8 columns in any order, as long
+// as A and B agree.  Lane (g, t) holds rows g and g + 8 and, in k-step ks,
+// the columns col0(ks) (slot t) and col1(ks) (slot t + 4) of the sub-chunk:
+//   VEC 4: col0 = 16 (ks / 2) + 4 t + 2 (ks % 2), col1 = col0 + 1
+//   VEC 2: col0 = 8 ks + 2 t,                   col1 = col0 + 1
+//   VEC 1: col0 = 8 ks + t,                     col1 = col0 + 4
+// so a VEC-wide load of one row fills slots of one or two k-steps.
+template <int VEC>
+__device__ __forceinline__ int frag_col0(int ks, int t4) {
+    if constexpr (VEC == 4) return 16 * (ks >> 1) + 4 * t4 + 2 * (ks & 1);
+    else if constexpr (VEC == 2) return 8 * ks + 2 * t4;
+    else return 8 * ks + t4;
+}
+template <int VEC>
+__device__ __forceinline__ int frag_col1(int ks, int t4) {
+    return frag_col0<VEC>(ks, t4) + (VEC == 1 ? 4 : 1);
+}
+
+// G or E block of one (sub-chunk, worker) into fragment order:
+// v[ks][0] = (row g, col0), v[ks][1] = (row g + 8, col0),
+// v[ks][2] = (row g, col1), v[ks][3] = (row g + 8, col1); zero outside the
+// layer.  base points at (tile row r0, sub-chunk column 0) of the buffer.
+template <int VEC, typename T>
+__device__ __forceinline__ void load_frag(const T* base, int64_t n, int g, int t4, bool ok_lo, bool ok_hi, int cols,
+                                          float (&v)[4][4]) {
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[ks][q] = 0.f;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const bool ok_row = half ? ok_hi : ok_lo;
+        const int q0 = half;   // 0: row g, 1: row g + 8
+        const T* rp = base + static_cast<int64_t>(g + 8 * half) * n;
+        if constexpr (VEC == 4) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int c = 16 * h + 4 * t4;
+                if (ok_row && c < cols) {
+                    float x[4];
+                    if constexpr (std::is_same<T, float>::value) ld_f32<4>(rp + c, x);
+                    else ld_grad<T, 4>(rp + c, x);
+                    v[2 * h][q0] = x[0];
+                    v[2 * h][q0 + 2] = x[1];
+                    v[2 * h + 1][q0] = x[2];
+                    v[2 * h + 1][q0 + 2] = x[3];
+                }
+            }
+        } else if constexpr (VEC == 2) {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const int c = 8 * ks + 2 * t4;
+                if (ok_row && c < cols) {
+                    float x[2];
+                    if constexpr (std::is_same<T, float>::value) ld_f32<2>(rp + c, x);
+                    else ld_grad<T, 2>(rp + c, x);
+                    v[ks][q0] = x[0];
+                    v[ks][q0 + 2] = x[1];
+                }
+            }
+        } else {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2) {
+                    const int c = 8 * ks + t4 + 4 * s2;
+                    if (ok_row && c < cols) {
+                        float x[1];
+                        if constexpr (std::is_same<T, float>::value) ld_f32<1>(rp + c, x);
+                        else ld_grad<T, 1>(rp + c, x);
+                        v[ks][q0 + 2 * s2] = x[0];
+                    }
+                }
+            }
+        }
+    }
+}
+
+// M block (fragment order) stored back over E, same addressing as load_frag.
+template <int VEC>
+__device__ __forceinline__ void store_frag(float* base, int64_t n, int g, int t4, bool ok_lo, bool ok_hi, int cols,
+                                           const float (&v)[4][4]) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const bool ok_row = half ? ok_hi : ok_lo;
+        const int q0 = half;
+        float* rp = base + static_cast<int64_t>(g + 8 * half) * n;
+        if constexpr (VEC == 4) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int c = 16 * h + 4 * t4;
+                if (ok_row && c < cols) {
+                    const float x[4] = {v[2 * h][q0], v[2 * h][q0 + 2], v[2 * h + 1][q0], v[2 * h + 1][q0 + 2]};
+                    st_f32<4>(rp + c, x);
+                }
+            }
+        } else if constexpr (VEC == 2) {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const int c = 8 * ks + 2 * t4;
+                if (ok_row && c < cols) {
+                    const float x[2] = {v[ks][q0], v[ks][q0 + 2]};
+                    st_f32<2>(rp + c, x);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2) {
+                    const int c = 8 * ks + t4 + 4 * s2;
+                    if (ok_row && c < cols) rp[c] = v[ks][q0 + 2 * s2];
+                }
+        }
+    }
+}
+
+template <int VEC, typename GT, bool LAZY, bool SF, bool READM>
+__device__ __forceinline__ void pass_a_mma(const Params& p, const LayerDesc& d, const TileCoord& tc,
+                                           const GT* const* gp, float* const* ep, const float* ph_prev,
+                                           unsigned char* wide) {
+    constexpr int R = 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int k = lane;
+    const int g = lane >> 2, t4 = lane & 3;
     const int r = p.r;
     const int W = p.workers;
     const int64_t n = d.n, m = d.m;
@@ -290,134 +456,172 @@ __device__ __forceinline__ void pass_a_wide(const Params& p, const LayerDesc& d,
     const int64_t jc = static_cast<int64_t>(tc.c) * d.slots * d.vec;
     const int width = static_cast<int>(min(static_cast<int64_t>(d.slots) * d.vec, n - jc));
     const int nsc = (width + kWideCols - 1) / kWideCols;
-    const int total = nsc * W;
-    const float* Q = p.t.q[tc.l];
-    const float* Qb = p.ws.qbar + d.qrow_off;
-    float* ms_w = m_s + warp * RPL * kWideCols;
+    const int nrg = d.tm / kMmaRows;            // 1, 2 or 4 row groups
+    const int parts = kWarps / nrg;
+    const int rg = warp % nrg, part = warp / nrg;
+    const int r0 = rg * kMmaRows;               // first tile row of this warp
+    const bool ok_lo = r0 + g < rows, ok_hi = r0 + g + 8 < rows;
+    float4* qf = reinterpret_cast<float4*>(wide);   // [k-step][rank tile][lane]
 
-    float gv[RPL], ev[RPL];
-    auto load = [&](int it) {
-        const int sc = it / W, w = it - sc * W;
-        const int64_t j0 = jc + sc * kWideCols;
-        const int ncols = min(kWideCols, width - sc * kWideCols);
+    // split B fragments of the chunk's Q in the same column order (zero
+    // beyond the chunk and rank r)
+    {
+        const float* Q = p.t.q[tc.l];
+        const int nks = nsc * 4;
+        for (int idx = threadIdx.x; idx < nks * 4 * 32; idx += kThreads) {
+            const int ln = idx & 31, nt = (idx >> 5) & 3, ksg = idx >> 7;
+            const int sc = ksg >> 2, ks = ksg & 3;
+            const int jj0 = sc * kWideCols + frag_col0<VEC>(ks, ln & 3);
+            const int jj1 = sc * kWideCols + frag_col1<VEC>(ks, ln & 3);
+            const int k = 8 * nt + (ln >> 2);
+            const float b0 = (jj0 < width && k < r) ? Q[(jc + jj0) * r + k] : 0.f;
+            const float b1 = (jj1 < width && k < r) ? Q[(jc + jj1) * r + k] : 0.f;
+            uint32_t h0, l0, h1, l1;
+            tf32_split(b0, h0, l0);
+            tf32_split(b1, h1, l1);
+            qf[idx] = make_float4(__uint_as_float(h0), __uint_as_float(h1), __uint_as_float(l0), __uint_as_float(l1));
+        }
+    }
+    __syncthreads();
+
+    // this part's workers: part, part + parts, ...
+    const int nw = W > part ? (W - part + parts - 1) / parts : 0;
+    const int total = nsc * nw;
+    const int64_t row0 = (i0 + r0) * n + jc;    // (first row of this warp, chunk column 0)
+    float gq[4][4], eq[4][4];
+    auto load = [&](int sc, int w) {
+        const int cols = width - sc * kWideCols;
+        load_frag<VEC>(ep[w] + row0 + sc * kWideCols, n, g, t4, ok_lo, ok_hi, cols, eq);
+        if constexpr (!READM) load_frag<VEC>(gp[w] + row0 + sc * kWideCols, n, g, t4, ok_lo, ok_hi, cols, gq);
+    };
+
+    double acc[4][4];
 #pragma unroll
-        for (int t = 0; t < RPL; ++t) {
-            const int ii = warp + kWarps * t;
-            gv[t] = 0.f;
-            ev[t] = 0.f;
-            if (ii < rows && lane < ncols) {
-                const int64_t off = (i0 + ii) * n + j0 + lane;
-                ev[t] = __ldcs(ep[w] + off);
-                if constexpr (!READM) {
-                    float g1[1];
-                    ld_grad<GT, 1>(gp[w] + off, g1);
-                    gv[t] = g1[0];
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[nt][c] = 0.0;
+    float* rt = reinterpret_cast<float*>(wide + kQfBytes) + warp * (kMmaRows * kRecStride);
+    float msum[SF ? 4 : 1][SF ? 4 : 1];
+
+    // products of an M block (fragment order) with the sub-chunk's k-steps
+    auto multiply = [&](int sc, const float (&mv)[4][4]) {
+        const int cols = width - sc * kWideCols;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            // does k-step ks hold a column of the sub-chunk? (VEC 4: k-steps
+            // 2h and 2h + 1 share columns 16h .. 16h + 15)
+            if ((VEC == 4 ? 16 * (ks >> 1) : 8 * ks) < cols) {
+                uint32_t ahi[4], alo[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) tf32_split(mv[ks][q], ahi[q], alo[q]);
+                const float4* qk = qf + ((sc * 4 + ks) * 4) * 32 + lane;
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    float c[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma_tf32x3(c, ahi, alo, qk[nt * 32]);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc[nt][q] += static_cast<double>(c[q]);
                 }
             }
         }
     };
 
-    double acc[RPL];
-#pragma unroll
-    for (int t = 0; t < RPL; ++t) acc[t] = 0.0;
-    float qreg[kWideCols];
-    float rec[LAZY ? RPL : 1];
-    float msum[SF ? RPL : 1];
-
-    // two float32 runs (even and odd columns) in one packed fp32x2 FMA, each
-    // 8 terms long (16 columns), then both added to the float64 accumulator
-    auto walk_rows = [&]() {
-#pragma unroll
-        for (int t = 0; t < RPL; ++t) {
-            const int ii = warp + kWarps * t;
-            if (ii < rows) {
-                const float4* mrow = reinterpret_cast<const float4*>(ms_w + t * kWideCols);
-                float2 run = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int q4 = 0; q4 < kWideCols / 4; ++q4) {
-                    const float4 mv = mrow[q4];
-                    run = __ffma2_rn(make_float2(mv.x, mv.y), make_float2(qreg[4 * q4 + 0], qreg[4 * q4 + 1]), run);
-                    run = __ffma2_rn(make_float2(mv.z, mv.w), make_float2(qreg[4 * q4 + 2], qreg[4 * q4 + 3]), run);
-                    if ((q4 & 3) == 3) {
-                        acc[t] += static_cast<double>(run.x) + static_cast<double>(run.y);
-                        run = make_float2(0.f, 0.f);
-                    }
-                }
-            }
-        }
-    };
-
-    load(0);
+    if (total > 0) load(0, part);
+    int sc = 0, wi = 0;
     for (int it = 0; it < total; ++it) {
-        const int sc = it / W, w = it - sc * W;
-        const int64_t j0 = jc + sc * kWideCols;
-        const int ncols = min(kWideCols, width - sc * kWideCols);
-        if (w == 0) {
-            // this lane's slice of Q for the sub-chunk: Q[j0 + jj][k]
-#pragma unroll
-            for (int jj = 0; jj < kWideCols; ++jj) qreg[jj] = (jj < ncols && k < r) ? Q[(j0 + jj) * r + k] : 0.f;
+        const int w = part + wi * parts;
+        const int cols = width - sc * kWideCols;
+        if (wi == 0) {
             if constexpr (LAZY) {
-                // the previous step's reconstruction of (row, this lane's column)
+                // the previous step's reconstruction of the block (lane =
+                // column), in recon_dot's operation order, parked in rt
+                const float* Qb = p.ws.qbar + d.qrow_off;
+                const bool okc = lane < cols && p.use_prev;
                 float qp[R];
 #pragma unroll
-                for (int kk = 0; kk < R; ++kk)
-                    qp[kk] = (lane < ncols && p.use_prev) ? Qb[(j0 + lane) * R + kk] : 0.f;
-#pragma unroll
-                for (int t = 0; t < RPL; ++t) {
-                    // recon_dot's operation order, P_hat row read from shared memory
-                    const int ii = min(warp + kWarps * t, rows - 1);
+                for (int kk = 0; kk < R; ++kk) qp[kk] = okc ? Qb[(jc + sc * kWideCols + lane) * R + kk] : 0.f;
+                __syncwarp();
+                for (int tt = 0; tt < kMmaRows; ++tt) {
+                    const int ii = min(r0 + tt, rows - 1);
                     float s2 = 0.f;
 #pragma unroll
                     for (int kk = 0; kk < R; ++kk) s2 = fmaf(ph_prev[ii * R + kk], qp[kk], s2);
-                    rec[t] = s2;
+                    rt[tt * kRecStride + lane] = s2;
                 }
+                __syncwarp();
             }
             if constexpr (SF) {
 #pragma unroll
-                for (int t = 0; t < RPL; ++t) msum[t] = 0.f;
+                for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) msum[ks][q] = 0.f;
             }
         }
-        // M for this worker's rows
+        // M for this worker's block, in the fragment registers
+        float mv[4][4];
 #pragma unroll
-        for (int t = 0; t < RPL; ++t) {
-            const int ii = warp + kWarps * t;
-            float mval = ev[t];
-            if (ii < rows && lane < ncols) {
+        for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float x = eq[ks][q];
                 if constexpr (!READM) {
-                    float e2 = ev[t];
-                    if constexpr (LAZY) e2 = e2 - rec[t];
-                    mval = gv[t] + e2;
-                    ep[w][(i0 + ii) * n + j0 + lane] = mval;
+                    if constexpr (LAZY) {
+                        const int c = (q & 2) ? frag_col1<VEC>(ks, t4) : frag_col0<VEC>(ks, t4);
+                        x = x - rt[(g + 8 * (q & 1)) * kRecStride + c];
+                    }
+                    x = gq[ks][q] + x;
                 }
-            } else {
-                mval = 0.f;
+                mv[ks][q] = x;
             }
-            if constexpr (SF) {
-                msum[t] += mval;
-            } else {
-                ms_w[t * kWideCols + lane] = mval;
-            }
+        if constexpr (!READM) store_frag<VEC>(ep[w] + row0 + sc * kWideCols, n, g, t4, ok_lo, ok_hi, cols, mv);
+        const bool last_w = wi == nw - 1;
+        // next (sub-chunk, worker) in flight while this block is multiplied
+        int sc2 = sc, wi2 = wi + 1;
+        if (wi2 == nw) {
+            wi2 = 0;
+            ++sc2;
         }
-        if (it + 1 < total) load(it + 1);   // in flight while the rows are walked
+        if (it + 1 < total) load(sc2, part + wi2 * parts);
         if constexpr (SF) {
-            if (w == W - 1) {
 #pragma unroll
-                for (int t = 0; t < RPL; ++t) ms_w[t * kWideCols + lane] = msum[t];
-                __syncwarp();
-                walk_rows();
-                __syncwarp();
-            }
+            for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) msum[ks][q] += mv[ks][q];
+            if (last_w) multiply(sc, msum);
         } else {
-            __syncwarp();
-            walk_rows();
-            __syncwarp();
+            multiply(sc, mv);
         }
+        sc = sc2;
+        wi = wi2;
     }
-    double* ppart = p.ws.ppart + d.ppart_off;
+
+    // parts' partials added in part order; part 0 writes the chunk's rows
+    __syncthreads();   // every warp is done with the Q fragments
+    double* cb = reinterpret_cast<double*>(wide);   // [warp][16 values][lane]
+    if (part > 0) {
 #pragma unroll
-    for (int t = 0; t < RPL; ++t) {
-        const int ii = warp + kWarps * t;
-        if (ii < rows) ppart[(static_cast<int64_t>(tc.c) * m + i0 + ii) * R + k] = acc[t];
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) cb[(warp * 16 + nt * 4 + q) * 32 + lane] = acc[nt][q];
+    }
+    __syncthreads();
+    if (part == 0) {
+        for (int pp = 1; pp < parts; ++pp) {
+            const int src = pp * nrg + rg;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[nt][q] += cb[(src * 16 + nt * 4 + q) * 32 + lane];
+        }
+        double* ppart = p.ws.ppart + d.ppart_off;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int ii = r0 + g + 8 * (q >> 1);
+                const int k = 8 * nt + 2 * t4 + (q & 1);
+                if (ii < rows) ppart[(static_cast<int64_t>(tc.c) * m + i0 + ii) * R + k] = acc[nt][q];
+            }
     }
 }
 
@@ -572,7 +776,10 @@ __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_a(Params p)
     __syncthreads();
 
     if constexpr (IsWide<R>::value) {
-        pass_a_wide<R, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s, wide);
+        unsigned char* wb = reinterpret_cast<unsigned char*>(wide);
+        if (d.vec == 4) pass_a_mma<4, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s, wb);
+        else if (d.vec == 2) pass_a_mma<2, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s, wb);
+        else pass_a_mma<1, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s, wb);
     } else {
         // VEC x R values of Q live in registers: VEC = 4 up to R = 4, 2 up to 16
         if (d.vec == 4) {
@@ -596,8 +803,9 @@ struct SmemB {
     static __host__ __device__ size_t t_bytes() { return R * R * sizeof(double); }
     static __host__ __device__ size_t red_bytes(int vec) {
         if (IsWide<R>::value) {
-            // rank-lane kernel: parked rows (tm x 32) + warp partials (8 x 32 x R)
-            return static_cast<size_t>(kWideRows * kWideCols + kWarps * kWideCols * R) * sizeof(float);
+            // tensor-core kernel: warp partials (8 x 32 columns x 33) + the
+            // warps' A fragments
+            return static_cast<size_t>(kWarps) * kWideCols * kRedStride * sizeof(float) + kPaBytes;
         }
         return static_cast<size_t>(kWarps) * R * vec * 32 * sizeof(float);
     }
@@ -720,107 +928,194 @@ __device__ __forceinline__ void pass_b_rows(const Params& p, const LayerDesc& d,
     }
 }
 
-// Rank-lane variant of the second pass (R = 32): lane k owns rank index k
-// and warp w rows w, w + 8, ... of the tile.  For every sub-chunk of 32
-// columns and every worker a warp parks its M rows in its own slice of
-// shared memory (prefetching the next ones into registers) and accumulates,
-// in float32, M[i][c] * P_hat[i][k] for its 32 columns; at the end of a
-// sub-chunk the 8 warps' partials are summed in float64 in warp order.
-template <int R, bool SF>
-__device__ __forceinline__ void pass_b_wide(const Params& p, const LayerDesc& d, const TileCoord& tc,
-                                            float* const* ep, const float* ph_s, float* sm) {
-    static_assert(R == 32, "rank-lane kernels map one lane per rank index");
-    constexpr int RPL = kWideRows / kWarps;
+// Tensor-core variant of the second pass (R = 32).  Warps split as in the
+// first pass: a row group of 16 rows per warp, the row group's warps
+// ("parts") dealing the workers.  The Q partial of a sub-chunk is
+// D (32 ranks x 32 columns) = P_hat^T (ranks x rows) * M (rows x columns):
+// the A fragments (P_hat^T of the warp's rows, split into tf32 hi and lo)
+// are formed once per tile in shared memory; the B fragments are M itself,
+// loaded straight from global memory.  Column order: lane (g, t) loads
+// columns 4g .. 4g + 3 of the rows it needs, and n-tile j takes column
+// 4g + j as its column g.  D accumulates in float32 over the warp's rows
+// and workers (one sub-chunk at a time); the 8 warps' D are then summed in
+// float64 in warp order, as in the CUDA-core passes.
+
+// Row ii (tile row) of M for the 32 columns of a sub-chunk, in the lane's
+// four columns 4g .. 4g + 3 (zero outside the layer).
+template <int VEC>
+__device__ __forceinline__ void load_cols4(const float* rp, bool ok, int c, int cols, float (&x)[4]) {
+    x[0] = x[1] = x[2] = x[3] = 0.f;
+    if (!ok) return;
+    if constexpr (VEC == 4) {
+        if (c < cols) ld_f32<4>(rp + c, x);
+    } else if constexpr (VEC == 2) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            if (c + 2 * h < cols) {
+                float y[2];
+                ld_f32<2>(rp + c + 2 * h, y);
+                x[2 * h] = y[0];
+                x[2 * h + 1] = y[1];
+            }
+    } else {
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+            if (c + h < cols) x[h] = rp[c + h];
+    }
+}
+
+template <int VEC, bool SF>
+__device__ __forceinline__ void pass_b_mma(const Params& p, const LayerDesc& d, const TileCoord& tc,
+                                           float* const* ep, const float* ph_s, float* red_s) {
+    constexpr int R = 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int k = lane;
+    const int g = lane >> 2, t4 = lane & 3;
     const int W = p.workers;
-    const int64_t n = d.n, m = d.m;
+    const int64_t n = d.n;
     const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
-    const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), m - i0));
+    const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), d.m - i0));
     const int64_t jc = static_cast<int64_t>(tc.c) * d.slots * d.vec;
     const int width = static_cast<int>(min(static_cast<int64_t>(d.slots) * d.vec, n - jc));
     const int nsc = (width + kWideCols - 1) / kWideCols;
-    float* ms_w = sm + warp * RPL * kWideCols;               // parked rows
-    float* red_s = sm + kWideRows * kWideCols;               // [warp][column][k]
+    const int nrg = d.tm / kMmaRows;
+    const int parts = kWarps / nrg;
+    const int rg = warp % nrg, part = warp / nrg;
+    const int r0 = rg * kMmaRows;
     double* qpart = p.ws.qpart + d.qpart_off;
+    float4* pa = reinterpret_cast<float4*>(red_s + kWarps * kWideCols * kRedStride);   // [warp][ks][mt][lane][hi, lo]
 
-    float ph[RPL];
+    // A fragments of this warp: A[rank][row] = P_hat[r0 + row][rank], rows
+    // outside the layer zero; slot t <- row 8 ks + t, slot t + 4 <- row 8 ks + t + 4
 #pragma unroll
-    for (int t = 0; t < RPL; ++t) {
-        const int ii = warp + kWarps * t;
-        ph[t] = (ii < rows) ? ph_s[ii * R + k] : 0.f;
-    }
-    float mv_in[RPL];
-    auto load = [&](int it) {
-        const int sc = it / W, w = it - sc * W;
-        const int ncols = min(kWideCols, width - sc * kWideCols);
+    for (int ks = 0; ks < 2; ++ks)
 #pragma unroll
-        for (int t = 0; t < RPL; ++t) {
-            const int ii = warp + kWarps * t;
-            mv_in[t] = (ii < rows && lane < ncols) ? __ldcs(ep[w] + (i0 + ii) * n + jc + sc * kWideCols + lane) : 0.f;
-        }
-    };
-    const int total = nsc * W;
-    load(0);
-    float2 acc[kWideCols / 2];   // columns (2c, 2c + 1)
-    float msum[SF ? RPL : 1];
-    for (int it = 0; it < total; ++it) {
-        const int sc = it / W, w = it - sc * W;
-        if (w == 0) {
+        for (int mt = 0; mt < 2; ++mt) {
+            float av[4];
 #pragma unroll
-            for (int c = 0; c < kWideCols / 2; ++c) acc[c] = make_float2(0.f, 0.f);
-            if constexpr (SF) {
-#pragma unroll
-                for (int t = 0; t < RPL; ++t) msum[t] = 0.f;
+            for (int q = 0; q < 4; ++q) {
+                const int row = r0 + 8 * ks + t4 + 4 * (q >> 1);
+                const int rank = 16 * mt + g + 8 * (q & 1);
+                av[q] = row < rows ? ph_s[row * R + rank] : 0.f;
             }
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) tf32_split(av[q], hi[q], lo[q]);
+            float4* dst = pa + (((warp * 2 + ks) * 2 + mt) * 32 + lane) * 2;
+            dst[0] = make_float4(__uint_as_float(hi[0]), __uint_as_float(hi[1]), __uint_as_float(hi[2]),
+                                 __uint_as_float(hi[3]));
+            dst[1] = make_float4(__uint_as_float(lo[0]), __uint_as_float(lo[1]), __uint_as_float(lo[2]),
+                                 __uint_as_float(lo[3]));
         }
-        bool walk = true;
+    __syncwarp();
+
+    // this part's workers: part, part + parts, ...
+    const int nw = W > part ? (W - part + parts - 1) / parts : 0;
+    const int64_t row0 = (i0 + r0) * n + jc;
+    // the lane's rows: 8 ks + t4 and 8 ks + t4 + 4 (tile rows r0 + ...)
+    auto load = [&](int sc, int w, float (&mv)[2][2][4]) {
+        const int cols = width - sc * kWideCols;
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = 8 * ks + t4 + 4 * hh;
+                load_cols4<VEC>(ep[w] + row0 + static_cast<int64_t>(row) * n + sc * kWideCols, r0 + row < rows,
+                                4 * g, cols, mv[ks][hh]);
+            }
+    };
+
+    float cur[2][2][4], nxt[2][2][4];
+    float msum[SF ? 2 : 1][SF ? 2 : 1][SF ? 4 : 1];
+    if (nw > 0) load(0, part, nxt);
+    for (int sc = 0; sc < nsc; ++sc) {
+        float dacc[2][4][4];   // [m-tile][n-tile][fragment]
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) dacc[mt][nt][q] = 0.f;
         if constexpr (SF) {
 #pragma unroll
-            for (int t = 0; t < RPL; ++t) msum[t] += mv_in[t];
-            walk = (w == W - 1);
-            if (walk) {
+            for (int ks = 0; ks < 2; ++ks)
 #pragma unroll
-                for (int t = 0; t < RPL; ++t) ms_w[t * kWideCols + lane] = msum[t];
-            }
-        } else {
+                for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-            for (int t = 0; t < RPL; ++t) ms_w[t * kWideCols + lane] = mv_in[t];
+                    for (int j = 0; j < 4; ++j) msum[ks][hh][j] = 0.f;
         }
-        if (it + 1 < total) load(it + 1);
-        if (walk) {
-            __syncwarp();
+        for (int wi = 0; wi < nw; ++wi) {
 #pragma unroll
-            for (int t = 0; t < RPL; ++t) {
-                const float4* mrow = reinterpret_cast<const float4*>(ms_w + t * kWideCols);
-                const float2 pp = make_float2(ph[t], ph[t]);
+            for (int ks = 0; ks < 2; ++ks)
 #pragma unroll
-                for (int c4 = 0; c4 < kWideCols / 4; ++c4) {
-                    const float4 mv = mrow[c4];
-                    acc[2 * c4 + 0] = __ffma2_rn(make_float2(mv.x, mv.y), pp, acc[2 * c4 + 0]);
-                    acc[2 * c4 + 1] = __ffma2_rn(make_float2(mv.z, mv.w), pp, acc[2 * c4 + 1]);
+                for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) cur[ks][hh][j] = nxt[ks][hh][j];
+            // next (sub-chunk, worker) in flight while this block is multiplied
+            if (wi + 1 < nw) load(sc, part + (wi + 1) * parts, nxt);
+            else if (sc + 1 < nsc) load(sc + 1, part, nxt);
+            bool go = true;
+            if constexpr (SF) {
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            msum[ks][hh][j] += cur[ks][hh][j];
+                            cur[ks][hh][j] = msum[ks][hh][j];
+                        }
+                go = wi == nw - 1;
+            }
+            if (go) {
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                    // B fragments of the four n-tiles: b0 = row t4, b1 = row t4 + 4
+                    uint32_t bh[4][2], bl[4][2];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        tf32_split(cur[ks][0][j], bh[j][0], bl[j][0]);
+                        tf32_split(cur[ks][1][j], bh[j][1], bl[j][1]);
+                    }
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt) {
+                        const float4* src = pa + (((warp * 2 + ks) * 2 + mt) * 32 + lane) * 2;
+                        const float4 h4 = src[0], l4 = src[1];
+                        const uint32_t ahi[4] = {__float_as_uint(h4.x), __float_as_uint(h4.y), __float_as_uint(h4.z),
+                                                 __float_as_uint(h4.w)};
+                        const uint32_t alo[4] = {__float_as_uint(l4.x), __float_as_uint(l4.y), __float_as_uint(l4.z),
+                                                 __float_as_uint(l4.w)};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            mma_tf32(dacc[mt][j], alo, bh[j][0], bh[j][1]);
+                            mma_tf32(dacc[mt][j], ahi, bl[j][0], bl[j][1]);
+                            mma_tf32(dacc[mt][j], ahi, bh[j][0], bh[j][1]);
+                        }
+                    }
                 }
             }
-            __syncwarp();
         }
-        if (w == W - 1) {
-            // sub-chunk done: sum the warps' partials in warp order
+        // sub-chunk done: every warp's D to shared memory, then summed over
+        // the warps in warp order (float64) per (column, rank)
 #pragma unroll
-            for (int c = 0; c < kWideCols / 2; ++c) {
-                red_s[(warp * kWideCols + 2 * c) * R + k] = acc[c].x;
-                red_s[(warp * kWideCols + 2 * c + 1) * R + k] = acc[c].y;
-            }
-            __syncthreads();
-            const int ncols = min(kWideCols, width - sc * kWideCols);
-            for (int idx = tid; idx < ncols * R; idx += kThreads) {
-                const int c = idx / R, kk = idx % R;
-                double s2 = 0.0;
+        for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                for (int wp = 0; wp < kWarps; ++wp) s2 += static_cast<double>(red_s[(wp * kWideCols + c) * R + kk]);
-                qpart[(static_cast<int64_t>(tc.rb) * n + jc + sc * kWideCols + c) * R + kk] = s2;
-            }
-            __syncthreads();
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int rank = 16 * mt + g + 8 * (q >> 1);
+                    const int col = 4 * (2 * t4 + (q & 1)) + j;
+                    red_s[(warp * kWideCols + col) * kRedStride + rank] = dacc[mt][j][q];
+                }
+        __syncthreads();
+        const int ncols = min(kWideCols, width - sc * kWideCols);
+        for (int idx = tid; idx < ncols * R; idx += kThreads) {
+            const int c = idx / R, kk = idx % R;
+            double s2 = 0.0;
+#pragma unroll
+            for (int wp = 0; wp < kWarps; ++wp) s2 += static_cast<double>(red_s[(wp * kWideCols + c) * kRedStride + kk]);
+            qpart[(static_cast<int64_t>(tc.rb) * n + jc + sc * kWideCols + c) * R + kk] = s2;
         }
+        __syncthreads();
     }
 }
 
@@ -913,7 +1208,9 @@ __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_b(Params p)
     load_phat_rows<R>(p, d, tc, ph_s, T_s, tc.c == 0);
 
     if constexpr (IsWide<R>::value) {
-        pass_b_wide<R, SF>(p, d, tc, ep, ph_s, red_s);
+        if (d.vec == 4) pass_b_mma<4, SF>(p, d, tc, ep, ph_s, red_s);
+        else if (d.vec == 2) pass_b_mma<2, SF>(p, d, tc, ep, ph_s, red_s);
+        else pass_b_mma<1, SF>(p, d, tc, ep, ph_s, red_s);
     } else {
         if (d.vec == 4) {
             if constexpr (R <= 4) pass_b_rows<R, 4, SF>(p, d, tc, ep, ph_s, red_s);

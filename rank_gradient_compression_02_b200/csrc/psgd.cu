@@ -67,6 +67,7 @@ LayerDesc layer_geometry(int64_t m, int64_t n, int R, int workers, LayerSizes* s
     tm = (tm + 7) / 8 * 8;
     tm = std::max<int64_t>(8, std::min<int64_t>(tm, std::min(R >= 32 ? psgd::kWideRows : 512, kRowsFloatsMax / R)));
     tm = std::min<int64_t>(tm, (m + 7) / 8 * 8);
+    if (R >= 32) tm = tm <= 16 ? 16 : (tm <= 32 ? 32 : 64);   // whole 16-row groups of the tensor-core pass
     d.tm = static_cast<int>(tm);
     d.nrb = static_cast<int>((m + tm - 1) / tm);
     d.nsup = (d.nrb + psgd::kSuper - 1) / psgd::kSuper;
