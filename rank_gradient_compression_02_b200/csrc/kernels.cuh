@@ -107,7 +107,10 @@ __device__ void factor_gram_warp(const double* Gs, double* Rs, double* Ts, int* 
 // (mma.sync m16n8k8 tf32, a warp per 16 rows); passes B and C map one lane
 // per rank index.  Tiles of the wide kernels have 16, 32 or 64 rows.
 template <int R>
-struct IsWide { static constexpr bool value = R >= 32; };
+struct IsWide { static constexpr bool value = R >= 16; };   // pass C: the wide variant
+// passes A and B on the tensor cores (rank 16 and 32)
+template <int R>
+struct UseMma { static constexpr bool value = R >= 16; };
 constexpr int kWideCols = 32;
 constexpr int kWideRows = 64;    // rows per tile cap for the wide kernels
 
@@ -166,7 +169,7 @@ struct SmemA {
     // lazy reconstruction tile
     static __host__ __device__ size_t wide_bytes(int tm) {
         (void)tm;
-        return IsWide<R>::value ? kQfBytes + kRecBytes : 0;
+        return UseMma<R>::value ? kQfBytes + kRecBytes : 0;
     }
     static __host__ __device__ size_t total(int W, int tm) {
         return ((ptr_bytes(W) + 15) & ~size_t(15)) + ((rows_bytes(tm) + 15) & ~size_t(15)) +
@@ -441,11 +444,12 @@ __device__ __forceinline__ void store_frag(float* base, int64_t n, int g, int t4
     }
 }
 
-template <int VEC, typename GT, bool LAZY, bool SF, bool READM>
+template <int R, int VEC, typename GT, bool LAZY, bool SF, bool READM>
 __device__ __forceinline__ void pass_a_mma(const Params& p, const LayerDesc& d, const TileCoord& tc,
                                            const GT* const* gp, float* const* ep, const float* ph_prev,
                                            unsigned char* wide) {
-    constexpr int R = 32;
+    static_assert(R == 16 || R == 32, "tensor-core pass A: rank 16 or 32");
+    constexpr int NT = R / 8;                   // n-tiles of 8 ranks
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t4 = lane & 3;
     const int r = p.r;
@@ -468,8 +472,8 @@ __device__ __forceinline__ void pass_a_mma(const Params& p, const LayerDesc& d, 
     {
         const float* Q = p.t.q[tc.l];
         const int nks = nsc * 4;
-        for (int idx = threadIdx.x; idx < nks * 4 * 32; idx += kThreads) {
-            const int ln = idx & 31, nt = (idx >> 5) & 3, ksg = idx >> 7;
+        for (int idx = threadIdx.x; idx < nks * NT * 32; idx += kThreads) {
+            const int ln = idx & 31, nt = (idx >> 5) % NT, ksg = (idx >> 5) / NT;
             const int sc = ksg >> 2, ks = ksg & 3;
             const int jj0 = sc * kWideCols + frag_col0<VEC>(ks, ln & 3);
             const int jj1 = sc * kWideCols + frag_col1<VEC>(ks, ln & 3);
@@ -495,9 +499,9 @@ __device__ __forceinline__ void pass_a_mma(const Params& p, const LayerDesc& d, 
         if constexpr (!READM) load_frag<VEC>(gp[w] + row0 + sc * kWideCols, n, g, t4, ok_lo, ok_hi, cols, gq);
     };
 
-    double acc[4][4];
+    double acc[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[nt][c] = 0.0;
     float* rt = reinterpret_cast<float*>(wide + kQfBytes) + warp * (kMmaRows * kRecStride);
@@ -514,9 +518,9 @@ __device__ __forceinline__ void pass_a_mma(const Params& p, const LayerDesc& d, 
                 uint32_t ahi[4], alo[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) tf32_split(mv[ks][q], ahi[q], alo[q]);
-                const float4* qk = qf + ((sc * 4 + ks) * 4) * 32 + lane;
+                const float4* qk = qf + ((sc * 4 + ks) * NT) * 32 + lane;
 #pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
+                for (int nt = 0; nt < NT; ++nt) {
                     float c[4] = {0.f, 0.f, 0.f, 0.f};
                     mma_tf32x3(c, ahi, alo, qk[nt * 32]);
 #pragma unroll
@@ -597,25 +601,25 @@ __device__ __forceinline__ void pass_a_mma(const Params& p, const LayerDesc& d, 
 
     // parts' partials added in part order; part 0 writes the chunk's rows
     __syncthreads();   // every warp is done with the Q fragments
-    double* cb = reinterpret_cast<double*>(wide);   // [warp][16 values][lane]
+    double* cb = reinterpret_cast<double*>(wide);   // [warp][4 NT values][lane]
     if (part > 0) {
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) cb[(warp * 16 + nt * 4 + q) * 32 + lane] = acc[nt][q];
+            for (int q = 0; q < 4; ++q) cb[(warp * 4 * NT + nt * 4 + q) * 32 + lane] = acc[nt][q];
     }
     __syncthreads();
     if (part == 0) {
         for (int pp = 1; pp < parts; ++pp) {
             const int src = pp * nrg + rg;
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int q = 0; q < 4; ++q) acc[nt][q] += cb[(src * 16 + nt * 4 + q) * 32 + lane];
+                for (int q = 0; q < 4; ++q) acc[nt][q] += cb[(src * 4 * NT + nt * 4 + q) * 32 + lane];
         }
         double* ppart = p.ws.ppart + d.ppart_off;
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int ii = r0 + g + 8 * (q >> 1);
@@ -775,11 +779,15 @@ __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_a(Params p)
     }
     __syncthreads();
 
-    if constexpr (IsWide<R>::value) {
+    if constexpr (UseMma<R>::value) {
         unsigned char* wb = reinterpret_cast<unsigned char*>(wide);
-        if (d.vec == 4) pass_a_mma<4, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s, wb);
-        else if (d.vec == 2) pass_a_mma<2, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s, wb);
-        else pass_a_mma<1, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s, wb);
+        if (d.vec == 4) {
+            pass_a_mma<R, 4, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s, wb);
+        } else if (d.vec == 2) {
+            pass_a_mma<R, 2, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s, wb);
+        } else {
+            pass_a_mma<R, 1, GT, LAZY, SF, READM>(p, d, tc, gp, ep, rows_s, wb);
+        }
     } else {
         // VEC x R values of Q live in registers: VEC = 4 up to R = 4, 2 up to 16
         if (d.vec == 4) {
@@ -802,7 +810,7 @@ struct SmemB {
     static __host__ __device__ size_t rows_bytes(int tm) { return static_cast<size_t>(tm) * R * sizeof(float); }
     static __host__ __device__ size_t t_bytes() { return R * R * sizeof(double); }
     static __host__ __device__ size_t red_bytes(int vec) {
-        if (IsWide<R>::value) {
+        if (UseMma<R>::value) {
             // tensor-core kernel: warp partials (8 x 32 columns x 33) + the
             // warps' A fragments
             return static_cast<size_t>(kWarps) * kWideCols * kRedStride * sizeof(float) + kPaBytes;
@@ -964,10 +972,11 @@ __device__ __forceinline__ void load_cols4(const float* rp, bool ok, int c, int 
     }
 }
 
-template <int VEC, bool SF>
+template <int R, int VEC, bool SF>
 __device__ __forceinline__ void pass_b_mma(const Params& p, const LayerDesc& d, const TileCoord& tc,
                                            float* const* ep, const float* ph_s, float* red_s) {
-    constexpr int R = 32;
+    static_assert(R == 16 || R == 32, "tensor-core pass B: rank 16 or 32");
+    constexpr int MT = R / 16;                  // m-tiles of 16 ranks
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t4 = lane & 3;
     const int W = p.workers;
@@ -989,7 +998,7 @@ __device__ __forceinline__ void pass_b_mma(const Params& p, const LayerDesc& d, 
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks)
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
+        for (int mt = 0; mt < MT; ++mt) {
             float av[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -1000,7 +1009,7 @@ __device__ __forceinline__ void pass_b_mma(const Params& p, const LayerDesc& d, 
             uint32_t hi[4], lo[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) tf32_split(av[q], hi[q], lo[q]);
-            float4* dst = pa + (((warp * 2 + ks) * 2 + mt) * 32 + lane) * 2;
+            float4* dst = pa + (((warp * 2 + ks) * MT + mt) * 32 + lane) * 2;
             dst[0] = make_float4(__uint_as_float(hi[0]), __uint_as_float(hi[1]), __uint_as_float(hi[2]),
                                  __uint_as_float(hi[3]));
             dst[1] = make_float4(__uint_as_float(lo[0]), __uint_as_float(lo[1]), __uint_as_float(lo[2]),
@@ -1028,9 +1037,9 @@ __device__ __forceinline__ void pass_b_mma(const Params& p, const LayerDesc& d, 
     float msum[SF ? 2 : 1][SF ? 2 : 1][SF ? 4 : 1];
     if (nw > 0) load(0, part, nxt);
     for (int sc = 0; sc < nsc; ++sc) {
-        float dacc[2][4][4];   // [m-tile][n-tile][fragment]
+        float dacc[MT][4][4];   // [m-tile][n-tile][fragment]
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -1077,8 +1086,8 @@ __device__ __forceinline__ void pass_b_mma(const Params& p, const LayerDesc& d, 
                         tf32_split(cur[ks][1][j], bh[j][1], bl[j][1]);
                     }
 #pragma unroll
-                    for (int mt = 0; mt < 2; ++mt) {
-                        const float4* src = pa + (((warp * 2 + ks) * 2 + mt) * 32 + lane) * 2;
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const float4* src = pa + (((warp * 2 + ks) * MT + mt) * 32 + lane) * 2;
                         const float4 h4 = src[0], l4 = src[1];
                         const uint32_t ahi[4] = {__float_as_uint(h4.x), __float_as_uint(h4.y), __float_as_uint(h4.z),
                                                  __float_as_uint(h4.w)};
@@ -1097,7 +1106,7 @@ __device__ __forceinline__ void pass_b_mma(const Params& p, const LayerDesc& d, 
         // sub-chunk done: every warp's D to shared memory, then summed over
         // the warps in warp order (float64) per (column, rank)
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -1207,10 +1216,14 @@ __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_b(Params p)
     for (int w = threadIdx.x; w < W; w += kThreads) ep[w] = p.t.errors[w * L + l];
     load_phat_rows<R>(p, d, tc, ph_s, T_s, tc.c == 0);
 
-    if constexpr (IsWide<R>::value) {
-        if (d.vec == 4) pass_b_mma<4, SF>(p, d, tc, ep, ph_s, red_s);
-        else if (d.vec == 2) pass_b_mma<2, SF>(p, d, tc, ep, ph_s, red_s);
-        else pass_b_mma<1, SF>(p, d, tc, ep, ph_s, red_s);
+    if constexpr (UseMma<R>::value) {
+        if (d.vec == 4) {
+            pass_b_mma<R, 4, SF>(p, d, tc, ep, ph_s, red_s);
+        } else if (d.vec == 2) {
+            pass_b_mma<R, 2, SF>(p, d, tc, ep, ph_s, red_s);
+        } else {
+            pass_b_mma<R, 1, SF>(p, d, tc, ep, ph_s, red_s);
+        }
     } else {
         if (d.vec == 4) {
             if constexpr (R <= 4) pass_b_rows<R, 4, SF>(p, d, tc, ep, ph_s, red_s);
@@ -1238,7 +1251,7 @@ struct SmemC {
     }
 };
 
-// Rank-lane variant of the third pass (R = 16 or 32).  The tile's
+// Wide variant of the third pass (R = 16 or 32).  The tile's
 // reconstruction rec = P_hat Q_bar^T (rows x chunk width) is formed once
 // from shared memory (Q_bar transposed, float4 per lane) with the same
 // float32 operation order as recon_dot, then applied to every worker:
@@ -1333,7 +1346,39 @@ __device__ __forceinline__ void pass_c_wide(const Params& p, const LayerDesc& d,
                 }
             }
         }
-        for (int w = 0; w < W; ++w) apply(ep[w], [&](float& x, int v) { x = x - rec[s2][v]; });
+        // E' = M - rec for every worker: a group's loads all in flight
+        // before its stores (8, 4, 2, 1 workers at a time)
+        auto group = [&](auto GC, int w0) {
+            constexpr int G = decltype(GC)::value;
+            if (full4) {
+                float4 v[G];
+#pragma unroll
+                for (int u = 0; u < G; ++u) v[u] = *reinterpret_cast<const float4*>(ep[w0 + u] + base);
+#pragma unroll
+                for (int u = 0; u < G; ++u) {
+                    v[u].x -= rec[s2][0];
+                    v[u].y -= rec[s2][1];
+                    v[u].z -= rec[s2][2];
+                    v[u].w -= rec[s2][3];
+                    *reinterpret_cast<float4*>(ep[w0 + u] + base) = v[u];
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < G; ++u)
+                    for (int v = 0; v < nv; ++v) ep[w0 + u][base + v] = ep[w0 + u][base + v] - rec[s2][v];
+            }
+        };
+        int w = 0;
+        for (; w + 8 <= W; w += 8) group(std::integral_constant<int, 8>{}, w);
+        if (w + 4 <= W) {
+            group(std::integral_constant<int, 4>{}, w);
+            w += 4;
+        }
+        if (w + 2 <= W) {
+            group(std::integral_constant<int, 2>{}, w);
+            w += 2;
+        }
+        if (w < W) group(std::integral_constant<int, 1>{}, w);
     }
 }
 

@@ -34,8 +34,9 @@ int pad_rank(int r) {
 }
 
 // lanes load VEC adjacent columns (a chunk is up to 32 * VEC columns); the
-// lane-per-column kernels keep VEC x R values of Q per lane in registers
-int max_vec_for_rank(int R) { return R <= 4 ? 4 : (R <= 16 ? 2 : 4); }
+// lane-per-column kernels (rank <= 8) keep VEC x R values of Q per lane in
+// registers, the tensor-core and wide kernels (rank 16, 32) do not
+int max_vec_for_rank(int R) { return R <= 4 ? 4 : (R <= 8 ? 2 : 4); }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -65,9 +66,9 @@ LayerDesc layer_geometry(int64_t m, int64_t n, int R, int workers, LayerSizes* s
     const int64_t cols = static_cast<int64_t>(d.slots) * d.vec;
     int64_t tm = (kTileTargetElems + cols * workers - 1) / (cols * workers);
     tm = (tm + 7) / 8 * 8;
-    tm = std::max<int64_t>(8, std::min<int64_t>(tm, std::min(R >= 32 ? psgd::kWideRows : 512, kRowsFloatsMax / R)));
+    tm = std::max<int64_t>(8, std::min<int64_t>(tm, std::min(R >= 16 ? psgd::kWideRows : 512, kRowsFloatsMax / R)));
     tm = std::min<int64_t>(tm, (m + 7) / 8 * 8);
-    if (R >= 32) tm = tm <= 16 ? 16 : (tm <= 32 ? 32 : 64);   // whole 16-row groups of the tensor-core pass
+    if (R >= 16) tm = tm <= 16 ? 16 : (tm <= 32 ? 32 : 64);   // whole 16-row groups of the tensor-core passes
     d.tm = static_cast<int>(tm);
     d.nrb = static_cast<int>((m + tm - 1) / tm);
     d.nsup = (d.nrb + psgd::kSuper - 1) / psgd::kSuper;
