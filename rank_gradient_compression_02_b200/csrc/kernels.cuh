@@ -155,8 +155,8 @@ constexpr int kMaxKSteps = 32 * 4 / 8;        // k-steps of 8 columns in the wid
 constexpr size_t kQfBytes = static_cast<size_t>(kMaxKSteps) * 4 * 32 * sizeof(float4);
 constexpr int kRedStride = 32 + 1;            // second pass: warp partial row stride (floats)
 constexpr size_t kPaBytes = static_cast<size_t>(kWarps) * 2 * 2 * 32 * 8 * sizeof(float);   // its A fragments
-constexpr int kRecStride = kWideCols + 1;     // lazy reconstruction tile row stride (floats)
-constexpr size_t kRecBytes = static_cast<size_t>(kWarps) * kMmaRows * kRecStride * sizeof(float);
+constexpr int kRecStride = 4 * kWideCols + 1;  // lazy reconstruction tile row stride (floats)
+constexpr size_t kRecBytes = static_cast<size_t>(kWideRows) * kRecStride * sizeof(float);
 
 template <int R>
 struct SmemA {
@@ -165,15 +165,14 @@ struct SmemA {
     static __host__ __device__ size_t rows_bytes(int tm) { return static_cast<size_t>(tm) * R * sizeof(double); }
     static __host__ __device__ size_t fac_bytes() { return 3 * R * R * sizeof(double) + 2 * R * sizeof(int) + 64; }
     // tensor-core kernel: the chunk's split Q fragments (later the parts'
-    // P partials, kWarps x 16 x 32 doubles, the same 32 KB) and every warp's
-    // lazy reconstruction tile
-    static __host__ __device__ size_t wide_bytes(int tm) {
-        (void)tm;
-        return UseMma<R>::value ? kQfBytes + kRecBytes : 0;
+    // P partials, kWarps x 16 x 32 doubles, the same 32 KB) and, in the
+    // lazy representation, the tile's reconstruction
+    static __host__ __device__ size_t wide_bytes(bool lazy) {
+        return UseMma<R>::value ? kQfBytes + (lazy ? kRecBytes : 0) : 0;
     }
-    static __host__ __device__ size_t total(int W, int tm) {
+    static __host__ __device__ size_t total(int W, int tm, bool lazy) {
         return ((ptr_bytes(W) + 15) & ~size_t(15)) + ((rows_bytes(tm) + 15) & ~size_t(15)) +
-               ((fac_bytes() + 15) & ~size_t(15)) + wide_bytes(tm);
+               ((fac_bytes() + 15) & ~size_t(15)) + wide_bytes(lazy);
     }
 };
 
@@ -504,8 +503,30 @@ __device__ __forceinline__ void pass_a_mma(const Params& p, const LayerDesc& d, 
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[nt][c] = 0.0;
-    float* rt = reinterpret_cast<float*>(wide + kQfBytes) + warp * (kMmaRows * kRecStride);
+    float* rt = reinterpret_cast<float*>(wide + kQfBytes);   // lazy: [tile row][chunk column]
     float msum[SF ? 4 : 1][SF ? 4 : 1];
+    if constexpr (LAZY) {
+        // the previous step's reconstruction of the whole tile (every row
+        // and every column slot, zero beyond the chunk), once, by all
+        // threads: recon_dot's operation order per element, two columns
+        // per packed FMA
+        const float* Qb = p.ws.qbar + d.qrow_off;
+        const int c0 = 2 * (threadIdx.x & 63), rq = threadIdx.x >> 6;
+        const bool ok0 = c0 < width && p.use_prev, ok1 = c0 + 1 < width && p.use_prev;
+        float2 qp[R];
+#pragma unroll
+        for (int kk = 0; kk < R; ++kk)
+            qp[kk] = make_float2(ok0 ? Qb[(jc + c0) * R + kk] : 0.f, ok1 ? Qb[(jc + c0 + 1) * R + kk] : 0.f);
+        for (int ii = rq; ii < d.tm; ii += 4) {
+            const float* ph = ph_prev + min(ii, rows - 1) * R;
+            float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int kk = 0; kk < R; ++kk) s2 = __ffma2_rn(make_float2(ph[kk], ph[kk]), qp[kk], s2);
+            rt[ii * kRecStride + c0] = s2.x;
+            rt[ii * kRecStride + c0 + 1] = s2.y;
+        }
+        __syncthreads();
+    }
 
     // products of an M block (fragment order) with the sub-chunk's k-steps
     auto multiply = [&](int sc, const float (&mv)[4][4]) {
@@ -536,24 +557,6 @@ __device__ __forceinline__ void pass_a_mma(const Params& p, const LayerDesc& d, 
         const int w = part + wi * parts;
         const int cols = width - sc * kWideCols;
         if (wi == 0) {
-            if constexpr (LAZY) {
-                // the previous step's reconstruction of the block (lane =
-                // column), in recon_dot's operation order, parked in rt
-                const float* Qb = p.ws.qbar + d.qrow_off;
-                const bool okc = lane < cols && p.use_prev;
-                float qp[R];
-#pragma unroll
-                for (int kk = 0; kk < R; ++kk) qp[kk] = okc ? Qb[(jc + sc * kWideCols + lane) * R + kk] : 0.f;
-                __syncwarp();
-                for (int tt = 0; tt < kMmaRows; ++tt) {
-                    const int ii = min(r0 + tt, rows - 1);
-                    float s2 = 0.f;
-#pragma unroll
-                    for (int kk = 0; kk < R; ++kk) s2 = fmaf(ph_prev[ii * R + kk], qp[kk], s2);
-                    rt[tt * kRecStride + lane] = s2;
-                }
-                __syncwarp();
-            }
             if constexpr (SF) {
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
@@ -571,7 +574,7 @@ __device__ __forceinline__ void pass_a_mma(const Params& p, const LayerDesc& d, 
                 if constexpr (!READM) {
                     if constexpr (LAZY) {
                         const int c = (q & 2) ? frag_col1<VEC>(ks, t4) : frag_col0<VEC>(ks, t4);
-                        x = x - rt[(g + 8 * (q & 1)) * kRecStride + c];
+                        x = x - rt[(r0 + g + 8 * (q & 1)) * kRecStride + sc * kWideCols + c];
                     }
                     x = gq[ks][q] + x;
                 }

@@ -284,10 +284,10 @@ void* kernel_ptr(int which, int R, int dtype, bool lazy, bool sf) {
 #undef PSGD_CASE
 }
 
-size_t smem_need(int which, int R, int W, int tm, int vec) {
+size_t smem_need(int which, int R, int W, int tm, int vec, bool lazy = false) {
 #define PSGD_CASE(RR)                                                         \
     case RR:                                                                  \
-        if (which == 0 || which == 3) return psgd::SmemA<RR>::total(W, tm);   \
+        if (which == 0 || which == 3) return psgd::SmemA<RR>::total(W, tm, lazy); \
         if (which == 1) return psgd::SmemB<RR>::total(W, tm, vec);            \
         return psgd::SmemC<RR>::total(W, tm);
     switch (R) {
@@ -406,7 +406,7 @@ int psgd_create(psgd_ctx** out, const psgd_layer* layers, int num_layers, int ra
         cnt += sz.cnt;
         for (int64_t t = 0; t < sz.tiles; ++t) tile_layer.push_back(l);
         ctx->desc.push_back(d);
-        ctx->smem_a = std::max(ctx->smem_a, smem_need(0, R, workers, d.tm, d.vec));
+        ctx->smem_a = std::max(ctx->smem_a, smem_need(0, R, workers, d.tm, d.vec, (flags & PSGD_FLAG_LAZY_ERRORS) != 0));
         ctx->smem_b = std::max(ctx->smem_b, smem_need(1, R, workers, d.tm, d.vec));
         ctx->smem_c = std::max(ctx->smem_c, smem_need(2, R, workers, d.tm, d.vec));
     }
