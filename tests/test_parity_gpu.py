@@ -29,7 +29,7 @@ def test_mixed_shapes_f32(rank, workers):
         H.assert_close(e, H.TOL["f32"], f"step {t}")
 
 
-@pytest.mark.parametrize("rank", [1, 4, 16])
+@pytest.mark.parametrize("rank", [1, 4, 16, 32])
 def test_mixed_shapes_bf16(rank):
     wl = H.small_workload(MIXED, rank, 4, dtype="bf16")
     _, _, hist = H.run_free(wl, steps=3)
@@ -40,7 +40,7 @@ def test_mixed_shapes_bf16(rank):
         H.assert_close(e, 1e-4, f"step {t} (fp32-level)")
 
 
-@pytest.mark.parametrize("rank", [2, 8])
+@pytest.mark.parametrize("rank", [2, 8, 16, 32])
 def test_sixteen_workers(rank):
     wl = H.small_workload(MIXED[:4], rank, 16)
     _, _, hist = H.run_free(wl, steps=2)
@@ -48,17 +48,19 @@ def test_sixteen_workers(rank):
         H.assert_close(e, H.TOL["f32"], f"step {t}")
 
 
+@pytest.mark.parametrize("rank", [4, 16, 32])
 @pytest.mark.parametrize("lazy,sum_first", [(True, False), (False, True), (True, True)])
-def test_modes(lazy, sum_first):
-    wl = H.small_workload(MIXED, 4, 3)
+def test_modes(lazy, sum_first, rank):
+    wl = H.small_workload(MIXED, rank, 3)
     _, _, hist = H.run_free(wl, steps=4, lazy=lazy, sum_first=sum_first)
     for t, e in enumerate(hist):
         H.assert_close(e, H.TOL["f32"], f"step {t}")
 
 
-@pytest.mark.parametrize("iters,lazy", [(2, False), (3, False), (2, True)])
-def test_power_iterations(iters, lazy):
-    wl = H.small_workload(MIXED, 4, 3)
+@pytest.mark.parametrize("iters,lazy,rank", [(2, False, 4), (3, False, 4), (2, True, 4), (2, False, 32),
+                                             (2, True, 16)])
+def test_power_iterations(iters, lazy, rank):
+    wl = H.small_workload(MIXED, rank, 3)
     run, _, hist = H.run_free(wl, steps=3, lazy=lazy, iters=iters)
     assert run.lib.step_launches == 2 * iters + (0 if lazy else 1)
     for t, e in enumerate(hist):
@@ -159,11 +161,13 @@ def test_bitwise_deterministic():
             assert torch.equal(a.E[w][l], b.E[w][l])
 
 
-def test_lazy_equals_eager_bitwise():
+@pytest.mark.parametrize("rank", [4, 16, 32])
+def test_lazy_equals_eager_bitwise(rank):
     # E' = M - P_hat Q_bar^T rebuilt in the next step's first pass is the
     # same float32 arithmetic as the eager residual, so the runs agree bit
-    # for bit
-    wl = H.small_workload(MIXED, 4, 3)
+    # for bit (ranks 16, 32: the tensor-core first pass rebuilds it on the
+    # CUDA cores in the residual pass's order)
+    wl = H.small_workload(MIXED, rank, 3)
     a = _run_steps(wl, 4, lazy=False)
     b = _run_steps(wl, 4, lazy=True)
     for l in range(len(wl.layers)):
@@ -397,6 +401,14 @@ def test_many_workers():
     _, _, hist = H.run_free(wl, steps=2)
     for t, e in enumerate(hist):
         H.assert_close(e, H.TOL["f32"], f"step {t}")
+
+
+@pytest.mark.parametrize("workers", [64, 256])
+def test_many_workers_rank32(workers):
+    # the tensor-core passes with 16-row tiles and every warp a worker part
+    wl = H.small_workload([(40, 130), (33, 37), (64, 576)], 32, workers)
+    _, _, hist = H.run_free(wl, steps=1)
+    H.assert_close(hist[0], H.TOL["f32"], "step 0")
 
 
 def test_max_workers_single_row():
