@@ -867,7 +867,9 @@ __device__ __forceinline__ void pass_b_rows(const Params& p, const LayerDesc& d,
     const int ns = min(d.slots, d.nvec - s0);
     const bool active = lane < ns;
     const int64_t j = static_cast<int64_t>(s0 + (active ? lane : 0)) * VEC;
-    constexpr int U = 8;   // 8 workers' loads in flight per lane (pass B only reads)
+    // pass B only reads: 128 bytes of loads in flight per lane (8, 16 or 32
+    // workers for 16-, 8- and 4-byte lanes)
+    constexpr int U = 32 / VEC;
 
     float qacc[VEC][R];
 #pragma unroll
@@ -875,7 +877,45 @@ __device__ __forceinline__ void pass_b_rows(const Params& p, const LayerDesc& d,
 #pragma unroll
         for (int k = 0; k < R; ++k) qacc[v][k] = 0.f;
 
-    if (active) {
+    if (active && W <= 4) {
+        // few workers: two rows' loads in flight together, then the
+        // products in the same order as the loop below (row, then worker)
+        for (int64_t i = i0 + warp; i < i1; i += 2 * kWarps) {
+            const bool two = i + kWarps < i1;
+            float e[2][4][VEC];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (u < W && (h == 0 || two)) ld_f32<VEC>(ep[u] + (i + h * kWarps) * n + j, e[h][u]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (h == 1 && !two) break;
+                float ph[R];
+#pragma unroll
+                for (int k = 0; k < R; ++k) ph[k] = ph_s[(i + h * kWarps - i0) * R + k];
+                float msum[VEC];
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) msum[v] = 0.f;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (u < W) {
+                        if constexpr (SF) {
+#pragma unroll
+                            for (int v = 0; v < VEC; ++v) msum[v] += e[h][u][v];
+                        } else {
+#pragma unroll
+                            for (int v = 0; v < VEC; ++v) axpy<R>(qacc[v], e[h][u][v], ph);
+                        }
+                    }
+                }
+                if constexpr (SF) {
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) axpy<R>(qacc[v], msum[v], ph);
+                }
+            }
+        }
+    } else if (active) {
         for (int64_t i = i0 + warp; i < i1; i += kWarps) {
             float ph[R];
 #pragma unroll
@@ -903,6 +943,18 @@ __device__ __forceinline__ void pass_b_rows(const Params& p, const LayerDesc& d,
             };
             int w = 0;
             for (; w + U <= W; w += U) group(std::integral_constant<int, U>{}, w);
+            if constexpr (U > 16) {
+                if (w + 16 <= W) {
+                    group(std::integral_constant<int, 16>{}, w);
+                    w += 16;
+                }
+            }
+            if constexpr (U > 8) {
+                if (w + 8 <= W) {
+                    group(std::integral_constant<int, 8>{}, w);
+                    w += 8;
+                }
+            }
             if (w + 4 <= W) {
                 group(std::integral_constant<int, 4>{}, w);
                 w += 4;
