@@ -44,13 +44,38 @@ def _peaks():
     return 6650.0, "fallback"
 
 
-def _kernel_source_hash() -> str:
+def _code_tokens(text: str) -> str:
+    """C++/CUDA source without comments and with whitespace collapsed: what
+    the compiler sees, so that editing a comment keeps the hash."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":                       # string or character literal
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
+def _kernel_source_hash(csrc: str = None) -> str:
+    """Hash of the CUDA sources' code (comments and layout ignored)."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "rank_gradient_compression_02_b200", "csrc")
+    csrc = csrc or os.path.join(ROOT, "rank_gradient_compression_02_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(_code_tokens(f.read()).encode())
     return h.hexdigest()[:16]
 
 

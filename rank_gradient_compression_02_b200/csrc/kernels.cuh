@@ -102,15 +102,16 @@ __device__ void factor_gram_warp(const double* Gs, double* Rs, double* Ts, int* 
 // ---------------------------------------------------------------------------
 // pass A
 
-// Rank 32 uses the wide kernels: a chunk (up to 32 * VEC columns) is walked
-// in sub-chunks of 32 columns.  Pass A forms M * Q on the tensor cores
-// (mma.sync m16n8k8 tf32, a warp per 16 rows); passes B and C map one lane
-// per rank index.  Tiles of the wide kernels have 16, 32 or 64 rows.
+// Ranks 16 and 32 use the wide kernels: a chunk (up to 32 * VEC columns) is
+// walked in sub-chunks of 32 columns.  Passes A and B form M * Q and
+// P_hat^T * M on the tensor cores (mma.sync m16n8k8 tf32, a warp per 16
+// rows); pass C forms the reconstruction once per tile on the CUDA cores
+// and applies it to every worker.  Tiles of the wide kernels have 16, 32 or
+// 64 rows.
 template <int R>
 struct IsWide { static constexpr bool value = R >= 16; };   // pass C: the wide variant
-// passes A and B on the tensor cores (rank 16 and 32)
 template <int R>
-struct UseMma { static constexpr bool value = R >= 16; };
+struct UseMma { static constexpr bool value = R >= 16; };   // passes A and B: tensor cores
 constexpr int kWideCols = 32;
 constexpr int kWideRows = 64;    // rows per tile cap for the wide kernels
 
