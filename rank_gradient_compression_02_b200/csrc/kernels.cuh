@@ -1775,8 +1775,17 @@ __global__ void k_vec_mean(const float* const* vecs, float* const* out, const in
     float* mo = (mom != nullptr) ? mom[k] : nullptr;
     for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < nk;
          e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        // workers summed in order; eight workers' loads in flight at a time
         float s = 0.f;
-        for (int w = 0; w < W; ++w) s += vecs[w * count + k][e];
+        int w = 0;
+        for (; w + 8 <= W; w += 8) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = vecs[(w + u) * count + k][e];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) s += v[u];
+        }
+        for (; w < W; ++w) s += vecs[w * count + k][e];
         const float g = s * inv_w;
         o[e] = g;
         if (x != nullptr && mo != nullptr) {
