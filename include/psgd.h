@@ -29,8 +29,11 @@
  * pages say nothing about rank deficiency; this is the rule the float64
  * oracle uses too).  NaN inputs propagate; they are not trapped.
  *
- * Precision: G is float32 or bfloat16; E, Q, P_hat, Q_bar, G_hat and all
- * accumulation are float32, Gram and Cholesky float64.
+ * Precision: G is float32 or bfloat16; E, Q, P_hat, Q_bar and G_hat are
+ * float32.  Products are float32 (ranks 16 and 32: tf32 tensor-core
+ * products of hi/lo-split factors, relative error below 2^-21), summed in
+ * float32 over short runs and then in float64; P_bar, the Gram matrix, its
+ * Cholesky factor and every partial sum across CTAs are float64.
  *
  * Ownership: the caller owns every tensor passed in (device memory, e.g.
  * PyTorch tensors).  The library owns its workspace and pointer tables,
