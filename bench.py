@@ -44,6 +44,27 @@ def _peaks():
     return 6650.0, "fallback"
 
 
+def compute_roofline(elements: int, rank: int, pass_a_ms: float, pass_b_ms: float, sm_mhz: float,
+                     bf16_tflops: float, sum_first: bool = False, workers: int = 1) -> dict:
+    """Compute side of the first two passes (the two products): their
+    algorithmic flops (2 r per worker element each; 2 r per matrix element
+    for the first pass with sum-first) per second of the two passes, against
+    the fp32 CUDA-core ceiling (148 SMs x 128 FMA lanes x 2 flop x SM clock)
+    and the tf32 tensor-core ceiling (the measured bf16 GEMM peak x the
+    nominal tf32 / bf16 ratio 1.1 / 2.25).  The tensor-core passes run three
+    split products per term, which this does not count."""
+    flops = 2 * rank * elements * (1.0 / workers if sum_first else 1.0) + 2 * rank * elements
+    sec = (pass_a_ms + pass_b_ms) * 1e-3
+    achieved = flops / sec / 1e12 if sec > 0 else 0.0
+    fp32_peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+    tf32_peak = bf16_tflops * 1.1 / 2.25
+    return {"unit": "TFLOP/s", "achieved": round(achieved, 2),
+            "fp32_cuda_core_peak": round(fp32_peak, 1), "fp32_frac": round(achieved / fp32_peak, 4),
+            "tf32_tensor_peak": round(tf32_peak, 1), "tf32_frac": round(achieved / tf32_peak, 4),
+            "note": "products of passes A and B only; ranks 16 and 32 run them on the tf32 tensor cores "
+                    "(mma.sync, three split products per term), ranks <= 8 on the CUDA cores"}
+
+
 def _code_tokens(text: str) -> str:
     """C++/CUDA source without comments and with whitespace collapsed: what
     the compiler sees, so that editing a comment keeps the hash."""
@@ -447,6 +468,17 @@ def main():
                 "peak_kind": f"{peak_kind} hbm_gbs",
                 "per_kernel_ms": {n: round(t, 4) for n, t in zip(names, per_launch_ms)},
                 "step_algorithmic_frac": round(step_min_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 4)}
+    if r >= 16:
+        # at ranks 16 and 32 the first two passes are bound by instruction
+        # issue, not HBM: report their compute side too
+        pk = {}
+        pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+        if os.path.exists(pp):
+            with open(pp) as f:
+                pk = json.load(f)
+        sm_mhz = (clk or {}).get("sm_mhz") or pk.get("sm_max_mhz", 1965.0)
+        roofline["compute"] = compute_roofline(wl.elements, r, per_launch_ms[0], per_launch_ms[1], sm_mhz,
+                                               pk.get("bf16_tflops", 1590.0), args.sum_first, wl.workers)
 
     # the lazy-error representation of the same step (E' rebuilt inside the
     # next step's first pass; bit-identical results), timed the same way

@@ -40,3 +40,17 @@ def test_committed_traffic_belongs_to_the_current_kernels():
     # still dirty in L2 at the end of the kernel)
     alg = 178_601_984 * 12
     assert 0.9 * alg < rec["dram_bytes_per_launch"] < 1.05 * alg
+
+
+def test_compute_roofline_arithmetic():
+    # 1e9 worker elements, r = 32, both passes 1 ms: 2 * 32 * 1e9 flop per
+    # pass -> 128 GFLOP in 2 ms = 64 TFLOP/s; fp32 ceiling at 2 GHz
+    # 148 * 128 * 2 * 2e9 = 75.8 TFLOP/s; tf32 ceiling 1600 * 1.1 / 2.25
+    c = bench.compute_roofline(10**9, 32, 1.0, 1.0, 2000.0, 1600.0)
+    assert abs(c["achieved"] - 64.0) < 1e-6
+    assert abs(c["fp32_cuda_core_peak"] - 75.8) < 0.05
+    assert abs(c["tf32_tensor_peak"] - 782.2) < 0.05
+    assert abs(c["fp32_frac"] - 64.0 / 75.776) < 1e-3
+    # sum-first: the first pass multiplies each matrix element once, not once per worker
+    s = bench.compute_roofline(10**9, 32, 1.0, 1.0, 2000.0, 1600.0, sum_first=True, workers=8)
+    assert abs(s["achieved"] - (2 * 32 * 1e9 / 8 + 2 * 32 * 1e9) / 2e-3 / 1e12) < 1e-6
