@@ -103,7 +103,9 @@ enum {
 typedef struct { int64_t m, n; } psgd_layer;   /* one gradient matrix */
 typedef struct psgd_ctx psgd_ctx;              /* opaque */
 
-/* Create a context on the current CUDA device.
+/* Create a context on the current CUDA device (the pages define no
+ * interface; a context holds what note-152 "Method" keeps between steps
+ * besides the caller's E and Q: P_hat and Q_bar of the last step).
  * layers[num_layers]: matrix shapes, m >= 1, n >= 1 (num_layers may be 0:
  *   every step is then a no-op).
  * rank: 1 <= rank <= 32 and rank <= min(m, n) for every layer.
@@ -115,6 +117,8 @@ typedef struct psgd_ctx psgd_ctx;              /* opaque */
 PSGD_API int psgd_create(psgd_ctx **out, const psgd_layer *layers, int num_layers, int rank, int workers,
                 uint64_t seed, int grad_dtype, unsigned flags);
 
+/* Release the context's workspace, tables and staging (NULL is a no-op);
+ * waits for the device first. */
 PSGD_API void psgd_destroy(psgd_ctx *ctx);
 
 /* Draw Q0 ~ N(0, 1) for every layer into q[l] (device, n x rank float32,
@@ -124,7 +128,8 @@ PSGD_API void psgd_destroy(psgd_ctx *ctx);
  * The initial Q is not orthogonalised and is shared by all workers. */
 PSGD_API int psgd_init_q(psgd_ctx *ctx, float *const *q, void *stream);
 
-/* One compression step for all layers and workers.
+/* One compression step for all layers and workers: the sequence of
+ * note-152 "Method" listed at the top of this file.
  * grads[w*L + l]:  device, m x n, grad dtype, read only.
  * errors[w*L + l]: device, m x n float32, E_w in, E'_w out (in place).  With
  *                  PSGD_FLAG_LAZY_ERRORS: M_w out (see the flag).
@@ -137,7 +142,8 @@ PSGD_API int psgd_init_q(psgd_ctx *ctx, float *const *q, void *stream);
 PSGD_API int psgd_step(psgd_ctx *ctx, const void *const *grads, float *const *errors, float *const *q,
               float *const *p_hat, float *const *recon, void *stream);
 
-/* The same step with HOST gradients: grads_host[w*L + l] are host pointers
+/* The same step with HOST gradients (an interface variant of psgd_step; no
+ * counterpart in the pages): grads_host[w*L + l] are host pointers
  * (pinned for asynchronous copies; pageable works but serialises).  The
  * library copies them into a device staging area it owns (allocated on
  * first use), runs psgd_step, and copies P_hat and Q_bar back to
@@ -160,8 +166,9 @@ PSGD_API int psgd_step_host_flat(psgd_ctx *ctx, const void *const *grads_host, c
                                  float *const *q_host, void *stream);
 
 /* PSGD_FLAG_LAZY_ERRORS only: write E'_w = M_w - P_hat Q_bar^T (from the
- * last step) into errors[w*L + l] in place.  The next step then starts from
- * E'_w as in the eager mode. */
+ * last step; the residual of note-152 "Concepts") into errors[w*L + l] in
+ * place.  The next step then starts from E'_w as in the eager mode.
+ * PSGD_ERR_STATE for a context without the flag. */
 PSGD_API int psgd_materialize_errors(psgd_ctx *ctx, float *const *errors, void *stream);
 
 /* Post-compression momentum (note-152, "Concepts"): for every layer, with
@@ -181,7 +188,8 @@ PSGD_API int psgd_momentum_step(psgd_ctx *ctx, float *const *params, float *cons
 PSGD_API int psgd_vec_mean(psgd_ctx *ctx, const float *const *vecs, float *const *out, const int64_t *len, int count,
                   float *const *params, float *const *mom, float lr, float beta, void *stream);
 
-/* Synchronise the last stream used and read the device status word:
+/* Service calls (no counterpart in the pages).
+ * Synchronise the last stream used and read the device status word:
  * PSGD_OK, or PSGD_ERR_DEVICE if a kernel flagged an inconsistency (e.g.
  * overlapping steps on one context), or PSGD_ERR_CUDA if a launch failed. */
 PSGD_API int psgd_status(psgd_ctx *ctx);
