@@ -273,9 +273,30 @@ def check_svd_refresh(ora):
     np.testing.assert_allclose(deep["G_hat"], o["G_hat"], atol=1e-9)
 
 
+def check_subspace_sin_max(ora):
+    """Principal angles by construction: with [U V] orthonormal, the
+    columns u_i cos t_i + v_i sin t_i span a subspace at angles t_i from
+    span(U); the largest sine must come back, also for a tiny angle (the
+    reason the oracle takes the spectral norm of the off-span part rather
+    than sqrt(1 - cos^2))."""
+    rng = np.random.default_rng(11)
+    n, r = 40, 3
+    B, _ = np.linalg.qr(rng.standard_normal((n, 2 * r)))
+    U, V = B[:, :r], B[:, r:]
+    for angles in ([0.3, 0.1, 0.05], [1e-9, 2e-9, 5e-10], [0.0, 0.0, 0.0], [np.pi / 2, 0.2, 0.1]):
+        t = np.array(angles)
+        P = U * np.cos(t) + V * np.sin(t)
+        # a rotation inside the span changes the basis, not the subspace
+        Rm, _ = np.linalg.qr(rng.standard_normal((r, r)))
+        got = ora.subspace_sin_max(U, P @ Rm)
+        want = float(np.max(np.sin(t)))
+        assert abs(got - want) <= 1e-12 + 1e-6 * want, (angles, got, want)
+
+
 ALL_CHECKS = [
     check_hand_cases, check_gram_schmidt_vs_householder, check_gram_schmidt_rank_deficient,
     check_rank1_closed_form, check_exact_low_rank, check_identities, check_linearity,
     check_jacobi_svd, check_warm_start_convergence, check_error_feedback_telescopes,
     check_momentum_closed_form, check_vec_mean, check_power_iterations, check_svd_refresh,
+    check_subspace_sin_max,
 ]
