@@ -26,6 +26,8 @@ pytestmark = pytest.mark.gpu
     (129, 1000, 2, 2, "f32"),
     (96, 130, 8, 4, "bf16"),
     (33, 37, 1, 1, "f32"),
+    (129, 1000, 32, 3, "f32"),    # the tensor-core passes, 16-byte lanes
+    (300, 650, 16, 2, "f32"),     # the tensor-core passes, 8-byte lanes
 ])
 def test_static_step_matches_context_step(m, n, rank, workers, dtype):
     wl = Workload(name="noalloc", layers=((m, n),), rank=rank, workers=workers, steps=2, grad_dtype=dtype)
