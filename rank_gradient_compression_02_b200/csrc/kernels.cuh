@@ -11,9 +11,11 @@
 //           G_hat = rec, optional momentum.
 //
 // Step order from "anthology-of-the-sota" note-152 on PowerSGD, "Method".
-// Every cross-CTA sum runs in a fixed order, so results are bitwise
-// reproducible.  No CTA waits on another: the last CTA to arrive at a
-// counter does the reduction.
+// At ranks 16 and 32 the two products of passes A and B run on the tf32
+// tensor cores (mma.sync, hi/lo-split factors); pass C and every other
+// rank use the CUDA cores.  Every cross-CTA sum runs in a fixed order, so
+// results are bitwise reproducible.  No CTA waits on another: the last CTA
+// to arrive at a counter does the reduction.
 #pragma once
 
 #include "device_common.cuh"
