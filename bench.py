@@ -7,9 +7,17 @@ HBM: psgd_step (error-feedback add, P = MQ, worker mean, orthogonalisation,
 Q = M^T P_hat, worker mean, residual), the uncompressed mean of the 1-D
 tensors and the post-compression momentum update, all through the C ABI.
 Metric: gradient elements compressed per second (W * sum(m*n) per step),
-whole job; with N GPUs each rank runs an independent replica (the method's
-workers are simulated on one GPU) and value = N * elements / max-over-ranks
-time.  Rank 0 prints one JSON line.
+whole job.  On one GPU the W workers are replica buffers and the worker
+means are on-device sums.  With N GPUs (torchrun, NCCL) every rank holds W
+workers and runs the distributed step: the P and Q partial sums (and the
+1-D gradients) are all-reduced between the library's three calls, so the
+job has N * W workers (weak scaling) and value = N * elements / max over
+ranks of the device time.  Rank 0 prints one JSON line with the roofline of
+the dominant kernel (HBM; plus the products' compute side at ranks 16 and
+32), the end-to-end figure through host buffers (psgd_step_host_flat), the
+clocks seen during the timed region and, on one GPU, the float64 oracle
+timed on the host cores.  --impl reference times that oracle as the
+reference arm.
 """
 from __future__ import annotations
 
