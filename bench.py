@@ -136,8 +136,8 @@ class ClockSampler:
 
     def start(self):
         try:
-            out_dir = os.path.join(ROOT, "gpurun_out") if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else "/tmp"
-            self.path = os.path.join(out_dir, f"clocks_bench_{os.getpid()}.csv")
+            import tempfile
+            self.path = os.path.join(tempfile.gettempdir(), f"clocks_bench_{os.getpid()}.csv")
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
