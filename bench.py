@@ -309,10 +309,13 @@ def launches_per_step(lib, B, dist: bool = False):
 # --------------------------------------------------------------------------
 # CPU oracle timing (bounded sample)
 
-def oracle_sample(wl, rank, budget_s=15.0, seed=1234, max_layers=None):
+def oracle_sample(wl, rank, budget_s=15.0, seed=1234, max_layers=None, carry_bytes=4 << 30):
     """Time the float64 oracle on a bounded sample of the workload: whole
-    layers (all workers) in list order until the oracle time passes
-    budget_s.  Returns (elements/s, elements, seconds, threads, text)."""
+    layers (all workers) in list order, step after step with each layer's
+    error memory and Q carried over, until the oracle time passes budget_s.
+    Steps after the first are taken only when the carried float64 state
+    (W * sum(m n) * 8 bytes) stays under carry_bytes.  Returns (elements/s,
+    elements, seconds, threads, text)."""
     import oracle.powersgd64 as ora
     try:
         from threadpoolctl import threadpool_info
@@ -320,25 +323,35 @@ def oracle_sample(wl, rank, budget_s=15.0, seed=1234, max_layers=None):
     except Exception:
         threads = os.cpu_count() or 1
     src = GradientSource(wl, seed)
-    done_el, spent, layers_done = 0, 0.0, 0
-    order = list(range(len(wl.layers)))
-    for l in order:
-        if max_layers is not None and layers_done >= max_layers:
-            break
-        m, n = wl.layers[l]
-        G = [src.layer_grad(0, w, l).to(torch.float64).numpy() for w in range(wl.workers)]
-        E = [np.zeros((m, n)) for _ in range(wl.workers)]
-        Q = src.initial_q(l, rank).to(torch.float64).numpy()
-        t0 = time.perf_counter()
-        ora.step(G, E, Q)
-        spent += time.perf_counter() - t0
-        done_el += wl.workers * m * n
-        layers_done += 1
-        del G, E
-        if spent >= budget_s:
-            break
-    text = (f"{layers_done} of {len(wl.layers)} layers (all {wl.workers} workers, one step, float64 NumPy; "
-            f"BLAS threads {threads}, elementwise ops single-threaded)")
+    done_el, spent, layers_done, steps_begun = 0, 0.0, 0, 0
+    nl = len(wl.layers) if max_layers is None else min(max_layers, len(wl.layers))
+    carry = wl.workers * sum(m * n for (m, n) in wl.layers[:nl]) * 8 <= carry_bytes
+    state = {}
+    step = 0
+    while spent < budget_s and nl > 0 and (step == 0 or carry):
+        steps_begun += 1
+        for l in range(nl):
+            m, n = wl.layers[l]
+            G = [src.layer_grad(step, w, l).to(torch.float64).numpy() for w in range(wl.workers)]
+            if l in state:
+                E, Q = state[l]
+            else:
+                E = [np.zeros((m, n)) for _ in range(wl.workers)]
+                Q = src.initial_q(l, rank).to(torch.float64).numpy()
+            t0 = time.perf_counter()
+            res = ora.step(G, E, Q)
+            spent += time.perf_counter() - t0
+            done_el += wl.workers * m * n
+            layers_done += 1
+            if carry:
+                state[l] = (res["E_new"], res["Q_bar"])
+            del G, E, res
+            if spent >= budget_s:
+                break
+        step += 1
+    text = (f"{layers_done} layer-steps over {steps_begun} step(s) of {len(wl.layers)} layers (all {wl.workers} "
+            f"workers, error memory and Q carried, float64 NumPy; BLAS threads {threads}, elementwise ops "
+            f"single-threaded)")
     return done_el / spent, done_el, spent, threads, text
 
 

@@ -1,6 +1,7 @@
 """Host-side logic of bench.py that needs no GPU: the kernel-source hash that
-decides whether committed ncu traffic still belongs to the kernels, and the
-committed traffic record itself."""
+decides whether committed ncu traffic still belongs to the kernels, the
+committed traffic record itself, the compute roofline arithmetic and the
+bounded oracle sample behind the CPU baseline."""
 import json
 import os
 import shutil
@@ -54,3 +55,17 @@ def test_compute_roofline_arithmetic():
     # sum-first: the first pass multiplies each matrix element once, not once per worker
     s = bench.compute_roofline(10**9, 32, 1.0, 1.0, 2000.0, 1600.0, sum_first=True, workers=8)
     assert abs(s["achieved"] - (2 * 32 * 1e9 / 8 + 2 * 32 * 1e9) / 2e-3 / 1e12) < 1e-6
+
+
+def test_oracle_sample_runs_later_steps_with_state_carried():
+    from tests import _harness as H
+    wl = H.small_workload([(24, 20), (9, 7)], 2, 2)
+    rate, elements, seconds, threads, text = bench.oracle_sample(wl, 2, budget_s=0.05)
+    per_step = wl.workers * (24 * 20 + 9 * 7)
+    # whole layers only: full steps plus possibly the first layer of the next
+    assert elements > per_step and elements % per_step in (0, wl.workers * 24 * 20)
+    assert rate > 0 and seconds >= 0.05 and threads >= 1
+    assert int(text.split(" over ")[1].split(" ")[0]) >= 2
+    # the carried state is bounded: with no room for it, only the first step runs
+    _, elements1, _, _, text1 = bench.oracle_sample(wl, 2, budget_s=10.0, carry_bytes=0)
+    assert elements1 == per_step and " over 1 step(s) " in text1
