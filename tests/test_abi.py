@@ -66,3 +66,18 @@ def test_null_context_is_an_argument_error(lib):
     assert lib.psgd_status(None) == _lib.PSGD_ERR_ARG
     assert lib.psgd_step_launches(None) == -1
     lib.psgd_destroy(None)
+
+
+def test_missing_library_is_an_error_not_a_fallback(tmp_path):
+    with pytest.raises(ImportError, match="libpsgd.so not found"):
+        _lib.load(str(tmp_path / "libpsgd.so"))
+
+
+def test_binding_has_no_cpu_or_oracle_path():
+    # the product path never reaches the oracle or a host implementation
+    pkg = os.path.join(ROOT, "rank_gradient_compression_02_b200")
+    for name in os.listdir(pkg):
+        if name.endswith(".py"):
+            text = open(os.path.join(pkg, name)).read()
+            assert "oracle" not in text, name
+            assert "numpy" not in text, name
