@@ -104,6 +104,26 @@ def check_exact_low_rank(ora):
         np.testing.assert_allclose(o["E_new"][w], Ms[w] - Mbar, atol=1e-12)
 
 
+def check_full_rank_is_lossless(ora):
+    """r = min(m, n): the factors span M_bar's whole column space, so the
+    decompressed gradient is the worker mean itself and each worker keeps
+    only its deviation from it: G_hat = mean(M), E'_w = M_w - mean(M).  With
+    r = m, P_hat is square and orthogonal."""
+    rng = _rng(12)
+    for m, n in ((6, 40), (40, 6)):
+        r = min(m, n)
+        W = 3
+        G = [rng.standard_normal((m, n)) for _ in range(W)]
+        E = [0.2 * rng.standard_normal((m, n)) for _ in range(W)]
+        o = ora.step(G, E, rng.standard_normal((n, r)))
+        Mbar = sum(g + e for g, e in zip(G, E)) / W
+        np.testing.assert_allclose(o["G_hat"], Mbar, atol=1e-11)
+        for w in range(W):
+            np.testing.assert_allclose(o["E_new"][w], G[w] + E[w] - Mbar, atol=1e-11)
+        if r == m:
+            np.testing.assert_allclose(o["P_hat"] @ o["P_hat"].T, np.eye(m), atol=1e-12)
+
+
 def check_identities(ora):
     """P_hat^T P_hat = I; P_hat Q_bar^T + E'_w = M_w; P_hat^T mean_w E'_w = 0;
     Q_bar = mean(M)^T P_hat ([N152] "Method")."""
@@ -295,6 +315,7 @@ def check_subspace_sin_max(ora):
 
 ALL_CHECKS = [
     check_hand_cases, check_gram_schmidt_vs_householder, check_gram_schmidt_rank_deficient,
+    check_full_rank_is_lossless,
     check_rank1_closed_form, check_exact_low_rank, check_identities, check_linearity,
     check_jacobi_svd, check_warm_start_convergence, check_error_feedback_telescopes,
     check_momentum_closed_form, check_vec_mean, check_power_iterations, check_svd_refresh,

@@ -411,6 +411,26 @@ def test_many_workers_rank32(workers):
     H.assert_close(hist[0], H.TOL["f32"], "step 0")
 
 
+# r = min(m, n): wide and tall layers of exactly the rank (no compression;
+# chunks of a few lanes at every lane width)
+FULL_RANK = {2: [(2, 64), (50, 2)], 4: [(4, 90), (70, 4)], 8: [(8, 100), (100, 8)],
+             16: [(16, 160), (200, 16)], 32: [(32, 400), (300, 32)]}
+
+
+@pytest.mark.parametrize("rank", sorted(FULL_RANK))
+def test_full_rank_is_lossless(rank):
+    wl = H.small_workload(FULL_RANK[rank], rank, 3)
+    run, orc, hist = H.run_free(wl, steps=3)
+    for t, e in enumerate(hist):
+        H.assert_close(e, H.TOL["f32"], f"step {t}")
+    # the decompressed gradient is the worker mean of M itself
+    for l in range(len(wl.layers)):
+        o = orc.last[l]
+        mbar = sum(o["M"]) / wl.workers
+        got = run.Rc[l].double().cpu().numpy()
+        assert np.linalg.norm(got - mbar) / np.linalg.norm(mbar) <= H.TOL["f32"]
+
+
 def test_max_workers_single_row():
     # the largest worker count the library accepts, on a one-row layer and an
     # odd-width layer
