@@ -1,8 +1,9 @@
-"""Host logic of the multi-GPU bench path on CPU with gloo, world size 2:
-max-over-ranks timing, whole-job throughput, and the distributed step's
-orchestration (the two all-reduces of the P and Q partials, the global
-worker count, the 1-D means) driven through a float64 stand-in for the
-library built from the oracle's functions."""
+"""Host logic of the multi-GPU bench path on CPU with gloo (world sizes 2
+and 3): max-over-ranks timing, whole-job throughput, and the distributed
+step's orchestration over two steps (the two all-reduces of the P and Q
+partials, the global worker count, error memory and warm start carried,
+momentum, the 1-D means) driven through a float64 stand-in for the library
+built from the oracle's functions."""
 import os
 import socket
 import types
@@ -132,14 +133,17 @@ LAYERS = [(12, 9), (7, 11)]
 R, WL = 2, 2
 
 
-def _grads(rank_id, w, l):
-    g = torch.Generator().manual_seed(1000 * rank_id + 10 * w + l)
+STEPS = 2
+
+
+def _grads(rank_id, w, l, t=0):
+    g = torch.Generator().manual_seed(100000 * t + 1000 * rank_id + 10 * w + l)
     m, n = LAYERS[l]
     return torch.randn(m, n, generator=g, dtype=torch.float64)
 
 
-def _vecs(rank_id, w):
-    g = torch.Generator().manual_seed(777 + 10 * rank_id + w)
+def _vecs(rank_id, w, t=0):
+    g = torch.Generator().manual_seed(777 + 100000 * t + 10 * rank_id + w)
     return [torch.randn(5, generator=g, dtype=torch.float64), torch.randn(3, generator=g, dtype=torch.float64)]
 
 
@@ -164,7 +168,15 @@ def _worker_dist(rank, world, port, q):
     db = bench.DistBuffers(lib, B, wl, torch.device("cpu"))
     db.p = db.p.double()
     db.q = db.q.double()
-    bench.dist_step(lib, B, wl, db, lambda t: dist.all_reduce(t, op=dist.ReduceOp.SUM))
+    for t in range(STEPS):
+        if t:
+            for w in range(WL):
+                for l in range(len(LAYERS)):
+                    B.G[w][l].copy_(_grads(rank, w, l, t))
+                for k, v in enumerate(_vecs(rank, w, t)):
+                    B.vecs[w][k].copy_(v)
+            db.pack(B.vecs)   # the flat all-reduce buffer holds the step's 1-D gradients
+        bench.dist_step(lib, B, wl, db, lambda x: dist.all_reduce(x, op=dist.ReduceOp.SUM))
     q.put((rank, [p.numpy().copy() for p in B.P], [x.numpy().copy() for x in B.Q],
            [[e.numpy().copy() for e in Ew] for Ew in B.E], [v.numpy().copy() for v in B.vout],
            [x.numpy().copy() for x in B.params]))
@@ -172,24 +184,32 @@ def _worker_dist(rank, world, port, q):
     dist.destroy_process_group()
 
 
-def test_distributed_step_orchestration_matches_oracle():
+@pytest.mark.parametrize("world", [2, 3])
+def test_distributed_step_orchestration_matches_oracle(world):
     import oracle.powersgd64 as ora
-    world = 2
     res = _spawn(_worker_dist, world)
     g = torch.Generator().manual_seed(5)
-    Q0 = [torch.randn(n, R, generator=g, dtype=torch.float64).numpy() for (_, n) in LAYERS]
-    for l in range(len(LAYERS)):
-        G = [_grads(r, w, l).numpy() for r in range(world) for w in range(WL)]
-        o = ora.step(G, [np.zeros_like(x) for x in G], Q0[l])
-        ghat = o["G_hat"]
-        for r, P, Q, E, vout, params in res:
+    Q = [torch.randn(n, R, generator=g, dtype=torch.float64).numpy() for (_, n) in LAYERS]
+    E = [[np.zeros(LAYERS[l]) for _ in range(world * WL)] for l in range(len(LAYERS))]
+    mom = [np.zeros(s) for s in LAYERS]
+    x = [np.zeros(s) for s in LAYERS]
+    for t in range(STEPS):
+        outs = []
+        for l in range(len(LAYERS)):
+            G = [_grads(r, w, l, t).numpy() for r in range(world) for w in range(WL)]
+            o = ora.step(G, E[l], Q[l])
+            E[l], Q[l] = o["E_new"], o["Q_bar"]
+            x[l], mom[l] = ora.momentum_update(x[l], mom[l], o["G_hat"], lr=0.1, beta=0.9)
+            outs.append(o)
+    for l, o in enumerate(outs):
+        for r, P, Qr, Er, vout, params in res:
             np.testing.assert_allclose(P[l], o["P_hat"], atol=1e-12)
-            np.testing.assert_allclose(Q[l], o["Q_bar"], atol=1e-12)
+            np.testing.assert_allclose(Qr[l], o["Q_bar"], atol=1e-12)
             for w in range(WL):
-                np.testing.assert_allclose(E[w][l], o["E_new"][r * WL + w], atol=1e-12)
-            np.testing.assert_allclose(params[l], -0.1 * ghat, atol=1e-12)
-    vec_want = [sum(_vecs(r, w)[k] for r in range(world) for w in range(WL)).numpy() / (world * WL)
+                np.testing.assert_allclose(Er[w][l], o["E_new"][r * WL + w], atol=1e-12)
+            np.testing.assert_allclose(params[l], x[l], atol=1e-12)
+    vec_want = [sum(_vecs(r, w, STEPS - 1)[k] for r in range(world) for w in range(WL)).numpy() / (world * WL)
                 for k in range(2)]
-    for r, P, Q, E, vout, params in res:
+    for r, P, Qr, Er, vout, params in res:
         for k in range(2):
             np.testing.assert_allclose(vout[k], vec_want[k], atol=1e-12)
