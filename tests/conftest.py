@@ -20,6 +20,10 @@ def pytest_collection_modifyitems(config, items):
     except Exception:  # pragma: no cover
         have_gpu = False
     if have_gpu:
+        # the GPU cases call the library: build it first when it is missing or
+        # older than its sources (a no-op otherwise; fails loudly without nvcc)
+        from rank_gradient_compression_02_b200 import build
+        build.build()
         return
     skip = pytest.mark.skip(reason="no CUDA device")
     for item in items:
