@@ -419,6 +419,11 @@ def main():
     torch.cuda.set_device(device)
 
     from rank_gradient_compression_02_b200 import PowerSGD
+    if world == 1:
+        # one process: build libpsgd.so if it is missing or stale (a no-op
+        # otherwise); several ranks never race on the build, they load it
+        from rank_gradient_compression_02_b200 import build
+        build.build()
     free, _ = torch.cuda.mem_get_info()
     need = device_bytes_needed(wl, r)
     if need > free * 0.95:
