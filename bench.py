@@ -494,6 +494,10 @@ def main():
                 "peak_kind": f"{peak_kind} hbm_gbs",
                 "per_kernel_ms": {n: round(t, 4) for n, t in zip(names, per_launch_ms)},
                 "step_algorithmic_frac": round(step_min_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 4)}
+    if args.iters == 1:
+        # achieved DRAM bandwidth of the whole step: the bytes the three
+        # passes move (ncu puts each pass's traffic at its design bytes)
+        roofline["step_dram_frac"] = round(sum(alg) / (ms_per_step * 1e-3) / 1e9 / peak, 4)
     if r >= 16:
         # at ranks 16 and 32 the first two passes are bound by instruction
         # issue, not HBM: report their compute side too
@@ -528,6 +532,8 @@ def main():
         lms = max_over_ranks(e0.elapsed_time(e1), world, device) / args.steps
         variants["lazy_errors"] = {"ms_per_step": lms, "value": job_value(wl.elements, world, lms),
                                    "step_algorithmic_frac": round(step_min_bytes / (lms * 1e-3) / 1e9 / peak, 4),
+                                   "step_dram_frac": (round(wl.elements * (gsz + 12) / (lms * 1e-3) / 1e9 / peak, 4)
+                                                      if args.iters == 1 else None),
                                    "note": "error buffers hold M between steps; E' materialised once at the end "
                                            "of the timed region"}
         lazy_lib.close()
