@@ -177,26 +177,6 @@ def svd_refresh_step(G: Sequence[np.ndarray], E: Sequence[np.ndarray], rank: int
     return dict(M=M, M_bar=M_bar, P_hat=P_hat, Q_bar=Q_bar, E_new=E_new, G_hat=G_hat, sigma=s)
 
 
-def run(layers_G, E0, Q0, drop_tol: float = DROP_TOL):
-    """Free-running multi-step driver.  layers_G[t][l][w] is the gradient of
-    worker w for layer l at step t; E0[l][w] and Q0[l] are the initial state.
-    The Q state of the next step is Q_bar exactly ([N152] "Concepts",
-    warm-start subspace iteration).  Yields the per-step result dicts (a list
-    over layers) and leaves the state in the returned E, Q lists."""
-    E = [[_f64(e) for e in El] for El in E0]
-    Q = [_f64(q) for q in Q0]
-    history = []
-    for Gt in layers_G:
-        outs = []
-        for l, Gl in enumerate(Gt):
-            o = step(Gl, E[l], Q[l], drop_tol)
-            E[l] = o["E_new"]
-            Q[l] = o["Q_bar"]
-            outs.append(o)
-        history.append(outs)
-    return history, E, Q
-
-
 # --- reference SVD for subspace checks ----------------------------------------
 
 def jacobi_svd(A, tol: float = 1e-15, max_sweeps: int = 60):

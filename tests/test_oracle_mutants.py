@@ -86,6 +86,39 @@ def _step_restarts_iterations(G, E, Q, drop_tol=ora.DROP_TOL, iters=1):
 
 _ORIG_STEP = ora.step
 
+
+def _step_residual_local_q(G, E, Q, drop_tol=ora.DROP_TOL, iters=1):
+    # each worker's residual against its own Q_w instead of the mean Q_bar
+    o = _ORIG_STEP(G, E, Q, drop_tol, iters)
+    o["E_new"] = [o["M"][w] - o["P_hat"] @ o["Qw"][w].T for w in range(len(G))]
+    return o
+
+
+def _step_q_bar_summed(G, E, Q, drop_tol=ora.DROP_TOL, iters=1):
+    # Q_bar is the sum over workers, not the mean
+    o = _ORIG_STEP(G, E, Q, drop_tol, iters)
+    W = len(G)
+    o["Q_bar"] = o["Q_bar"] * W
+    o["E_new"] = [o["M"][w] - o["P_hat"] @ o["Q_bar"].T for w in range(W)]
+    o["G_hat"] = o["P_hat"] @ o["Q_bar"].T
+    return o
+
+
+def _step_residual_from_g(G, E, Q, drop_tol=ora.DROP_TOL, iters=1):
+    # the new error memory forgets the old one: E' = G_w - P_hat Q_bar^T
+    o = _ORIG_STEP(G, E, Q, drop_tol, iters)
+    o["E_new"] = [np.asarray(G[w], dtype=np.float64) - o["G_hat"] for w in range(len(G))]
+    return o
+
+
+def _gs_reversed_order(P, drop_tol=ora.DROP_TOL):
+    # orthogonalises the columns last to first
+    P = np.asarray(P, dtype=np.float64)
+    return _ORIG_GS(P[:, ::-1], drop_tol)[:, ::-1].copy()
+
+
+_ORIG_GS = ora.gram_schmidt
+
 MUTANTS = {
     "iterations_restart": {"step": _step_restarts_iterations},
     "ef_ignores_error": {"error_feedback_add": _ef_ignores_error},
@@ -99,6 +132,10 @@ MUTANTS = {
     "left_multiply_scaled": {"left_multiply": _left_multiply_no_transpose_of_phat},
     "momentum_ignores_mom": {"momentum_update": _momentum_ignores_mom},
     "momentum_dampened": {"momentum_update": _momentum_dampened},
+    "residual_local_q": {"step": _step_residual_local_q},
+    "q_bar_summed": {"step": _step_q_bar_summed},
+    "residual_from_g": {"step": _step_residual_from_g},
+    "gs_reversed_order": {"gram_schmidt": _gs_reversed_order},
 }
 
 
