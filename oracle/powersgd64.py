@@ -12,6 +12,8 @@ Sources (cited by page title and section):
           warm-start paragraphs.
   [ABS]   "PowerSGD: Practical Low-Rank Gradient Compression for Distributed
           Optimization", Abstract.
+  [PLUS]  "From PowerSGD to PowerSGD+ ...", Abstract (the periodic SVD
+          refresh of the projection subspace).
 
 Everything is computed in float64 with plain NumPy; matrix products use
 ``@`` (a library primitive), every other step is written out as the method
