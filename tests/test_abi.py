@@ -81,3 +81,48 @@ def test_binding_has_no_cpu_or_oracle_path():
             text = open(os.path.join(pkg, name)).read()
             assert "oracle" not in text, name
             assert "numpy" not in text, name
+
+
+_C_CALLER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "psgd.h"
+
+int main(void) {
+    psgd_layer layers[2] = {{64, 48}, {10, 512}};
+    psgd_ctx *ctx = (psgd_ctx *)1;
+    /* rank 0, rank above min(m, n), 0 workers, unknown flag: refused before any device work */
+    if (psgd_create(&ctx, layers, 2, 0, 4, 7u, PSGD_F32, 0u) != PSGD_ERR_ARG || ctx != NULL) return 1;
+    if (psgd_create(&ctx, layers, 2, 11, 4, 7u, PSGD_F32, 0u) != PSGD_ERR_ARG) return 2;
+    if (psgd_create(&ctx, layers, 2, 2, 0, 7u, PSGD_BF16, 0u) != PSGD_ERR_ARG) return 3;
+    if (psgd_create(&ctx, layers, 2, 2, 4, 7u, PSGD_F32, 8u) != PSGD_ERR_ARG) return 4;
+    if (strlen(psgd_last_error(NULL)) == 0) return 5;
+    if (psgd_step(NULL, NULL, NULL, NULL, NULL, NULL, NULL) != PSGD_ERR_ARG) return 6;
+    if (psgd_status(NULL) != PSGD_ERR_ARG) return 7;
+    if (psgd_step_launches(NULL) != -1) return 8;
+    psgd_destroy(NULL);
+    printf("ok\n");
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no gcc")
+    src = tmp_path / "caller.c"
+    src.write_text(_C_CALLER)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.dirname(HEADER),
+                    str(src), "-o", str(exe), "-L", libdir, "-lpsgd", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stdout, out.stderr)
+    # and as C++: the extern "C" block keeps the names unmangled
+    gxx = shutil.which("g++")
+    if gxx is not None:
+        subprocess.run([gxx, "-std=c++11", "-Wall", "-Werror", "-fsyntax-only", "-x", "c++", "-I",
+                        os.path.dirname(HEADER), str(src)], check=True)
