@@ -126,3 +126,21 @@ def test_header_is_plain_c_and_links(lib, tmp_path):
     if gxx is not None:
         subprocess.run([gxx, "-std=c++11", "-Wall", "-Werror", "-fsyntax-only", "-x", "c++", "-I",
                         os.path.dirname(HEADER), str(src)], check=True)
+
+
+def test_static_step_checks_need_no_device(lib):
+    # every check of the allocation-free step happens before device work;
+    # the pointer values are never dereferenced
+    W = 2
+    ok = (ctypes.c_void_p * W)(*([16] * W))
+    odd = (ctypes.c_void_p * W)(16, 20)
+    null = (ctypes.c_void_p * W)(16, None)
+    step = lib.psgd_step_static
+    assert step(8192, 8192, 32, W, 0, ok, ok, 16, None, None, None) == _lib.PSGD_ERR_ARG   # beyond the scratch
+    assert "static scratch" in lib.psgd_last_error(None).decode()
+    assert step(64, 48, 49, W, 0, ok, ok, 16, None, None, None) == _lib.PSGD_ERR_ARG       # rank > min(m, n)
+    assert step(64, 48, 2, 0, 0, ok, ok, 16, None, None, None) == _lib.PSGD_ERR_ARG        # no workers
+    assert step(64, 48, 2, W, 2, ok, ok, 16, None, None, None) == _lib.PSGD_ERR_ARG        # bad dtype
+    assert step(64, 48, 2, W, 0, null, ok, 16, None, None, None) == _lib.PSGD_ERR_ARG      # null gradient
+    assert step(64, 48, 2, W, 0, odd, ok, 16, None, None, None) == _lib.PSGD_ERR_ALIGN     # 4-byte offset
+    assert step(64, 48, 2, W, 0, ok, ok, 24, None, None, None) == _lib.PSGD_ERR_ALIGN      # q misaligned
