@@ -144,3 +144,21 @@ def test_static_step_checks_need_no_device(lib):
     assert step(64, 48, 2, W, 0, null, ok, 16, None, None, None) == _lib.PSGD_ERR_ARG      # null gradient
     assert step(64, 48, 2, W, 0, odd, ok, 16, None, None, None) == _lib.PSGD_ERR_ALIGN     # 4-byte offset
     assert step(64, 48, 2, W, 0, ok, ok, 24, None, None, None) == _lib.PSGD_ERR_ALIGN      # q misaligned
+
+
+def test_readme_c_example_compiles(tmp_path):
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no gcc")
+    text = open(os.path.join(ROOT, "README.md")).read()
+    block = re.search(r"```c\n(.*?)```", text, re.S).group(1)
+    body = "\n".join(ln for ln in block.splitlines() if not ln.startswith("#include"))
+    src = tmp_path / "example.c"
+    src.write_text('#include <stdio.h>\n#include "psgd.h"\n'
+                   "void example(float *const *q, void *stream, const void *const *grads, float *const *errors,\n"
+                   "             float *const *p_hat, float *const *recon, float *const *params,\n"
+                   "             float *const *mom) {\n" + body + "\n}\n")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-fsyntax-only", "-I",
+                    os.path.dirname(HEADER), str(src)], check=True)
