@@ -172,6 +172,7 @@ def test_reference_arm_line(fake_gpu, monkeypatch, capsys):
     d = _run(monkeypatch, capsys, "--impl", "reference", "--steps", "2", "--warmup", "3")
     assert d["impl"] == "reference" and d["dtype"] == "f64" and d["value"] > 0
     assert d["cpu_baseline"]["value"] == d["value"] and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["cpu_baseline"]["sample"].startswith("each step: the whole workload step")
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 
@@ -200,3 +201,10 @@ def test_json_line_distributed_step_one_rank(fake_gpu, monkeypatch, capsys):
     assert ("set_global_workers", fake_gpu.workers) in lib.calls
     i = lib.calls.index("dist_p")
     assert lib.calls[i:i + 3] == ["dist_p", "dist_q", "dist_finish"]
+
+
+def test_reference_arm_falls_back_to_one_layer_per_step(fake_gpu, monkeypatch, capsys):
+    monkeypatch.setattr(bench, "run_reference",
+                        lambda *a, _f=bench.run_reference: _f(*a, full_max_elements=0))
+    d = _run(monkeypatch, capsys, "--impl", "reference", "--steps", "3", "--warmup", "3")
+    assert d["value"] > 0 and d["cpu_baseline"]["sample"].startswith("each step: one layer")
