@@ -1,8 +1,8 @@
 """The parity cases are fair tests: on every shape set, rank and worker
 count the GPU parity tests gate, the oracle itself moves by at most half
 the float32 tolerance (1e-4) when its inputs are perturbed by one float32
-ulp, over the same free-running steps (the largest, 2.1e-5, is rank 32
-with three workers at the third step).  A case above the tolerance would
+ulp, over the same free-running steps (the largest, 3.4e-5, is rank 32
+with three workers at the fourth step).  A case above the tolerance would
 have to be reported rather than gated."""
 import pytest
 
@@ -17,6 +17,22 @@ MARGIN = 0.5 * H.TOL["f32"]
 @pytest.mark.parametrize("workers", [1, 3])
 def test_mixed_shapes_are_well_conditioned(rank, workers):
     assert max_sensitivity(H.small_workload(MIXED, rank, workers), steps=3) <= MARGIN
+
+
+@pytest.mark.parametrize("rank", [4, 16, 32])
+def test_four_step_mode_cases_are_well_conditioned(rank):
+    # lazy errors, sum-first and power iterations run four steps on these
+    assert max_sensitivity(H.small_workload(MIXED, rank, 3), steps=4) <= MARGIN
+
+
+@pytest.mark.parametrize("rank", [2, 8, 16, 32])
+def test_sixteen_worker_cases_are_well_conditioned(rank):
+    assert max_sensitivity(H.small_workload(MIXED[:4], rank, 16), steps=2) <= MARGIN
+
+
+@pytest.mark.parametrize("workers", [64, 256])
+def test_many_worker_cases_are_well_conditioned(workers):
+    assert max_sensitivity(H.small_workload([(40, 130), (33, 37), (64, 576)], 32, workers), steps=1) <= MARGIN
 
 
 @pytest.mark.parametrize("rank", sorted(FULL_RANK))
