@@ -3,7 +3,7 @@ oracle's own results move when its inputs are perturbed by one float32
 ulp.  A parity case is a fair test at a tolerance only if this sensitivity
 sits well below it: otherwise rounding alone, in any correct float32
 implementation, could exceed the bar."""
-from typing import Dict, List, Sequence, Tuple
+from typing import Dict, List, Optional, Sequence, Tuple
 
 import numpy as np
 
@@ -17,25 +17,30 @@ def _perturb(a: np.ndarray, rng) -> np.ndarray:
     return a * (1.0 + ULP * rng.choice([-1.0, 1.0], size=a.shape))
 
 
-def ulp_sensitivity(wl: Workload, steps: int, seed: int = 1234, probe_seed: int = 5) -> List[Dict[str, float]]:
+def ulp_sensitivity(wl: Workload, steps: int, seed: int = 1234, probe_seed: int = 5,
+                    layers_idx: Optional[Sequence[int]] = None) -> List[Dict[str, float]]:
     """Free-running steps of the oracle on the workload's gradients, once as
     generated and once with every gradient and the initial Q perturbed by
     one float32 ulp (random sign).  Returns, per step, the largest relative
     Frobenius change over the layers of P_hat, Q_bar, G_hat and E'_w (E'
-    relative to ||M_w||), the same measures the parity tests use."""
+    relative to ||M_w||), the same measures the parity tests use.
+    layers_idx: the layers to follow (default all), with the workload's own
+    per-layer inputs."""
     src = GradientSource(wl, seed)
     rng = np.random.default_rng(probe_seed)
     W = wl.workers
+    idx = list(range(len(wl.layers))) if layers_idx is None else list(layers_idx)
     a_state: Dict[int, Tuple] = {}
     b_state: Dict[int, Tuple] = {}
-    for l, (m, n) in enumerate(wl.layers):
+    for l in idx:
+        m, n = wl.layers[l]
         q = src.initial_q(l).double().numpy()
         a_state[l] = ([np.zeros((m, n)) for _ in range(W)], q)
         b_state[l] = ([np.zeros((m, n)) for _ in range(W)], _perturb(q, rng))
     out = []
     for t in range(steps):
         worst: Dict[str, float] = {}
-        for l in range(len(wl.layers)):
+        for l in idx:
             G = [src.layer_grad(t, w, l).double().numpy() for w in range(W)]
             a = ora.step(G, *a_state[l])
             b = ora.step([_perturb(g, rng) for g in G], *b_state[l])
@@ -50,5 +55,5 @@ def ulp_sensitivity(wl: Workload, steps: int, seed: int = 1234, probe_seed: int 
     return out
 
 
-def max_sensitivity(wl: Workload, steps: int, seed: int = 1234) -> float:
-    return max(max(d.values()) for d in ulp_sensitivity(wl, steps, seed))
+def max_sensitivity(wl: Workload, steps: int, seed: int = 1234, layers_idx=None) -> float:
+    return max(max(d.values()) for d in ulp_sensitivity(wl, steps, seed, layers_idx=layers_idx))

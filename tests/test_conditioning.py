@@ -46,3 +46,16 @@ def test_probe_detects_an_ill_conditioned_case():
     # their orthogonalisation amplifies a one-ulp change past the tolerance
     wl = H.small_workload([(64, 48)], 8, 1, noise=("abs", 1e-5))
     assert max_sensitivity(wl, steps=3) > H.TOL["f32"]
+
+
+def test_resnet18_full_size_is_well_conditioned():
+    # every layer of the ResNet-18 set at full size, three steps, as the
+    # full-size GPU parity test runs it
+    from synth import C1
+    assert max_sensitivity(C1, steps=3) <= MARGIN
+
+
+@pytest.mark.parametrize("rank", [1, 4, 32])
+def test_sweep_1024_sampled_layers_are_well_conditioned(rank):
+    from synth import C4B
+    assert max_sensitivity(C4B.with_rank(rank), steps=3, layers_idx=[0, 97, 255]) <= MARGIN
