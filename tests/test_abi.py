@@ -162,3 +162,17 @@ def test_readme_c_example_compiles(tmp_path):
                    "             float *const *mom) {\n" + body + "\n}\n")
     subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-fsyntax-only", "-I",
                     os.path.dirname(HEADER), str(src)], check=True)
+
+
+def test_binding_constants_match_the_header():
+    text = open(HEADER).read()
+    values = {k: int(v) for k, v in re.findall(r"\b(PSGD_(?:OK|ERR_\w+|F32|BF16|FLAG_\w+))\s*=\s*(\d+)u?\b", text)}
+    assert values["PSGD_OK"] == _lib.PSGD_OK
+    for name in ("ARG", "ALIGN", "CUDA", "OOM", "STATE", "DEVICE"):
+        assert values[f"PSGD_ERR_{name}"] == getattr(_lib, f"PSGD_ERR_{name}"), name
+        assert _lib._ERR_NAMES[values[f"PSGD_ERR_{name}"]] == f"PSGD_ERR_{name}"
+    assert values["PSGD_F32"] == _lib.PSGD_F32 and values["PSGD_BF16"] == _lib.PSGD_BF16
+    for name in ("LAZY_ERRORS", "SUM_FIRST", "NO_WARM_START"):
+        assert values[f"PSGD_FLAG_{name}"] == getattr(_lib, f"FLAG_{name}"), name
+    m = re.search(r"#define PSGD_STATIC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
+    assert m and int(m.group(1)) << int(m.group(2)) == 16 << 20
