@@ -1,9 +1,12 @@
 """ctypes binding of libpsgd.so (the C ABI in include/psgd.h).
 
 Argument marshalling only: tensors become device pointers, lists become
-pointer arrays, the current torch stream becomes a cudaStream_t.  Every
-step of the computation runs in the library's kernels; there is no fallback
-of any kind, and a missing library is an error.
+pointer arrays, the current torch stream becomes a cudaStream_t.  Before an
+address crosses the ABI, each tensor's side (device or host), dtype,
+contiguity and size and each list's length are checked (again only when a
+call's buffers change).  Every step of the computation runs in the
+library's kernels; there is no fallback of any kind, and a missing library
+is an error.
 """
 from __future__ import annotations
 
@@ -90,16 +93,69 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     return lib
 
 
+def _on_device(t: torch.Tensor) -> bool:
+    return t.is_cuda
+
+
+def _check_buf(t, what: str, numel: int, dtypes, on_device: bool, at_least: bool = False):
+    """Host-side check of one buffer before its address crosses the ABI: a
+    tensor must sit on the right side (device or host), have a listed
+    dtype, be contiguous and hold numel elements (at least numel with
+    at_least).  Raw addresses (ints) and None pass through unchecked; the
+    library checks those for null and alignment itself."""
+    if t is None or isinstance(t, int):
+        return
+    if not isinstance(t, torch.Tensor):
+        raise PsgdError(PSGD_ERR_ARG, f"{what}: expected a tensor or an address, got {type(t).__name__}")
+    if _on_device(t) != on_device:
+        raise PsgdError(PSGD_ERR_ARG, f"{what}: expected a {'device' if on_device else 'host'} tensor")
+    if t.dtype not in dtypes:
+        raise PsgdError(PSGD_ERR_ARG, f"{what}: dtype {t.dtype} not in {list(dtypes)}")
+    if not t.is_contiguous():
+        raise PsgdError(PSGD_ERR_ARG, f"{what}: not contiguous")
+    n = t.numel()
+    if (n < numel) if at_least else (n != numel):
+        raise PsgdError(PSGD_ERR_ARG, f"{what}: {n} elements, expected {'at least ' if at_least else ''}{numel}")
+
+
+def _check_list(values, what: str, count: int):
+    if values is None or len(values) != count:
+        raise PsgdError(PSGD_ERR_ARG, f"{what}: expected {count} entries, got "
+                                      f"{'none' if values is None else len(values)}")
+
+
+_F32 = (torch.float32,)
+_F64 = (torch.float64,)
+
+
+def _addr(v):
+    # tensors give their address; ints and None pass as they are (anything
+    # else is refused by the checks before it reaches the library)
+    return v.data_ptr() if isinstance(v, torch.Tensor) else v
+
+
+def _arr(addrs: Sequence) -> ctypes.Array:
+    return (ctypes.c_void_p * max(1, len(addrs)))(*addrs)
+
+
 def _ptrs(values: Sequence) -> ctypes.Array:
-    arr = (ctypes.c_void_p * max(1, len(values)))()
-    for i, v in enumerate(values):
-        if v is None:
-            arr[i] = None
-        elif isinstance(v, int):
-            arr[i] = v
-        else:
-            arr[i] = v.data_ptr()
-    return arr
+    return _arr([_addr(v) for v in values])
+
+
+def _sig(values: Sequence) -> tuple:
+    """Addresses and element counts of a call's buffers: the checks run again
+    only when these change (the library re-uploads its pointer tables on
+    the same condition).  Entries that are raw addresses or None count -1
+    elements."""
+    try:
+        return [v.data_ptr() for v in values], [v.numel() for v in values]
+    except AttributeError:
+        return ([_addr(v) for v in values],
+                [v.numel() if isinstance(v, torch.Tensor) else -1 for v in values])
+
+
+def _arr_sig(sig: tuple) -> ctypes.Array:
+    return _arr(sig[0])
 
 
 def _stream_handle(stream) -> int:
@@ -117,6 +173,15 @@ def step_static(m: int, n: int, rank: int, grads, errors, q, p_hat=None, recon=N
     array.  For callers that cannot allocate device memory."""
     lib = load()
     W = len(grads)
+    m, n, rank = int(m), int(n), int(rank)
+    gdt = (torch.bfloat16,) if grad_dtype == "bf16" else _F32
+    _check_list(errors, "errors", W)
+    for w in range(W):
+        _check_buf(grads[w], f"grads[{w}]", m * n, gdt, True)
+        _check_buf(errors[w], f"errors[{w}]", m * n, _F32, True)
+    _check_buf(q, "q", n * rank, _F32, True)
+    _check_buf(p_hat, "p_hat", m * rank, _F32, True)
+    _check_buf(recon, "recon", m * n, _F32, True)
     rc = lib.psgd_step_static(int(m), int(n), int(rank), W, PSGD_BF16 if grad_dtype == "bf16" else PSGD_F32,
                               _ptrs(grads), _ptrs(errors), q.data_ptr(),
                               p_hat.data_ptr() if p_hat is not None else None,
@@ -160,52 +225,135 @@ class PowerSGD:
         if rc:
             raise PsgdError(rc, self.lib.psgd_last_error(self._h).decode())
 
-    def _wl(self, per_worker: Sequence[Sequence]) -> ctypes.Array:
+    @staticmethod
+    def _flat(per_worker: Sequence[Sequence]) -> List:
         flat: List = []
+        for row in per_worker:
+            flat.extend(row)
+        return flat
+
+    def _validated(self, name: str, parts: Sequence, check) -> List:
+        """Signatures of the call's buffer lists (None for an absent list);
+        check() runs unless they equal those of the last validated call of
+        this kind.  The library reads W*L (or L) entries from each list, so
+        a list is only ever passed after a check of its length."""
+        sigs = [None if p is None else _sig(p) for p in parts]
+        seen = self.__dict__.setdefault("_seen", {})
+        if seen.get(name) != sigs:
+            check()
+            seen[name] = sigs
+        return sigs
+
+    @staticmethod
+    def _opt(sig):
+        return None if sig is None else _arr_sig(sig)
+
+    def _gdt(self):
+        return (torch.bfloat16,) if self.grad_dtype == "bf16" else _F32
+
+    def _check_wl(self, per_worker, what: str, dtypes, on_device: bool = True):
+        """per_worker[w][l]: W lists of L matrices m x n."""
+        _check_list(per_worker, what, self.workers)
         for w in range(self.workers):
-            flat.extend(per_worker[w])
-        return _ptrs(flat)
+            _check_list(per_worker[w], f"{what}[{w}]", len(self.layers))
+            for l, (m, n) in enumerate(self.layers):
+                _check_buf(per_worker[w][l], f"{what}[{w}][{l}]", m * n, dtypes, on_device)
+
+    def _check_layers(self, bufs, what: str, cols, on_device: bool = True, optional: bool = False):
+        """bufs[l]: one m x cols (cols = 'n' for m x n, 'r' for m x rank, 'nr'
+        for n x rank) float32 buffer per layer; optional lists may be None."""
+        if bufs is None and optional:
+            return
+        _check_list(bufs, what, len(self.layers))
+        for l, (m, n) in enumerate(self.layers):
+            numel = {"n": m * n, "r": m * self.rank, "nr": n * self.rank}[cols]
+            _check_buf(bufs[l], f"{what}[{l}]", numel, _F32, on_device)
 
     # -- API
     def init_q(self, q: Sequence, stream=None):
-        self._check(self.lib.psgd_init_q(self._h, _ptrs(q), _stream_handle(stream)))
+        (sq,) = self._validated("init_q", (q,), lambda: self._check_layers(q, "q", "nr"))
+        self._check(self.lib.psgd_init_q(self._h, _arr_sig(sq), _stream_handle(stream)))
+
+    def _check_step_bufs(self, grads, errors, q, p_hat, recon, grads_on_device=True):
+        self._check_wl(grads, "grads", self._gdt(), on_device=grads_on_device)
+        self._check_wl(errors, "errors", _F32)
+        self._check_layers(q, "q", "nr")
+        self._check_layers(p_hat, "p_hat", "r", on_device=grads_on_device, optional=True)
+        self._check_layers(recon, "recon", "n", optional=True)
 
     def step(self, grads, errors, q, p_hat=None, recon=None, stream=None):
-        self._check(self.lib.psgd_step(self._h, self._wl(grads), self._wl(errors), _ptrs(q),
-                                       _ptrs(p_hat) if p_hat is not None else None,
-                                       _ptrs(recon) if recon is not None else None,
-                                       _stream_handle(stream)))
+        sg, se, sq, sp, sr = self._validated(
+            "step", (self._flat(grads), self._flat(errors), q, p_hat, recon),
+            lambda: self._check_step_bufs(grads, errors, q, p_hat, recon))
+        self._check(self.lib.psgd_step(self._h, _arr_sig(sg), _arr_sig(se), _arr_sig(sq), self._opt(sp),
+                                       self._opt(sr), _stream_handle(stream)))
 
     def step_host(self, grads_host, errors, q, p_hat_host=None, q_host=None, stream=None):
-        self._check(self.lib.psgd_step_host(self._h, self._wl(grads_host), self._wl(errors), _ptrs(q),
-                                            _ptrs(p_hat_host) if p_hat_host is not None else None,
-                                            _ptrs(q_host) if q_host is not None else None,
-                                            _stream_handle(stream)))
+        def check():
+            self._check_step_bufs(grads_host, errors, q, p_hat_host, None, grads_on_device=False)
+            self._check_layers(q_host, "q_host", "nr", on_device=False, optional=True)
+        sg, se, sq, sp, sh = self._validated(
+            "step_host", (self._flat(grads_host), self._flat(errors), q, p_hat_host, q_host), check)
+        self._check(self.lib.psgd_step_host(self._h, _arr_sig(sg), _arr_sig(se), _arr_sig(sq), self._opt(sp),
+                                            self._opt(sh), _stream_handle(stream)))
 
     def step_host_flat(self, grads_host, layer_offsets, errors, q, p_hat_host=None, q_host=None, stream=None):
         """grads_host[w]: one host buffer per worker holding every layer,
         layer l starting at element layer_offsets[l]."""
-        offs = (ctypes.c_int64 * max(1, len(layer_offsets)))(*[int(o) for o in layer_offsets])
-        self._check(self.lib.psgd_step_host_flat(self._h, _ptrs(grads_host), offs, self._wl(errors), _ptrs(q),
-                                                 _ptrs(p_hat_host) if p_hat_host is not None else None,
-                                                 _ptrs(q_host) if q_host is not None else None,
-                                                 _stream_handle(stream)))
+        offsets = [int(o) for o in layer_offsets]
+
+        def check():
+            _check_list(offsets, "layer_offsets", len(self.layers))
+            _check_list(grads_host, "grads_host", self.workers)
+            span = max((o + m * n for o, (m, n) in zip(offsets, self.layers)), default=0)
+            for w in range(self.workers):
+                _check_buf(grads_host[w], f"grads_host[{w}]", span, self._gdt(), False, at_least=True)
+            self._check_wl(errors, "errors", _F32)
+            self._check_layers(q, "q", "nr")
+            self._check_layers(p_hat_host, "p_hat_host", "r", on_device=False, optional=True)
+            self._check_layers(q_host, "q_host", "nr", on_device=False, optional=True)
+        sg, so, se, sq, sp, sh = self._validated(
+            "step_host_flat", (grads_host, offsets, self._flat(errors), q, p_hat_host, q_host), check)
+        offs = (ctypes.c_int64 * max(1, len(offsets)))(*offsets)
+        self._check(self.lib.psgd_step_host_flat(self._h, _arr_sig(sg), offs, _arr_sig(se), _arr_sig(sq),
+                                                 self._opt(sp), self._opt(sh), _stream_handle(stream)))
 
     def materialize_errors(self, errors, stream=None):
-        self._check(self.lib.psgd_materialize_errors(self._h, self._wl(errors), _stream_handle(stream)))
+        (se,) = self._validated("materialize_errors", (self._flat(errors),),
+                                lambda: self._check_wl(errors, "errors", _F32))
+        self._check(self.lib.psgd_materialize_errors(self._h, _arr_sig(se), _stream_handle(stream)))
 
     def momentum_step(self, params, mom, lr: float, beta: float, stream=None):
-        self._check(self.lib.psgd_momentum_step(self._h, _ptrs(params), _ptrs(mom), lr, beta,
+        def check():
+            self._check_layers(params, "params", "n")
+            self._check_layers(mom, "mom", "n")
+        sx, sm = self._validated("momentum_step", (params, mom), check)
+        self._check(self.lib.psgd_momentum_step(self._h, _arr_sig(sx), _arr_sig(sm), lr, beta,
                                                 _stream_handle(stream)))
 
     def vec_mean(self, vecs, out, params=None, mom=None, lr: float = 0.0, beta: float = 0.0, stream=None):
         """vecs[w][k] -> out[k] = mean over workers (+ momentum if params, mom)."""
         K = len(out)
-        lens = (ctypes.c_int64 * max(1, K))(*[int(t.numel()) for t in out])
-        self._check(self.lib.psgd_vec_mean(self._h, self._wl(vecs), _ptrs(out), lens, K,
-                                           _ptrs(params) if params is not None else None,
-                                           _ptrs(mom) if mom is not None else None, lr, beta,
-                                           _stream_handle(stream)))
+
+        def check():
+            for k, t in enumerate(out):
+                if not isinstance(t, torch.Tensor):
+                    raise PsgdError(PSGD_ERR_ARG, f"out[{k}]: expected a tensor (its length sets the vector's)")
+                _check_buf(t, f"out[{k}]", t.numel(), _F32, True)
+            _check_list(vecs, "vecs", self.workers)
+            for w in range(self.workers):
+                _check_list(vecs[w], f"vecs[{w}]", K)
+                for k in range(K):
+                    _check_buf(vecs[w][k], f"vecs[{w}][{k}]", out[k].numel(), _F32, True)
+            for name, lst in (("params", params), ("mom", mom)):
+                if lst is not None:
+                    _check_list(lst, name, K)
+                    for k in range(K):
+                        _check_buf(lst[k], f"{name}[{k}]", out[k].numel(), _F32, True)
+        sv, so, sx, sm = self._validated("vec_mean", (self._flat(vecs), out, params, mom), check)
+        lens = (ctypes.c_int64 * max(1, K))(*so[1])
+        self._check(self.lib.psgd_vec_mean(self._h, _arr_sig(sv), _arr_sig(so), lens, K, self._opt(sx),
+                                           self._opt(sm), lr, beta, _stream_handle(stream)))
 
     # -- distributed step (the caller all-reduces p_send and q_send, SUM)
     def set_global_workers(self, total: int):
@@ -217,15 +365,22 @@ class PowerSGD:
         return int(pe.value), int(qe.value)
 
     def dist_p(self, grads, errors, q, p_send, p_hat=None, recon=None, stream=None):
-        self._check(self.lib.psgd_dist_p(self._h, self._wl(grads), self._wl(errors), _ptrs(q),
-                                         _ptrs(p_hat) if p_hat is not None else None,
-                                         _ptrs(recon) if recon is not None else None,
-                                         p_send.data_ptr(), _stream_handle(stream)))
+        def check():
+            self._check_step_bufs(grads, errors, q, p_hat, recon)
+            _check_buf(p_send, "p_send", 0, _F64, True, at_least=True)
+        sg, se, sq, sp, sr = self._validated(
+            "dist_p", (self._flat(grads), self._flat(errors), q, p_hat, recon), check)
+        _check_buf(p_send, "p_send", 0, _F64, True, at_least=True)
+        self._check(self.lib.psgd_dist_p(self._h, _arr_sig(sg), _arr_sig(se), _arr_sig(sq), self._opt(sp),
+                                         self._opt(sr), p_send.data_ptr(), _stream_handle(stream)))
 
     def dist_q(self, p_sum, q_send, stream=None):
+        _check_buf(p_sum, "p_sum", 0, _F64, True, at_least=True)
+        _check_buf(q_send, "q_send", 0, _F64, True, at_least=True)
         self._check(self.lib.psgd_dist_q(self._h, p_sum.data_ptr(), q_send.data_ptr(), _stream_handle(stream)))
 
     def dist_finish(self, q_sum, stream=None):
+        _check_buf(q_sum, "q_sum", 0, _F64, True, at_least=True)
         self._check(self.lib.psgd_dist_finish(self._h, q_sum.data_ptr(), _stream_handle(stream)))
 
     def profile(self, enable: bool = True):
