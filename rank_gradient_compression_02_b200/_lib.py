@@ -4,7 +4,7 @@ Argument marshalling only: tensors become device pointers, lists become
 pointer arrays, the current torch stream becomes a cudaStream_t.  Before an
 address crosses the ABI, each tensor's side (device or host), dtype,
 contiguity and size and each list's length are checked (again only when a
-call's buffers change).  Every step of the computation runs in the
+buffer address of the call changes).  Every step of the computation runs in the
 library's kernels; there is no fallback of any kind, and a missing library
 is an error.
 """
@@ -142,20 +142,18 @@ def _ptrs(values: Sequence) -> ctypes.Array:
     return _arr([_addr(v) for v in values])
 
 
-def _sig(values: Sequence) -> tuple:
-    """Addresses and element counts of a call's buffers: the checks run again
-    only when these change (the library re-uploads its pointer tables on
-    the same condition).  Entries that are raw addresses or None count -1
-    elements."""
+def _sig(values: Sequence) -> List:
+    """The addresses of a call's buffers (ints and None as they are): the
+    checks run again only when these change, the same condition on which
+    the library re-uploads its pointer tables."""
     try:
-        return [v.data_ptr() for v in values], [v.numel() for v in values]
+        return [v.data_ptr() for v in values]
     except AttributeError:
-        return ([_addr(v) for v in values],
-                [v.numel() if isinstance(v, torch.Tensor) else -1 for v in values])
+        return [_addr(v) for v in values]
 
 
-def _arr_sig(sig: tuple) -> ctypes.Array:
-    return _arr(sig[0])
+def _arr_sig(sig: List) -> ctypes.Array:
+    return _arr(sig)
 
 
 def _stream_handle(stream) -> int:
@@ -351,7 +349,7 @@ class PowerSGD:
                     for k in range(K):
                         _check_buf(lst[k], f"{name}[{k}]", out[k].numel(), _F32, True)
         sv, so, sx, sm = self._validated("vec_mean", (self._flat(vecs), out, params, mom), check)
-        lens = (ctypes.c_int64 * max(1, K))(*so[1])
+        lens = (ctypes.c_int64 * max(1, K))(*[t.numel() for t in out])
         self._check(self.lib.psgd_vec_mean(self._h, _arr_sig(sv), _arr_sig(so), lens, K, self._opt(sx),
                                            self._opt(sm), lr, beta, _stream_handle(stream)))
 

@@ -1,8 +1,8 @@
 """The binding's host-side checks (CPU, stub library): every buffer is
 checked for side (device or host), dtype, contiguity and size, and every
 list for its length, before an address crosses the ABI; the addresses
-passed are the tensors' own, worker-major; checks run again only when a
-call's buffers change.  "Device" tensors are CPU tensors marked as such."""
+passed are the tensors' own, worker-major; checks run again only when an
+address of the call changes.  "Device" tensors are CPU tensors marked as such."""
 import ctypes
 
 import pytest
