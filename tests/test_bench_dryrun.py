@@ -208,3 +208,22 @@ def test_reference_arm_falls_back_to_one_layer_per_step(fake_gpu, monkeypatch, c
                         lambda *a, _f=bench.run_reference: _f(*a, full_max_elements=0))
     d = _run(monkeypatch, capsys, "--impl", "reference", "--steps", "3", "--warmup", "3")
     assert d["value"] > 0 and d["cpu_baseline"]["sample"].startswith("each step: one layer")
+
+
+def test_json_line_lazy_mode(fake_gpu, monkeypatch, capsys):
+    wl = fake_gpu
+    d = _run(monkeypatch, capsys, "--lazy", "--steps", "3", "--warmup", "3", "--no-cpu-baseline", "--no-e2e")
+    assert d["config"]["mode"] == "lazy" and d["variants"] == {}
+    rl = d["roofline"]
+    # lazy: no third pass; the step moves G, E and M once each plus M again in pass B
+    assert rl["per_kernel_ms"]["pass_c"] == 0.2   # the recorder's figure; the bytes model ignores it
+    assert rl["step_dram_frac"] == pytest.approx(wl.elements * 16 / (d["ms_per_step"] * 1e-3) / 1e9 / rl["peak"],
+                                                 rel=1e-3, abs=1e-4)
+    assert _Recorder.created[0].lazy
+
+
+def test_json_line_sum_first_and_power_iterations(fake_gpu, monkeypatch, capsys):
+    d = _run(monkeypatch, capsys, "--sum-first", "--iters", "2", "--steps", "3", "--warmup", "3",
+             "--no-cpu-baseline", "--no-e2e", "--no-variants")
+    assert d["config"]["mode"] == "eager+sumfirst+iters2"
+    assert "step_dram_frac" not in d["roofline"]       # the bytes model covers one iteration only
