@@ -306,6 +306,45 @@ def launches_per_step(lib, B, dist: bool = False):
     return n
 
 
+def roofline_block(wl, r: int, mode: str, kern_ms, kern_steps: int, ms_per_step: float, clk,
+                   lazy: bool = False, sum_first: bool = False, iters: int = 1) -> dict:
+    """The JSON line's roofline object: the dominant pass's algorithmic
+    bytes per launch over its average event-timed launch (pass A reads G
+    and E, or M, and writes M; pass B reads M; pass C reads M and writes
+    E'), against the measured copy bandwidth; the step's minimum and design
+    bytes over the step time; at r >= 16 the products' compute side."""
+    peak, peak_kind = _peaks()
+    gsz = 2 if wl.grad_dtype == "bf16" else 4
+    per_launch_ms = [k / max(1, kern_steps) for k in kern_ms]
+    alg = [wl.elements * (gsz + 8), wl.elements * 4, 0 if lazy else wl.elements * 8]
+    names = ["pass_a", "pass_b", "pass_c"]
+    dom = max(range(3), key=lambda i: per_launch_ms[i])
+    achieved = alg[dom] / (per_launch_ms[dom] * 1e-3) / 1e9 if per_launch_ms[dom] > 0 else 0.0
+    traffic = _traffic_record(wl.name, mode) if dom == 0 else None
+    step_min_bytes = wl.elements * (gsz + 8)
+    roofline = {"bound": "hbm", "kernel": names[dom], "achieved": round(achieved, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_kind": f"{peak_kind} hbm_gbs",
+                "per_kernel_ms": {n: round(t, 4) for n, t in zip(names, per_launch_ms)},
+                "step_algorithmic_frac": round(step_min_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 4)}
+    if iters == 1:
+        # achieved DRAM bandwidth of the whole step: the bytes the three
+        # passes move (ncu puts each pass's traffic at its design bytes)
+        roofline["step_dram_frac"] = round(sum(alg) / (ms_per_step * 1e-3) / 1e9 / peak, 4)
+    if r >= 16:
+        # at ranks 16 and 32 the first two passes are bound by instruction
+        # issue, not HBM: report their compute side too
+        pk = {}
+        pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+        if os.path.exists(pp):
+            with open(pp) as f:
+                pk = json.load(f)
+        sm_mhz = (clk or {}).get("sm_mhz") or pk.get("sm_max_mhz", 1965.0)
+        roofline["compute"] = compute_roofline(wl.elements, r, per_launch_ms[0], per_launch_ms[1], sm_mhz,
+                                               pk.get("bf16_tflops", 1590.0), sum_first, wl.workers)
+    return roofline
+
+
 # --------------------------------------------------------------------------
 # CPU oracle timing (bounded sample)
 
@@ -477,38 +516,11 @@ def main():
     ms_per_step = ms / args.steps
     value = job_value(wl.elements, world, ms_per_step)
 
-    # roofline of the dominant kernel (first pass unless measured otherwise)
-    peak, peak_kind = _peaks()
+    roofline = roofline_block(wl, r, mode, kern_ms, kern_steps, ms_per_step, clk, lazy=args.lazy,
+                              sum_first=args.sum_first, iters=args.iters)
+    peak = roofline["peak"]
     gsz = 2 if wl.grad_dtype == "bf16" else 4
-    per_launch_ms = [k / max(1, kern_steps) for k in kern_ms]
-    # algorithmic bytes per launch: pass A reads G and E (or M) and writes M;
-    # pass B reads M; pass C reads M and writes E'
-    alg = [wl.elements * (gsz + 8), wl.elements * 4, 0 if args.lazy else wl.elements * 8]
-    names = ["pass_a", "pass_b", "pass_c"]
-    dom = max(range(3), key=lambda i: per_launch_ms[i])
-    achieved = alg[dom] / (per_launch_ms[dom] * 1e-3) / 1e9 if per_launch_ms[dom] > 0 else 0.0
-    traffic = _traffic_record(wl.name, mode) if dom == 0 else None
     step_min_bytes = wl.elements * (gsz + 8)
-    roofline = {"bound": "hbm", "kernel": names[dom], "achieved": round(achieved, 1), "peak": peak,
-                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-                "peak_kind": f"{peak_kind} hbm_gbs",
-                "per_kernel_ms": {n: round(t, 4) for n, t in zip(names, per_launch_ms)},
-                "step_algorithmic_frac": round(step_min_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 4)}
-    if args.iters == 1:
-        # achieved DRAM bandwidth of the whole step: the bytes the three
-        # passes move (ncu puts each pass's traffic at its design bytes)
-        roofline["step_dram_frac"] = round(sum(alg) / (ms_per_step * 1e-3) / 1e9 / peak, 4)
-    if r >= 16:
-        # at ranks 16 and 32 the first two passes are bound by instruction
-        # issue, not HBM: report their compute side too
-        pk = {}
-        pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
-        if os.path.exists(pp):
-            with open(pp) as f:
-                pk = json.load(f)
-        sm_mhz = (clk or {}).get("sm_mhz") or pk.get("sm_max_mhz", 1965.0)
-        roofline["compute"] = compute_roofline(wl.elements, r, per_launch_ms[0], per_launch_ms[1], sm_mhz,
-                                               pk.get("bf16_tflops", 1590.0), args.sum_first, wl.workers)
 
     # the lazy-error representation of the same step (E' rebuilt inside the
     # next step's first pass; bit-identical results), timed the same way

@@ -6,6 +6,8 @@ import json
 import os
 import shutil
 
+import pytest
+
 import bench
 
 
@@ -69,3 +71,26 @@ def test_oracle_sample_runs_later_steps_with_state_carried():
     # the carried state is bounded: with no room for it, only the first step runs
     _, elements1, _, _, text1 = bench.oracle_sample(wl, 2, budget_s=10.0, carry_bytes=0)
     assert elements1 == per_step and " over 1 step(s) " in text1
+
+
+def test_roofline_block_picks_the_dominant_pass():
+    from synth import Workload
+    wl = Workload(name="t", layers=((1000, 1000),), rank=2, workers=4, steps=1)
+    el = wl.elements
+    # pass C the slowest: its bytes (read M, write E') over its time
+    rl = bench.roofline_block(wl, 2, "eager", [1.0, 0.5, 2.0], 2, 2.0, None)
+    assert rl["kernel"] == "pass_c" and rl["traffic"] is None
+    assert rl["achieved"] == pytest.approx(el * 8 / 1e-3 / 1e9, abs=0.051)
+    assert rl["step_dram_frac"] == pytest.approx(el * 24 / 2e-3 / 1e9 / rl["peak"], abs=1e-4)
+    assert rl["step_algorithmic_frac"] == pytest.approx(el * 12 / 2e-3 / 1e9 / rl["peak"], abs=1e-4)
+    assert "compute" not in rl
+    # lazy mode moves 16 bytes per worker element; bf16 gradients 2 fewer
+    rl = bench.roofline_block(wl, 2, "lazy", [1.0, 0.5, 0.0], 1, 1.0, None, lazy=True)
+    assert rl["kernel"] == "pass_a" and rl["step_dram_frac"] == pytest.approx(el * 16 / 1e-3 / 1e9 / rl["peak"],
+                                                                              abs=1e-4)
+    from dataclasses import replace
+    rl = bench.roofline_block(replace(wl, grad_dtype="bf16"), 2, "eager", [1.0, 0.5, 0.5], 1, 2.0, None)
+    assert rl["achieved"] == pytest.approx(el * 10 / 1e-3 / 1e9, abs=0.051)
+    # ranks 16 and 32 add the compute side; power iterations drop the bytes model
+    rl = bench.roofline_block(wl, 16, "eager", [1.0, 0.5, 0.5], 1, 2.0, {"sm_mhz": 1965.0}, iters=2)
+    assert "compute" in rl and "step_dram_frac" not in rl
