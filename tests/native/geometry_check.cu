@@ -1,0 +1,40 @@
+// Host-side check of the library's own tile geometry and shared-memory
+// sizing (csrc/psgd.cu included as is) over the shapes, ranks and worker
+// counts the GPU tests use; run on the CPU, no device call is made.
+#include "psgd.cu"
+#include <cstdio>
+int main() {
+    struct Case { int64_t m, n; int r, W; };
+    std::vector<Case> cs;
+    int64_t mixed[][2] = {{300,650},{64,576},{40,130},{256,128},{33,37},{700,33},{129,1000}};
+    for (int r : {1,2,3,4,8,16,32}) for (int W : {1,3,16,64,256}) for (auto& s : mixed) cs.push_back({s[0], s[1], r, W});
+    int64_t full[][3] = {{2,64,2},{50,2,2},{4,90,4},{70,4,4},{8,100,8},{100,8,8},{16,160,16},{200,16,16},{32,400,32},{300,32,32},
+                         {96,130,16},{40,64,16},{1,64,1},{9,7,1},{35,33,8},{1,40,1},{8,8,1}};
+    for (auto& f : full) for (int W : {1,2,3,256}) cs.push_back({f[0], f[1], (int)f[2], W});
+    int bad = 0, n = 0;
+    for (auto& c : cs) {
+        if (c.r > c.m || c.r > c.n) continue;
+        const int R = pad_rank(c.r);
+        LayerSizes sz{};
+        LayerDesc d = layer_geometry(c.m, c.n, R, c.W, &sz);
+        ++n;
+        auto fail = [&](const char* what) { ++bad; std::printf("FAIL %s: m=%lld n=%lld r=%d W=%d tm=%d vec=%d slots=%d nchunk=%d\n", what,
+            (long long)c.m, (long long)c.n, c.r, c.W, d.tm, d.vec, d.slots, d.nchunk); };
+        if (c.n % d.vec) fail("vec divides n");
+        if (d.vec > max_vec_for_rank(R)) fail("vec within the rank's limit");
+        if (d.slots < 1 || d.slots > 32) fail("slots in 1..32");
+        if ((int64_t)d.nchunk * d.slots < d.nvec || (int64_t)(d.nchunk - 1) * d.slots >= d.nvec) fail("chunks cover the row, none empty");
+        if ((int64_t)d.nrb * d.tm < c.m || (int64_t)(d.nrb - 1) * d.tm >= c.m) fail("row blocks cover the matrix, none empty");
+        if (d.tm % 8) fail("tm multiple of 8");
+        if (R >= 16 && d.tm != 16 && d.tm != 32 && d.tm != 64) fail("tensor-core tiles of 16/32/64 rows");
+        if ((int64_t)d.tm * R > kRowsFloatsMax) fail("rows buffer");
+        if (d.slots * d.vec > 4 * psgd::kWideCols) fail("chunk within the k-steps");
+        for (int lazy = 0; lazy < 2; ++lazy) {
+            size_t a = smem_need(0, R, c.W, d.tm, d.vec, lazy), b = smem_need(1, R, c.W, d.tm, d.vec), cc = smem_need(2, R, c.W, d.tm, d.vec);
+            if (a > 232448 || b > 232448 || cc > 232448 || !a || !b || !cc) fail("shared memory within 227 KB");
+        }
+        if (sz.tiles != (int64_t)d.nrb * d.nchunk) fail("tile count");
+    }
+    std::printf("%d cases, %d failures\n", n, bad);
+    return bad != 0;
+}
