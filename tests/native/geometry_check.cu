@@ -11,6 +11,19 @@ int main() {
     int64_t full[][3] = {{2,64,2},{50,2,2},{4,90,4},{70,4,4},{8,100,8},{100,8,8},{16,160,16},{200,16,16},{32,400,32},{300,32,32},
                          {96,130,16},{40,64,16},{1,64,1},{9,7,1},{35,33,8},{1,40,1},{8,8,1}};
     for (auto& f : full) for (int W : {1,2,3,256}) cs.push_back({f[0], f[1], (int)f[2], W});
+    // the full-size workloads: ResNet-18 set (r = 2, W = 16), LSTM set (r = 4,
+    // W = 16), transformer set (r = 4, W = 4), the two sweeps (W = 8, r = 1..32)
+    int64_t resnet[][2] = {{64,576},{128,576},{128,1152},{256,1152},{256,2304},{512,2304},{512,4608},
+                           {128,64},{256,128},{512,256},{10,512}};
+    for (auto& s : resnet) cs.push_back({s[0], s[1], 2, 16});
+    cs.push_back({2600, 650, 4, 16});
+    cs.push_back({33280, 650, 4, 16});
+    int64_t tf[][2] = {{4096,12288},{4096,4096},{16384,4096},{4096,16384}};
+    for (auto& s : tf) cs.push_back({s[0], s[1], 4, 4});
+    for (int r : {1,2,3,4,8,16,32}) {
+        cs.push_back({8192, 8192, r, 8});
+        cs.push_back({1024, 1024, r, 8});
+    }
     int bad = 0, n = 0;
     for (auto& c : cs) {
         if (c.r > c.m || c.r > c.n) continue;

@@ -1,6 +1,7 @@
 """The library's tile geometry, checked in its own host code on the CPU:
 tests/native/geometry_check.cu includes csrc/psgd.cu unchanged and checks,
-for every shape, rank and worker count the GPU tests use, that the lane
+for every shape, rank and worker count the GPU tests and the full-size
+workloads use, that the lane
 width divides the row, chunks and row blocks cover the matrix with none
 empty, the tensor-core tiles are whole 16-row groups, the rows buffer and
 the widest chunk fit, and each pass's shared memory fits in 227 KB."""
