@@ -1,23 +1,30 @@
 """Benchmark of the PowerSGD compression step on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 3] [--impl ours|reference]
 
 One step = the whole hot path over one batch of synthetic gradients held in
 HBM: psgd_step (error-feedback add, P = MQ, worker mean, orthogonalisation,
-Q = M^T P_hat, worker mean, residual), the uncompressed mean of the 1-D
-tensors and the post-compression momentum update, all through the C ABI.
-Metric: gradient elements compressed per second (W * sum(m*n) per step),
-whole job.  On one GPU the W workers are replica buffers and the worker
-means are on-device sums.  With N GPUs (torchrun, NCCL) every rank holds W
-workers and runs the distributed step: the P and Q partial sums (and the
-1-D gradients) are all-reduced between the library's three calls, so the
-job has N * W workers (weak scaling) and value = N * elements / max over
-ranks of the device time.  Rank 0 prints one JSON line with the roofline of
-the dominant kernel (HBM; plus the products' compute side at ranks 16 and
-32), the end-to-end figure through host buffers (psgd_step_host_flat), the
-clocks seen during the timed region and, on one GPU, the float64 oracle
-timed on the host cores.  --impl reference times that oracle as the
-reference arm.
+Q = M^T P_hat, worker mean, residual), plus, where the workload has them,
+the uncompressed mean of the 1-D tensors and the post-compression momentum
+update, all through the C ABI.  The default workload is the transformer-block
+set (24 x (4096x12288, 4096x4096, 16384x4096, 4096x16384), bf16 gradients,
+fp32 error memory, rank 4, 4 workers: 19.3 G worker elements per step), the
+largest that fits one GPU.  Metric: gradient elements compressed per second
+(W * sum(m*n) per step), whole job.  On one GPU the W workers are replica
+buffers and the worker means are on-device sums.  With N GPUs (torchrun,
+NCCL) every rank holds W workers and runs the distributed step: the P and Q
+partial sums (and the 1-D gradients) are all-reduced between the library's
+three calls, so the job has N * W workers (weak scaling) and value = N *
+elements / max over ranks of the device time.
+
+Rank 0 prints one JSON line: the roofline of the dominant kernel (HBM; plus
+the products' compute side at ranks 16 and 32), the end-to-end figure
+through host buffers (psgd_step_host_flat), the clocks seen from the
+warm-up to the end of the timed region, the compression ratio and payload,
+on one GPU the float64 oracle timed on the host cores, and "workloads": the
+other workloads' eager steps (the LSTM set, the 8192^2 and 256 x 1024^2
+rank sweeps with the subspace error of the latter, the ResNet-18 set), each
+timed the same way.  --impl reference times the oracle as the reference arm.
 """
 from __future__ import annotations
 
@@ -134,16 +141,27 @@ class ClockSampler:
         self.proc = None
         self.path = None
 
-    def start(self):
+    def start(self, interval_ms: int = 50, wait_first_s: float = 5.0):
+        """Start sampling; waits (up to wait_first_s) for the first sample so
+        that a short timed region is still covered."""
         try:
             import tempfile
             self.path = os.path.join(tempfile.gettempdir(), f"clocks_bench_{os.getpid()}.csv")
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+                 "-lms", str(interval_ms)], stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        t0 = time.time()
+        while time.time() - t0 < wait_first_s and self.proc.poll() is None:
+            try:
+                if os.path.getsize(self.path) > 0:
+                    break
+            except OSError:
+                pass
+            time.sleep(0.05)
 
     def stop(self):
         if self.proc is None:
@@ -210,9 +228,9 @@ class Buffers:
                   for w in range(W)]
         src = GradientSource(wl, seed)
         self.src = src
+        self.device = device
         src.fill(0, self.G)
-        self.Q = [src.initial_q(l, rank).to(device) for l in range(L)]
-        self.P = [torch.empty(m, rank, device=device) for (m, _) in wl.layers]
+        self.set_rank(rank)
         self.params = self.mom = None
         if wl.momentum:
             self.params = [torch.zeros(m, n, device=device) for (m, n) in wl.layers]
@@ -223,6 +241,21 @@ class Buffers:
             self.vout = [torch.empty(k, device=device) for k in wl.vectors]
             self.vx = [torch.zeros(k, device=device) for k in wl.vectors]
             self.vmom = [torch.zeros(k, device=device) for k in wl.vectors]
+
+    def set_rank(self, rank):
+        """Initial Q and P_hat buffers for rank r; the error memory starts
+        from zero again (a fresh run of the same gradients at another rank)."""
+        self.rank = rank
+        L = len(self.wl.layers)
+        self.Q = [self.src.initial_q(l, rank).to(self.device) for l in range(L)]
+        self.P = [torch.empty(m, rank, device=self.device) for (m, _) in self.wl.layers]
+        for e in self.E_flat:
+            e.zero_()
+
+    def release(self):
+        """Drop every device buffer (the caller then empties torch's cache)."""
+        for name in ("G_flat", "E_flat", "G", "E", "Q", "P", "params", "mom", "vecs", "vout", "vx", "vmom"):
+            setattr(self, name, None)
 
 
 def device_bytes_needed(wl, rank):
@@ -366,6 +399,7 @@ def oracle_sample(wl, rank, budget_s=15.0, seed=1234, max_layers=None, carry_byt
     nl = len(wl.layers) if max_layers is None else min(max_layers, len(wl.layers))
     carry = wl.workers * sum(m * n for (m, n) in wl.layers[:nl]) * 8 <= carry_bytes
     state = {}
+    shapes = []
     step = 0
     while spent < budget_s and nl > 0 and (step == 0 or carry):
         steps_begun += 1
@@ -382,16 +416,215 @@ def oracle_sample(wl, rank, budget_s=15.0, seed=1234, max_layers=None, carry_byt
             spent += time.perf_counter() - t0
             done_el += wl.workers * m * n
             layers_done += 1
+            if (m, n) not in shapes:
+                shapes.append((m, n))
             if carry:
                 state[l] = (res["E_new"], res["Q_bar"])
             del G, E, res
             if spent >= budget_s:
                 break
         step += 1
+    distinct = len(set(wl.layers[:nl]))
     text = (f"{layers_done} layer-steps over {steps_begun} step(s) of {len(wl.layers)} layers (all {wl.workers} "
             f"workers, error memory and Q carried, float64 NumPy; BLAS threads {threads}, elementwise ops "
-            f"single-threaded)")
+            f"single-threaded); shapes sampled {len(shapes)} of {distinct}: "
+            + ", ".join(f"{m}x{n}" for m, n in shapes))
     return done_el / spent, done_el, spent, threads, text
+
+
+# --------------------------------------------------------------------------
+# reports that need no timing
+
+def compression_report(wl, r: int) -> dict:
+    """What one worker sends per step with and without compression: the
+    factors P (m x r) and Q (n x r) in float32, against the gradient itself
+    (the "PowerSGD" glossary page: O(r(m + n)) instead of O(mn)); also the
+    float64 P and Q partial sums the library's distributed step all-reduces
+    (rank padded to a power of two)."""
+    smn = sum(m * n for m, n in wl.layers)
+    smpn = sum(m + n for m, n in wl.layers)
+    R = 1
+    while R < r:
+        R *= 2
+    gsz = 2 if wl.grad_dtype == "bf16" else 4
+    return {"ratio": round(smn / (r * smpn), 2), "factor_bytes_per_worker": 4 * r * smpn,
+            "gradient_bytes_per_worker": gsz * smn, "dist_partial_bytes_per_rank": 8 * R * smpn}
+
+
+def sin_theta_max(U_ref: np.ndarray, P: np.ndarray) -> float:
+    """Largest principal-angle sine between span(U_ref) and span(P) (both
+    with orthonormal columns): the spectral norm of (I - U_ref U_ref^T) P."""
+    Rm = P - U_ref @ (U_ref.T @ P)
+    return float(np.linalg.norm(Rm, 2))
+
+
+# --------------------------------------------------------------------------
+# timing helpers
+
+def timed_steps(step_fn, steps: int, warmup: int, lib, stream, barrier=lambda: None, before_timed=None):
+    """warmup untimed steps, then exactly `steps` steps between two CUDA
+    events on `stream`, with the library's per-pass events on.  Returns
+    (ms per step, summed per-pass ms, profiled steps)."""
+    for _ in range(warmup):
+        step_fn()
+    lib.status()
+    barrier()
+    torch.cuda.synchronize()
+    if before_timed is not None:
+        before_timed()
+    lib.profile(True)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        step_fn()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    kern_ms, kern_steps = lib.profile_read()
+    lib.profile(False)
+    lib.status()
+    return ms / max(1, steps), kern_ms, kern_steps
+
+
+def _host_ram_available() -> float:
+    try:
+        with open("/proc/meminfo") as f:
+            for line in f:
+                if line.startswith("MemAvailable"):
+                    return int(line.split()[1]) * 1024.0
+    except Exception:
+        pass
+    return 0.0
+
+
+def _pinned_empty(numel: int, dtype):
+    return torch.empty(numel, dtype=dtype, pin_memory=True)
+
+
+def _free_device_cache():
+    import gc
+    gc.collect()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+# --------------------------------------------------------------------------
+# the other workloads (one GPU): eager step per workload and rank
+
+def workload_line(wl, r: int, steps: int, warmup: int, stream, B=None, lazy_variant=False) -> dict:
+    """Time the eager step of one workload at rank r (buffers B reused when
+    given) and return its figures: ms per step, elements/s, the step's
+    design-byte (DRAM) and minimum-byte fractions of the measured peak, and
+    the per-pass times."""
+    from rank_gradient_compression_02_b200 import PowerSGD
+    lib = PowerSGD(wl.layers, r, wl.workers, grad_dtype=wl.grad_dtype)
+    try:
+        ms, kern_ms, ks = timed_steps(lambda: run_step(lib, B, wl), steps, warmup, lib, stream)
+    finally:
+        lib.close()
+    rl = roofline_block(wl, r, "eager", kern_ms, ks, ms, None)
+    out = {"rank": r, "ms_per_step": round(ms, 4), "value": job_value(wl.elements, 1, ms),
+           "step_dram_frac": rl.get("step_dram_frac"), "step_algorithmic_frac": rl["step_algorithmic_frac"],
+           "dominant": rl["kernel"], "dominant_frac": rl["frac"], "per_kernel_ms": rl["per_kernel_ms"],
+           "pass_a_frac": round(wl.elements * ((2 if wl.grad_dtype == "bf16" else 4) + 8)
+                                / (rl["per_kernel_ms"]["pass_a"] * 1e-3) / 1e9 / rl["peak"], 4)
+           if rl["per_kernel_ms"]["pass_a"] > 0 else None,
+           "steps": steps}
+    if "compute" in rl:
+        out["compute"] = {k: rl["compute"][k] for k in ("achieved", "unit", "fp32_frac", "tf32_frac")}
+    if lazy_variant:
+        B.set_rank(r)
+        lib = PowerSGD(wl.layers, r, wl.workers, grad_dtype=wl.grad_dtype, lazy_errors=True)
+        try:
+            lms, _, _ = timed_steps(lambda: run_step(lib, B, wl), steps, warmup, lib, stream)
+        finally:
+            lib.close()
+        peak = rl["peak"]
+        gsz = 2 if wl.grad_dtype == "bf16" else 4
+        out["lazy_errors"] = {"ms_per_step": round(lms, 4), "value": job_value(wl.elements, 1, lms),
+                              "step_dram_frac": round(wl.elements * (gsz + 12) / (lms * 1e-3) / 1e9 / peak, 4),
+                              "step_algorithmic_frac": round(wl.elements * (gsz + 8) / (lms * 1e-3) / 1e9 / peak,
+                                                             4)}
+    return out
+
+
+def subspace_error_report(wl, ranks, device, steps: int, seed: int = 1234) -> dict:
+    """Per rank: run `steps` warm-started steps of the workload's first
+    matrix (its own seeded, slowly rotating gradients, all workers, error
+    feedback) through the library and report sin of the largest principal
+    angle between the last step's P_hat and the top-r left singular
+    subspace of that step's worker mean M_bar = mean_w(G_w + E_w), from a
+    float64 LAPACK SVD on the host."""
+    from dataclasses import replace
+    from rank_gradient_compression_02_b200 import PowerSGD
+    one = replace(wl, layers=wl.layers[:1])
+    m, n = one.layers[0]
+    W = one.workers
+    out = {}
+    for r in ranks:
+        src = GradientSource(one.with_rank(r), seed)
+        gdt = torch.bfloat16 if one.grad_dtype == "bf16" else torch.float32
+        G = [[torch.empty(m, n, dtype=gdt, device=device)] for _ in range(W)]
+        E = [[torch.zeros(m, n, device=device)] for _ in range(W)]
+        Q = [src.initial_q(0, r).to(device)]
+        P = [torch.empty(m, r, device=device)]
+        lib = PowerSGD(one.layers, r, W, grad_dtype=one.grad_dtype)
+        try:
+            for t in range(steps):
+                src.fill(t, G)
+                if t == steps - 1:
+                    Mbar = sum(G[w][0].double() + E[w][0].double() for w in range(W)) / W
+                lib.step(G, E, Q, P, None)
+            torch.cuda.synchronize()
+            lib.status()
+        finally:
+            lib.close()
+        U = np.linalg.svd(Mbar.cpu().numpy(), full_matrices=False)[0][:, :r]
+        Ph = P[0].double().cpu().numpy()
+        gated = r <= one.spectrum_terms
+        out[str(r)] = {"sin_theta_max": sin_theta_max(U, Ph), "steps": steps,
+                       "status": "gated" if gated else "reported, not gated (directions beyond the "
+                                                         f"{one.spectrum_terms}-term spectrum are noise)"}
+        del G, E, Q, P, Mbar
+    return {"matrix": f"{m}x{n}", "workers": W,
+            "reference": "float64 LAPACK SVD of the last step's worker mean (numpy.linalg.svd)", "by_rank": out}
+
+
+def run_workloads(keys, steps: int, warmup: int, device, stream, subspace_steps=None) -> dict:
+    """The other workloads' eager steps on this GPU, one after another (each
+    allocated, timed and released), with the rank sweeps of the sweep
+    workloads, their compression figures and, for the 1024 x 1024 sweep,
+    the subspace error."""
+    res = {}
+    for key in keys:
+        wl = get_workload(key)
+        ranks = list(wl.ranks) if wl.ranks else [wl.rank]
+        if device_bytes_needed(wl, ranks[-1]) > torch.cuda.mem_get_info()[0] * 0.9:
+            res[wl.name] = {"skipped": "not enough free device memory"}
+            continue
+        B = Buffers(wl, ranks[0], device)
+        entry = {"elements_per_step": wl.elements, "workers": wl.workers, "grad_dtype": wl.grad_dtype,
+                 "l2": "inputs larger than L2 (no flush needed)" if wl.elements * 4 > 4 * 126e6 else "inputs fit L2"}
+        if wl.ranks:
+            entry["by_rank"] = {}
+            for r in ranks:
+                B.set_rank(r)
+                line = workload_line(wl.with_rank(r), r, steps, warmup, stream, B)
+                line["compression"] = compression_report(wl, r)
+                entry["by_rank"][str(r)] = line
+        else:
+            entry.update(workload_line(wl, wl.rank, steps, warmup, stream, B, lazy_variant=True))
+            entry["compression"] = compression_report(wl, wl.rank)
+        B.release()
+        del B
+        _free_device_cache()
+        if wl.rotate and len(wl.layers) > 1:
+            entry["subspace_error"] = subspace_error_report(wl, ranks, device,
+                                                            subspace_steps or wl.steps)
+        res[wl.name] = entry
+    return res
 
 
 # --------------------------------------------------------------------------
@@ -399,21 +632,28 @@ def oracle_sample(wl, rank, budget_s=15.0, seed=1234, max_layers=None, carry_byt
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="1", help="workload: 0, 1, 2, 3, 4a, 4b or a name")
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="3", help="workload: 0, 1, 2, 3, 4a, 4b or a name (default 3, the "
+                                                  "transformer set: the largest that fits one GPU)")
     ap.add_argument("--rank", type=int, default=None, help="rank r (default: the workload's)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--lazy", action="store_true", help="lazy error representation")
     ap.add_argument("--sum-first", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--oracle-budget", type=float, default=15.0)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--oracle-budget", type=float, default=20.0)
     ap.add_argument("--layers", default=None, help="comma-separated layer indices (a subset, for small captures)")
     ap.add_argument("--workers", type=int, default=None, help="override the worker count (small captures)")
     ap.add_argument("--iters", type=int, default=1, help="power iterations per step")
     ap.add_argument("--no-variants", action="store_true", help="skip timing the lazy-error variant")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other workloads' sub-lines (LSTM, ResNet-18, the two sweeps)")
+    ap.add_argument("--workloads", default="2,4a,4b,1", help="workloads of the sub-lines")
+    ap.add_argument("--workload-steps", type=int, default=10)
+    ap.add_argument("--subspace-steps", type=int, default=None,
+                    help="steps of the subspace-error runs (default: the workload's own)")
     ap.add_argument("--dist", action="store_true",
                     help="use the distributed step with NCCL all-reduces even on one GPU")
     args = ap.parse_args()
@@ -490,30 +730,13 @@ def main():
         if world > 1:
             dist.barrier()
 
-    for _ in range(args.warmup):
-        step_fn()
-    lib.status()
-    barrier()
-    torch.cuda.synchronize()
+    # clocks sampled from before the warm-up to the end of the timed region
     clocks = ClockSampler(local if world > 1 else 0)
     clocks.start()
-    lib.profile(True)
     stream = torch.cuda.current_stream()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step_fn()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    ms = ev0.elapsed_time(ev1)
-    kern_ms, kern_steps = lib.profile_read()
-    lib.profile(False)
+    ms_per_step, kern_ms, kern_steps = timed_steps(step_fn, args.steps, args.warmup, lib, stream, barrier)
     clk = clocks.stop()
-    lib.status()
-    ms = max_over_ranks(ms, world, device)
-    ms_per_step = ms / args.steps
+    ms_per_step = max_over_ranks(ms_per_step * args.steps, world, device) / args.steps
     value = job_value(wl.elements, world, ms_per_step)
 
     roofline = roofline_block(wl, r, mode, kern_ms, kern_steps, ms_per_step, clk, lazy=args.lazy,
@@ -550,26 +773,39 @@ def main():
                                            "of the timed region"}
         lazy_lib.close()
 
-    e2e = None
-    if not args.no_e2e:
-        e2e = run_e2e(lib, B, wl, r, args, world, device, DB if dist_mode else None)
-
     cpu = None
     if rank_id == 0 and world == 1 and not args.no_cpu_baseline:
         v, el, sec, threads, text = oracle_sample(wl, r, budget_s=args.oracle_budget)
         cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": text,
                "seconds": round(sec, 2)}
 
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(lib, B, wl, r, args, world, device, DB if dist_mode else None)
+
+    launches = args.steps * launches_per_step(lib, B, dist_mode)
+    lib.close()
+    B.release()
+    del B
+    if dist_mode:
+        del DB
+    _free_device_cache()
+
+    workloads = None
+    if world == 1 and not dist_mode and not args.no_workloads and not args.layers and not args.workers:
+        keys = [k for k in args.workloads.split(",") if k and get_workload(k).name != wl.name]
+        workloads = run_workloads(keys, args.workload_steps, 3, device, stream, args.subspace_steps)
+
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f32" if wl.grad_dtype == "f32" else "bf16-in/f32",
            "data": "synthetic (seeded low-rank + noise gradients, resident in HBM)",
-           "config": config, "gpu_launches": args.steps * launches_per_step(lib, B, dist_mode),
+           "config": config, "gpu_launches": launches,
            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "variants": variants,
-           "hbm_gbs_step": round(step_min_bytes / (ms_per_step * 1e-3) / 1e9, 1)}
+           "hbm_gbs_step": round(step_min_bytes / (ms_per_step * 1e-3) / 1e9, 1),
+           "compression": compression_report(wl, r), "workloads": workloads}
     if rank_id == 0:
         print(json.dumps(out), flush=True)
-    lib.close()
     if world > 1 or args.dist:
         dist.destroy_process_group()
 
@@ -579,20 +815,32 @@ def run_e2e(lib, B, wl, r, args, world, device, DB=None):
     host gradients, one flat buffer per worker, copied in every step
     (psgd_step_host_flat on one GPU; one copy per worker into the device
     buffers before the distributed step on several), P_hat and Q_bar (and
-    the 1-D means) read back."""
+    the 1-D means) read back.  When the library's device staging of the
+    host gradients would not fit beside the resident buffers (the
+    transformer set: 38.7 GB of bf16 gradients beside 77 GB of error
+    memory), the device gradient buffers are released first: the staging
+    takes their place."""
     gsz = 2 if wl.grad_dtype == "bf16" else 4
-    host_bytes = wl.elements * gsz
-    if host_bytes > 16e9:
-        return {"value": None, "unit": UNIT, "skipped": "host copy of the gradients exceeds 16 GB"}
     import torch.distributed as dist
     W, L = wl.workers, len(wl.layers)
+    span = max(B.offs[l] + m * n for l, (m, n) in enumerate(wl.layers))
+    host_bytes = W * B.offs[-1] * gsz
+    if host_bytes * 1.25 + 8e9 > _host_ram_available():
+        return {"value": None, "unit": UNIT,
+                "skipped": f"host RAM too small for {host_bytes / 1e9:.1f} GB of pinned gradients"}
     # one pinned host buffer per worker holding every layer (a flat gradient
     # bucket), uploaded with one copy per worker
-    Gh = [torch.empty(B.offs[-1], dtype=B.G_flat[0].dtype).pin_memory() for _ in range(W)]
+    Gh = [_pinned_empty(B.offs[-1], B.G_flat[0].dtype) for _ in range(W)]
     for w in range(W):
         Gh[w].copy_(B.G_flat[w])
+    stage_bytes = W * ((span * gsz + 255) // 256 * 256)
+    released = False
+    if DB is None and stage_bytes > torch.cuda.mem_get_info()[0] * 0.9:
+        B.G_flat = None
+        B.G = None
+        _free_device_cache()
+        released = True
     layer_offs = [B.offs[l] for l in range(L)]
-    span = max(B.offs[l] + m * n for l, (m, n) in enumerate(wl.layers))
     Ph = [torch.empty(m, r).pin_memory() for (m, _) in wl.layers]
     Qh = [torch.empty(n, r).pin_memory() for (_, n) in wl.layers]
     vbytes = 0
@@ -667,8 +915,12 @@ def run_e2e(lib, B, wl, r, args, world, device, DB=None):
     per = ms / args.e2e_steps
     h2d = W * span * gsz + vbytes
     d2h = sum((m + n) * r * 4 for (m, n) in wl.layers) + (vout_h.numel() * 4 if B.vecs is not None else 0)
-    return {"value": wl.elements * world / (per * 1e-3), "unit": UNIT, "ms_per_step": per,
-            "steps": args.e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    out = {"value": wl.elements * world / (per * 1e-3), "unit": UNIT, "ms_per_step": per,
+           "steps": args.e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    if released:
+        out["note"] = "device gradient buffers released first; the library's staging holds the uploads"
+    del Gh
+    return out
 
 
 def run_reference(args, wl, r, config, world, full_max_elements=2e8, budget_s=180.0):

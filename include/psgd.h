@@ -215,9 +215,11 @@ PSGD_API int psgd_step_launches(const psgd_ctx *ctx);
  * partials, T, counters) lives in one file-scope static device array of
  * PSGD_STATIC_SCRATCH_BYTES (16 MiB).  Every GPU that loads the library
  * holds that array until the process exits.  The call allocates no device
- * memory and calls no allocating routine (the descriptor and pointer table
- * are staged from the stack); only a failed call stores its message in
- * thread-local host memory for psgd_last_error(NULL).
+ * memory and calls no allocating routine: a small set-up kernel, launched
+ * on `stream` with the layer descriptor and the pointer table passed by
+ * value, writes them into the array and clears the counters and the status
+ * word; only a failed call stores its message in thread-local host memory
+ * for psgd_last_error(NULL).
  *
  * grads[w], errors[w]: HOST arrays of W device pointers (m x n, grad dtype
  * and float32); q: device n x rank (warm start in, Q_bar out); p_hat:
@@ -237,6 +239,14 @@ PSGD_API int psgd_step_launches(const psgd_ctx *ctx);
 PSGD_API int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int grad_dtype,
                               const void *const *grads, float *const *errors, float *q, float *p_hat,
                               float *recon, void *stream);
+
+/* Status of the last psgd_step_static call on the current device (no
+ * counterpart in the pages): synchronises `stream`, then reads the status
+ * word at the head of the static array.  PSGD_OK, or PSGD_ERR_DEVICE when a
+ * kernel of that call found a reduction counter inconsistent (what calls
+ * that overlap on the GPU produce: their results are then wrong), or
+ * PSGD_ERR_CUDA.  Allocates nothing. */
+PSGD_API int psgd_step_static_status(void *stream);
 
 /* Distributed step.  On a real data-parallel job every rank (GPU) holds
  * its own workers (the context's `workers`, usually 1) and the two means of

@@ -60,6 +60,7 @@ _SIGS = {
     "psgd_last_error": (ctypes.c_char_p, [_P]),
     "psgd_step_static": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         _PP, _PP, _P, _P, _P, _P]),
+    "psgd_step_static_status": (ctypes.c_int, [_P]),
     "psgd_set_power_iters": (ctypes.c_int, [_P, ctypes.c_int]),
     "psgd_set_global_workers": (ctypes.c_int, [_P, ctypes.c_int]),
     "psgd_dist_sizes": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]),
@@ -184,6 +185,16 @@ def step_static(m: int, n: int, rank: int, grads, errors, q, p_hat=None, recon=N
                               _ptrs(grads), _ptrs(errors), q.data_ptr(),
                               p_hat.data_ptr() if p_hat is not None else None,
                               recon.data_ptr() if recon is not None else None, _stream_handle(stream))
+    if rc:
+        raise PsgdError(rc, lib.psgd_last_error(None).decode())
+
+
+def step_static_status(stream=None) -> None:
+    """Synchronise `stream` and raise if the last allocation-free step on
+    this device flagged a device-side inconsistency
+    (psgd_step_static_status)."""
+    lib = load()
+    rc = lib.psgd_step_static_status(_stream_handle(stream))
     if rc:
         raise PsgdError(rc, lib.psgd_last_error(None).decode())
 

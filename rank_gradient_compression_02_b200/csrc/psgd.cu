@@ -895,16 +895,29 @@ int psgd_vec_mean(psgd_ctx* ctx, const float* const* vecs, float* const* out, co
 // ---- allocation-free single-layer step ------------------------------------
 // All scratch of psgd_step_static lives in this array; host code never uses
 // its name as an address: the device address comes from
-// cudaGetSymbolAddress, looked up once per device.
+// cudaGetSymbolAddress, looked up once per device.  The first 256 bytes
+// hold the status word of the last call (kStaticStatusOffset); the layer's
+// scratch follows.
 static __device__ __align__(256) unsigned char g_psgd_static_scratch[PSGD_STATIC_SCRATCH_BYTES];
 
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr size_t kStaticStatusOffset = 0;
+constexpr size_t kStaticHeader = 256;
 std::mutex g_static_mu;
 void* g_static_addr[kMaxDevices] = {};
+// dynamic shared memory each kernel was opted in to on each device by this
+// entry point: [device][pass][log2 R][dtype] (bytes, 0 = not yet)
+size_t g_static_smem[kMaxDevices][3][6][2] = {};
 
-cudaError_t static_scratch_address(void** out) {
+int log2_rank(int R) {
+    int k = 0;
+    while ((1 << k) < R) ++k;
+    return k;
+}
+
+cudaError_t static_scratch_address(void** out, int* dev_out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -917,7 +930,54 @@ cudaError_t static_scratch_address(void** out) {
         g_static_addr[dev] = p;
     }
     *out = g_static_addr[dev];
+    *dev_out = dev;
     return cudaSuccess;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per (device, kernel,
+// size): later calls only read the cache.
+cudaError_t static_smem_opt_in(int dev, int which, int R, int dtype, const void* fn, size_t need) {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    size_t& have = g_static_smem[dev][which][log2_rank(R)][dtype == PSGD_BF16 ? 1 : 0];
+    if (have >= need) return cudaSuccess;
+    cudaFuncAttributes fa{};
+    cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+    if (e != cudaSuccess) return e;
+    if (static_cast<size_t>(fa.maxDynamicSharedSizeBytes) < need) {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(need));
+        if (e != cudaSuccess) return e;
+    }
+    have = need;
+    return cudaSuccess;
+}
+
+// Everything a call writes into the scratch before its three passes,
+// passed by value (no host staging buffer): the layer descriptor, the
+// pointer table (grads[W], errors[W], q, p_hat, recon) and the extents to
+// clear (tile map, counters) plus the status word.
+struct StaticSetup {
+    LayerDesc desc;
+    uint64_t tab[2 * psgd::kMaxWorkers + 3];
+    LayerDesc* desc_dst;
+    uint64_t* tab_dst;
+    int* tile_dst;
+    unsigned* cnt_dst;
+    int* status_dst;
+    int ntab;
+    int64_t ntiles, ncnt;
+};
+
+__global__ void k_static_setup(const StaticSetup s) {
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    if (tid == 0) {
+        *s.desc_dst = s.desc;
+        *s.status_dst = 0;
+    }
+    for (int64_t i = tid; i < s.ntab; i += stride) s.tab_dst[i] = s.tab[i];
+    // one layer: every tile maps to layer 0; counters start at zero
+    for (int64_t i = tid; i < s.ntiles; i += stride) s.tile_dst[i] = 0;
+    for (int64_t i = tid; i < s.ncnt; i += stride) s.cnt_dst[i] = 0u;
 }
 
 }  // namespace
@@ -946,8 +1006,8 @@ int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int grad_dtype
     LayerDesc d = layer_geometry(m, n, R, workers, &sz);
     const int64_t ntiles = sz.tiles;
 
-    // scratch layout inside the static array
-    size_t off = 0;
+    // scratch layout inside the static array (after the status header)
+    size_t off = kStaticHeader;
     auto carve = [&](size_t bytes) {
         const size_t o = off;
         off = align_up(off + std::max<size_t>(bytes, 1), 256);
@@ -967,7 +1027,6 @@ int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int grad_dtype
     const size_t o_qsup = carve(sizeof(double) * sz.qsup);
     const size_t o_T = carve(sizeof(double) * sz.t);
     const size_t o_cnt = carve(sizeof(unsigned) * sz.cnt);
-    const size_t o_status = carve(sizeof(int));
     if (off > PSGD_STATIC_SCRATCH_BYTES)
         return fail(nullptr, PSGD_ERR_ARG, "layer %lld x %lld at rank %d with %d workers needs %zu bytes of scratch; "
                     "the static scratch holds %u", (long long)m, (long long)n, rank, workers, off,
@@ -978,27 +1037,47 @@ int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int grad_dtype
         d.cnt_off = 0;
 
     void* base_v = nullptr;
-    cudaError_t e = static_scratch_address(&base_v);
+    int dev = 0;
+    cudaError_t e = static_scratch_address(&base_v, &dev);
     if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "static scratch address: %s", cudaGetErrorString(e));
     unsigned char* base = static_cast<unsigned char*>(base_v);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    // descriptor and pointer table from host stack memory (no allocation)
-    uint64_t tab[2 * psgd::kMaxWorkers + 3];
-    for (int w = 0; w < workers; ++w) {
-        tab[w] = reinterpret_cast<uint64_t>(grads[w]);
-        tab[workers + w] = reinterpret_cast<uint64_t>(errors[w]);
+    const size_t smem[3] = {smem_need(0, R, workers, d.tm, d.vec), smem_need(1, R, workers, d.tm, d.vec),
+                            smem_need(2, R, workers, d.tm, d.vec)};
+    void* fns[3];
+    for (int which = 0; which < 3; ++which) {
+        fns[which] = kernel_ptr(which, R, grad_dtype, false, false);
+        e = static_smem_opt_in(dev, which, R, grad_dtype, fns[which], smem[which]);
+        if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "shared-memory opt-in: %s", cudaGetErrorString(e));
     }
-    tab[2 * workers] = reinterpret_cast<uint64_t>(q);
-    tab[2 * workers + 1] = reinterpret_cast<uint64_t>(p_hat);
-    tab[2 * workers + 2] = reinterpret_cast<uint64_t>(recon);
-    e = cudaMemcpyAsync(base + o_desc, &d, sizeof(LayerDesc), cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess)
-        e = cudaMemcpyAsync(base + o_tab, tab, sizeof(uint64_t) * ntab, cudaMemcpyHostToDevice, s);
-    // tile -> layer map is all zeros (one layer); counters and status start at zero
-    if (e == cudaSuccess) e = cudaMemsetAsync(base + o_tile, 0, sizeof(int) * ntiles, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(base + o_cnt, 0, o_status + sizeof(int) - o_cnt, s);
-    if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "scratch set-up: %s", cudaGetErrorString(e));
+
+    // descriptor, pointer table, tile map, counters and status written on
+    // the device by one set-up kernel that takes them by value
+    StaticSetup su{};
+    su.desc = d;
+    for (int w = 0; w < workers; ++w) {
+        su.tab[w] = reinterpret_cast<uint64_t>(grads[w]);
+        su.tab[workers + w] = reinterpret_cast<uint64_t>(errors[w]);
+    }
+    su.tab[2 * workers] = reinterpret_cast<uint64_t>(q);
+    su.tab[2 * workers + 1] = reinterpret_cast<uint64_t>(p_hat);
+    su.tab[2 * workers + 2] = reinterpret_cast<uint64_t>(recon);
+    su.desc_dst = reinterpret_cast<LayerDesc*>(base + o_desc);
+    su.tab_dst = reinterpret_cast<uint64_t*>(base + o_tab);
+    su.tile_dst = reinterpret_cast<int*>(base + o_tile);
+    su.cnt_dst = reinterpret_cast<unsigned*>(base + o_cnt);
+    su.status_dst = reinterpret_cast<int*>(base + kStaticStatusOffset);
+    su.ntab = ntab;
+    su.ntiles = ntiles;
+    su.ncnt = sz.cnt;
+    {
+        const int64_t work = std::max<int64_t>({ntiles, sz.cnt, static_cast<int64_t>(ntab), 1});
+        const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(148, (work + 255) / 256));
+        k_static_setup<<<blocks, 256, 0, s>>>(su);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "scratch set-up: %s", cudaGetErrorString(e));
+    }
 
     psgd::Params p{};
     uint64_t* tab_d = reinterpret_cast<uint64_t*>(base + o_tab);
@@ -1019,31 +1098,42 @@ int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int grad_dtype
     p.ws.qsup = reinterpret_cast<double*>(base + o_qsup);
     p.ws.T = reinterpret_cast<double*>(base + o_T);
     p.ws.cnt = reinterpret_cast<unsigned*>(base + o_cnt);
-    p.ws.status = reinterpret_cast<int*>(base + o_status);
+    p.ws.status = reinterpret_cast<int*>(base + kStaticStatusOffset);
     p.num_layers = 1;
     p.workers = workers;
     p.r = rank;
     p.inv_w = 1.0f / static_cast<float>(workers);
     p.drop_tol = kDropTol;
+    p.inv_w_global = 1.0 / static_cast<double>(workers);
 
-    const size_t smem[3] = {smem_need(0, R, workers, d.tm, d.vec), smem_need(1, R, workers, d.tm, d.vec),
-                            smem_need(2, R, workers, d.tm, d.vec)};
     for (int which = 0; which < 3; ++which) {
-        void* fn = kernel_ptr(which, R, grad_dtype, false, false);
-        cudaFuncAttributes fa{};
-        e = cudaFuncGetAttributes(&fa, fn);
-        if (e == cudaSuccess && static_cast<size_t>(fa.maxDynamicSharedSizeBytes) < smem[which])
-            e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem[which]));
-        if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "shared-memory opt-in: %s", cudaGetErrorString(e));
         psgd::Params pw = p;
         if (which == 2) {
             pw.do_resid = 1;
             pw.do_recon = recon ? 1 : 0;
         }
         void* args[] = {&pw};
-        e = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(ntiles)), dim3(psgd::kThreads), args, smem[which], s);
+        e = cudaLaunchKernel(fns[which], dim3(static_cast<unsigned>(ntiles)), dim3(psgd::kThreads), args,
+                             smem[which], s);
         if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
     }
+    return PSGD_OK;
+}
+
+int psgd_step_static_status(void* stream) {
+    g_create_error.clear();
+    void* base_v = nullptr;
+    int dev = 0;
+    cudaError_t e = static_scratch_address(&base_v, &dev);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    int word = 0;
+    if (e == cudaSuccess)
+        e = cudaMemcpy(&word, static_cast<unsigned char*>(base_v) + kStaticStatusOffset, sizeof(int),
+                       cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "static status: %s", cudaGetErrorString(e));
+    if (word != 0)
+        return fail(nullptr, PSGD_ERR_DEVICE, "device status word 0x%x: a reduction counter was inconsistent "
+                    "(calls overlapping on the GPU)", word);
     return PSGD_OK;
 }
 

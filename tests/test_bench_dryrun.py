@@ -28,7 +28,7 @@ class _Event:
 
 _FAKE_CUDA = types.SimpleNamespace(
     synchronize=lambda *a, **k: None, mem_get_info=lambda *a: (180e9, 183e9), set_device=lambda *a: None,
-    current_stream=lambda *a: None, Event=_Event, is_available=lambda: True)
+    current_stream=lambda *a: None, Event=_Event, is_available=lambda: True, empty_cache=lambda: None)
 
 
 class _TorchProxy(types.ModuleType):
@@ -47,10 +47,15 @@ class _Recorder:
         self.profiling = False
         _Recorder.created.append(self)
 
-    def step(self, *a, **k):
+    def step(self, G, E, Q, P, recon=None):
         self.calls.append("step")
         if self.profiling:
             self.steps_profiled += 1
+        # P_hat stand-in with orthonormal columns (the first r unit vectors),
+        # so that reports built from it are computable
+        for p in P or []:
+            p.zero_()
+            p[:p.shape[1]].copy_(torch.eye(p.shape[1]))
 
     def step_host_flat(self, *a, **k):
         self.calls.append("step_host_flat")
@@ -110,6 +115,7 @@ def fake_gpu(monkeypatch):
     monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
     monkeypatch.setattr(pkg, "PowerSGD", _Recorder)
     monkeypatch.setattr(build, "build", lambda *a, **k: None)
+    monkeypatch.setattr(bench, "_pinned_empty", lambda numel, dtype: torch.empty(numel, dtype=dtype))
     wl = Workload(name="tiny", layers=((64, 48), (24, 32)), rank=2, workers=3, steps=3,
                   vectors=(5, 3), momentum=(0.9, 0.1))
     monkeypatch.setattr(bench, "get_workload", lambda key: wl)
@@ -227,3 +233,72 @@ def test_json_line_sum_first_and_power_iterations(fake_gpu, monkeypatch, capsys)
              "--no-cpu-baseline", "--no-e2e", "--no-variants")
     assert d["config"]["mode"] == "eager+sumfirst+iters2"
     assert "step_dram_frac" not in d["roofline"]       # the bytes model covers one iteration only
+
+
+def test_json_line_workloads_and_reports(fake_gpu, monkeypatch, capsys):
+    main_wl = fake_gpu
+    lstm = Workload(name="tiny_lstm", layers=((40, 26),) * 2, rank=4, workers=4, steps=3)
+    sweep = Workload(name="tiny_sweep", layers=((32, 32),) * 3, rank=1, workers=2, steps=4, rotate=0.05,
+                     ranks=(1, 2, 8))
+    table = {"m": main_wl, "l": lstm, "s": sweep}
+    monkeypatch.setattr(bench, "get_workload", lambda key: table[key])
+    d = _run(monkeypatch, capsys, "--config", "m", "--steps", "3", "--warmup", "3", "--no-cpu-baseline",
+             "--no-e2e", "--no-variants", "--workloads", "m,l,s", "--workload-steps", "2")
+    wls = d["workloads"]
+    # the main workload is not repeated among the sub-lines
+    assert set(wls) == {"tiny_lstm", "tiny_sweep"}
+    lw = wls["tiny_lstm"]
+    for key in ("ms_per_step", "value", "step_dram_frac", "step_algorithmic_frac", "per_kernel_ms", "lazy_errors",
+                "compression"):
+        assert key in lw, key
+    assert lw["rank"] == 4 and lw["compression"]["ratio"] == round(2 * 40 * 26 / (4 * 2 * 66), 2)
+    sw = wls["tiny_sweep"]
+    assert set(sw["by_rank"]) == {"1", "2", "8"}
+    for r, line in sw["by_rank"].items():
+        assert line["rank"] == int(r) and line["value"] > 0 and "compression" in line
+    se = sw["subspace_error"]["by_rank"]
+    assert set(se) == {"1", "2", "8"} and se["1"]["steps"] == 4
+    assert se["2"]["status"] == "gated" and se["8"]["status"].startswith("reported, not gated")
+    for v in se.values():
+        assert 0.0 <= v["sin_theta_max"] <= 1.0 + 1e-12
+    assert d["compression"]["ratio"] == round((64 * 48 + 24 * 32) / (2 * (64 + 48 + 24 + 32)), 2)
+
+
+def test_e2e_releases_device_gradients_when_staging_does_not_fit(fake_gpu, monkeypatch, capsys):
+    monkeypatch.setattr(_FAKE_CUDA, "mem_get_info", lambda *a: (1e3, 183e9))
+    real_need = bench.device_bytes_needed
+    monkeypatch.setattr(bench, "device_bytes_needed", lambda *a: 0)
+    d = _run(monkeypatch, capsys, "--steps", "2", "--warmup", "3", "--no-cpu-baseline", "--no-variants",
+             "--e2e-steps", "2", "--no-workloads")
+    assert d["e2e"]["value"] > 0 and "released" in d["e2e"]["note"]
+    assert real_need is not None
+
+
+def test_compression_report_of_the_workloads():
+    from synth import C1, C3
+    c1 = bench.compression_report(C1, 2)
+    smpn = sum(m + n for m, n in C1.layers)
+    assert c1["ratio"] == round(11_162_624 / (2 * smpn), 2)
+    assert c1["factor_bytes_per_worker"] == 4 * 2 * smpn and c1["gradient_bytes_per_worker"] == 4 * 11_162_624
+    c3 = bench.compression_report(C3, 4)
+    # 24 blocks x (16384 + 8192 + 20480 + 20480) rows + columns
+    assert c3["ratio"] == round(4_831_838_208 / (4 * 24 * 65536), 2) and c3["gradient_bytes_per_worker"] == \
+        2 * 4_831_838_208
+    assert c3["dist_partial_bytes_per_rank"] == 8 * 4 * 24 * 65536
+
+
+def test_sin_theta_max_known_angles():
+    import numpy as np
+    # span(e0, e1) against span(e0, cos t e1 + sin t e2): largest angle t
+    for t in (1e-9, 1e-3, 0.3, 1.2):
+        U = np.eye(5)[:, :2]
+        P = np.zeros((5, 2))
+        P[0, 0] = 1.0
+        P[1, 1], P[2, 1] = np.cos(t), np.sin(t)
+        assert abs(bench.sin_theta_max(U, P) - np.sin(t)) < 1e-12 * max(1.0, t) + 1e-15
+    # invariant under a rotation of either basis
+    rng = np.random.default_rng(3)
+    U = np.linalg.qr(rng.standard_normal((9, 3)))[0]
+    P = np.linalg.qr(rng.standard_normal((9, 3)))[0]
+    Rt = np.linalg.qr(rng.standard_normal((3, 3)))[0]
+    assert abs(bench.sin_theta_max(U, P) - bench.sin_theta_max(U @ Rt, P @ Rt.T)) < 1e-12

@@ -1,0 +1,225 @@
+"""Parity over the workloads' own step counts: free-running trajectories of
+the library (warm start, error feedback, and momentum where the workload
+has it) against the float64 oracle, gated at every step.
+
+Layers are independent ("anthology-of-the-sota" note-152, "Method":
+per-layer approximation), and a layer's tiles, reductions and summation
+order depend only on its own shape, the rank and the worker count, so the
+library context of the longer runs holds only the sampled layers; the
+first test checks that a sampled layer's results are bit for bit those of
+the full workload's context.  Gradients come from the full workload's
+generator (same layer indices, so the same seeds and the same rotating
+subspace).  P_hat, Q_bar and G_hat are compared at every step; the error
+memory and the momentum state every `e_every` steps and at the last."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.powersgd64 as ora
+from synth import C1, C2, C3, C4B, GradientSource
+
+from . import _harness as H
+
+pytestmark = pytest.mark.gpu
+
+
+def _host_ram_gb():
+    try:
+        with open("/proc/meminfo") as f:
+            for line in f:
+                if line.startswith("MemAvailable"):
+                    return int(line.split()[1]) / 1e6
+    except Exception:
+        pass
+    return 0.0
+
+
+class _Trajectory:
+    """The library on `run_layers` of a workload (device buffers per layer,
+    gradients generated on the device), the oracle on `sample`."""
+
+    def __init__(self, wl, run_layers, sample, momentum=False, vectors=False, seed=1234):
+        from rank_gradient_compression_02_b200 import PowerSGD
+        self.wl, self.W = wl, wl.workers
+        self.run_layers, self.sample = list(run_layers), list(sample)
+        self.pos = {l: i for i, l in enumerate(self.run_layers)}
+        self.src = GradientSource(wl, seed)
+        shapes = [wl.layers[l] for l in self.run_layers]
+        gdt = torch.bfloat16 if wl.grad_dtype == "bf16" else torch.float32
+        self.lib = PowerSGD(shapes, wl.rank, self.W, seed=seed, grad_dtype=wl.grad_dtype)
+        self.G = [[torch.empty(m, n, dtype=gdt, device="cuda") for (m, n) in shapes] for _ in range(self.W)]
+        self.E = [[torch.zeros(m, n, device="cuda") for (m, n) in shapes] for _ in range(self.W)]
+        Q0 = {l: self.src.initial_q(l) for l in self.run_layers}
+        self.Q = [Q0[l].cuda() for l in self.run_layers]
+        self.P = [torch.empty(m, wl.rank, device="cuda") for (m, _) in shapes]
+        self.Rc = [torch.empty(m, n, device="cuda") if l in self.sample else None
+                   for l, (m, n) in zip(self.run_layers, shapes)]
+        self.orc = H.OracleRun(self.sample, {l: [np.zeros(wl.layers[l]) for _ in range(self.W)] for l in self.sample},
+                               {l: Q0[l].double().numpy() for l in self.sample})
+        self.momentum = wl.momentum if momentum else None
+        if self.momentum:
+            self.params = [torch.zeros(m, n, device="cuda") for (m, n) in shapes]
+            self.mom = [torch.zeros(m, n, device="cuda") for (m, n) in shapes]
+            self.xr = {l: np.zeros(wl.layers[l]) for l in self.sample}
+            self.mr = {l: np.zeros(wl.layers[l]) for l in self.sample}
+        self.vectors = vectors and bool(wl.vectors)
+        if self.vectors:
+            K = len(wl.vectors)
+            self.vout = [torch.empty(k, device="cuda") for k in wl.vectors]
+            self.vx = [torch.zeros(k, device="cuda") for k in wl.vectors]
+            self.vm = [torch.zeros(k, device="cuda") for k in wl.vectors]
+            self.vxr = [np.zeros(k) for k in wl.vectors]
+            self.vmr = [np.zeros(k) for k in wl.vectors]
+            self.K = K
+
+    def fill(self, t):
+        for i, l in enumerate(self.run_layers):
+            low = self.src.lowrank(t, l, "cuda")
+            for w in range(self.W):
+                self.src.layer_grad(t, w, l, "cuda", lowrank=low, out=self.G[w][i])
+
+    def step(self, t):
+        self.fill(t)
+        torch.cuda.synchronize()
+        G_host = {l: [H.to64(self.G[w][self.pos[l]]) for w in range(self.W)] for l in self.sample}
+        self.lib.step(self.G, self.E, self.Q, self.P, self.Rc)
+        beta, lr = self.momentum if self.momentum else (0.0, 0.0)
+        if self.momentum:
+            self.lib.momentum_step(self.params, self.mom, lr, beta)
+        vhost = None
+        if self.vectors:
+            vhost = [self.src.vector_grads(t, w) for w in range(self.W)]
+            vdev = [[v.cuda() for v in row] for row in vhost]
+            self.lib.vec_mean(vdev, self.vout, self.vx, self.vm, lr=lr, beta=beta)
+        torch.cuda.synchronize()
+        self.orc.step(G_host)
+        if self.momentum:
+            for l in self.sample:
+                self.xr[l], self.mr[l] = ora.momentum_update(self.xr[l], self.mr[l], self.orc.last[l]["G_hat"],
+                                                             lr, beta)
+        vmeans = None
+        if self.vectors:
+            vmeans = []
+            for k in range(self.K):
+                mean = ora.vec_mean([vhost[w][k].double().numpy() for w in range(self.W)])
+                self.vxr[k], self.vmr[k] = ora.momentum_update(self.vxr[k], self.vmr[k], mean, lr, beta)
+                vmeans.append(mean)
+        return G_host, vmeans
+
+    def errors(self, full: bool, vmeans=None):
+        errs = {}
+        for l in self.sample:
+            o, i = self.orc.last[l], self.pos[l]
+            e = {"P_hat": H.rel_fro(H.to64(self.P[i]), o["P_hat"]), "Q_bar": H.rel_fro(H.to64(self.Q[i]), o["Q_bar"]),
+                 "G_hat": H.rel_fro(H.to64(self.Rc[i]), o["G_hat"])}
+            if full:
+                e["E_new"] = max(H.rel_fro(H.to64(self.E[w][i]), o["E_new"][w], denom=np.linalg.norm(o["M"][w]))
+                                 for w in range(self.W))
+                if self.momentum:
+                    e["params"] = H.rel_fro(H.to64(self.params[i]), self.xr[l])
+                    e["mom"] = H.rel_fro(H.to64(self.mom[i]), self.mr[l])
+            for k, v in e.items():
+                errs[k] = max(errs.get(k, 0.0), v)
+        if full and self.vectors:
+            errs["vec_params"] = max(H.rel_fro(H.to64(self.vx[k]), self.vxr[k]) for k in range(self.K))
+            errs["vec_mean"] = max(H.rel_fro(H.to64(self.vout[k]), vmeans[k]) for k in range(self.K))
+        return errs
+
+
+def _run(traj, steps, e_every, tol, what):
+    worst = {}
+    for t in range(steps):
+        _, vm = traj.step(t)
+        full = (t + 1) % e_every == 0 or t == steps - 1
+        errs = traj.errors(full, vm)
+        H.assert_close(errs, tol, f"{what}, step {t}")
+        for k, v in errs.items():
+            worst[k] = max(worst.get(k, 0.0), v)
+    traj.lib.status()
+    return worst
+
+
+def test_sampled_context_is_bitwise_the_full_context():
+    # two steps of the ResNet-18 set: every layer in one context, and three
+    # of its layers in a context of their own, on the same gradients
+    sample = [3, 12, 19]
+    full = _Trajectory(C1, range(len(C1.layers)), sample)
+    part = _Trajectory(C1, sample, sample)
+    for t in range(2):
+        full.fill(t)
+        part.fill(t)
+        full.lib.step(full.G, full.E, full.Q, full.P, full.Rc)
+        part.lib.step(part.G, part.E, part.Q, part.P, part.Rc)
+        torch.cuda.synchronize()
+        for l in sample:
+            i, j = full.pos[l], part.pos[l]
+            assert torch.equal(full.P[i], part.P[j]) and torch.equal(full.Q[i], part.Q[j])
+            assert torch.equal(full.Rc[i], part.Rc[j])
+            for w in range(C1.workers):
+                assert torch.equal(full.G[w][i], part.G[w][j]) and torch.equal(full.E[w][i], part.E[w][j])
+    full.lib.status()
+    part.lib.status()
+
+
+def test_resnet18_100_steps_with_momentum():
+    # every layer, 16 workers, rank 2, 100 steps, post-compression momentum
+    # on the matrices and the 1-D tensors (beta 0.9, lr 0.1)
+    traj = _Trajectory(C1, range(len(C1.layers)), range(len(C1.layers)), momentum=True, vectors=True)
+    worst = _run(traj, C1.steps, 10, H.TOL["f32"], "resnet18")
+    assert set(worst) >= {"P_hat", "Q_bar", "G_hat", "E_new", "params", "mom", "vec_params"}
+
+
+@pytest.mark.parametrize("rank", [1, 4, 32])
+def test_sweep_1024_50_rotating_steps(rank):
+    # the first and last of the 256 matrices, 8 workers, subspace turned by
+    # 0.05 rad before every step, 50 steps
+    wl = C4B.with_rank(rank)
+    traj = _Trajectory(wl, [0, 255], [0, 255])
+    _run(traj, wl.steps, 10, H.TOL["f32"], f"1024^2 sweep r={rank}")
+
+
+def test_lstm_gate_weights_50_steps():
+    # two 2600 x 650 gate matrices (the same lane width, column chunks and
+    # two-level row-block reduction as the 33280 x 650 decoder, which the
+    # full-size test runs), 16 workers, rank 4, 50 steps
+    traj = _Trajectory(C2, [0, 5], [0, 5])
+    _run(traj, C2.steps, 10, H.TOL["f32"], "lstm gates")
+
+
+def test_transformer_bf16_20_steps():
+    # the 4096 x 4096 out-projection and the 4096 x 16384 down-projection,
+    # bf16 gradients, 4 workers, rank 4, 20 steps
+    if _host_ram_gb() < 48:
+        pytest.skip("host RAM too small for the float64 oracle of the sampled layers")
+    traj = _Trajectory(C3, [1, 3], [1, 3])
+    _run(traj, C3.steps, 5, H.TOL["bf16"], "transformer")
+
+
+@pytest.mark.parametrize("rank", [1, 2, 4])
+def test_subspace_error_report_matches_the_oracle(rank):
+    # the benchmark's subspace-error figure for the 1024 x 1024 sweep (its
+    # own run through the library over the workload's 50 rotating steps)
+    # against the same figure on the oracle's trajectory: sin of the largest
+    # principal angle between the last P_hat and the top-r left singular
+    # vectors of the last step's worker mean
+    import bench
+    wl = C4B
+    rep = bench.subspace_error_report(wl, [rank], torch.device("cuda"), wl.steps)
+    got = rep["by_rank"][str(rank)]["sin_theta_max"]
+    src = GradientSource(wl.with_rank(rank), 1234)
+    m, n = wl.layers[0]
+    E = [np.zeros((m, n)) for _ in range(wl.workers)]
+    Q = src.initial_q(0, rank).double().numpy()
+    for t in range(wl.steps):
+        # the same device-generated gradients the library's run consumed
+        low = src.lowrank(t, 0, "cuda")
+        G = [H.to64(src.layer_grad(t, w, 0, "cuda", lowrank=low)) for w in range(wl.workers)]
+        if t == wl.steps - 1:
+            Mbar = ora.worker_mean([ora.error_feedback_add(G[w], E[w]) for w in range(wl.workers)])
+        o = ora.step(G, E, Q)
+        E, Q = o["E_new"], o["Q_bar"]
+    U = np.linalg.svd(Mbar, full_matrices=False)[0][:, :rank]
+    want = ora.subspace_sin_max(U, o["P_hat"])
+    assert abs(got - want) <= 1e-4 + 1e-3 * want, (got, want)

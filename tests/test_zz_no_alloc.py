@@ -1,5 +1,5 @@
-"""The allocation-free entry point (psgd_step_static) against the
-context-based psgd_step, through the C ABI.
+"""The allocation-free entry point (psgd_step_static) through the C ABI:
+against the context-based psgd_step and against the float64 oracle.
 
 psgd_step_static is for callers that cannot allocate device memory: its
 scratch lives in a static device array inside the library.  This file is
@@ -13,6 +13,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle.powersgd64 as ora
 from rank_gradient_compression_02_b200 import PowerSGD, PsgdError, _lib
 from synth import GradientSource, Workload
 
@@ -29,32 +30,46 @@ pytestmark = pytest.mark.gpu
     (129, 1000, 32, 3, "f32"),    # the tensor-core passes, 16-byte lanes
     (300, 650, 16, 2, "f32"),     # the tensor-core passes, 8-byte lanes
 ])
-def test_static_step_matches_context_step(m, n, rank, workers, dtype):
+def test_static_step_matches_context_step_and_oracle(m, n, rank, workers, dtype):
     wl = Workload(name="noalloc", layers=((m, n),), rank=rank, workers=workers, steps=2, grad_dtype=dtype)
     src = GradientSource(wl, seed=11)
     gdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     ctx = PowerSGD(wl.layers, rank, workers, grad_dtype=dtype)
-    q0 = src.initial_q(0).cuda()
-    # two independent states, the same inputs
+    q0 = src.initial_q(0)
+    # two independent device states and a float64 oracle state, the same inputs
     G = [torch.empty(m, n, device="cuda", dtype=gdt) for _ in range(workers)]
     E_ctx = [torch.zeros(m, n, device="cuda") for _ in range(workers)]
     E_st = [torch.zeros(m, n, device="cuda") for _ in range(workers)]
-    q_ctx, q_st = q0.clone(), q0.clone()
+    q_ctx, q_st = q0.cuda(), q0.cuda()
     P_ctx = torch.empty(m, rank, device="cuda")
     P_st = torch.empty(m, rank, device="cuda")
     R_ctx = torch.empty(m, n, device="cuda")
     R_st = torch.empty(m, n, device="cuda")
+    E_ora = [np.zeros((m, n)) for _ in range(workers)]
+    Q_ora = q0.double().numpy()
     for t in range(2):          # two calls in a row, state carried in place
+        host = [src.layer_grad(t, w, 0) for w in range(workers)]
         for w in range(workers):
-            G[w].copy_(src.layer_grad(t, w, 0))
+            G[w].copy_(host[w])
         ctx.step([[g] for g in G], [[e] for e in E_ctx], [q_ctx], [P_ctx], [R_ctx])
         _lib.step_static(m, n, rank, G, E_st, q_st, P_st, R_st, grad_dtype=dtype)
+        _lib.step_static_status()
         torch.cuda.synchronize()
-        errs = {"P_hat": H.rel_fro(H.to64(P_st), H.to64(P_ctx)),
-                "Q_bar": H.rel_fro(H.to64(q_st), H.to64(q_ctx)),
-                "G_hat": H.rel_fro(H.to64(R_st), H.to64(R_ctx)),
-                "E_new": max(H.rel_fro(H.to64(E_st[w]), H.to64(E_ctx[w])) for w in range(workers))}
-        H.assert_close(errs, H.TOL["f32"], f"call {t}")
+        # the same kernels in the same order on the same inputs: bit for bit
+        # the context step's results
+        assert torch.equal(P_st, P_ctx), f"call {t}: P_hat"
+        assert torch.equal(q_st, q_ctx), f"call {t}: Q_bar"
+        assert torch.equal(R_st, R_ctx), f"call {t}: G_hat"
+        for w in range(workers):
+            assert torch.equal(E_st[w], E_ctx[w]), f"call {t}: E'_{w}"
+        # and against the float64 oracle, free-running from the same state
+        o = ora.step([g.double().numpy() for g in host], E_ora, Q_ora)
+        E_ora, Q_ora = o["E_new"], o["Q_bar"]
+        errs = {"P_hat": H.rel_fro(H.to64(P_st), o["P_hat"]), "Q_bar": H.rel_fro(H.to64(q_st), o["Q_bar"]),
+                "G_hat": H.rel_fro(H.to64(R_st), o["G_hat"]),
+                "E_new": max(H.rel_fro(H.to64(E_st[w]), o["E_new"][w], denom=np.linalg.norm(o["M"][w]))
+                             for w in range(workers))}
+        H.assert_close(errs, H.TOL[dtype], f"call {t} against the oracle")
     ctx.status()
 
 
