@@ -290,17 +290,34 @@ PSGD_API int psgd_set_power_iters(psgd_ctx *ctx, int iters);
 /* PowerSGD+ periodic SVD refresh ("From PowerSGD to PowerSGD+", Abstract:
  * the projection subspace is periodically re-aligned with the optimal one
  * through a singular value decomposition).  With every > 0, every step
- * whose number (1, 2, ...) is a multiple of `every` runs `iters` subspace
- * iterations (1 <= iters <= 64) from the warm start and then a
- * Rayleigh-Ritz rotation: C = Q_bar^T Q_bar = W Lambda W^T (Jacobi,
- * float64, eigenvalues descending, each column of W signed so that its
- * largest-magnitude entry is positive), P_hat <- P_hat W, Q_bar <- Q_bar W.
- * Once the iterations have converged, P_hat = U_r and Q_bar = V_r Sigma_r
- * (singular vectors up to sign) of the worker-mean matrix, and the
- * residual is taken against that truncated SVD.  every = 0 turns it off
- * (the default).  Adds 2 * (iters - power_iters) + 1 launches on refresh
- * steps. */
+ * whose number (1, 2, ...) is a multiple of `every` replaces the step's
+ * factors by the rank-r truncated SVD of the worker mean M_bar:
+ * P_hat = U_r, Q_bar = V_r Sigma_r (singular vectors up to sign), and the
+ * residual is taken against it.  The SVD is computed by subspace iteration
+ * on an oversampled block of r' = r + p columns (p from
+ * psgd_set_svd_oversampling, default 8; r' capped by 32 and by the smallest
+ * side of every layer; Halko, Martinsson and Tropp, SIAM Review 2011,
+ * section 4.5), started from [warm-start Q | fresh N(0, 1) draws] (the
+ * psgd_init_q generator with draw index 2^62 + step number), followed by a
+ * Rayleigh-Ritz rotation: C = Q_bar^T Q_bar = W Lambda W^T (Jacobi, float64,
+ * eigenvalues descending, each column of W signed so that its
+ * largest-magnitude entry is positive), of which the top r directions are
+ * kept.  The top-r subspace converges as (sigma_{r'+1} / sigma_r)^(2 J) in
+ * J iterations; each layer stops once the estimate of that factor from the
+ * orthogonalisation's Cholesky diagonal, (lambda_{r'} / lambda_r)^(J - 1),
+ * is at most 1e-10, and after `iters` iterations at most (1 <= iters <= 64).
+ * every = 0 turns refresh off (the default).  A refresh step makes
+ * 2 * iters + 2 launches, + 1 for the residual pass (eager mode, or when
+ * G_hat is wanted), + 1 in lazy mode to write out the previous E' first; a
+ * converged layer's later iterations return at once.  With oversampling 0
+ * (or when no column can be added) the block is the rank-r factors
+ * themselves: `iters` iterations from the warm start, the rotation in
+ * place, 2 * (iters - power_iters) + 1 more launches than a regular step. */
 PSGD_API int psgd_set_svd_refresh(psgd_ctx *ctx, int every, int iters);
+
+/* Oversampling p of the refresh block above, 0 <= p <= 31 (default 8).  The
+ * context holds a second workspace of rank r + p while refresh is on. */
+PSGD_API int psgd_set_svd_oversampling(psgd_ctx *ctx, int extra);
 
 /* Per-kernel timing of psgd_step, for measurement: with enable != 0 every
  * later psgd_step records CUDA events (on its stream) around each of its

@@ -68,6 +68,7 @@ _SIGS = {
     "psgd_dist_q": (ctypes.c_int, [_P, _P, _P, _P]),
     "psgd_dist_finish": (ctypes.c_int, [_P, _P, _P]),
     "psgd_set_svd_refresh": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int]),
+    "psgd_set_svd_oversampling": (ctypes.c_int, [_P, ctypes.c_int]),
     "psgd_profile_enable": (ctypes.c_int, [_P, ctypes.c_int]),
     "psgd_profile_read": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
 }
@@ -208,7 +209,8 @@ class PowerSGD:
 
     def __init__(self, layers: Sequence[Sequence[int]], rank: int, workers: int, seed: int = 1234,
                  grad_dtype: str = "f32", lazy_errors: bool = False, sum_first: bool = False,
-                 power_iters: int = 1, warm_start: bool = True, svd_every: int = 0, svd_iters: int = 8):
+                 power_iters: int = 1, warm_start: bool = True, svd_every: int = 0, svd_iters: int = 8,
+                 svd_oversampling: Optional[int] = None):
         self.lib = load()
         self.layers = [(int(m), int(n)) for m, n in layers]
         self.rank = int(rank)
@@ -226,6 +228,8 @@ class PowerSGD:
         self._h = h
         if power_iters != 1:
             self._check(self.lib.psgd_set_power_iters(self._h, int(power_iters)))
+        if svd_oversampling is not None:
+            self._check(self.lib.psgd_set_svd_oversampling(self._h, int(svd_oversampling)))
         if svd_every:
             self._check(self.lib.psgd_set_svd_refresh(self._h, int(svd_every), int(svd_iters)))
 

@@ -87,6 +87,9 @@ struct Work {
     double* T;
     unsigned* cnt;
     int* status;
+    // SVD refresh with oversampling: the iteration after which each layer
+    // stops (set by the first pass once its convergence bound is met)
+    int* conv_iter;
 };
 
 struct Params {
@@ -105,6 +108,12 @@ struct Params {
     double* dist_out;
     const double* dist_in;
     double inv_w_global;
+    // subspace iterations of an SVD refresh: this launch's iteration number
+    // (1, 2, ...); with track_conv, layers whose conv_iter is below it are
+    // skipped, and the first pass's factorisation sets conv_iter once
+    // (lambda_{r'} / lambda_{r_conv})^(iter - 1) <= conv_eps
+    int iter, track_conv, r_conv;
+    double conv_eps;
 };
 
 enum : int { kStatusCounter = 1 };

@@ -750,6 +750,22 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
         factor_gram_warp<R>(Gs, Rs, Ts, drop, p.r, p.drop_tol, tid);
         double* T = p.ws.T + d.t_off;
         for (int idx = tid; idx < R * R; idx += 32) T[idx] = Ts[idx];
+        if (p.track_conv && tid == 0 && p.iter >= 3) {
+            // Subspace iteration on A = M_bar M_bar^T: from the second
+            // iteration on, P_bar = A P_hat_prev, so the factor's diagonal
+            // estimates the eigenvalues lambda_j = sigma_j^2 of A in
+            // decreasing order.  The top r_conv directions of an r-column
+            // block converge as (lambda_{r+1} / lambda_{r_conv})^iterations
+            // (Halko, Martinsson and Tropp, SIAM Review 2011, section 4.5);
+            // with the block's last estimate lambda_r standing in for
+            // lambda_{r+1} >= ..., the layer stops after this iteration once
+            // that factor is at most conv_eps.  A zero lambda_{r_conv} (rank
+            // below r_conv: the range is captured exactly) stops it too.
+            const double lam_keep = Rs[(p.r_conv - 1) * R + (p.r_conv - 1)];
+            const double lam_last = Rs[(p.r - 1) * R + (p.r - 1)];
+            const bool done = !(lam_keep > 0.0) || pow(lam_last / lam_keep, p.iter - 1) <= p.conv_eps;
+            if (done) p.ws.conv_iter[tc.l] = p.iter;
+        }
     }
     if (tid == 0) cnt[cl.a_layer] = 0u;
 }
@@ -761,6 +777,7 @@ __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_a(Params p)
     extern __shared__ __align__(16) unsigned char smem[];
     const int t = tile_index<false>();
     const int l = p.t.tile_layer[t];
+    if (p.track_conv && p.iter > p.ws.conv_iter[l]) return;   // converged refresh layer
     const LayerDesc d = p.t.layers[l];
     const TileCoord tc = decode_tile(d, t, l);
     const int W = p.workers;
@@ -1260,6 +1277,7 @@ __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_b(Params p)
     extern __shared__ __align__(16) unsigned char smem[];
     const int t = tile_index<true>();
     const int l = p.t.tile_layer[t];
+    if (p.track_conv && p.iter > p.ws.conv_iter[l]) return;   // converged refresh layer
     const LayerDesc d = p.t.layers[l];
     const TileCoord tc = decode_tile(d, t, l);
     const int W = p.workers;
@@ -1618,15 +1636,55 @@ __global__ void k_dist_qbar(Params p) {
 }
 
 // ---------------------------------------------------------------------------
-// Rayleigh-Ritz rotation after converged subspace iterations (SVD refresh):
-// C = Q_bar^T Q_bar = W diag(lambda) W^T (cyclic Jacobi, float64, one warp,
-// eigenvalues sorted descending, every column of W signed so that its
-// largest-magnitude entry is positive), then P_hat <- P_hat W and
-// Q_bar <- Q_bar W.  When span(P_hat) is the top-r left singular subspace of
-// the worker mean, this makes P_hat = U_r and Q_bar = V_r Sigma_r; P_hat Q_bar^T
-// is unchanged.  One CTA per layer.
+// initial Q: Philox4x64-10 (Salmon et al., SC'11) + Box-Muller (1958)
+struct Philox4x64 {
+    static constexpr uint64_t M0 = 0xD2E7470EE14C6C93ull;
+    static constexpr uint64_t M1 = 0xCA5A826395121157ull;
+    static constexpr uint64_t W0 = 0x9E3779B97F4A7C15ull;
+    static constexpr uint64_t W1 = 0xBB67AE8584CAA73Bull;
+    __device__ static void run(uint64_t (&x)[4], uint64_t k0, uint64_t k1) {
+#pragma unroll
+        for (int rnd = 0; rnd < 10; ++rnd) {
+            if (rnd) {
+                k0 += W0;
+                k1 += W1;
+            }
+            const uint64_t hi0 = __umul64hi(M0, x[0]), lo0 = M0 * x[0];
+            const uint64_t hi1 = __umul64hi(M1, x[2]), lo1 = M1 * x[2];
+            const uint64_t y0 = hi1 ^ x[1] ^ k0;
+            const uint64_t y2 = hi0 ^ x[3] ^ k1;
+            x[0] = y0;
+            x[1] = lo1;
+            x[2] = y2;
+            x[3] = lo0;
+        }
+    }
+};
+
+// ---------------------------------------------------------------------------
+// Rayleigh-Ritz rotation after the subspace iterations of an SVD refresh:
+// C = Q_bar^T Q_bar = W diag(lambda) W^T over the block's r columns (cyclic
+// Jacobi, float64, one warp, eigenvalues sorted descending, every column of
+// W signed so that its largest-magnitude entry is positive); then
+// P_hat W and Q_bar W, of which the first dst.r_out columns are kept.  When
+// span(P_hat) holds the top left singular subspace of the worker mean, the
+// kept columns are P_hat = U_r and Q_bar = V_r Sigma_r.  The source is the
+// launching context's workspace (rank r = p.r, stride R); the destination
+// is a context of rank dst.r_out (stride dst.RD, columns r_out..RD-1 set to
+// zero) with the caller's Q and P_hat: the same context (in place, r_out =
+// r) or the rank-r context an oversampled block was iterated for.  One CTA
+// per layer; each row is read whole before it is written.
+struct RRDst {
+    const LayerDesc* layers;   // destination geometry (prow_off, qrow_off)
+    float* phat;               // destination workspace rows, stride RD
+    float* qbar;
+    float* const* q_out;       // caller's Q, n x r_out
+    float* const* p_out;       // caller's P_hat, m x r_out (table may be null, entries too)
+    int RD, r_out;
+};
+
 template <int R>
-__global__ void __launch_bounds__(kThreads) k_rayleigh_ritz(Params p) {
+__global__ void __launch_bounds__(kThreads) k_rayleigh_ritz(Params p, RRDst dst) {
     __shared__ double C[R * R];
     __shared__ double V[R * R];
     __shared__ double Wm[R * R];
@@ -1634,11 +1692,12 @@ __global__ void __launch_bounds__(kThreads) k_rayleigh_ritz(Params p) {
     __shared__ int order[R];
     const int l = blockIdx.x;
     const LayerDesc d = p.t.layers[l];
+    const LayerDesc dd = dst.layers[l];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int r = p.r;
     constexpr int NG = R * (R + 1) / 2;
-    float* qbar = p.ws.qbar + d.qrow_off;
-    float* phat = p.ws.phat + d.prow_off;
+    const float* qbar = p.ws.qbar + d.qrow_off;
+    const float* phat = p.ws.phat + d.prow_off;
 
     // 1) C = Q_bar^T Q_bar (pairs over warps, rows over lanes, fixed order)
     for (int pidx = warp; pidx < NG; pidx += kWarps) {
@@ -1733,35 +1792,66 @@ __global__ void __launch_bounds__(kThreads) k_rayleigh_ritz(Params p) {
     }
     __syncthreads();
 
-    // 3) rotate Q_bar and P_hat in place (one row per thread)
-    float* qout = p.t.q[l];
-    float* pout = (p.t.p_hat_out != nullptr) ? p.t.p_hat_out[l] : nullptr;
-    for (int64_t j = tid; j < d.n; j += kThreads) {
-        double row[R];
+    // 3) rotate Q_bar and P_hat (one row per thread), keep r_out columns
+    const int RD = dst.RD, ro = dst.r_out;
+    float* qd = dst.qbar + dd.qrow_off;
+    float* pd = dst.phat + dd.prow_off;
+    float* qout = dst.q_out[l];
+    float* pout = (dst.p_out != nullptr) ? dst.p_out[l] : nullptr;
+    auto rotate_rows = [&](const float* src, float* dws, float* out, int64_t rows) {
+        for (int64_t j = tid; j < rows; j += kThreads) {
+            double row[R];
 #pragma unroll
-        for (int k = 0; k < R; ++k) row[k] = qbar[j * R + k];
+            for (int k = 0; k < R; ++k) row[k] = src[j * R + k];
+            for (int k = 0; k < RD; ++k) {
+                double v = 0.0;
+                if (k < ro) {
 #pragma unroll
-        for (int k = 0; k < R; ++k) {
-            double v = 0.0;
-#pragma unroll
-            for (int a = 0; a < R; ++a) v += row[a] * Wm[a * R + k];
-            const float f = static_cast<float>(v);
-            qbar[j * R + k] = f;
-            if (k < r) qout[j * r + k] = f;
+                    for (int a = 0; a < R; ++a) v += row[a] * Wm[a * R + k];
+                }
+                const float f = static_cast<float>(v);
+                dws[j * RD + k] = f;
+                if (out != nullptr && k < ro) out[j * ro + k] = f;
+            }
         }
-    }
-    for (int64_t i = tid; i < d.m; i += kThreads) {
-        double row[R];
+    };
+    rotate_rows(qbar, qd, qout, d.n);
+    rotate_rows(phat, pd, pout, d.m);
+}
+
+// Q block of an oversampled refresh: the caller's warm start Q (n x r) in
+// the first r columns, fresh N(0, 1) draws in the other rp - r (the
+// k_init_q generator: Philox4x64-10 keyed by (seed, l), counter
+// (b, draw, 0, 0) for block b = e / 4 of the extra elements
+// e = j * (rp - r) + (k - r), Box-Muller in float64).
+__global__ void k_assemble_q(float* const* qdst, float* const* qsrc, const LayerDesc* layers, int r, int rp,
+                             uint64_t seed, uint64_t draw) {
+    const int l = blockIdx.y;
+    const int64_t n = layers[l].n;
+    const int px = rp - r;
+    float* out = qdst[l];
+    const float* in = qsrc[l];
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t e = t0; e < n * r; e += stride) out[(e / r) * rp + e % r] = in[e];
+    const int64_t total = n * px;
+    constexpr double kTwoPi = 2.0 * 3.141592653589793;
+    for (int64_t b = t0; b < (total + 3) / 4; b += stride) {
+        uint64_t x[4] = {static_cast<uint64_t>(b), draw, 0ull, 0ull};
+        Philox4x64::run(x, seed, static_cast<uint64_t>(l));
+        double z[4];
 #pragma unroll
-        for (int k = 0; k < R; ++k) row[k] = phat[i * R + k];
+        for (int h = 0; h < 2; ++h) {
+            const double u0 = (static_cast<double>(x[2 * h] >> 11) + 0.5) * (1.0 / 9007199254740992.0);
+            const double u1 = (static_cast<double>(x[2 * h + 1] >> 11) + 0.5) * (1.0 / 9007199254740992.0);
+            const double rho = sqrt(-2.0 * log(u0));
+            z[2 * h] = rho * cos(kTwoPi * u1);
+            z[2 * h + 1] = rho * sin(kTwoPi * u1);
+        }
 #pragma unroll
-        for (int k = 0; k < R; ++k) {
-            double v = 0.0;
-#pragma unroll
-            for (int a = 0; a < R; ++a) v += row[a] * Wm[a * R + k];
-            const float f = static_cast<float>(v);
-            phat[i * R + k] = f;
-            if (pout != nullptr && k < r) pout[i * r + k] = f;
+        for (int t = 0; t < 4; ++t) {
+            const int64_t e = 4 * b + t;
+            if (e < total) out[(e / px) * rp + r + e % px] = static_cast<float>(z[t]);
         }
     }
 }
@@ -1797,32 +1887,6 @@ __global__ void k_vec_mean(const float* const* vecs, float* const* out, const in
         }
     }
 }
-
-// ---------------------------------------------------------------------------
-// initial Q: Philox4x64-10 (Salmon et al., SC'11) + Box-Muller (1958)
-struct Philox4x64 {
-    static constexpr uint64_t M0 = 0xD2E7470EE14C6C93ull;
-    static constexpr uint64_t M1 = 0xCA5A826395121157ull;
-    static constexpr uint64_t W0 = 0x9E3779B97F4A7C15ull;
-    static constexpr uint64_t W1 = 0xBB67AE8584CAA73Bull;
-    __device__ static void run(uint64_t (&x)[4], uint64_t k0, uint64_t k1) {
-#pragma unroll
-        for (int rnd = 0; rnd < 10; ++rnd) {
-            if (rnd) {
-                k0 += W0;
-                k1 += W1;
-            }
-            const uint64_t hi0 = __umul64hi(M0, x[0]), lo0 = M0 * x[0];
-            const uint64_t hi1 = __umul64hi(M1, x[2]), lo1 = M1 * x[2];
-            const uint64_t y0 = hi1 ^ x[1] ^ k0;
-            const uint64_t y2 = hi0 ^ x[3] ^ k1;
-            x[0] = y0;
-            x[1] = lo1;
-            x[2] = y2;
-            x[3] = lo0;
-        }
-    }
-};
 
 __global__ void k_init_q(float* const* q, const LayerDesc* layers, int r, uint64_t seed, uint64_t draw) {
     const int l = blockIdx.y;

@@ -24,6 +24,11 @@ using psgd::LayerDesc;
 namespace {
 
 constexpr double kDropTol = 1e-12;
+// An oversampled refresh stops a layer once the estimated convergence
+// factor of its top-r subspace, (lambda_{r'} / lambda_r)^(iterations), is
+// at most this: well below the float32 resolution of the iterates, with a
+// margin for the unknown angle of the starting block.
+constexpr double kRefreshEps = 1e-10;
 constexpr int64_t kTileTargetElems = 65536;  // worker elements per tile (all W workers)
 constexpr int kRowsFloatsMax = 4096;         // TM * R bound (shared-memory rows buffer)
 
@@ -195,7 +200,12 @@ struct psgd_ctx {
     bool tab_l_has_recon = false;
     cudaEvent_t* dist_ev = nullptr;   // profiling events of the step in progress
     int svd_every = 0;      // SVD refresh period in steps (0: off)
-    int svd_iters = 0;      // subspace iterations on a refresh step
+    int svd_iters = 0;      // subspace iterations on a refresh step (the cap)
+    int svd_over = 8;       // oversampling columns of a refresh step
+    psgd_ctx* sub = nullptr;   // rank r + p context iterated on refresh steps
+    float* qsub = nullptr;     // its Q block per layer (n x (r + p)), one allocation
+    DevTable tab_sub;          // q' table | L null p_hat | L null recon
+    std::vector<uint64_t> tab_sub_vals;
     uint64_t steps_done = 0;
 
     bool have_step = false;
@@ -436,6 +446,7 @@ int psgd_create(psgd_ctx** out, const psgd_layer* layers, int num_layers, int ra
     const size_t o_T = carve(sizeof(double) * tt);
     const size_t o_cnt = carve(sizeof(unsigned) * cnt);
     const size_t o_status = carve(sizeof(int));
+    const size_t o_conv = carve(sizeof(int) * std::max(1, num_layers));
     ctx->ws_bytes = off;
     cudaError_t e = cudaMalloc(&ctx->ws, ctx->ws_bytes);
     if (e != cudaSuccess) {
@@ -457,6 +468,7 @@ int psgd_create(psgd_ctx** out, const psgd_layer* layers, int num_layers, int ra
     ctx->work.T = reinterpret_cast<double*>(base + o_T);
     ctx->work.cnt = reinterpret_cast<unsigned*>(base + o_cnt);
     ctx->work.status = reinterpret_cast<int*>(base + o_status);
+    ctx->work.conv_iter = reinterpret_cast<int*>(base + o_conv);
 
     e = cudaMemset(ctx->ws, 0, ctx->ws_bytes);
     if (e == cudaSuccess && num_layers > 0)
@@ -504,6 +516,9 @@ void psgd_destroy(psgd_ctx* ctx) {
     if (!ctx) return;
     DeviceGuard g(ctx->device);
     cudaDeviceSynchronize();
+    if (ctx->sub) psgd_destroy(ctx->sub);
+    if (ctx->qsub) cudaFree(ctx->qsub);
+    ctx->tab_sub.release();
     if (ctx->ws) cudaFree(ctx->ws);
     if (ctx->stage) cudaFree(ctx->stage);
     ctx->tab_w.release();
@@ -571,6 +586,68 @@ static cudaEvent_t* profile_events(psgd_ctx* ctx, cudaError_t* err) {
     return ctx->prof_ev[ctx->prof_used++].data();
 }
 
+// A PowerSGD+ refresh step with an oversampled block ("From PowerSGD to
+// PowerSGD+", Abstract: the projection subspace is re-aligned through an
+// SVD): subspace iterations on r' = r + p columns in the rank-r' context
+// ctx->sub, starting from Q' = [warm-start Q | fresh draws], each layer
+// stopping once its convergence bound is met (at most svd_iters
+// iterations); then Rayleigh-Ritz keeps the top r directions in this
+// context's workspace and the caller's Q and P_hat.  The first iteration
+// forms M = G + E over the error buffers (in lazy mode after the previous
+// step's E' has been written out), so that pass C can follow as usual.
+static int refresh_oversampled(psgd_ctx* ctx, const psgd::Params& p, bool lazy, cudaStream_t s, cudaEvent_t* ev) {
+    psgd_ctx* sub = ctx->sub;
+    int rc = PSGD_OK;
+    if (lazy && ctx->errors_hold_m) {
+        psgd::Params pm = p;
+        pm.use_prev = 0;
+        pm.do_resid = 1;
+        rc = launch(ctx, 2, true, pm, ctx->smem_c, s);
+        if (rc) return rc;
+    }
+    cudaError_t e = ctx->tab_sub.update(ctx->tab_sub_vals, s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "table upload");
+    float* const* qs = static_cast<float* const*>(ctx->tab_sub.dev());
+    int64_t maxn = 0;
+    for (auto& d : ctx->desc) maxn = std::max(maxn, d.n);
+    const unsigned gx = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(1024, (maxn * sub->r + 255) / 256)));
+    psgd::k_assemble_q<<<dim3(gx, ctx->L), 256, 0, s>>>(qs, p.t.q, ctx->desc_d, ctx->r, sub->r, ctx->seed,
+                                                        (uint64_t(1) << 62) | (ctx->steps_done + 1));
+    e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaMemsetAsync(sub->work.conv_iter, 0x7f, sizeof(int) * ctx->L, s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "refresh set-up");
+
+    psgd::Params ps = base_params(sub);
+    ps.t.grads = p.t.grads;
+    ps.t.errors = p.t.errors;
+    ps.t.q = qs;
+    ps.t.p_hat_out = qs + ctx->L;     // null entries: the block's P_hat stays inside
+    ps.t.recon_out = qs + 2 * ctx->L;
+    ps.track_conv = 1;
+    ps.r_conv = ctx->r;
+    ps.conv_eps = kRefreshEps;
+    for (int it = 1; it <= ctx->svd_iters && !rc; ++it) {
+        ps.iter = it;
+        rc = launch(sub, it == 1 ? 0 : 3, false, ps, sub->smem_a, s);
+        if (it == 1 && ev) {
+            cudaEventRecord(ev[1], s);
+            cudaEventRecord(ev[2], s);
+        }
+        if (!rc) rc = launch(sub, 1, false, ps, sub->smem_b, s);
+    }
+    if (rc) return fail(ctx, rc, "refresh iterations: %s", sub->err.c_str());
+    void* fn = kernel_ptr(4, sub->R, sub->dtype, false, false);
+    psgd::RRDst dst{ctx->desc_d, ctx->work.phat, ctx->work.qbar, p.t.q, p.t.p_hat_out, ctx->R, ctx->r};
+    void* args[] = {&ps, &dst};
+    e = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(ctx->L)), dim3(psgd::kThreads), args, 0, s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "Rayleigh-Ritz launch");
+    if (ev) {
+        cudaEventRecord(ev[3], s);
+        cudaEventRecord(ev[4], s);
+    }
+    return PSGD_OK;
+}
+
 static int step_impl(psgd_ctx* ctx, const void* const* grads, float* const* errors, float* const* q,
                      float* const* p_hat, float* const* recon, cudaStream_t s) {
     const size_t WL = static_cast<size_t>(ctx->W) * ctx->L;
@@ -615,30 +692,35 @@ static int step_impl(psgd_ctx* ctx, const void* const* grads, float* const* erro
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(ctx, e, "fresh Q launch");
     }
-    rc = launch(ctx, 0, lazy, p, ctx->smem_a, s);
-    if (ev) {
-        cudaEventRecord(ev[1], s);
-        cudaEventRecord(ev[2], s);
-    }
-    if (!rc) rc = launch(ctx, 1, lazy, p, ctx->smem_b, s);
     const bool refresh = ctx->svd_every > 0 && (ctx->steps_done + 1) % ctx->svd_every == 0;
-    const int iters = refresh ? ctx->svd_iters : ctx->iters;
-    for (int it = 1; it < iters && !rc; ++it) {
-        psgd::Params pi = p;
-        pi.use_prev = 0;
-        rc = launch(ctx, 3, false, pi, ctx->smem_a, s);
-        if (!rc) rc = launch(ctx, 1, lazy, pi, ctx->smem_b, s);
-    }
-    if (refresh && !rc) {
-        // Rayleigh-Ritz: one CTA per layer
-        void* fn = kernel_ptr(4, ctx->R, ctx->dtype, false, false);
-        void* args[] = {&p};
-        e = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(ctx->L)), dim3(psgd::kThreads), args, 0, s);
-        if (e != cudaSuccess) return cuda_fail(ctx, e, "Rayleigh-Ritz launch");
-    }
-    if (ev) {
-        cudaEventRecord(ev[3], s);
-        cudaEventRecord(ev[4], s);
+    if (refresh && ctx->sub) {
+        rc = refresh_oversampled(ctx, p, lazy, s, ev);
+    } else {
+        rc = launch(ctx, 0, lazy, p, ctx->smem_a, s);
+        if (ev) {
+            cudaEventRecord(ev[1], s);
+            cudaEventRecord(ev[2], s);
+        }
+        if (!rc) rc = launch(ctx, 1, lazy, p, ctx->smem_b, s);
+        const int iters = refresh ? ctx->svd_iters : ctx->iters;
+        for (int it = 1; it < iters && !rc; ++it) {
+            psgd::Params pi = p;
+            pi.use_prev = 0;
+            rc = launch(ctx, 3, false, pi, ctx->smem_a, s);
+            if (!rc) rc = launch(ctx, 1, lazy, pi, ctx->smem_b, s);
+        }
+        if (refresh && !rc) {
+            // Rayleigh-Ritz in place: one CTA per layer
+            void* fn = kernel_ptr(4, ctx->R, ctx->dtype, false, false);
+            psgd::RRDst dst{ctx->desc_d, ctx->work.phat, ctx->work.qbar, p.t.q, p.t.p_hat_out, ctx->R, ctx->r};
+            void* args[] = {&p, &dst};
+            e = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(ctx->L)), dim3(psgd::kThreads), args, 0, s);
+            if (e != cudaSuccess) return cuda_fail(ctx, e, "Rayleigh-Ritz launch");
+        }
+        if (ev) {
+            cudaEventRecord(ev[3], s);
+            cudaEventRecord(ev[4], s);
+        }
     }
     if (!rc && (!lazy || recon)) {
         psgd::Params pc = p;
@@ -1304,6 +1386,46 @@ int psgd_set_power_iters(psgd_ctx* ctx, int iters) {
     return PSGD_OK;
 }
 
+// (Re)build the rank r + p context of oversampled refresh steps, or drop it
+// when refresh is off or no column can be added (r + p capped by 32 and by
+// the smallest side of every layer).
+static int configure_refresh(psgd_ctx* ctx) {
+    int rp = std::min(psgd::kMaxRank, ctx->r + ctx->svd_over);
+    for (auto& sh : ctx->shapes) rp = static_cast<int>(std::min<int64_t>(rp, std::min(sh.m, sh.n)));
+    const bool want = ctx->svd_every > 0 && rp > ctx->r && ctx->L > 0;
+    if (ctx->sub && (!want || ctx->sub->r != rp)) {
+        psgd_destroy(ctx->sub);
+        ctx->sub = nullptr;
+        if (ctx->qsub) cudaFree(ctx->qsub);
+        ctx->qsub = nullptr;
+        ctx->tab_sub.release();
+        ctx->tab_sub_vals.clear();
+    }
+    if (!want || ctx->sub) return PSGD_OK;
+    DeviceGuard g(ctx->device);
+    psgd_ctx* sub = nullptr;
+    int rc = psgd_create(&sub, ctx->shapes.data(), ctx->L, rp, ctx->W, ctx->seed, ctx->dtype,
+                         ctx->flags & PSGD_FLAG_SUM_FIRST);
+    if (rc) return fail(ctx, rc, "refresh context: %s", psgd_last_error(nullptr));
+    std::vector<size_t> offs(ctx->L);
+    size_t total = 0;
+    for (int l = 0; l < ctx->L; ++l) {
+        offs[l] = total;
+        total = align_up(total + static_cast<size_t>(ctx->shapes[l].n) * rp * sizeof(float), 256);
+    }
+    cudaError_t e = cudaMalloc(&ctx->qsub, total);
+    if (e != cudaSuccess) {
+        psgd_destroy(sub);
+        return fail(ctx, PSGD_ERR_OOM, "refresh Q block of %zu bytes: %s", total, cudaGetErrorString(e));
+    }
+    ctx->sub = sub;
+    ctx->tab_sub_vals.assign(3 * static_cast<size_t>(ctx->L), 0);
+    for (int l = 0; l < ctx->L; ++l)
+        ctx->tab_sub_vals[l] = reinterpret_cast<uint64_t>(static_cast<unsigned char*>(static_cast<void*>(ctx->qsub)) +
+                                                          offs[l]);
+    return PSGD_OK;
+}
+
 int psgd_set_svd_refresh(psgd_ctx* ctx, int every, int iters) {
     if (!ctx) return PSGD_ERR_ARG;
     if (every < 0) return fail(ctx, PSGD_ERR_ARG, "refresh period %d < 0", every);
@@ -1311,7 +1433,15 @@ int psgd_set_svd_refresh(psgd_ctx* ctx, int every, int iters) {
         return fail(ctx, PSGD_ERR_ARG, "refresh iterations %d not in [1, 64]", iters);
     ctx->svd_every = every;
     ctx->svd_iters = every > 0 ? iters : 0;
-    return PSGD_OK;
+    return configure_refresh(ctx);
+}
+
+int psgd_set_svd_oversampling(psgd_ctx* ctx, int extra) {
+    if (!ctx) return PSGD_ERR_ARG;
+    if (extra < 0 || extra > psgd::kMaxRank - 1)
+        return fail(ctx, PSGD_ERR_ARG, "oversampling %d not in [0, %d]", extra, psgd::kMaxRank - 1);
+    ctx->svd_over = extra;
+    return configure_refresh(ctx);
 }
 
 int psgd_profile_enable(psgd_ctx* ctx, int enable) {

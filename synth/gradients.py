@@ -4,7 +4,8 @@ Serves both sides of every check (the CUDA library and the float64 oracle)
 and holds none of the method's arithmetic.
 
 Per layer l (m x n) the generator fixes orthonormal U (m x K), V (n x K) from
-QR of seeded Gaussians and sigma_k = 10 * 2^-k (k = 1..K).  The gradient of
+QR of seeded Gaussians and sigma_k = 10 * 2^-k (k = 1..K), or the workload's
+explicit spectrum when it gives one.  The gradient of
 worker w at step t is
 
     G = U diag(sigma) V^T + s * N(0, 1)
@@ -89,7 +90,7 @@ class GradientSource:
         self._U: List[np.ndarray] = []
         self._V: List[np.ndarray] = []
         for l, (m, n) in enumerate(wl.layers):
-            K = min(wl.spectrum_terms, m, n)
+            K = min(len(wl.spectrum) if wl.spectrum else wl.spectrum_terms, m, n)
             self._U.append(_orthonormal(m, K, mix_seed(seed, _TAG_BASIS, l, 0)))
             self._V.append(_orthonormal(n, K, mix_seed(seed, _TAG_BASIS, l, 1)))
         self._basis_step = 0
@@ -112,7 +113,12 @@ class GradientSource:
     def basis(self, step: int, l: int):
         self._advance_to(step)
         U, V = self._U[l], self._V[l]
-        return U, V, sigmas(U.shape[1])
+        return U, V, self._sigmas(U.shape[1])
+
+    def _sigmas(self, K: int) -> np.ndarray:
+        if self.wl.spectrum:
+            return np.asarray(self.wl.spectrum[:K], dtype=np.float64)
+        return sigmas(K)
 
     def lowrank(self, step: int, l: int, device="cpu") -> torch.Tensor:
         U, V, s = self.basis(step, l)
@@ -125,8 +131,8 @@ class GradientSource:
         if kind == "abs":
             return float(val)
         m, n = self.wl.layers[l]
-        K = min(self.wl.spectrum_terms, m, n)
-        rms = math.sqrt(float(np.sum(sigmas(K) ** 2))) / math.sqrt(m * n)
+        K = min(len(self.wl.spectrum) if self.wl.spectrum else self.wl.spectrum_terms, m, n)
+        rms = math.sqrt(float(np.sum(self._sigmas(K) ** 2))) / math.sqrt(m * n)
         return float(val) * rms
 
     def _torch_dtype(self):

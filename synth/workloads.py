@@ -26,6 +26,7 @@ class Workload:
     rotate: float = 0.0                      # subspace rotation angle per step (radians)
     ranks: Tuple[int, ...] = ()              # rank sweep (rank is the first entry)
     spectrum_terms: int = 4                  # K in sum_k sigma_k u_k v_k^T, sigma_k = 10 * 2^-k
+    spectrum: Tuple[float, ...] = ()         # explicit sigma_1 >= sigma_2 >= ... (replaces the default)
 
     @property
     def elements_per_worker(self) -> int:

@@ -38,14 +38,14 @@ class LibRun:
 
     def __init__(self, wl: Workload, seed: int = 1234, lazy: bool = False, sum_first: bool = False,
                  recon: bool = True, device: str = "cuda", iters: int = 1, warm_start: bool = True,
-                 svd_every: int = 0, svd_iters: int = 8):
+                 svd_every: int = 0, svd_iters: int = 8, svd_oversampling=None):
         from rank_gradient_compression_02_b200 import PowerSGD
         self.wl = wl
         self.seed = seed
         self.src = GradientSource(wl, seed)
         self.lib = PowerSGD(wl.layers, wl.rank, wl.workers, seed=seed, grad_dtype=wl.grad_dtype,
                             lazy_errors=lazy, sum_first=sum_first, power_iters=iters, warm_start=warm_start,
-                            svd_every=svd_every, svd_iters=svd_iters)
+                            svd_every=svd_every, svd_iters=svd_iters, svd_oversampling=svd_oversampling)
         self.lazy = lazy
         gdt = torch.bfloat16 if wl.grad_dtype == "bf16" else torch.float32
         W, L = wl.workers, len(wl.layers)
