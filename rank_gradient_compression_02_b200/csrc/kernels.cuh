@@ -124,6 +124,18 @@ constexpr int kWideRows = 64;    // rows per tile cap for the wide kernels
 // and the rounding of the lo parts leave a relative error below 2^-21
 // (split-precision products on tensor cores: Markidis et al., "NVIDIA
 // Tensor Core Programmability, Performance & Precision", IPDPSW 2018).
+// Rounding to tf32 on the bit pattern: the magnitude bits plus half a unit of
+// the 13 dropped bits, then truncated.  IEEE sign-magnitude encoding makes
+// this round-to-nearest with ties away from zero (a carry out of the
+// mantissa moves to the next binade; infinity stays infinity), computed on
+// the integer pipe instead of the conversion unit.  Any rounding to tf32
+// would do: hi + lo = x holds exactly whichever way hi is rounded.
+// The first pass is bound by the conversion unit (its float64 flushes), so
+// it rounds on the integer pipe; the second pass, whose conversion unit is
+// idle and whose registers are at their limit, uses cvt.rna.tf32.f32.
+__device__ __forceinline__ uint32_t tf32_round_int(float x) {
+    return (__float_as_uint(x) + 0x1000u) & 0xffffe000u;
+}
 __device__ __forceinline__ uint32_t tf32_round(float x) {
     uint32_t r;
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
@@ -132,6 +144,10 @@ __device__ __forceinline__ uint32_t tf32_round(float x) {
 __device__ __forceinline__ void tf32_split(float x, uint32_t& hi, uint32_t& lo) {
     hi = tf32_round(x);
     lo = tf32_round(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void tf32_split_int(float x, uint32_t& hi, uint32_t& lo) {
+    hi = tf32_round_int(x);
+    lo = tf32_round_int(x - __uint_as_float(hi));
 }
 // c += A (16 x 8, row-major fragment) * B (8 x 8, column fragment), float32
 // accumulate.  Fragment of lane (g = lane / 4, t = lane % 4): a = A[g][t],
@@ -152,6 +168,28 @@ __device__ __forceinline__ void mma_tf32x3(float (&c)[4], const uint32_t (&ahi)[
     mma_tf32(c, ahi, __float_as_uint(b.z), __float_as_uint(b.w));
     mma_tf32(c, ahi, __float_as_uint(b.x), __float_as_uint(b.y));
 }
+
+// ---- asynchronous global -> shared copies (16 bytes, no register staging) --
+// cp.async with a source size of 0 writes zeros (used for rows and columns
+// outside the layer; the source address is then never read).
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, bool valid) {
+    const unsigned dst = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    const int n = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(gsrc), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
+// Staged second pass (ranks 16, 32; rows 16-byte aligned, i.e. n % 4 == 0):
+// one worker's 64 x 128 block of M at a time goes to shared memory by
+// cp.async (kStages buffers), row stride kStgStride floats (the padding
+// keeps a quarter-warp's 8-byte fragment loads on distinct banks).
+constexpr int kStgRows = 64;
+constexpr int kStgCols = 128;
+constexpr int kStgStride = kStgCols + 8;
+constexpr int kStages = 2;
+constexpr size_t kStgBytes = static_cast<size_t>(kStages) * kStgRows * kStgStride * sizeof(float);
 
 constexpr int kMmaRows = 16;                  // rows per warp in the tensor-core pass A
 constexpr int kMaxKSteps = 32 * 4 / 8;        // k-steps of 8 columns in the widest chunk
@@ -325,9 +363,9 @@ __device__ __forceinline__ void pass_a_rows(const Params& p, const LayerDesc& d,
 // the mma A fragments (VEC-wide loads), forms M = G + E there, stores M
 // over E, prefetches the next block and multiplies: per k-step of 8
 // columns and 8 ranks, three tf32 products (mma_tf32x3) summed in float32,
-// then added to a float64 accumulator, i.e. float32 runs of 8 terms as in
-// the CUDA-core passes.  At the end the parts' partials are added in part
-// order and written per chunk.
+// then added to a Kahan-compensated float32 accumulator, which is widened to
+// float64 at the end of the tile.  The parts' partials are then added in
+// part order (float64) and written per chunk.
 //
 // Fragment columns.  An mma k-step takes 8 columns in any order, as long
 // as A and B agree.  Lane (g, t) holds rows g and g + 8 and, in k-step ks,
@@ -501,11 +539,15 @@ __device__ __forceinline__ void pass_a_mma(const Params& p, const LayerDesc& d, 
         if constexpr (!READM) load_frag<VEC>(gp[w] + row0 + sc * kWideCols, n, g, t4, ok_lo, ok_hi, cols, gq);
     };
 
-    double acc[NT][4];
+    // Kahan-compensated float32 sums of the k-steps' products (Kahan 1965):
+    // the running sum and its compensation stay on the FMA pipe, accurate
+    // to about one float32 rounding of the sum however many k-steps it
+    // takes; the tile's result is widened to float64 once, below.
+    float accf[NT][4], comp[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[nt][c] = 0.0;
+        for (int c = 0; c < 4; ++c) accf[nt][c] = comp[nt][c] = 0.f;
     float* rt = reinterpret_cast<float*>(wide + kQfBytes);   // lazy: [tile row][chunk column]
     float msum[SF ? 4 : 1][SF ? 4 : 1];
     if constexpr (LAZY) {
@@ -541,14 +583,19 @@ __device__ __forceinline__ void pass_a_mma(const Params& p, const LayerDesc& d, 
             if ((VEC == 4 ? 16 * (ks >> 1) : 8 * ks) < cols) {
                 uint32_t ahi[4], alo[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) tf32_split(mv[ks][q], ahi[q], alo[q]);
+                for (int q = 0; q < 4; ++q) tf32_split_int(mv[ks][q], ahi[q], alo[q]);
                 const float4* qk = qf + ((sc * 4 + ks) * NT) * 32 + lane;
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     float c[4] = {0.f, 0.f, 0.f, 0.f};
                     mma_tf32x3(c, ahi, alo, qk[nt * 32]);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) acc[nt][q] += static_cast<double>(c[q]);
+                    for (int q = 0; q < 4; ++q) {
+                        const float y = c[q] - comp[nt][q];
+                        const float t = accf[nt][q] + y;
+                        comp[nt][q] = (t - accf[nt][q]) - y;
+                        accf[nt][q] = t;
+                    }
                 }
             }
         }
@@ -604,6 +651,12 @@ __device__ __forceinline__ void pass_a_mma(const Params& p, const LayerDesc& d, 
         sc = sc2;
         wi = wi2;
     }
+
+    double acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[nt][q] = static_cast<double>(accf[nt][q]) - static_cast<double>(comp[nt][q]);
 
     // parts' partials added in part order; part 0 writes the chunk's rows
     __syncthreads();   // every warp is done with the Q fragments
@@ -833,6 +886,12 @@ struct SmemB {
     static __host__ __device__ size_t rows_bytes(int tm) { return static_cast<size_t>(tm) * R * sizeof(float); }
     static __host__ __device__ size_t t_bytes() { return R * R * sizeof(double); }
     static __host__ __device__ size_t red_bytes(int vec) {
+        if (UseMma<R>::value && vec == 4) {
+            // staged kernel: the M stages + the split P_hat^T fragments of
+            // every k-step of the tile (8 k-steps x R / 16 m-tiles x 32 lanes
+            // x hi, lo float4)
+            return kStgBytes + static_cast<size_t>(kStgRows / 8) * (R / 16) * 32 * 2 * sizeof(float4);
+        }
         if (UseMma<R>::value) {
             // tensor-core kernel: warp partials (8 x 32 columns x 33) + the
             // warps' A fragments
@@ -1203,6 +1262,188 @@ __device__ __forceinline__ void pass_b_mma(const Params& p, const LayerDesc& d, 
     }
 }
 
+// Staged tensor-core second pass (R = 16, 32; VEC 4).  The tile (tm <= 64
+// rows x a chunk of <= 128 columns) is processed one worker at a time: the
+// worker's block is copied into a shared-memory stage by cp.async while the
+// previous worker's block is multiplied, so several 32 KB blocks per SM are
+// in flight without holding registers.  Warp w owns the chunk columns
+// 16 w .. 16 w + 15 over all the tile's rows: D (R ranks x 16 columns) =
+// P_hat^T (ranks x rows) * M (rows x columns), two n-tiles of 8 columns,
+// n-tile j taking column 16 w + 2 g + j as its column g, so that lane
+// (g, t) reads one 8-byte pair per row.  A = P_hat^T of all the tile's
+// rows, split into tf32 hi and lo once per tile.  D accumulates one worker
+// (tm rows, three split products per term) in float32 and is then added to
+// a float64 sum: float32 runs of at most 64 rows, as in the other
+// tensor-core kernels.  No cross-warp reduction: every warp writes its own
+// columns' row-block partial.
+template <int R, bool SF>
+__device__ __forceinline__ void pass_b_staged(const Params& p, const LayerDesc& d, const TileCoord& tc,
+                                              float* const* ep, const float* ph_s, float* red_s) {
+    static_assert(R == 16 || R == 32, "staged pass B: rank 16 or 32");
+    constexpr int MT = R / 16;                  // m-tiles of 16 ranks
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int W = p.workers;
+    const int64_t n = d.n;
+    const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
+    const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), d.m - i0));
+    const int64_t jc = static_cast<int64_t>(tc.c) * d.slots * 4;
+    const int width = static_cast<int>(min(static_cast<int64_t>(d.slots) * 4, n - jc));
+    const int nks = d.tm / 8;                   // k-steps of 8 rows (tm = 16, 32 or 64)
+    float* stg = red_s;                         // [stage][row][kStgStride]
+    float4* pa = reinterpret_cast<float4*>(reinterpret_cast<unsigned char*>(red_s) + kStgBytes);  // [ks][mt][lane][hi, lo]
+
+    // A fragments: A[rank][row] = P_hat[row][rank] (zero outside the
+    // layer); slot t <- row 8 ks + t, slot t + 4 <- row 8 ks + t + 4
+    for (int idx = tid; idx < nks * MT * 32; idx += kThreads) {
+        const int ln = idx & 31, mt = (idx >> 5) % MT, ks = (idx >> 5) / MT;
+        const int gg = ln >> 2, tt = ln & 3;
+        float av[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int row = 8 * ks + tt + 4 * (q >> 1);
+            const int rank = 16 * mt + gg + 8 * (q & 1);
+            av[q] = row < rows ? ph_s[row * R + rank] : 0.f;
+        }
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tf32_split(av[q], hi[q], lo[q]);
+        pa[2 * idx] = make_float4(__uint_as_float(hi[0]), __uint_as_float(hi[1]), __uint_as_float(hi[2]),
+                                  __uint_as_float(hi[3]));
+        pa[2 * idx + 1] = make_float4(__uint_as_float(lo[0]), __uint_as_float(lo[1]), __uint_as_float(lo[2]),
+                                      __uint_as_float(lo[3]));
+    }
+
+    // one worker's block into stage s: (tm rows) x (32 x 16 bytes)
+    auto issue = [&](int w, int stage) {
+        float* dst = stg + static_cast<size_t>(stage) * kStgRows * kStgStride;
+        const float* src = ep[w] + i0 * n + jc;
+        for (int idx = tid; idx < d.tm * (kStgCols / 4); idx += kThreads) {
+            const int row = idx >> 5, c4 = (idx & 31) * 4;
+            const bool ok = row < rows && c4 < width;
+            cp_async16(dst + row * kStgStride + c4, ok ? src + static_cast<int64_t>(row) * n + c4 : src, ok);
+        }
+    };
+
+    const int col0 = 16 * warp + 2 * g;          // this lane's column pair (n-tiles 0 and 1)
+    const bool active = 16 * warp < width;
+    float dacc[MT][2][4];
+    double dsum[MT][2][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) dsum[mt][j][q] = 0.0;
+    float msum[SF ? 8 : 1][SF ? 4 : 1];
+    if constexpr (SF) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) msum[ks][q] = 0.f;
+    }
+
+    // products of one block (x[ks] = rows 8 ks + t, 8 ks + t + 4 at the
+    // lane's two columns) into dsum
+    auto multiply = [&](const float* blk) {
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) dacc[mt][j][q] = 0.f;
+#pragma unroll(SF ? 8 : 1)
+        for (int ks = 0; ks < (SF ? 8 : nks); ++ks) {
+            if (SF && ks >= nks) break;
+            float x[4];
+            if constexpr (SF) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) x[q] = msum[ks][q];
+            } else {
+                const float2 a = *reinterpret_cast<const float2*>(blk + (8 * ks + t4) * kStgStride + col0);
+                const float2 b = *reinterpret_cast<const float2*>(blk + (8 * ks + t4 + 4) * kStgStride + col0);
+                x[0] = a.x; x[1] = b.x; x[2] = a.y; x[3] = b.y;
+            }
+            // B fragments of the two n-tiles: b0 = row t, b1 = row t + 4
+            uint32_t bh[4], bl[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) tf32_split(x[q], bh[q], bl[q]);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const float4 h4 = pa[2 * ((ks * MT + mt) * 32 + lane)];
+                const float4 l4 = pa[2 * ((ks * MT + mt) * 32 + lane) + 1];
+                const uint32_t ahi[4] = {__float_as_uint(h4.x), __float_as_uint(h4.y), __float_as_uint(h4.z),
+                                         __float_as_uint(h4.w)};
+                const uint32_t alo[4] = {__float_as_uint(l4.x), __float_as_uint(l4.y), __float_as_uint(l4.z),
+                                         __float_as_uint(l4.w)};
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    mma_tf32(dacc[mt][j], alo, bh[2 * j], bh[2 * j + 1]);
+                    mma_tf32(dacc[mt][j], ahi, bl[2 * j], bl[2 * j + 1]);
+                    mma_tf32(dacc[mt][j], ahi, bh[2 * j], bh[2 * j + 1]);
+                }
+            }
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) dsum[mt][j][q] += static_cast<double>(dacc[mt][j][q]);
+    };
+
+    // pipeline over the workers: kStages - 1 blocks ahead
+#pragma unroll
+    for (int s0 = 0; s0 < kStages - 1; ++s0) {
+        if (s0 < W) issue(s0, s0);
+        cp_async_commit();
+    }
+    __syncthreads();   // the A fragments are in shared memory
+    for (int w = 0; w < W; ++w) {
+        const int ahead = w + kStages - 1;
+        if (ahead < W) issue(ahead, ahead % kStages);
+        cp_async_commit();                       // (an empty group keeps the count uniform)
+        cp_async_wait<kStages - 1>();            // worker w's block has landed
+        __syncthreads();
+        const float* blk = stg + static_cast<size_t>(w % kStages) * kStgRows * kStgStride;
+        if (active) {
+            if constexpr (SF) {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    if (ks >= nks) break;
+                    const float2 a = *reinterpret_cast<const float2*>(blk + (8 * ks + t4) * kStgStride + col0);
+                    const float2 b = *reinterpret_cast<const float2*>(blk + (8 * ks + t4 + 4) * kStgStride + col0);
+                    msum[ks][0] += a.x;
+                    msum[ks][1] += b.x;
+                    msum[ks][2] += a.y;
+                    msum[ks][3] += b.y;
+                }
+                if (w == W - 1) multiply(blk);
+            } else {
+                multiply(blk);
+            }
+        }
+        __syncthreads();   // stage w % kStages may be refilled next
+    }
+    cp_async_wait<0>();
+
+    // this warp's columns of the row block's partial Q rows
+    if (active) {
+        double* qpart = p.ws.qpart + d.qpart_off;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int rank = 16 * mt + g + 8 * (q >> 1);
+                    const int col = 16 * warp + 2 * (2 * t4 + (q & 1)) + j;
+                    if (col < width)
+                        qpart[(static_cast<int64_t>(tc.rb) * n + jc + col) * R + rank] = dsum[mt][j][q];
+                }
+    }
+}
+
 template <int R>
 __device__ void pass_b_epilogue(const Params& p, const LayerDesc& d, const TileCoord& tc) {
     __shared__ int s_flag;
@@ -1294,7 +1535,7 @@ __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_b(Params p)
 
     if constexpr (UseMma<R>::value) {
         if (d.vec == 4) {
-            pass_b_mma<R, 4, SF>(p, d, tc, ep, ph_s, red_s);
+            pass_b_staged<R, SF>(p, d, tc, ep, ph_s, red_s);
         } else if (d.vec == 2) {
             pass_b_mma<R, 2, SF>(p, d, tc, ep, ph_s, red_s);
         } else {
@@ -1767,7 +2008,7 @@ __global__ void __launch_bounds__(kThreads) k_rayleigh_ritz(Params p, RRDst dst)
                 int best = a;
                 for (int b = a + 1; b < r; ++b)
                     if (lam[order[b]] > lam[order[best]]) best = b;
-                const int tmp = order[a];
+                const int tmp = order[best];
                 for (int b = best; b > a; --b) order[b] = order[b - 1];
                 order[a] = tmp;
             }
