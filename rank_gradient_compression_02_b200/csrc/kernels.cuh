@@ -190,6 +190,11 @@ constexpr int kStgCols = 128;
 constexpr int kStgStride = kStgCols + 8;
 constexpr int kStages = 2;
 constexpr size_t kStgBytes = static_cast<size_t>(kStages) * kStgRows * kStgStride * sizeof(float);
+// Staged CUDA-core second pass (R <= 4, rows 16-byte aligned): units of
+// 32 rows x 128 columns of one worker (16 KB), three stages.
+constexpr int kUnitRows = 32;
+constexpr int kUnitStages = 3;
+constexpr size_t kUnitBytes = static_cast<size_t>(kUnitStages) * kUnitRows * kStgCols * sizeof(float);
 
 constexpr int kMmaRows = 16;                  // rows per warp in the tensor-core pass A
 constexpr int kMaxKSteps = 32 * 4 / 8;        // k-steps of 8 columns in the widest chunk
@@ -897,7 +902,7 @@ struct SmemB {
             // warps' A fragments
             return static_cast<size_t>(kWarps) * kWideCols * kRedStride * sizeof(float) + kPaBytes;
         }
-        return static_cast<size_t>(kWarps) * R * vec * 32 * sizeof(float);
+        return static_cast<size_t>(kWarps) * R * vec * 32 * sizeof(float) + (vec == 4 ? kUnitBytes : 0);
     }
     static __host__ __device__ size_t total(int W, int tm, int vec) {
         return ((ptr_bytes(W) + 15) & ~size_t(15)) + ((rows_bytes(tm) + 15) & ~size_t(15)) + t_bytes() +
@@ -1067,6 +1072,125 @@ __device__ __forceinline__ void pass_b_rows(const Params& p, const LayerDesc& d,
 #pragma unroll
         for (int wp = 0; wp < kWarps; ++wp) s += static_cast<double>(red_s[((wp * R + k) * VEC + v) * 32 + ln]);
         qpart[(static_cast<int64_t>(tc.rb) * n + static_cast<int64_t>(s0) * VEC + cc) * R + k] = s;
+    }
+}
+
+// Staged CUDA-core second pass (R <= 4, VEC 4).  The tile's rows are
+// walked in units of 32 rows x the chunk's columns of one worker, copied
+// into a three-stage shared-memory ring by cp.async (rows and columns
+// outside the layer zero-filled), so that about two units per CTA are in
+// flight while one is multiplied; units go row group by row group, the
+// workers in order inside each group.  Warp w takes rows w, w + 8, w + 16,
+// w + 24 of a unit; lane l the 4 columns of vector slot l, read from shared
+// memory (a warp reads one contiguous 512-byte row: no bank conflicts).
+// The products are summed per lane in float32 over the tile's rows and
+// workers and then across warps in float64 (as in pass_b_rows).
+template <int R, bool SF>
+__device__ __forceinline__ void pass_b_rows_staged(const Params& p, const LayerDesc& d, const TileCoord& tc,
+                                                   float* const* ep, const float* ph_s, float* red_s) {
+    static_assert(R <= 4, "staged CUDA-core pass B: 16-byte lanes need R <= 4");
+    constexpr int VEC = 4;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int W = p.workers;
+    const int64_t n = d.n, m = d.m;
+    const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
+    const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), m - i0));
+    const int s0 = tc.c * d.slots;
+    const int ns = min(d.slots, d.nvec - s0);
+    const bool active = lane < ns;
+    const int64_t jc = static_cast<int64_t>(s0) * VEC;
+    const int width = ns * VEC;
+    const int ur = min(kUnitRows, d.tm);        // rows per unit (tiles of many workers have few rows)
+    const int ngroups = (rows + ur - 1) / ur;
+    const int nunits = ngroups * W;
+    float* ring = red_s + static_cast<size_t>(kWarps) * R * VEC * 32;   // after the warp partials
+
+    auto issue = [&](int u, int stage) {
+        const int g = u / W, w = u - (u / W) * W;
+        float* dst = ring + static_cast<size_t>(stage) * kUnitRows * kStgCols;
+        const float* src = ep[w] + (i0 + static_cast<int64_t>(g) * ur) * n + jc;
+        const int grows = min(ur, rows - g * ur);
+        for (int idx = tid; idx < ur * (kStgCols / 4); idx += kThreads) {
+            const int row = idx >> 5, c4 = (idx & 31) * 4;
+            const bool ok = row < grows && c4 < width;
+            cp_async16(dst + row * kStgCols + c4, ok ? src + static_cast<int64_t>(row) * n + c4 : src, ok);
+        }
+    };
+
+    float qacc[VEC][R];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v)
+#pragma unroll
+        for (int k = 0; k < R; ++k) qacc[v][k] = 0.f;
+    float msum[SF ? 4 : 1][SF ? VEC : 1];
+    if constexpr (SF) {
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) msum[rr][v] = 0.f;
+    }
+
+#pragma unroll
+    for (int s0u = 0; s0u < kUnitStages - 1; ++s0u) {
+        if (s0u < nunits) issue(s0u, s0u);
+        cp_async_commit();
+    }
+    for (int u = 0; u < nunits; ++u) {
+        const int ahead = u + kUnitStages - 1;
+        if (ahead < nunits) issue(ahead, ahead % kUnitStages);
+        cp_async_commit();
+        cp_async_wait<kUnitStages - 1>();
+        __syncthreads();
+        const float* blk = ring + static_cast<size_t>(u % kUnitStages) * kUnitRows * kStgCols;
+        const int g = u / W, w = u - (u / W) * W;
+        if (active) {
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                const int row = warp + kWarps * rr;
+                const int gi = g * ur + row;
+                if (row < ur && gi < rows) {
+                    const float4 x4 = *reinterpret_cast<const float4*>(blk + row * kStgCols + VEC * lane);
+                    const float x[VEC] = {x4.x, x4.y, x4.z, x4.w};
+                    float ph[R];
+#pragma unroll
+                    for (int k = 0; k < R; ++k) ph[k] = ph_s[gi * R + k];
+                    if constexpr (SF) {
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) msum[rr][v] += x[v];
+                        if (w == W - 1) {
+#pragma unroll
+                            for (int v = 0; v < VEC; ++v) {
+                                axpy<R>(qacc[v], msum[rr][v], ph);
+                                msum[rr][v] = 0.f;
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) axpy<R>(qacc[v], x[v], ph);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+    cp_async_wait<0>();
+
+    // this warp's partial, laid out [warp][k][v][lane] (conflict-free)
+#pragma unroll
+    for (int k = 0; k < R; ++k)
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) red_s[((warp * R + k) * VEC + v) * 32 + lane] = qacc[v][k];
+    __syncthreads();
+    // sum over warps in order; write the row block's partial Q rows
+    double* qpart = p.ws.qpart + d.qpart_off;
+    for (int idx = tid; idx < width * R; idx += kThreads) {
+        const int cc = idx / R;
+        const int k = idx % R;
+        const int ln = cc / VEC, v = cc % VEC;
+        double s = 0.0;
+#pragma unroll
+        for (int wp = 0; wp < kWarps; ++wp) s += static_cast<double>(red_s[((wp * R + k) * VEC + v) * 32 + ln]);
+        qpart[(static_cast<int64_t>(tc.rb) * n + jc + cc) * R + k] = s;
     }
 }
 
@@ -1543,7 +1667,7 @@ __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_b(Params p)
         }
     } else {
         if (d.vec == 4) {
-            if constexpr (R <= 4) pass_b_rows<R, 4, SF>(p, d, tc, ep, ph_s, red_s);
+            if constexpr (R <= 4) pass_b_rows_staged<R, SF>(p, d, tc, ep, ph_s, red_s);
         } else if (d.vec == 2) {
             if constexpr (R <= 16) pass_b_rows<R, 2, SF>(p, d, tc, ep, ph_s, red_s);
         } else {

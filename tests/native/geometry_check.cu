@@ -45,6 +45,11 @@ int main() {
         for (int lazy = 0; lazy < 2; ++lazy) {
             size_t a = smem_need(0, R, c.W, d.tm, d.vec, lazy), b = smem_need(1, R, c.W, d.tm, d.vec), cc = smem_need(2, R, c.W, d.tm, d.vec);
             if (a > 232448 || b > 232448 || cc > 232448 || !a || !b || !cc) fail("shared memory within 227 KB");
+            // the CTAs per SM the launch bounds aim at (228 KB per SM, 1 KB
+            // reserved per CTA): 3 for passes A and B at R <= 8, else 2
+            const size_t per3 = 228 * 1024 / 3 - 1024, per2 = 228 * 1024 / 2 - 1024;
+            if (a > (R <= 8 ? per3 : per2) || b > (R <= 8 ? per3 : per2) || cc > per2)
+                fail("shared memory lets the intended CTAs per SM reside");
         }
         if (sz.tiles != (int64_t)d.nrb * d.nchunk) fail("tile count");
     }

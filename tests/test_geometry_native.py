@@ -4,7 +4,8 @@ for every shape, rank and worker count the GPU tests and the full-size
 workloads use, that the lane
 width divides the row, chunks and row blocks cover the matrix with none
 empty, the tensor-core tiles are whole 16-row groups, the rows buffer and
-the widest chunk fit, and each pass's shared memory fits in 227 KB."""
+the widest chunk fit, and each pass's shared memory fits in 227 KB and
+leaves room for the CTAs per SM its launch bounds aim at."""
 import os
 import shutil
 import subprocess
