@@ -190,11 +190,6 @@ constexpr int kStgCols = 128;
 constexpr int kStgStride = kStgCols + 8;
 constexpr int kStages = 2;
 constexpr size_t kStgBytes = static_cast<size_t>(kStages) * kStgRows * kStgStride * sizeof(float);
-// Staged CUDA-core second pass (R <= 4, rows 16-byte aligned): units of
-// 32 rows x 128 columns of one worker (16 KB), three stages.
-constexpr int kUnitRows = 32;
-constexpr int kUnitStages = 3;
-constexpr size_t kUnitBytes = static_cast<size_t>(kUnitStages) * kUnitRows * kStgCols * sizeof(float);
 
 constexpr int kMmaRows = 16;                  // rows per warp in the tensor-core pass A
 constexpr int kMaxKSteps = 32 * 4 / 8;        // k-steps of 8 columns in the widest chunk
@@ -889,20 +884,21 @@ template <int R>
 struct SmemB {
     static __host__ __device__ size_t ptr_bytes(int W) { return static_cast<size_t>(W) * sizeof(void*); }
     static __host__ __device__ size_t rows_bytes(int tm) { return static_cast<size_t>(tm) * R * sizeof(float); }
-    static __host__ __device__ size_t t_bytes() { return R * R * sizeof(double); }
+    // rounded up to 16 bytes: the region after it takes 16-byte accesses
+    static __host__ __device__ size_t t_bytes() { return (R * R * sizeof(double) + 15) & ~size_t(15); }
     static __host__ __device__ size_t red_bytes(int vec) {
         if (UseMma<R>::value && vec == 4) {
-            // staged kernel: the M stages + the split P_hat^T fragments of
-            // every k-step of the tile (8 k-steps x R / 16 m-tiles x 32 lanes
-            // x hi, lo float4)
-            return kStgBytes + static_cast<size_t>(kStgRows / 8) * (R / 16) * 32 * 2 * sizeof(float4);
+            // staged kernel: the M stages, reused at the end for the warps'
+            // partials (8 warps x 64 columns x (R + 1) floats)
+            const size_t red = static_cast<size_t>(kWarps) * 64 * (R + 1) * sizeof(float);
+            return kStgBytes > red ? kStgBytes : red;
         }
         if (UseMma<R>::value) {
             // tensor-core kernel: warp partials (8 x 32 columns x 33) + the
             // warps' A fragments
             return static_cast<size_t>(kWarps) * kWideCols * kRedStride * sizeof(float) + kPaBytes;
         }
-        return static_cast<size_t>(kWarps) * R * vec * 32 * sizeof(float) + (vec == 4 ? kUnitBytes : 0);
+        return static_cast<size_t>(kWarps) * R * vec * 32 * sizeof(float);
     }
     static __host__ __device__ size_t total(int W, int tm, int vec) {
         return ((ptr_bytes(W) + 15) & ~size_t(15)) + ((rows_bytes(tm) + 15) & ~size_t(15)) + t_bytes() +
@@ -1072,125 +1068,6 @@ __device__ __forceinline__ void pass_b_rows(const Params& p, const LayerDesc& d,
 #pragma unroll
         for (int wp = 0; wp < kWarps; ++wp) s += static_cast<double>(red_s[((wp * R + k) * VEC + v) * 32 + ln]);
         qpart[(static_cast<int64_t>(tc.rb) * n + static_cast<int64_t>(s0) * VEC + cc) * R + k] = s;
-    }
-}
-
-// Staged CUDA-core second pass (R <= 4, VEC 4).  The tile's rows are
-// walked in units of 32 rows x the chunk's columns of one worker, copied
-// into a three-stage shared-memory ring by cp.async (rows and columns
-// outside the layer zero-filled), so that about two units per CTA are in
-// flight while one is multiplied; units go row group by row group, the
-// workers in order inside each group.  Warp w takes rows w, w + 8, w + 16,
-// w + 24 of a unit; lane l the 4 columns of vector slot l, read from shared
-// memory (a warp reads one contiguous 512-byte row: no bank conflicts).
-// The products are summed per lane in float32 over the tile's rows and
-// workers and then across warps in float64 (as in pass_b_rows).
-template <int R, bool SF>
-__device__ __forceinline__ void pass_b_rows_staged(const Params& p, const LayerDesc& d, const TileCoord& tc,
-                                                   float* const* ep, const float* ph_s, float* red_s) {
-    static_assert(R <= 4, "staged CUDA-core pass B: 16-byte lanes need R <= 4");
-    constexpr int VEC = 4;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int W = p.workers;
-    const int64_t n = d.n, m = d.m;
-    const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
-    const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), m - i0));
-    const int s0 = tc.c * d.slots;
-    const int ns = min(d.slots, d.nvec - s0);
-    const bool active = lane < ns;
-    const int64_t jc = static_cast<int64_t>(s0) * VEC;
-    const int width = ns * VEC;
-    const int ur = min(kUnitRows, d.tm);        // rows per unit (tiles of many workers have few rows)
-    const int ngroups = (rows + ur - 1) / ur;
-    const int nunits = ngroups * W;
-    float* ring = red_s + static_cast<size_t>(kWarps) * R * VEC * 32;   // after the warp partials
-
-    auto issue = [&](int u, int stage) {
-        const int g = u / W, w = u - (u / W) * W;
-        float* dst = ring + static_cast<size_t>(stage) * kUnitRows * kStgCols;
-        const float* src = ep[w] + (i0 + static_cast<int64_t>(g) * ur) * n + jc;
-        const int grows = min(ur, rows - g * ur);
-        for (int idx = tid; idx < ur * (kStgCols / 4); idx += kThreads) {
-            const int row = idx >> 5, c4 = (idx & 31) * 4;
-            const bool ok = row < grows && c4 < width;
-            cp_async16(dst + row * kStgCols + c4, ok ? src + static_cast<int64_t>(row) * n + c4 : src, ok);
-        }
-    };
-
-    float qacc[VEC][R];
-#pragma unroll
-    for (int v = 0; v < VEC; ++v)
-#pragma unroll
-        for (int k = 0; k < R; ++k) qacc[v][k] = 0.f;
-    float msum[SF ? 4 : 1][SF ? VEC : 1];
-    if constexpr (SF) {
-#pragma unroll
-        for (int rr = 0; rr < 4; ++rr)
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) msum[rr][v] = 0.f;
-    }
-
-#pragma unroll
-    for (int s0u = 0; s0u < kUnitStages - 1; ++s0u) {
-        if (s0u < nunits) issue(s0u, s0u);
-        cp_async_commit();
-    }
-    for (int u = 0; u < nunits; ++u) {
-        const int ahead = u + kUnitStages - 1;
-        if (ahead < nunits) issue(ahead, ahead % kUnitStages);
-        cp_async_commit();
-        cp_async_wait<kUnitStages - 1>();
-        __syncthreads();
-        const float* blk = ring + static_cast<size_t>(u % kUnitStages) * kUnitRows * kStgCols;
-        const int g = u / W, w = u - (u / W) * W;
-        if (active) {
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
-                const int row = warp + kWarps * rr;
-                const int gi = g * ur + row;
-                if (row < ur && gi < rows) {
-                    const float4 x4 = *reinterpret_cast<const float4*>(blk + row * kStgCols + VEC * lane);
-                    const float x[VEC] = {x4.x, x4.y, x4.z, x4.w};
-                    float ph[R];
-#pragma unroll
-                    for (int k = 0; k < R; ++k) ph[k] = ph_s[gi * R + k];
-                    if constexpr (SF) {
-#pragma unroll
-                        for (int v = 0; v < VEC; ++v) msum[rr][v] += x[v];
-                        if (w == W - 1) {
-#pragma unroll
-                            for (int v = 0; v < VEC; ++v) {
-                                axpy<R>(qacc[v], msum[rr][v], ph);
-                                msum[rr][v] = 0.f;
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int v = 0; v < VEC; ++v) axpy<R>(qacc[v], x[v], ph);
-                    }
-                }
-            }
-        }
-        __syncthreads();
-    }
-    cp_async_wait<0>();
-
-    // this warp's partial, laid out [warp][k][v][lane] (conflict-free)
-#pragma unroll
-    for (int k = 0; k < R; ++k)
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) red_s[((warp * R + k) * VEC + v) * 32 + lane] = qacc[v][k];
-    __syncthreads();
-    // sum over warps in order; write the row block's partial Q rows
-    double* qpart = p.ws.qpart + d.qpart_off;
-    for (int idx = tid; idx < width * R; idx += kThreads) {
-        const int cc = idx / R;
-        const int k = idx % R;
-        const int ln = cc / VEC, v = cc % VEC;
-        double s = 0.0;
-#pragma unroll
-        for (int wp = 0; wp < kWarps; ++wp) s += static_cast<double>(red_s[((wp * R + k) * VEC + v) * 32 + ln]);
-        qpart[(static_cast<int64_t>(tc.rb) * n + jc + cc) * R + k] = s;
     }
 }
 
@@ -1386,57 +1263,38 @@ __device__ __forceinline__ void pass_b_mma(const Params& p, const LayerDesc& d, 
     }
 }
 
-// Staged tensor-core second pass (R = 16, 32; VEC 4).  The tile (tm <= 64
-// rows x a chunk of <= 128 columns) is processed one worker at a time: the
-// worker's block is copied into a shared-memory stage by cp.async while the
-// previous worker's block is multiplied, so several 32 KB blocks per SM are
-// in flight without holding registers.  Warp w owns the chunk columns
-// 16 w .. 16 w + 15 over all the tile's rows: D (R ranks x 16 columns) =
-// P_hat^T (ranks x rows) * M (rows x columns), two n-tiles of 8 columns,
-// n-tile j taking column 16 w + 2 g + j as its column g, so that lane
-// (g, t) reads one 8-byte pair per row.  A = P_hat^T of all the tile's
-// rows, split into tf32 hi and lo once per tile.  D accumulates one worker
-// (tm rows, three split products per term) in float32 and is then added to
-// a float64 sum: float32 runs of at most 64 rows, as in the other
-// tensor-core kernels.  No cross-warp reduction: every warp writes its own
-// columns' row-block partial.
+// Staged second pass for R = 16, 32 with 16-byte rows (n % 4 == 0), on the
+// CUDA cores.  The tile (tm <= 64 rows x a chunk of <= 128 columns) is
+// processed one worker at a time: the worker's block is copied into a
+// shared-memory stage by cp.async while the previous worker's block is
+// multiplied, so that 32 KB blocks are in flight without holding registers.
+// Warp w takes the chunk columns 64 (w & 1) .. 64 (w & 1) + 63 and the tile
+// rows (w >> 1) + 4 i.  Lane l takes 4 columns, 4 (l % 16) .. + 3 of that
+// half, and half of the ranks, R / 2 (l / 16) .. + R / 2 - 1: per row, one
+// 16-byte load of M and R / 8 broadcast 16-byte loads of the P_hat row feed
+// 2 R fused multiply-adds (packed, two ranks per instruction, accumulators
+// kept as pairs), summed in float32 over the warp's rows and the workers.
+// (Measured on the B200, the tf32 mma.sync path needs three split products
+// per term and its tensor pipe saturated at the CUDA cores' multiply-add
+// rate.)  At the end the four row-quarter warps of each column half are
+// added in float64, in order.
 template <int R, bool SF>
 __device__ __forceinline__ void pass_b_staged(const Params& p, const LayerDesc& d, const TileCoord& tc,
                                               float* const* ep, const float* ph_s, float* red_s) {
     static_assert(R == 16 || R == 32, "staged pass B: rank 16 or 32");
-    constexpr int MT = R / 16;                  // m-tiles of 16 ranks
+    constexpr int RH = R / 2;                   // ranks per lane
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g = lane >> 2, t4 = lane & 3;
     const int W = p.workers;
     const int64_t n = d.n;
     const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
     const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), d.m - i0));
     const int64_t jc = static_cast<int64_t>(tc.c) * d.slots * 4;
     const int width = static_cast<int>(min(static_cast<int64_t>(d.slots) * 4, n - jc));
-    const int nks = d.tm / 8;                   // k-steps of 8 rows (tm = 16, 32 or 64)
     float* stg = red_s;                         // [stage][row][kStgStride]
-    float4* pa = reinterpret_cast<float4*>(reinterpret_cast<unsigned char*>(red_s) + kStgBytes);  // [ks][mt][lane][hi, lo]
-
-    // A fragments: A[rank][row] = P_hat[row][rank] (zero outside the
-    // layer); slot t <- row 8 ks + t, slot t + 4 <- row 8 ks + t + 4
-    for (int idx = tid; idx < nks * MT * 32; idx += kThreads) {
-        const int ln = idx & 31, mt = (idx >> 5) % MT, ks = (idx >> 5) / MT;
-        const int gg = ln >> 2, tt = ln & 3;
-        float av[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int row = 8 * ks + tt + 4 * (q >> 1);
-            const int rank = 16 * mt + gg + 8 * (q & 1);
-            av[q] = row < rows ? ph_s[row * R + rank] : 0.f;
-        }
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tf32_split(av[q], hi[q], lo[q]);
-        pa[2 * idx] = make_float4(__uint_as_float(hi[0]), __uint_as_float(hi[1]), __uint_as_float(hi[2]),
-                                  __uint_as_float(hi[3]));
-        pa[2 * idx + 1] = make_float4(__uint_as_float(lo[0]), __uint_as_float(lo[1]), __uint_as_float(lo[2]),
-                                      __uint_as_float(lo[3]));
-    }
+    const int half = warp & 1, rq = warp >> 1;
+    const int lc = 64 * half + 4 * (lane & 15); // the lane's first column in the chunk
+    const int k0 = RH * (lane >> 4);            // the lane's first rank
+    const bool active = lc < width;
 
     // one worker's block into stage s: (tm rows) x (32 x 16 bytes)
     auto issue = [&](int w, int stage) {
@@ -1449,71 +1307,30 @@ __device__ __forceinline__ void pass_b_staged(const Params& p, const LayerDesc& 
         }
     };
 
-    const int col0 = 16 * warp + 2 * g;          // this lane's column pair (n-tiles 0 and 1)
-    const bool active = 16 * warp < width;
-    float dacc[MT][2][4];
-    double dsum[MT][2][4];
+    float2 acc[4][RH / 2];                      // [column][rank pair]
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
+    for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) dsum[mt][j][q] = 0.0;
-    float msum[SF ? 8 : 1][SF ? 4 : 1];
+        for (int k = 0; k < RH / 2; ++k) acc[c][k] = make_float2(0.f, 0.f);
+    float4 msum[SF ? kStgRows / 4 : 1];
     if constexpr (SF) {
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) msum[ks][q] = 0.f;
+        for (int i = 0; i < kStgRows / 4; ++i) msum[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-
-    // products of one block (x[ks] = rows 8 ks + t, 8 ks + t + 4 at the
-    // lane's two columns) into dsum
-    auto multiply = [&](const float* blk) {
+    auto rank_update = [&](const float4 x, int row) {
+        const float4* ph4 = reinterpret_cast<const float4*>(ph_s + row * R + k0);
+        const float2 xs[4] = {make_float2(x.x, x.x), make_float2(x.y, x.y), make_float2(x.z, x.z),
+                              make_float2(x.w, x.w)};
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
+        for (int k4 = 0; k4 < RH / 4; ++k4) {
+            const float4 pv = ph4[k4];
+            const float2 p01 = make_float2(pv.x, pv.y), p23 = make_float2(pv.z, pv.w);
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) dacc[mt][j][q] = 0.f;
-#pragma unroll(SF ? 8 : 1)
-        for (int ks = 0; ks < (SF ? 8 : nks); ++ks) {
-            if (SF && ks >= nks) break;
-            float x[4];
-            if constexpr (SF) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) x[q] = msum[ks][q];
-            } else {
-                const float2 a = *reinterpret_cast<const float2*>(blk + (8 * ks + t4) * kStgStride + col0);
-                const float2 b = *reinterpret_cast<const float2*>(blk + (8 * ks + t4 + 4) * kStgStride + col0);
-                x[0] = a.x; x[1] = b.x; x[2] = a.y; x[3] = b.y;
-            }
-            // B fragments of the two n-tiles: b0 = row t, b1 = row t + 4
-            uint32_t bh[4], bl[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) tf32_split(x[q], bh[q], bl[q]);
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                const float4 h4 = pa[2 * ((ks * MT + mt) * 32 + lane)];
-                const float4 l4 = pa[2 * ((ks * MT + mt) * 32 + lane) + 1];
-                const uint32_t ahi[4] = {__float_as_uint(h4.x), __float_as_uint(h4.y), __float_as_uint(h4.z),
-                                         __float_as_uint(h4.w)};
-                const uint32_t alo[4] = {__float_as_uint(l4.x), __float_as_uint(l4.y), __float_as_uint(l4.z),
-                                         __float_as_uint(l4.w)};
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    mma_tf32(dacc[mt][j], alo, bh[2 * j], bh[2 * j + 1]);
-                    mma_tf32(dacc[mt][j], ahi, bl[2 * j], bl[2 * j + 1]);
-                    mma_tf32(dacc[mt][j], ahi, bh[2 * j], bh[2 * j + 1]);
-                }
+            for (int c = 0; c < 4; ++c) {
+                acc[c][2 * k4] = __ffma2_rn(xs[c], p01, acc[c][2 * k4]);
+                acc[c][2 * k4 + 1] = __ffma2_rn(xs[c], p23, acc[c][2 * k4 + 1]);
             }
         }
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) dsum[mt][j][q] += static_cast<double>(dacc[mt][j][q]);
     };
 
     // pipeline over the workers: kStages - 1 blocks ahead
@@ -1522,7 +1339,6 @@ __device__ __forceinline__ void pass_b_staged(const Params& p, const LayerDesc& 
         if (s0 < W) issue(s0, s0);
         cp_async_commit();
     }
-    __syncthreads();   // the A fragments are in shared memory
     for (int w = 0; w < W; ++w) {
         const int ahead = w + kStages - 1;
         if (ahead < W) issue(ahead, ahead % kStages);
@@ -1531,40 +1347,48 @@ __device__ __forceinline__ void pass_b_staged(const Params& p, const LayerDesc& 
         __syncthreads();
         const float* blk = stg + static_cast<size_t>(w % kStages) * kStgRows * kStgStride;
         if (active) {
-            if constexpr (SF) {
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    if (ks >= nks) break;
-                    const float2 a = *reinterpret_cast<const float2*>(blk + (8 * ks + t4) * kStgStride + col0);
-                    const float2 b = *reinterpret_cast<const float2*>(blk + (8 * ks + t4 + 4) * kStgStride + col0);
-                    msum[ks][0] += a.x;
-                    msum[ks][1] += b.x;
-                    msum[ks][2] += a.y;
-                    msum[ks][3] += b.y;
+#pragma unroll 2
+            for (int i = 0; i < kStgRows / 4; ++i) {
+                const int row = rq + 4 * i;
+                if (row < rows) {
+                    const float4 x = *reinterpret_cast<const float4*>(blk + row * kStgStride + lc);
+                    if constexpr (SF) {
+                        msum[i].x += x.x;
+                        msum[i].y += x.y;
+                        msum[i].z += x.z;
+                        msum[i].w += x.w;
+                        if (w == W - 1) rank_update(msum[i], row);
+                    } else {
+                        rank_update(x, row);
+                    }
                 }
-                if (w == W - 1) multiply(blk);
-            } else {
-                multiply(blk);
             }
         }
         __syncthreads();   // stage w % kStages may be refilled next
     }
     cp_async_wait<0>();
 
-    // this warp's columns of the row block's partial Q rows
-    if (active) {
-        double* qpart = p.ws.qpart + d.qpart_off;
+    // the four row quarters of each column half, in float64 and in order;
+    // the stages are free now: red[warp][col (64)][R + 1] floats
+    constexpr int RS = R + 1;
+    float* red = stg;
+    const int cl = 4 * (lane & 15);
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
+    for (int c = 0; c < 4; ++c)
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
+        for (int k = 0; k < RH / 2; ++k) {
+            red[(warp * 64 + cl + c) * RS + k0 + 2 * k] = acc[c][k].x;
+            red[(warp * 64 + cl + c) * RS + k0 + 2 * k + 1] = acc[c][k].y;
+        }
+    __syncthreads();
+    double* qpart = p.ws.qpart + d.qpart_off;
+    for (int idx = tid; idx < width * R; idx += kThreads) {
+        const int col = idx / R, k = idx - (idx / R) * R;
+        const int h = col >> 6, c = col & 63;
+        double s2 = 0.0;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int rank = 16 * mt + g + 8 * (q >> 1);
-                    const int col = 16 * warp + 2 * (2 * t4 + (q & 1)) + j;
-                    if (col < width)
-                        qpart[(static_cast<int64_t>(tc.rb) * n + jc + col) * R + rank] = dsum[mt][j][q];
-                }
+        for (int q = 0; q < 4; ++q) s2 += static_cast<double>(red[((2 * q + h) * 64 + c) * RS + k]);
+        qpart[(static_cast<int64_t>(tc.rb) * n + jc + col) * R + k] = s2;
     }
 }
 
@@ -1652,7 +1476,7 @@ __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_b(Params p)
     float* ph_s = reinterpret_cast<float*>(smem + ((SmemB<R>::ptr_bytes(W) + 15) & ~size_t(15)));
     double* T_s = reinterpret_cast<double*>(reinterpret_cast<unsigned char*>(ph_s) +
                                             ((SmemB<R>::rows_bytes(d.tm) + 15) & ~size_t(15)));
-    float* red_s = reinterpret_cast<float*>(T_s + R * R);
+    float* red_s = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(T_s) + SmemB<R>::t_bytes());
 
     for (int w = threadIdx.x; w < W; w += kThreads) ep[w] = p.t.errors[w * L + l];
     load_phat_rows<R>(p, d, tc, ph_s, T_s, tc.c == 0);
@@ -1667,7 +1491,7 @@ __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_b(Params p)
         }
     } else {
         if (d.vec == 4) {
-            if constexpr (R <= 4) pass_b_rows_staged<R, SF>(p, d, tc, ep, ph_s, red_s);
+            if constexpr (R <= 4) pass_b_rows<R, 4, SF>(p, d, tc, ep, ph_s, red_s);
         } else if (d.vec == 2) {
             if constexpr (R <= 16) pass_b_rows<R, 2, SF>(p, d, tc, ep, ph_s, red_s);
         } else {
