@@ -239,7 +239,7 @@ def test_json_line_workloads_and_reports(fake_gpu, monkeypatch, capsys):
     main_wl = fake_gpu
     lstm = Workload(name="tiny_lstm", layers=((40, 26),) * 2, rank=4, workers=4, steps=3)
     sweep = Workload(name="tiny_sweep", layers=((32, 32),) * 3, rank=1, workers=2, steps=4, rotate=0.05,
-                     ranks=(1, 2, 8))
+                     ranks=(1, 2, 16))
     table = {"m": main_wl, "l": lstm, "s": sweep}
     monkeypatch.setattr(bench, "get_workload", lambda key: table[key])
     d = _run(monkeypatch, capsys, "--config", "m", "--steps", "3", "--warmup", "3", "--no-cpu-baseline",
@@ -253,12 +253,14 @@ def test_json_line_workloads_and_reports(fake_gpu, monkeypatch, capsys):
         assert key in lw, key
     assert lw["rank"] == 4 and lw["compression"]["ratio"] == round(2 * 40 * 26 / (4 * 2 * 66), 2)
     sw = wls["tiny_sweep"]
-    assert set(sw["by_rank"]) == {"1", "2", "8"}
+    assert set(sw["by_rank"]) == {"1", "2", "16"}
     for r, line in sw["by_rank"].items():
         assert line["rank"] == int(r) and line["value"] > 0 and "compression" in line
+        # ranks 16 and 32 also time the sum-first mode
+        assert ("sum_first" in line) == (int(r) >= 16)
     se = sw["subspace_error"]["by_rank"]
-    assert set(se) == {"1", "2", "8"} and se["1"]["steps"] == 4
-    assert se["2"]["status"].startswith("checked against the oracle") and se["8"]["status"].startswith("reported")
+    assert set(se) == {"1", "2", "16"} and se["1"]["steps"] == 4
+    assert se["2"]["status"].startswith("checked against the oracle") and se["16"]["status"].startswith("reported")
     for v in se.values():
         assert 0.0 <= v["sin_theta_max"] <= 1.0 + 1e-12
     assert d["compression"]["ratio"] == round((64 * 48 + 24 * 32) / (2 * (64 + 48 + 24 + 32)), 2)
