@@ -534,20 +534,6 @@ def workload_line(wl, r: int, steps: int, warmup: int, stream, B=None, lazy_vari
            "steps": steps}
     if "compute" in rl:
         out["compute"] = {k: rl["compute"][k] for k in ("achieved", "unit", "fp32_frac", "tf32_frac")}
-    if r >= 16:
-        # the sum-first mode (workers' M summed before the products, one
-        # product per matrix element instead of one per worker element)
-        B.set_rank(r)
-        lib = PowerSGD(wl.layers, r, wl.workers, grad_dtype=wl.grad_dtype, sum_first=True)
-        try:
-            sms, skern, sks = timed_steps(lambda: run_step(lib, B, wl), steps, warmup, lib, stream)
-        finally:
-            lib.close()
-        srl = roofline_block(wl, r, "eager+sumfirst", skern, sks, sms, None, sum_first=True)
-        out["sum_first"] = {"ms_per_step": round(sms, 4), "value": job_value(wl.elements, 1, sms),
-                            "step_dram_frac": srl.get("step_dram_frac"),
-                            "step_algorithmic_frac": srl["step_algorithmic_frac"],
-                            "per_kernel_ms": srl["per_kernel_ms"]}
     if lazy_variant:
         B.set_rank(r)
         lib = PowerSGD(wl.layers, r, wl.workers, grad_dtype=wl.grad_dtype, lazy_errors=True)

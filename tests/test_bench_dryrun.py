@@ -256,8 +256,6 @@ def test_json_line_workloads_and_reports(fake_gpu, monkeypatch, capsys):
     assert set(sw["by_rank"]) == {"1", "2", "16"}
     for r, line in sw["by_rank"].items():
         assert line["rank"] == int(r) and line["value"] > 0 and "compression" in line
-        # ranks 16 and 32 also time the sum-first mode
-        assert ("sum_first" in line) == (int(r) >= 16)
     se = sw["subspace_error"]["by_rank"]
     assert set(se) == {"1", "2", "16"} and se["1"]["steps"] == 4
     assert se["2"]["status"].startswith("checked against the oracle") and se["16"]["status"].startswith("reported")
