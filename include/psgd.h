@@ -198,8 +198,10 @@ PSGD_API int psgd_status(psgd_ctx *ctx);
 PSGD_API int psgd_workspace_bytes(const psgd_ctx *ctx, size_t *bytes);
 
 /* Number of kernel launches one regular psgd_step makes for this context
- * (for launch accounting; an SVD-refresh step adds the launches stated at
- * psgd_set_svd_refresh). */
+ * (for launch accounting): per power iteration the first pass, the P_hat
+ * kernel and the second pass, + 1 for the third pass in eager mode, + 1
+ * with PSGD_FLAG_NO_WARM_START.  An SVD-refresh step makes the launches
+ * stated at psgd_set_svd_refresh. */
 PSGD_API int psgd_step_launches(const psgd_ctx *ctx);
 
 /* Allocation-free step for one layer.  No counterpart in the pages: this
@@ -307,12 +309,12 @@ PSGD_API int psgd_set_power_iters(psgd_ctx *ctx, int iters);
  * orthogonalisation's Cholesky diagonal, (lambda_{r'} / lambda_r)^(J - 1),
  * is at most 1e-10, and after `iters` iterations at most (1 <= iters <= 64).
  * every = 0 turns refresh off (the default).  A refresh step makes
- * 2 * iters + 2 launches, + 1 for the residual pass (eager mode, or when
+ * 3 * iters + 2 launches, + 1 for the residual pass (eager mode, or when
  * G_hat is wanted), + 1 in lazy mode to write out the previous E' first; a
  * converged layer's later iterations return at once.  With oversampling 0
  * (or when no column can be added) the block is the rank-r factors
  * themselves: `iters` iterations from the warm start, the rotation in
- * place, 2 * (iters - power_iters) + 1 more launches than a regular step. */
+ * place, 3 * (iters - power_iters) + 1 more launches than a regular step. */
 PSGD_API int psgd_set_svd_refresh(psgd_ctx *ctx, int every, int iters);
 
 /* Oversampling p of the refresh block above, 0 <= p <= 31 (default 8).  The
@@ -323,7 +325,7 @@ PSGD_API int psgd_set_svd_oversampling(psgd_ctx *ctx, int extra);
  * later psgd_step records CUDA events (on its stream) around each of its
  * kernel launches.  psgd_profile_read synchronises on those events, writes
  * the summed device milliseconds of the first pass (error feedback + P),
- * the second pass (Q, plus every later power iteration) and the third pass
+ * the second pass (P_hat and Q, plus every later power iteration) and the third pass
  * (residual / decompression, 0 in lazy mode) to ms[0..2] and the number of recorded steps to *steps, and
  * clears the record.  Recording adds six event records per step.  The
  * distributed calls are recorded too (pass A in psgd_dist_p; the

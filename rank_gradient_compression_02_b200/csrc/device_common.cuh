@@ -11,6 +11,7 @@ constexpr int kThreads = 256;          // threads per CTA in every streaming ker
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxWorkers = 256;
 constexpr int kMaxRank = 32;
+constexpr int kRowsFloatsMax = 4096;   // tile rows x R bound (the second pass's P_hat rows)
 
 // Per-layer geometry and workspace offsets (element counts), built on the
 // host at context creation.  A "tile" is TM rows x one column chunk of a
@@ -116,7 +117,10 @@ struct Params {
     double conv_eps;
 };
 
-enum : int { kStatusCounter = 1 };
+enum : int {
+    kStatusCounter = 1,   // a reduction counter held an impossible value
+    kStatusTimeout = 2    // a bounded wait on the tensor cores ran out (about one second)
+};
 
 // ---- loads and stores ------------------------------------------------------
 

@@ -141,6 +141,22 @@ __device__ __forceinline__ uint32_t tf32_round(float x) {
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
     return r;
 }
+// sum_{j < count} src[j * stride] in index order, eight loads in flight at a
+// time (the partials were written by other CTAs of this launch: L2 loads)
+__device__ __forceinline__ double sum_in_order(const double* src, int64_t stride, int count) {
+    double s = 0.0;
+    int j = 0;
+    for (; j + 8 <= count; j += 8) {
+        double v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (j + u) * stride);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) s += v[u];
+    }
+    for (; j < count; ++j) s += __ldcg(src + j * stride);
+    return s;
+}
+
 __device__ __forceinline__ void tf32_split(float x, uint32_t& hi, uint32_t& lo) {
     hi = tf32_round(x);
     lo = tf32_round(x - __uint_as_float(hi));
@@ -181,6 +197,68 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
+// ---- 5th-generation tensor cores (tcgen05) --------------------------------
+// Shared-memory matrix descriptor, no swizzle, K-major operand: core
+// matrices of 8 rows (of M or N) x 16 bytes (4 tf32 of K) stored as 128
+// contiguous bytes; LBO is the byte distance between core matrices adjacent
+// in K, SBO between core matrices adjacent in M or N.  Field layout of the
+// sm_100 matrix descriptor: start address >> 4 in bits [0, 14), LBO >> 4 in
+// [16, 30), SBO >> 4 in [32, 46), descriptor version 1 in [46, 48), base
+// offset 0, layout type 0 (no swizzle) in [61, 64).
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3fffu) | (static_cast<uint64_t>((lbo >> 4) & 0x3fffu) << 16) |
+           (static_cast<uint64_t>((sbo >> 4) & 0x3fffu) << 32) | (1ull << 46);
+}
+// Instruction descriptor of kind::tf32 with both operands K-major: D
+// float32 (bits [4, 6) = 1), A and B tf32 (bits [7, 10), [10, 13) = 2),
+// N >> 3 in bits [17, 23), M >> 4 in bits [24, 29).  (Operands marked
+// MN-major in bits 15 and 16 were measured to contribute nothing to D for
+// tf32 on this part; the kernels transpose into K-major instead.)
+__host__ __device__ constexpr uint32_t umma_idesc_tf32(int M, int N) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+__device__ __forceinline__ void umma_tf32(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait for the phase `parity` of an mbarrier to complete: about one
+// second at most, after which the status word gets kStatusTimeout and false
+// is returned (the caller then winds down without using the results).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int* status) {
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+            "selp.b32 %0, 1, 0, P1;\n\t}\n"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (global_timer_ns() - t0 > 1000000000ull) {
+            atomicOr(status, kStatusTimeout);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // Staged second pass (ranks 16, 32; rows 16-byte aligned, i.e. n % 4 == 0):
 // one worker's 64 x 128 block of M at a time goes to shared memory by
 // cp.async (kStages buffers), row stride kStgStride floats (the padding
@@ -190,6 +268,29 @@ constexpr int kStgCols = 128;
 constexpr int kStgStride = kStgCols + 8;
 constexpr int kStages = 2;
 constexpr size_t kStgBytes = static_cast<size_t>(kStages) * kStgRows * kStgStride * sizeof(float);
+// Tensor-core second pass: the worker's block split into tf32 hi and lo,
+// both transposed to K-major, B = [P_hat hi | P_hat lo] K-major, then the
+// mbarrier, the TMEM address and the wind-down flag.  In A, each group of 8
+// columns holds 16 core matrices (64 rows of K) and is padded by 16 bytes
+// (kTcSboA), so the 16-byte stores of 8 consecutive column quads land in 8
+// distinct bank groups.
+constexpr uint32_t kTcSboA = 16 * 128 + 16;
+constexpr uint32_t kTcSboB = 16 * 128;
+// workers whose products accumulate in tensor memory (float32, at most 64
+// MMA accumulations per element and half) before D is read back into the
+// float64 sums
+constexpr int kTcGroup = 4;
+// independent accumulators (k-step ks goes to ks % kTcChains), so that
+// successive MMAs do not wait on one another's result
+constexpr int kTcChains = 4;
+constexpr size_t kTcABytes = static_cast<size_t>(kStgCols / 8) * kTcSboA;   // one A buffer (33 KB)
+template <int R>
+struct TcSmem {
+    static constexpr size_t b_bytes = static_cast<size_t>(2 * R / 8) * kTcSboB;   // 2R rows of N x 64 of K
+    static constexpr size_t total = 2 * kTcABytes + b_bytes + 16;
+    // per chain D = [hi*hi + lo*hi | hi*lo]; a power of two >= 32
+    static constexpr uint32_t tmem_cols = 2 * R * kTcChains;
+};
 
 constexpr int kMmaRows = 16;                  // rows per warp in the tensor-core pass A
 constexpr int kMaxKSteps = 32 * 4 / 8;        // k-steps of 8 columns in the widest chunk
@@ -720,8 +821,7 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
     for (int idx = tid; idx < rows * R; idx += kThreads) {
         const int64_t i = i0 + idx / R;
         const int k = idx % R;
-        double s = 0.0;
-        for (int c = 0; c < d.nchunk; ++c) s += __ldcg(&ppart[(static_cast<int64_t>(c) * m + i) * R + k]);
+        double s = sum_in_order(ppart + i * R + k, m * R, d.nchunk);
         if (p.dist) {
             // this rank's share of the all-reduce: the row's sum over its workers
             p.dist_out[d.prow_off + i * R + k] = s;
@@ -764,8 +864,7 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
     __threadfence();
     double* gsup = p.ws.gsup + d.gsup_off;
     for (int pidx = tid; pidx < NG; pidx += kThreads) {
-        double s = 0.0;
-        for (int k = 0; k < nin; ++k) s += __ldcg(&gram[static_cast<int64_t>(rb0 + k) * NG + pidx]);
+        double s = sum_in_order(gram + static_cast<int64_t>(rb0) * NG + pidx, NG, nin);
         gsup[static_cast<int64_t>(sup) * NG + pidx] = s;
     }
     if (tid == 0) cnt[cl.a_sup + sup] = 0u;
@@ -793,8 +892,7 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
             ++a;
         }
         const int b = a + rem;
-        double s = 0.0;
-        for (int k = 0; k < d.nsup; ++k) s += __ldcg(&gsup[static_cast<int64_t>(k) * NG + pidx]);
+        double s = sum_in_order(gsup + pidx, NG, d.nsup);
         Gs[a * R + b] = s;
         Gs[b * R + a] = s;
     }
@@ -884,14 +982,13 @@ template <int R>
 struct SmemB {
     static __host__ __device__ size_t ptr_bytes(int W) { return static_cast<size_t>(W) * sizeof(void*); }
     static __host__ __device__ size_t rows_bytes(int tm) { return static_cast<size_t>(tm) * R * sizeof(float); }
-    // rounded up to 16 bytes: the region after it takes 16-byte accesses
-    static __host__ __device__ size_t t_bytes() { return (R * R * sizeof(double) + 15) & ~size_t(15); }
     static __host__ __device__ size_t red_bytes(int vec) {
         if (UseMma<R>::value && vec == 4) {
             // staged kernel: the M stages, reused at the end for the warps'
             // partials (8 warps x 64 columns x (R + 1) floats)
             const size_t red = static_cast<size_t>(kWarps) * 64 * (R + 1) * sizeof(float);
-            return kStgBytes > red ? kStgBytes : red;
+            const size_t staged = kStgBytes > red ? kStgBytes : red;
+            return staged > TcSmem<R>::total ? staged : TcSmem<R>::total;
         }
         if (UseMma<R>::value) {
             // tensor-core kernel: warp partials (8 x 32 columns x 33) + the
@@ -901,36 +998,31 @@ struct SmemB {
         return static_cast<size_t>(kWarps) * R * vec * 32 * sizeof(float);
     }
     static __host__ __device__ size_t total(int W, int tm, int vec) {
-        return ((ptr_bytes(W) + 15) & ~size_t(15)) + ((rows_bytes(tm) + 15) & ~size_t(15)) + t_bytes() +
-               red_bytes(vec);
+        return ((ptr_bytes(W) + 15) & ~size_t(15)) + ((rows_bytes(tm) + 15) & ~size_t(15)) + red_bytes(vec);
     }
 };
 
-// P_hat rows [i0, i0+rows) of a layer into shared memory: P_bar T, float64
-// accumulation in column order.  Chunk 0 also writes them out.
+// The tile's P_hat rows [i0, i0+rows) from the workspace (formed once per
+// layer by k_phat) into shared memory; a thread's loads are all in flight
+// together.
 template <int R>
 __device__ __forceinline__ void load_phat_rows(const Params& p, const LayerDesc& d, const TileCoord& tc,
-                                               float* ph_s, double* T_s, bool write_out) {
+                                               float* ph_s) {
+    constexpr int kE = kRowsFloatsMax / kThreads;   // elements per thread at most
     const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
     const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), d.m - i0));
-    const double* T = p.ws.T + d.t_off;
-    for (int idx = threadIdx.x; idx < R * R; idx += kThreads) T_s[idx] = T[idx];
-    __syncthreads();
-    const double* pbar = p.ws.pbar + d.prow_off + i0 * R;
-    float* phat_ws = p.ws.phat + d.prow_off + i0 * R;
-    float* out = (p.t.p_hat_out != nullptr) ? p.t.p_hat_out[tc.l] : nullptr;
-    const int r = p.r;
-    for (int idx = threadIdx.x; idx < rows * R; idx += kThreads) {
-        const int ii = idx / R;
-        const int k = idx % R;
-        double s = 0.0;
-        for (int a = 0; a <= k; ++a) s += pbar[ii * R + a] * T_s[a * R + k];
-        const float v = static_cast<float>(s);
-        ph_s[idx] = v;
-        if (write_out) {
-            phat_ws[idx] = v;
-            if (out != nullptr && k < r) out[(i0 + ii) * r + k] = v;
-        }
+    const int total = rows * R;
+    const float* src = p.ws.phat + d.prow_off + i0 * R;
+    float v[kE];
+#pragma unroll
+    for (int e = 0; e < kE; ++e) {
+        const int idx = threadIdx.x + e * kThreads;
+        v[e] = idx < total ? __ldg(src + idx) : 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < kE; ++e) {
+        const int idx = threadIdx.x + e * kThreads;
+        if (idx < total) ph_s[idx] = v[e];
     }
     __syncthreads();
 }
@@ -1392,6 +1484,243 @@ __device__ __forceinline__ void pass_b_staged(const Params& p, const LayerDesc& 
     }
 }
 
+// Second pass on the 5th-generation tensor cores (R = 16, 32; 16-byte rows).
+// For every worker, D (128 chunk columns x ranks, float32, in tensor memory)
+// = M^T P_hat over the tile's rows.  tf32 operands are read K-major (K = the
+// tile's rows), so the worker's block of M, held row-major in global memory,
+// is transposed on its way into shared memory: each thread loads 4 x 4
+// blocks (four rows of one column quad) one worker ahead into registers,
+// splits them into hi (the top 19 bits) and lo = x - hi, and stores every
+// column's four rows as one 16-byte K row of a core matrix.  B = [P_hat hi |
+// P_hat lo] (round-to-nearest split), K-major, once per tile.  Per k-step of
+// 8 rows two MMAs give fp32 accuracy from tf32 products (split-precision
+// products, Markidis et al. 2018): A_hi [B_hi | B_lo] (N = 2R) and A_lo B_hi
+// (N = R, accumulated into the first half), so D = [hi*hi + lo*hi | hi*lo],
+// in kTcChains independent accumulators (k-step ks into ks % kTcChains).
+// One thread issues them and commits to an mbarrier, and one thread waits
+// on it before the next worker's block is stored.  D accumulates over
+// groups of kTcGroup workers; after each group all eight warps read it back
+// (tcgen05.ld: four lane quarters x two rank halves; chains and halves
+// summed in float32) into float64 sums, so float32 runs stay within
+// kTcGroup workers' rows of one tile.  Every wait is bounded
+// (about a second), after which the status word is set and the tile winds
+// down; the tensor memory is released on every path.
+
+__device__ __forceinline__ uint32_t tc_kmajor(int mn, int k, uint32_t sbo) {   // bytes; K extent 64
+    return static_cast<uint32_t>((mn >> 3) * sbo + (k >> 2) * 128 + (mn & 7) * 16 + (k & 3) * 4);
+}
+
+// 32 TMEM lanes x N consecutive columns (N = 8 or 16) into this warp; the
+// values are valid after tmem_wait_ld()
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&u)[N]) {
+    if constexpr (N == 16) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+            "%14, %15}, [%16];"
+            : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+              "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
+            : "r"(taddr));
+    } else {
+        static_assert(N == 8, "tmem_ld: 8 or 16 columns");
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                     : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+                       "=r"(u[7])
+                     : "r"(taddr));
+    }
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+template <int R>
+__device__ __forceinline__ void pass_b_tc(const Params& p, const LayerDesc& d, const TileCoord& tc,
+                                          float* const* ep, const float* ph_s, unsigned char* buf) {
+    static_assert(R == 16 || R == 32, "tensor-core pass B: rank 16 or 32");
+    constexpr int RH = R / 2;                             // ranks per reading warp
+    constexpr int kQ = (kStgRows / 4) / kWarps;           // row quads per thread and block (2)
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int W = p.workers;
+    const int64_t n = d.n;
+    const int64_t i0 = static_cast<int64_t>(tc.rb) * d.tm;
+    const int rows = static_cast<int>(min(static_cast<int64_t>(d.tm), d.m - i0));
+    const int64_t jc = static_cast<int64_t>(tc.c) * d.slots * 4;
+    const int width = static_cast<int>(min(static_cast<int64_t>(d.slots) * 4, n - jc));
+    const int nks = d.tm / 8;
+    unsigned char* a_hi = buf;
+    unsigned char* a_lo = buf + kTcABytes;
+    unsigned char* b_s = a_lo + kTcABytes;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(b_s + TcSmem<R>::b_bytes);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
+    int* flag = reinterpret_cast<int*>(tslot + 1);
+    const uint32_t bar_a = static_cast<uint32_t>(__cvta_generic_to_shared(bar));
+    constexpr uint32_t kIdescHL = umma_idesc_tf32(128, 2 * R);
+    constexpr uint32_t kIdescL = umma_idesc_tf32(128, R);
+
+    // this thread: column quad `lane` (a warp's loads take 512 contiguous
+    // bytes of one row) of row quads warp + 8 i; x[i][r] = row 4 (warp + 8 i) + r
+    const int c4 = 4 * lane;
+    const bool col_ok = c4 < width;
+    auto load = [&](int w, float4 (&v)[kQ][4]) {
+        const float* src = ep[w] + i0 * n + jc + c4;
+#pragma unroll
+        for (int i = 0; i < kQ; ++i)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int row = 4 * (warp + kWarps * i) + r;
+                v[i][r] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (col_ok && row < rows) v[i][r] = __ldcg(reinterpret_cast<const float4*>(src + row * n));
+            }
+    };
+    // column c4 + j, rows 4q..4q+3: one 16-byte K row of a core matrix at
+    // (col >> 3) kTcSboA + q 128 + (col & 7) 16
+    auto split_store = [&](const float4 (&v)[kQ][4]) {
+#pragma unroll
+        for (int i = 0; i < kQ; ++i) {
+            const int q = warp + kWarps * i;   // uniform over the warp
+            if (4 * q < d.tm) {
+                const uint32_t base = (lane >> 1) * kTcSboA + q * 128 + (lane & 1) * 64;
+                const float4 t[4] = {make_float4(v[i][0].x, v[i][1].x, v[i][2].x, v[i][3].x),
+                                     make_float4(v[i][0].y, v[i][1].y, v[i][2].y, v[i][3].y),
+                                     make_float4(v[i][0].z, v[i][1].z, v[i][2].z, v[i][3].z),
+                                     make_float4(v[i][0].w, v[i][1].w, v[i][2].w, v[i][3].w)};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float4 h;
+                    h.x = __uint_as_float(__float_as_uint(t[j].x) & 0xffffe000u);
+                    h.y = __uint_as_float(__float_as_uint(t[j].y) & 0xffffe000u);
+                    h.z = __uint_as_float(__float_as_uint(t[j].z) & 0xffffe000u);
+                    h.w = __uint_as_float(__float_as_uint(t[j].w) & 0xffffe000u);
+                    *reinterpret_cast<float4*>(a_hi + base + j * 16) = h;
+                    *reinterpret_cast<float4*>(a_lo + base + j * 16) =
+                        make_float4(t[j].x - h.x, t[j].y - h.y, t[j].z - h.z, t[j].w - h.w);
+                }
+            }
+        }
+    };
+
+    // set-up: barrier, tensor memory, B
+    if (tid == 0) {
+        mbar_init(bar_a, 1);
+        *flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         static_cast<uint32_t>(__cvta_generic_to_shared(tslot))),
+                     "r"(TcSmem<R>::tmem_cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    for (int idx = tid; idx < d.tm * R; idx += kThreads) {
+        const int row = idx / R, k = idx - (idx / R) * R;
+        uint32_t hi = 0, lo = 0;
+        if (row < rows) tf32_split(ph_s[row * R + k], hi, lo);
+        *reinterpret_cast<uint32_t*>(b_s + tc_kmajor(k, row, kTcSboB)) = hi;
+        *reinterpret_cast<uint32_t*>(b_s + tc_kmajor(R + k, row, kTcSboB)) = lo;
+    }
+    float4 x[kQ][4], xn[kQ][4];
+    if (W > 0) load(0, x);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+
+    double dsum[RH];
+#pragma unroll
+    for (int k = 0; k < RH; ++k) dsum[k] = 0.0;
+    const int kh = (warp >> 2) * RH;                                                // this warp's ranks
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);   // its TMEM lanes
+    // the chains' two halves summed in float32 (chains beyond the tile's
+    // k-steps hold nothing), then added to the float64 sums; 8 ranks at a time
+    auto read_back = [&]() {
+#pragma unroll
+        for (int k0 = 0; k0 < RH; k0 += 8) {
+            uint32_t u[8];
+            float f[8];
+            tmem_ld<8>(t_lane + static_cast<uint32_t>(kh + k0), u);   // chain 0, hi*hi + lo*hi
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(u[k]);
+#pragma unroll
+            for (int c = 0; c < kTcChains; ++c)
+#pragma unroll
+                for (int h = (c == 0 ? 1 : 0); h < 2; ++h) {
+                    if (c < nks) {   // uniform over the block
+                        tmem_ld<8>(t_lane + static_cast<uint32_t>(c * 2 * R + h * R + kh + k0), u);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) f[k] += __uint_as_float(u[k]);
+                    }
+                }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) dsum[k0 + k] += static_cast<double>(f[k]);
+        }
+    };
+    // one thread waits for worker w's products; the others at the barrier
+    auto wait_products = [&](int w) -> bool {
+        if (tid == 0 && !mbar_wait_bounded(bar_a, static_cast<uint32_t>(w & 1), p.ws.status)) *flag = 1;
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        return *flag == 0;
+    };
+
+    bool ok = true;
+    for (int w = 0; w < W; ++w) {
+        if (w + 1 < W) load(w + 1, xn);
+        if (w > 0) {
+            // worker w - 1's products are done: D and the A buffers are free
+            if (!wait_products(w - 1)) {
+                ok = false;
+                break;
+            }
+            if ((w - 1) % kTcGroup == kTcGroup - 1) read_back();
+        }
+        split_store(x);
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0) {
+            const uint32_t ah = static_cast<uint32_t>(__cvta_generic_to_shared(a_hi));
+            const uint32_t al = static_cast<uint32_t>(__cvta_generic_to_shared(a_lo));
+            const uint32_t bb = static_cast<uint32_t>(__cvta_generic_to_shared(b_s));
+            for (int ks = 0; ks < nks; ++ks) {
+                const uint32_t ko = static_cast<uint32_t>(ks) * 256;   // 8 rows = two K core matrices
+                const uint32_t dc = tmem + static_cast<uint32_t>((ks % kTcChains) * 2 * R);
+                const uint64_t db = umma_desc(bb + ko, 128, kTcSboB);
+                umma_tf32(dc, umma_desc(ah + ko, 128, kTcSboA), db, kIdescHL,
+                          (ks >= kTcChains || w % kTcGroup) ? 1u : 0u);
+                umma_tf32(dc, umma_desc(al + ko, 128, kTcSboA), db, kIdescL, 1u);
+            }
+            umma_commit(bar_a);
+        }
+#pragma unroll
+        for (int i = 0; i < kQ; ++i)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) x[i][r] = xn[i][r];
+    }
+    if (ok && W > 0) {
+        ok = wait_products(W - 1);
+        if (ok) read_back();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TcSmem<R>::tmem_cols)
+                     : "memory");
+    }
+    if (!ok) return;   // the status word says why; this tile's partial is not written
+    // this thread's chunk column (TMEM lane) and rank half of the row block's partial Q rows
+    const int col = (warp & 3) * 32 + lane;
+    if (col < width) {
+        double* qp = p.ws.qpart + d.qpart_off + (static_cast<int64_t>(tc.rb) * n + jc + col) * R + kh;
+#pragma unroll
+        for (int k = 0; k < RH; ++k) qp[k] = dsum[k];
+    }
+}
+
 template <int R>
 __device__ void pass_b_epilogue(const Params& p, const LayerDesc& d, const TileCoord& tc) {
     __shared__ int s_flag;
@@ -1424,8 +1753,7 @@ __device__ void pass_b_epilogue(const Params& p, const LayerDesc& d, const TileC
     for (int idx = tid; idx < cols * R; idx += kThreads) {
         const int64_t col = col0 + idx / R;
         const int k = idx % R;
-        double s = 0.0;
-        for (int j = 0; j < nin; ++j) s += __ldcg(&qpart[(static_cast<int64_t>(rb0 + j) * n + col) * R + k]);
+        const double s = sum_in_order(qpart + (static_cast<int64_t>(rb0) * n + col) * R + k, n * R, nin);
         qsup[(static_cast<int64_t>(sup) * n + col) * R + k] = s;
     }
     if (tid == 0) *c1 = 0u;
@@ -1448,8 +1776,7 @@ __device__ void pass_b_epilogue(const Params& p, const LayerDesc& d, const TileC
     for (int idx = tid; idx < cols * R; idx += kThreads) {
         const int64_t col = col0 + idx / R;
         const int k = idx % R;
-        double s = 0.0;
-        for (int j = 0; j < d.nsup; ++j) s += __ldcg(&qsup[(static_cast<int64_t>(j) * n + col) * R + k]);
+        const double s = sum_in_order(qsup + col * R + k, n * R, d.nsup);
         if (p.dist) {
             p.dist_out[d.qrow_off + col * R + k] = s;   // this rank's share of the all-reduce
             continue;
@@ -1474,16 +1801,16 @@ __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_b(Params p)
 
     float** ep = reinterpret_cast<float**>(smem);
     float* ph_s = reinterpret_cast<float*>(smem + ((SmemB<R>::ptr_bytes(W) + 15) & ~size_t(15)));
-    double* T_s = reinterpret_cast<double*>(reinterpret_cast<unsigned char*>(ph_s) +
+    float* red_s = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(ph_s) +
                                             ((SmemB<R>::rows_bytes(d.tm) + 15) & ~size_t(15)));
-    float* red_s = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(T_s) + SmemB<R>::t_bytes());
 
     for (int w = threadIdx.x; w < W; w += kThreads) ep[w] = p.t.errors[w * L + l];
-    load_phat_rows<R>(p, d, tc, ph_s, T_s, tc.c == 0);
+    load_phat_rows<R>(p, d, tc, ph_s);
 
     if constexpr (UseMma<R>::value) {
         if (d.vec == 4) {
-            pass_b_staged<R, SF>(p, d, tc, ep, ph_s, red_s);
+            if constexpr (SF) pass_b_staged<R, SF>(p, d, tc, ep, ph_s, red_s);
+            else pass_b_tc<R>(p, d, tc, ep, ph_s, reinterpret_cast<unsigned char*>(red_s));
         } else if (d.vec == 2) {
             pass_b_mma<R, 2, SF>(p, d, tc, ep, ph_s, red_s);
         } else {
@@ -1499,6 +1826,44 @@ __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_b(Params p)
         }
     }
     pass_b_epilogue<R>(p, d, tc);
+}
+
+// P_hat = P_bar T (T = R^-1 from the orthogonalisation) for every layer,
+// once per layer: float64 sums in column order over the upper-triangular T,
+// rounded to float32, into the workspace (read by the second and third
+// passes) and the caller's P_hat.  Grid (x, L): layer blockIdx.y, its m R
+// elements strided over blockIdx.x; a thread's loads of its row are all in
+// flight together.
+template <int R>
+__global__ void __launch_bounds__(kThreads) k_phat(Params p) {
+    __shared__ double T_s[R * R];
+    const int l = blockIdx.y;
+    if (p.track_conv && p.iter > p.ws.conv_iter[l]) return;   // converged refresh layer
+    const LayerDesc d = p.t.layers[l];
+    const double* T = p.ws.T + d.t_off;
+    for (int idx = threadIdx.x; idx < R * R; idx += kThreads) T_s[idx] = T[idx];
+    __syncthreads();
+    const int64_t total = d.m * R;
+    const double* pbar = p.ws.pbar + d.prow_off;
+    float* phat = p.ws.phat + d.prow_off;
+    float* out = (p.t.p_hat_out != nullptr) ? p.t.p_hat_out[l] : nullptr;
+    const int r = p.r;
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * kThreads) {
+        const int64_t row = idx / R;
+        const int k = static_cast<int>(idx - row * R);
+        const double* pr = pbar + row * R;
+        double pv[R];
+#pragma unroll
+        for (int a = 0; a < R; ++a) pv[a] = a <= k ? __ldg(pr + a) : 0.0;
+        double s = 0.0;
+#pragma unroll
+        for (int a = 0; a < R; ++a)
+            if (a <= k) s += pv[a] * T_s[a * R + k];
+        const float v = static_cast<float>(s);
+        phat[idx] = v;
+        if (out != nullptr && k < r) out[row * r + k] = v;
+    }
 }
 
 // ---------------------------------------------------------------------------

@@ -30,7 +30,7 @@ constexpr double kDropTol = 1e-12;
 // margin for the unknown angle of the starting block.
 constexpr double kRefreshEps = 1e-10;
 constexpr int64_t kTileTargetElems = 65536;  // worker elements per tile (all W workers)
-constexpr int kRowsFloatsMax = 4096;         // TM * R bound (shared-memory rows buffer)
+constexpr int kRowsFloatsMax = psgd::kRowsFloatsMax;   // TM * R bound (shared-memory rows buffer)
 
 int pad_rank(int r) {
     int R = 1;
@@ -269,6 +269,7 @@ struct Launch {
     static void* rayleigh_ritz() { return (void*)psgd::k_rayleigh_ritz<R>; }
     static void* dist_orth() { return (void*)psgd::k_dist_orth<R>; }
     static void* dist_qbar() { return (void*)psgd::k_dist_qbar<R>; }
+    static void* phat() { return (void*)psgd::k_phat<R>; }
 };
 
 void* kernel_ptr(int which, int R, int dtype, bool lazy, bool sf) {
@@ -280,6 +281,7 @@ void* kernel_ptr(int which, int R, int dtype, bool lazy, bool sf) {
         if (which == 4) return Launch<RR>::rayleigh_ritz();  \
         if (which == 5) return Launch<RR>::dist_orth();      \
         if (which == 6) return Launch<RR>::dist_qbar();      \
+        if (which == 7) return Launch<RR>::phat();           \
         return Launch<RR>::pass_c();
     switch (R) {
         PSGD_CASE(1)
@@ -327,11 +329,27 @@ psgd::Params base_params(psgd_ctx* ctx) {
     return p;
 }
 
+// Grid of k_phat: (x, L), x covering the largest layer's m R elements
+// (grid-stride beyond 4096 blocks).
+dim3 phat_grid(const std::vector<LayerDesc>& desc, int R) {
+    int64_t maxm = 1;
+    for (auto& d : desc) maxm = std::max(maxm, d.m);
+    const int64_t gx = std::min<int64_t>(4096, (maxm * R + psgd::kThreads - 1) / psgd::kThreads);
+    return dim3(static_cast<unsigned>(std::max<int64_t>(1, gx)), static_cast<unsigned>(desc.size()));
+}
+
+// The second pass (which == 1) is preceded by k_phat, which forms P_hat
+// from P_bar and T once per layer.
 int launch(psgd_ctx* ctx, int which, bool lazy, const psgd::Params& p, size_t smem, cudaStream_t stream) {
     if (ctx->ntiles == 0) return PSGD_OK;
     void* fn = kernel_ptr(which, ctx->R, ctx->dtype, lazy, (ctx->flags & PSGD_FLAG_SUM_FIRST) != 0);
     if (!fn) return fail(ctx, PSGD_ERR_ARG, "no kernel for rank %d", ctx->r);
     void* args[] = {const_cast<psgd::Params*>(&p)};
+    if (which == 1) {
+        cudaError_t e = cudaLaunchKernel(kernel_ptr(7, ctx->R, ctx->dtype, false, false), phat_grid(ctx->desc, ctx->R),
+                                         dim3(psgd::kThreads), args, 0, stream);
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "P_hat launch");
+    }
     cudaError_t e = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(ctx->ntiles)), dim3(psgd::kThreads), args, smem,
                                      stream);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "kernel launch");
@@ -541,7 +559,7 @@ int psgd_workspace_bytes(const psgd_ctx* ctx, size_t* bytes) {
 int psgd_step_launches(const psgd_ctx* ctx) {
     if (!ctx) return -1;
     if (ctx->ntiles == 0) return 0;
-    int n = 2 * ctx->iters + ((ctx->flags & PSGD_FLAG_LAZY_ERRORS) ? 0 : 1);
+    int n = 3 * ctx->iters + ((ctx->flags & PSGD_FLAG_LAZY_ERRORS) ? 0 : 1);
     if (ctx->flags & PSGD_FLAG_NO_WARM_START) n += 1;
     return n;
 }
@@ -1195,6 +1213,11 @@ int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int grad_dtype
             pw.do_recon = recon ? 1 : 0;
         }
         void* args[] = {&pw};
+        if (which == 1) {
+            e = cudaLaunchKernel(kernel_ptr(7, R, grad_dtype, false, false), phat_grid({d}, R),
+                                 dim3(psgd::kThreads), args, 0, s);
+            if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "P_hat launch: %s", cudaGetErrorString(e));
+        }
         e = cudaLaunchKernel(fns[which], dim3(static_cast<unsigned>(ntiles)), dim3(psgd::kThreads), args,
                              smem[which], s);
         if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));

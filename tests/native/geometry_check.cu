@@ -50,6 +50,15 @@ int main() {
             const size_t per3 = 228 * 1024 / 3 - 1024, per2 = 228 * 1024 / 2 - 1024;
             if (a > (R <= 8 ? per3 : per2) || b > (R <= 8 ? per3 : per2) || cc > per2)
                 fail("shared memory lets the intended CTAs per SM reside");
+            // pass B on the 5th-generation tensor cores (R >= 16, 16-byte
+            // rows): the CTAs that shared memory lets reside on one SM never
+            // ask for more than its 512 TMEM columns, so no allocation waits
+            if (R >= 16 && d.vec == 4) {
+                const size_t resident = 228 * 1024 / (b + 1024);
+                const uint32_t cols = R == 16 ? psgd::TcSmem<16>::tmem_cols : psgd::TcSmem<32>::tmem_cols;
+                if (resident * cols > 512) fail("tensor memory of the resident CTAs within 512 columns");
+                if (b < (R == 16 ? psgd::TcSmem<16>::total : psgd::TcSmem<32>::total)) fail("tensor-core pass B buffers");
+            }
         }
         if (sz.tiles != (int64_t)d.nrb * d.nchunk) fail("tile count");
     }
