@@ -157,6 +157,36 @@ __device__ __forceinline__ double sum_in_order(const double* src, int64_t stride
     return s;
 }
 
+// elements summed together by sums_in_order: four at ranks 16 and 32, two
+// below (those kernels run at 80 registers per thread)
+template <int R>
+struct SumBatch { static constexpr int value = R >= 16 ? 4 : 2; };
+
+// s[e] = sum_{j < count} src[e][j * stride] for E elements at once, each in
+// index order (the same order as sum_in_order), eight loads per element in
+// flight; elements with valid[e] false read nothing and their s[e] is 0
+template <int E>
+__device__ __forceinline__ void sums_in_order(const double* const (&src)[E], const bool (&valid)[E],
+                                              int64_t stride, int count, double (&s)[E]) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) s[e] = 0.0;
+    int j = 0;
+    for (; j + 8 <= count; j += 8) {
+        double v[E][8];
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[e][u] = valid[e] ? __ldcg(src[e] + (j + u) * stride) : 0.0;
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+#pragma unroll
+            for (int u = 0; u < 8; ++u) s[e] += v[e][u];
+    }
+    for (; j < count; ++j)
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            if (valid[e]) s[e] += __ldcg(src[e] + j * stride);
+}
 __device__ __forceinline__ void tf32_split(float x, uint32_t& hi, uint32_t& lo) {
     hi = tf32_round(x);
     lo = tf32_round(x - __uint_as_float(hi));
@@ -224,6 +254,39 @@ __device__ __forceinline__ void umma_tf32(uint32_t tmem_d, uint64_t da, uint64_t
         "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(tmem_d),
         "l"(da), "l"(db), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
 }
+// The same with A read from tensor memory (K-major: lane = row of M, one
+// column per tf32 element of K) at tmem_a.
+__device__ __forceinline__ void umma_tf32_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc,
+                                             uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(db), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+// 16 consecutive columns of this thread's TMEM lane (the warp's 32 lanes)
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&u)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16};" ::"r"(taddr),
+        "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]), "r"(u[8]),
+        "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15])
+        : "memory");
+}
+// 8 consecutive columns of this thread's TMEM lane (the warp's 32 lanes)
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&u)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// one lane of the (converged) warp: true there, false elsewhere
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}\n"
+        : "=r"(pred));
+    return pred != 0;
+}
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
@@ -268,28 +331,32 @@ constexpr int kStgCols = 128;
 constexpr int kStgStride = kStgCols + 8;
 constexpr int kStages = 2;
 constexpr size_t kStgBytes = static_cast<size_t>(kStages) * kStgRows * kStgStride * sizeof(float);
-// Tensor-core second pass: the worker's block split into tf32 hi and lo,
-// both transposed to K-major, B = [P_hat hi | P_hat lo] K-major, then the
-// mbarrier, the TMEM address and the wind-down flag.  In A, each group of 8
-// columns holds 16 core matrices (64 rows of K) and is padded by 16 bytes
-// (kTcSboA), so the 16-byte stores of 8 consecutive column quads land in 8
-// distinct bank groups.
-constexpr uint32_t kTcSboA = 16 * 128 + 16;
+// Tensor-core second pass: B = [P_hat hi | P_hat lo] K-major in shared
+// memory (8 rows of N x 16 bytes per core matrix, 16 core matrices = 64
+// rows of K per group of 8 N rows), the threads' float64 sums, then the
+// mbarrier, the TMEM address and the wind-down flag.  A (the worker's block split into hi and lo) and the
+// accumulators live in tensor memory.
 constexpr uint32_t kTcSboB = 16 * 128;
 // workers whose products accumulate in tensor memory (float32, at most 64
 // MMA accumulations per element and half) before D is read back into the
 // float64 sums
 constexpr int kTcGroup = 4;
-// independent accumulators (k-step ks goes to ks % kTcChains), so that
-// successive MMAs do not wait on one another's result
-constexpr int kTcChains = 4;
-constexpr size_t kTcABytes = static_cast<size_t>(kStgCols / 8) * kTcSboA;   // one A buffer (33 KB)
+// independent accumulators (k-step ks goes to ks % kTcChains)
+constexpr int kTcChains = 2;
+// tensor-memory columns: A hi (64 rows of K), A lo, then the chains' D
+constexpr uint32_t kTcAHi = 0, kTcALo = 64, kTcD = 128;
 template <int R>
 struct TcSmem {
     static constexpr size_t b_bytes = static_cast<size_t>(2 * R / 8) * kTcSboB;   // 2R rows of N x 64 of K
-    static constexpr size_t total = 2 * kTcABytes + b_bytes + 16;
-    // per chain D = [hi*hi + lo*hi | hi*lo]; a power of two >= 32
-    static constexpr uint32_t tmem_cols = 2 * R * kTcChains;
+    // each thread's float64 sums of its column and rank half: [R / 2][threads]
+    static constexpr size_t sum_bytes = static_cast<size_t>(R / 2) * kThreads * sizeof(double);
+    // at least 76 KB, so that no more than two CTAs reside on an SM (228 KB)
+    // and their tensor memory (tmem_cols each) fits in the SM's 512 columns
+    static constexpr size_t need = b_bytes + sum_bytes + 16;
+    static constexpr size_t total = need > 76 * 1024 ? need : 76 * 1024;
+    // per chain D = [hi*hi + lo*hi | hi*lo]; the allocation is a power of two
+    static constexpr uint32_t tmem_cols = 256;
+    static_assert(kTcD + kTcChains * 2 * R <= tmem_cols, "tensor memory of the second pass");
 };
 
 constexpr int kMmaRows = 16;                  // rows per warp in the tensor-core pass A
@@ -818,18 +885,33 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
     const double* ppart = p.ws.ppart + d.ppart_off;
     double* pbar = p.ws.pbar + d.prow_off;
     const double inv_w = 1.0 / static_cast<double>(p.workers);
-    for (int idx = tid; idx < rows * R; idx += kThreads) {
-        const int64_t i = i0 + idx / R;
-        const int k = idx % R;
-        double s = sum_in_order(ppart + i * R + k, m * R, d.nchunk);
-        if (p.dist) {
-            // this rank's share of the all-reduce: the row's sum over its workers
-            p.dist_out[d.prow_off + i * R + k] = s;
-            continue;
+    for (int base = tid; base < rows * R; base += SumBatch<R>::value * kThreads) {
+        constexpr int E = SumBatch<R>::value;
+        const double* src[E];
+        bool valid[E];
+        double sums[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int idx = base + e * kThreads;
+            valid[e] = idx < rows * R;
+            src[e] = ppart + (i0 + (valid[e] ? idx / R : 0)) * R + (valid[e] ? idx % R : 0);
         }
-        const double v = s * inv_w;
-        pb_s[idx] = v;
-        pbar[i * R + k] = v;
+        sums_in_order<E>(src, valid, m * R, d.nchunk, sums);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int idx = base + e * kThreads;
+            if (!valid[e]) continue;
+            const int64_t i = i0 + idx / R;
+            const int k = idx % R;
+            if (p.dist) {
+                // this rank's share of the all-reduce: the row's sum over its workers
+                p.dist_out[d.prow_off + i * R + k] = sums[e];
+                continue;
+            }
+            const double v = sums[e] * inv_w;
+            pb_s[idx] = v;
+            pbar[i * R + k] = v;
+        }
     }
     if (tid == 0) cnt[cl.a_rb + tc.rb] = 0u;
     if (p.dist) return;
@@ -1486,25 +1568,26 @@ __device__ __forceinline__ void pass_b_staged(const Params& p, const LayerDesc& 
 
 // Second pass on the 5th-generation tensor cores (R = 16, 32; 16-byte rows).
 // For every worker, D (128 chunk columns x ranks, float32, in tensor memory)
-// = M^T P_hat over the tile's rows.  tf32 operands are read K-major (K = the
-// tile's rows), so the worker's block of M, held row-major in global memory,
-// is transposed on its way into shared memory: each thread loads 4 x 4
-// blocks (four rows of one column quad) one worker ahead into registers,
-// splits them into hi (the top 19 bits) and lo = x - hi, and stores every
-// column's four rows as one 16-byte K row of a core matrix.  B = [P_hat hi |
-// P_hat lo] (round-to-nearest split), K-major, once per tile.  Per k-step of
-// 8 rows two MMAs give fp32 accuracy from tf32 products (split-precision
-// products, Markidis et al. 2018): A_hi [B_hi | B_lo] (N = 2R) and A_lo B_hi
-// (N = R, accumulated into the first half), so D = [hi*hi + lo*hi | hi*lo],
-// in kTcChains independent accumulators (k-step ks into ks % kTcChains).
-// One thread issues them and commits to an mbarrier, and one thread waits
-// on it before the next worker's block is stored.  D accumulates over
-// groups of kTcGroup workers; after each group all eight warps read it back
-// (tcgen05.ld: four lane quarters x two rank halves; chains and halves
-// summed in float32) into float64 sums, so float32 runs stay within
-// kTcGroup workers' rows of one tile.  Every wait is bounded
-// (about a second), after which the status word is set and the tile winds
-// down; the tensor memory is released on every path.
+// = M^T P_hat over the tile's rows.  A = the worker's block of M, K-major in
+// tensor memory: each thread owns one TMEM lane (a chunk column) and half
+// of the tile's rows; it loads its 32 rows one worker ahead into registers
+// (a warp's loads take 128 contiguous bytes of a row), splits them into hi
+// (the top 19 bits) and lo = x - hi, and writes both with tcgen05.st.
+// B = [P_hat hi | P_hat lo] (round-to-nearest split), K-major in shared
+// memory, once per tile.  Per k-step of 8 rows two MMAs give fp32 accuracy
+// from tf32 products (split-precision products, Markidis et al. 2018):
+// A_hi [B_hi | B_lo] (N = 2R) and A_lo B_hi (N = R, accumulated into the
+// first half), so D = [hi*hi + lo*hi | hi*lo], in kTcChains independent
+// accumulators (k-step ks into ks % kTcChains).  Warp 0 runs the issue loop,
+// one elected lane issues them and commits to an mbarrier, and one thread
+// waits on it before the next worker's block is written.  D accumulates
+// over groups of kTcGroup workers; after each group all eight warps read it
+// back (tcgen05.ld: four lane quarters x two rank halves; chains and halves
+// summed in float32) into float64 sums (each thread's own slots in shared
+// memory), so float32 runs stay within kTcGroup workers' rows of one tile.
+// Every wait is bounded (about a
+// second), after which the status word is set and the tile winds down; the
+// tensor memory is released on every path.
 
 __device__ __forceinline__ uint32_t tc_kmajor(int mn, int k, uint32_t sbo) {   // bytes; K extent 64
     return static_cast<uint32_t>((mn >> 3) * sbo + (k >> 2) * 128 + (mn & 7) * 16 + (k & 3) * 4);
@@ -1535,8 +1618,8 @@ template <int R>
 __device__ __forceinline__ void pass_b_tc(const Params& p, const LayerDesc& d, const TileCoord& tc,
                                           float* const* ep, const float* ph_s, unsigned char* buf) {
     static_assert(R == 16 || R == 32, "tensor-core pass B: rank 16 or 32");
-    constexpr int RH = R / 2;                             // ranks per reading warp
-    constexpr int kQ = (kStgRows / 4) / kWarps;           // row quads per thread and block (2)
+    constexpr int RH = R / 2;   // ranks per reading warp
+    constexpr int KH = 32;      // rows of K per thread (half of the 64-row tile)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int W = p.workers;
     const int64_t n = d.n;
@@ -1545,55 +1628,28 @@ __device__ __forceinline__ void pass_b_tc(const Params& p, const LayerDesc& d, c
     const int64_t jc = static_cast<int64_t>(tc.c) * d.slots * 4;
     const int width = static_cast<int>(min(static_cast<int64_t>(d.slots) * 4, n - jc));
     const int nks = d.tm / 8;
-    unsigned char* a_hi = buf;
-    unsigned char* a_lo = buf + kTcABytes;
-    unsigned char* b_s = a_lo + kTcABytes;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(b_s + TcSmem<R>::b_bytes);
+    unsigned char* b_s = buf;
+    double* dsum = reinterpret_cast<double*>(b_s + TcSmem<R>::b_bytes);   // [RH][kThreads]
+    uint64_t* bar = reinterpret_cast<uint64_t*>(b_s + TcSmem<R>::b_bytes + TcSmem<R>::sum_bytes);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
     int* flag = reinterpret_cast<int*>(tslot + 1);
     const uint32_t bar_a = static_cast<uint32_t>(__cvta_generic_to_shared(bar));
     constexpr uint32_t kIdescHL = umma_idesc_tf32(128, 2 * R);
     constexpr uint32_t kIdescL = umma_idesc_tf32(128, R);
 
-    // this thread: column quad `lane` (a warp's loads take 512 contiguous
-    // bytes of one row) of row quads warp + 8 i; x[i][r] = row 4 (warp + 8 i) + r
-    const int c4 = 4 * lane;
-    const bool col_ok = c4 < width;
-    auto load = [&](int w, float4 (&v)[kQ][4]) {
-        const float* src = ep[w] + i0 * n + jc + c4;
+    // this thread: TMEM lane (chunk column) 32 (warp & 3) + lane, rows
+    // KH (warp >> 2) .. + KH - 1 of the tile
+    const int col = (warp & 3) * 32 + lane;
+    const int r0 = KH * (warp >> 2);
+    const bool has_rows = r0 < d.tm;   // uniform over the warp
+    const bool col_ok = col < width;
+    const int nr = col_ok ? max(0, min(KH, rows - r0)) : 0;   // rows this thread loads
+    auto load = [&](int w, float (&v)[KH]) {
+        const float* src = ep[w] + (i0 + r0) * n + jc + col;
 #pragma unroll
-        for (int i = 0; i < kQ; ++i)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int row = 4 * (warp + kWarps * i) + r;
-                v[i][r] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (col_ok && row < rows) v[i][r] = __ldcg(reinterpret_cast<const float4*>(src + row * n));
-            }
-    };
-    // column c4 + j, rows 4q..4q+3: one 16-byte K row of a core matrix at
-    // (col >> 3) kTcSboA + q 128 + (col & 7) 16
-    auto split_store = [&](const float4 (&v)[kQ][4]) {
-#pragma unroll
-        for (int i = 0; i < kQ; ++i) {
-            const int q = warp + kWarps * i;   // uniform over the warp
-            if (4 * q < d.tm) {
-                const uint32_t base = (lane >> 1) * kTcSboA + q * 128 + (lane & 1) * 64;
-                const float4 t[4] = {make_float4(v[i][0].x, v[i][1].x, v[i][2].x, v[i][3].x),
-                                     make_float4(v[i][0].y, v[i][1].y, v[i][2].y, v[i][3].y),
-                                     make_float4(v[i][0].z, v[i][1].z, v[i][2].z, v[i][3].z),
-                                     make_float4(v[i][0].w, v[i][1].w, v[i][2].w, v[i][3].w)};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float4 h;
-                    h.x = __uint_as_float(__float_as_uint(t[j].x) & 0xffffe000u);
-                    h.y = __uint_as_float(__float_as_uint(t[j].y) & 0xffffe000u);
-                    h.z = __uint_as_float(__float_as_uint(t[j].z) & 0xffffe000u);
-                    h.w = __uint_as_float(__float_as_uint(t[j].w) & 0xffffe000u);
-                    *reinterpret_cast<float4*>(a_hi + base + j * 16) = h;
-                    *reinterpret_cast<float4*>(a_lo + base + j * 16) =
-                        make_float4(t[j].x - h.x, t[j].y - h.y, t[j].z - h.z, t[j].w - h.w);
-                }
-            }
+        for (int r = 0; r < KH; ++r) {
+            v[r] = r < nr ? __ldcg(src) : 0.f;
+            src += n;
         }
     };
 
@@ -1617,19 +1673,40 @@ __device__ __forceinline__ void pass_b_tc(const Params& p, const LayerDesc& d, c
         *reinterpret_cast<uint32_t*>(b_s + tc_kmajor(k, row, kTcSboB)) = hi;
         *reinterpret_cast<uint32_t*>(b_s + tc_kmajor(R + k, row, kTcSboB)) = lo;
     }
-    float4 x[kQ][4], xn[kQ][4];
-    if (W > 0) load(0, x);
+    float x[KH], xn[KH];
+    if (W > 0 && has_rows) load(0, x);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);   // this warp's TMEM lanes
 
-    double dsum[RH];
+    // hi and lo of this thread's rows into its TMEM lane (v is left holding lo)
+    auto store_a = [&](float (&v)[KH]) {
 #pragma unroll
-    for (int k = 0; k < RH; ++k) dsum[k] = 0.0;
-    const int kh = (warp >> 2) * RH;                                                // this warp's ranks
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);   // its TMEM lanes
+        for (int j = 0; j < KH; j += 8) {
+            uint32_t u[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                u[k] = __float_as_uint(v[j + k]) & 0xffffe000u;
+                v[j + k] -= __uint_as_float(u[k]);
+            }
+            tmem_st8(t_lane + kTcAHi + static_cast<uint32_t>(r0 + j), u);
+        }
+#pragma unroll
+        for (int j = 0; j < KH; j += 8) {
+            uint32_t u[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) u[k] = __float_as_uint(v[j + k]);
+            tmem_st8(t_lane + kTcALo + static_cast<uint32_t>(r0 + j), u);
+        }
+        tmem_wait_st();
+    };
+
+#pragma unroll
+    for (int k = 0; k < RH; ++k) dsum[k * kThreads + tid] = 0.0;   // this thread's own slots
+    const int kh = (warp >> 2) * RH;   // this warp's ranks
     // the chains' two halves summed in float32 (chains beyond the tile's
     // k-steps hold nothing), then added to the float64 sums; 8 ranks at a time
     auto read_back = [&]() {
@@ -1637,7 +1714,7 @@ __device__ __forceinline__ void pass_b_tc(const Params& p, const LayerDesc& d, c
         for (int k0 = 0; k0 < RH; k0 += 8) {
             uint32_t u[8];
             float f[8];
-            tmem_ld<8>(t_lane + static_cast<uint32_t>(kh + k0), u);   // chain 0, hi*hi + lo*hi
+            tmem_ld<8>(t_lane + kTcD + static_cast<uint32_t>(kh + k0), u);   // chain 0, hi*hi + lo*hi
             tmem_wait_ld();
 #pragma unroll
             for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(u[k]);
@@ -1646,14 +1723,14 @@ __device__ __forceinline__ void pass_b_tc(const Params& p, const LayerDesc& d, c
 #pragma unroll
                 for (int h = (c == 0 ? 1 : 0); h < 2; ++h) {
                     if (c < nks) {   // uniform over the block
-                        tmem_ld<8>(t_lane + static_cast<uint32_t>(c * 2 * R + h * R + kh + k0), u);
+                        tmem_ld<8>(t_lane + kTcD + static_cast<uint32_t>(c * 2 * R + h * R + kh + k0), u);
                         tmem_wait_ld();
 #pragma unroll
                         for (int k = 0; k < 8; ++k) f[k] += __uint_as_float(u[k]);
                     }
                 }
 #pragma unroll
-            for (int k = 0; k < 8; ++k) dsum[k0 + k] += static_cast<double>(f[k]);
+            for (int k = 0; k < 8; ++k) dsum[(k0 + k) * kThreads + tid] += static_cast<double>(f[k]);
         }
     };
     // one thread waits for worker w's products; the others at the barrier
@@ -1665,40 +1742,43 @@ __device__ __forceinline__ void pass_b_tc(const Params& p, const LayerDesc& d, c
         return *flag == 0;
     };
 
+    // worker w: its rows are in `cur`; the next worker's are loaded into
+    // `nxt` (the two register sets alternate, so no copy waits on the loads)
     bool ok = true;
-    for (int w = 0; w < W; ++w) {
-        if (w + 1 < W) load(w + 1, xn);
+    auto worker = [&](int w, float (&cur)[KH], float (&nxt)[KH]) -> bool {
+        if (w + 1 < W && has_rows) load(w + 1, nxt);
         if (w > 0) {
-            // worker w - 1's products are done: D and the A buffers are free
-            if (!wait_products(w - 1)) {
-                ok = false;
-                break;
-            }
+            // worker w - 1's products are done: A and D are free
+            if (!wait_products(w - 1)) return false;
             if ((w - 1) % kTcGroup == kTcGroup - 1) read_back();
         }
-        split_store(x);
-        fence_async_smem();
+        if (has_rows) store_a(cur);
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        if (tid == 0) {
-            const uint32_t ah = static_cast<uint32_t>(__cvta_generic_to_shared(a_hi));
-            const uint32_t al = static_cast<uint32_t>(__cvta_generic_to_shared(a_lo));
+        if (warp == 0) {
+            // warp-uniform loop; one elected lane issues
+            const bool leader = elect_one();
+            const uint32_t acc0 = (w % kTcGroup) ? 1u : 0u;
             const uint32_t bb = static_cast<uint32_t>(__cvta_generic_to_shared(b_s));
             for (int ks = 0; ks < nks; ++ks) {
-                const uint32_t ko = static_cast<uint32_t>(ks) * 256;   // 8 rows = two K core matrices
-                const uint32_t dc = tmem + static_cast<uint32_t>((ks % kTcChains) * 2 * R);
-                const uint64_t db = umma_desc(bb + ko, 128, kTcSboB);
-                umma_tf32(dc, umma_desc(ah + ko, 128, kTcSboA), db, kIdescHL,
-                          (ks >= kTcChains || w % kTcGroup) ? 1u : 0u);
-                umma_tf32(dc, umma_desc(al + ko, 128, kTcSboA), db, kIdescL, 1u);
+                const uint32_t dc = tmem + kTcD + static_cast<uint32_t>((ks % kTcChains) * 2 * R);
+                if (leader) {
+                    // 8 rows of K: 8 TMEM columns of A, two K core matrices (256 bytes) of B
+                    const uint64_t db = umma_desc(bb + static_cast<uint32_t>(ks) * 256, 128, kTcSboB);
+                    umma_tf32_ts(dc, tmem + kTcAHi + static_cast<uint32_t>(ks) * 8, db, kIdescHL,
+                                 ks >= kTcChains ? 1u : acc0);
+                    umma_tf32_ts(dc, tmem + kTcALo + static_cast<uint32_t>(ks) * 8, db, kIdescL, 1u);
+                }
             }
-            umma_commit(bar_a);
+            if (leader) umma_commit(bar_a);
+            __syncwarp();
         }
-#pragma unroll
-        for (int i = 0; i < kQ; ++i)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) x[i][r] = xn[i][r];
+        return true;
+    };
+    for (int w = 0; w < W && ok; w += 2) {
+        ok = worker(w, x, xn);
+        if (ok && w + 1 < W) ok = worker(w + 1, xn, x);
     }
     if (ok && W > 0) {
         ok = wait_products(W - 1);
@@ -1713,11 +1793,10 @@ __device__ __forceinline__ void pass_b_tc(const Params& p, const LayerDesc& d, c
     }
     if (!ok) return;   // the status word says why; this tile's partial is not written
     // this thread's chunk column (TMEM lane) and rank half of the row block's partial Q rows
-    const int col = (warp & 3) * 32 + lane;
-    if (col < width) {
+    if (col_ok) {
         double* qp = p.ws.qpart + d.qpart_off + (static_cast<int64_t>(tc.rb) * n + jc + col) * R + kh;
 #pragma unroll
-        for (int k = 0; k < RH; ++k) qp[k] = dsum[k];
+        for (int k = 0; k < RH; ++k) qp[k] = dsum[k * kThreads + tid];
     }
 }
 
@@ -1750,11 +1829,24 @@ __device__ void pass_b_epilogue(const Params& p, const LayerDesc& d, const TileC
     __threadfence();
     const double* qpart = p.ws.qpart + d.qpart_off;
     double* qsup = p.ws.qsup + d.qsup_off;
-    for (int idx = tid; idx < cols * R; idx += kThreads) {
-        const int64_t col = col0 + idx / R;
-        const int k = idx % R;
-        const double s = sum_in_order(qpart + (static_cast<int64_t>(rb0) * n + col) * R + k, n * R, nin);
-        qsup[(static_cast<int64_t>(sup) * n + col) * R + k] = s;
+    for (int base = tid; base < cols * R; base += SumBatch<R>::value * kThreads) {
+        constexpr int E = SumBatch<R>::value;
+        const double* src[E];
+        bool valid[E];
+        double s[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int idx = base + e * kThreads;
+            valid[e] = idx < cols * R;
+            const int64_t col = col0 + (valid[e] ? idx / R : 0);
+            src[e] = qpart + (static_cast<int64_t>(rb0) * n + col) * R + (valid[e] ? idx % R : 0);
+        }
+        sums_in_order<E>(src, valid, n * R, nin, s);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int idx = base + e * kThreads;
+            if (valid[e]) qsup[(static_cast<int64_t>(sup) * n + col0 + idx / R) * R + idx % R] = s[e];
+        }
     }
     if (tid == 0) *c1 = 0u;
 
@@ -1773,17 +1865,33 @@ __device__ void pass_b_epilogue(const Params& p, const LayerDesc& d, const TileC
     float* qout = p.t.q[tc.l];
     const int r = p.r;
     const double inv_w = 1.0 / static_cast<double>(p.workers);
-    for (int idx = tid; idx < cols * R; idx += kThreads) {
-        const int64_t col = col0 + idx / R;
-        const int k = idx % R;
-        const double s = sum_in_order(qsup + col * R + k, n * R, d.nsup);
-        if (p.dist) {
-            p.dist_out[d.qrow_off + col * R + k] = s;   // this rank's share of the all-reduce
-            continue;
+    for (int base = tid; base < cols * R; base += SumBatch<R>::value * kThreads) {
+        constexpr int E = SumBatch<R>::value;
+        const double* src[E];
+        bool valid[E];
+        double sums[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int idx = base + e * kThreads;
+            valid[e] = idx < cols * R;
+            src[e] = qsup + (col0 + (valid[e] ? idx / R : 0)) * R + (valid[e] ? idx % R : 0);
         }
-        const float v = static_cast<float>(s * inv_w);
-        qbar[col * R + k] = v;
-        if (k < r) qout[col * r + k] = v;
+        sums_in_order<E>(src, valid, n * R, d.nsup, sums);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int idx = base + e * kThreads;
+            if (!valid[e]) continue;
+            const int64_t col = col0 + idx / R;
+            const int k = idx % R;
+            const double s = sums[e];
+            if (p.dist) {
+                p.dist_out[d.qrow_off + col * R + k] = s;   // this rank's share of the all-reduce
+                continue;
+            }
+            const float v = static_cast<float>(s * inv_w);
+            qbar[col * R + k] = v;
+            if (k < r) qout[col * r + k] = v;
+        }
     }
     if (tid == 0) cnt[cl.b_chunk + tc.c] = 0u;
 }
