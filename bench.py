@@ -77,7 +77,8 @@ def compute_roofline(elements: int, rank: int, pass_a_ms: float, pass_b_ms: floa
             "fp32_cuda_core_peak": round(fp32_peak, 1), "fp32_frac": round(achieved / fp32_peak, 4),
             "tf32_tensor_peak": round(tf32_peak, 1), "tf32_frac": round(achieved / tf32_peak, 4),
             "note": "products of passes A and B only; ranks 16 and 32 run them on the tf32 tensor cores "
-                    "(mma.sync, three split products per term), ranks <= 8 on the CUDA cores"}
+                    "with three split products per term (pass A mma.sync; pass B tcgen05 with A in tensor "
+                    "memory on 16-byte rows), ranks <= 8 on the CUDA cores"}
 
 
 def _code_tokens(text: str) -> str:

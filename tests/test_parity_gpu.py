@@ -446,6 +446,18 @@ def test_many_workers_rank32(workers):
     H.assert_close(hist[0], H.TOL["f32"], "step 0")
 
 
+@pytest.mark.parametrize("rank", [16, 32])
+@pytest.mark.parametrize("workers", [64, 256])
+def test_many_workers_tensor_memory_pass(workers, rank):
+    # the second pass on the 5th-generation tensor cores (16-byte rows):
+    # float32 runs of up to four workers' rows inside the tensor core, then
+    # float64; three free-running steps, full and ragged tiles and chunks
+    wl = H.small_workload([(64, 576), (256, 128), (129, 1000)], rank, workers)
+    _, _, hist = H.run_free(wl, steps=3)
+    for t, e in enumerate(hist):
+        H.assert_close(e, H.TOL["f32"], f"step {t}")
+
+
 # r = min(m, n): wide and tall layers of exactly the rank (no compression;
 # chunks of a few lanes at every lane width)
 FULL_RANK = {2: [(2, 64), (50, 2)], 4: [(4, 90), (70, 4)], 8: [(8, 100), (100, 8)],
