@@ -331,11 +331,14 @@ psgd::Params base_params(psgd_ctx* ctx) {
 
 // Grid of k_phat: (x, L), x covering the largest layer's m R elements
 // (grid-stride beyond 4096 blocks).
+dim3 phat_grid(int64_t maxm, size_t num_layers, int R) {
+    const int64_t gx = std::min<int64_t>(4096, (std::max<int64_t>(1, maxm) * R + psgd::kThreads - 1) / psgd::kThreads);
+    return dim3(static_cast<unsigned>(std::max<int64_t>(1, gx)), static_cast<unsigned>(num_layers));
+}
 dim3 phat_grid(const std::vector<LayerDesc>& desc, int R) {
     int64_t maxm = 1;
     for (auto& d : desc) maxm = std::max(maxm, d.m);
-    const int64_t gx = std::min<int64_t>(4096, (maxm * R + psgd::kThreads - 1) / psgd::kThreads);
-    return dim3(static_cast<unsigned>(std::max<int64_t>(1, gx)), static_cast<unsigned>(desc.size()));
+    return phat_grid(maxm, desc.size(), R);
 }
 
 // The second pass (which == 1) is preceded by k_phat, which forms P_hat
@@ -1214,7 +1217,7 @@ int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int grad_dtype
         }
         void* args[] = {&pw};
         if (which == 1) {
-            e = cudaLaunchKernel(kernel_ptr(7, R, grad_dtype, false, false), phat_grid({d}, R),
+            e = cudaLaunchKernel(kernel_ptr(7, R, grad_dtype, false, false), phat_grid(d.m, 1, R),
                                  dim3(psgd::kThreads), args, 0, s);
             if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "P_hat launch: %s", cudaGetErrorString(e));
         }

@@ -29,6 +29,16 @@ def test_mixed_shapes_f32(rank, workers):
         H.assert_close(e, H.TOL["f32"], f"step {t}")
 
 
+@pytest.mark.parametrize("rank", [1, 2, 4, 8])
+def test_eight_byte_rows_odd_row_counts(rank):
+    # 8-byte lanes (n % 4 == 2, and every even n at r = 8) on layers with an
+    # odd number of rows and ragged row blocks
+    wl = H.small_workload([(33, 650), (9, 10), (301, 26), (64, 576)], rank, 3)
+    _, _, hist = H.run_free(wl, steps=3)
+    for t, e in enumerate(hist):
+        H.assert_close(e, H.TOL["f32"], f"step {t}")
+
+
 @pytest.mark.parametrize("rank", [1, 4, 16, 32])
 def test_mixed_shapes_bf16(rank):
     wl = H.small_workload(MIXED, rank, 4, dtype="bf16")
@@ -315,7 +325,8 @@ def test_vec_mean_and_momentum():
 
 
 def test_momentum_step_matches_oracle():
-    wl = H.small_workload(MIXED[:4], 2, 3)
+    # (33, 650): 8-byte lanes with an odd row count
+    wl = H.small_workload(MIXED[:4] + [(33, 650)], 2, 3)
     run = H.LibRun(wl)
     L = len(wl.layers)
     params = [torch.zeros(m, n, device="cuda") for (m, n) in wl.layers]
