@@ -190,9 +190,22 @@ PSGD_API int psgd_vec_mean(psgd_ctx *ctx, const float *const *vecs, float *const
 
 /* Service calls (no counterpart in the pages).
  * Synchronise the last stream used and read the device status word:
- * PSGD_OK, or PSGD_ERR_DEVICE if a kernel flagged an inconsistency (e.g.
- * overlapping steps on one context), or PSGD_ERR_CUDA if a launch failed. */
+ * PSGD_OK, or PSGD_ERR_DEVICE if a kernel flagged an inconsistency (bit 0x1:
+ * a reduction counter held an impossible value, e.g. overlapping steps on
+ * one context; bit 0x2: a bounded wait of a tensor-core pass ran out, about
+ * one second, and that tile wrote nothing), or PSGD_ERR_CUDA if a launch
+ * failed.  A set word is reported once and then cleared, so the steps that
+ * follow report their own state (the context's counters stay consistent
+ * either way). */
 PSGD_API int psgd_status(psgd_ctx *ctx);
+
+/* For testing the bounded waits (no counterpart in the pages): with on != 0
+ * the tensor-core second pass (ranks 16 and 32, 16-byte rows) of later
+ * steps issues no products and commits none, so each of its tiles waits
+ * out its one-second limit, sets bit 0x2 of the status word, releases its
+ * tensor memory and writes no partial; that step's results are not valid.
+ * on = 0 (the default) restores normal steps. */
+PSGD_API int psgd_test_stall_products(psgd_ctx *ctx, int on);
 
 /* Bytes of device workspace the context holds (excluding host staging). */
 PSGD_API int psgd_workspace_bytes(const psgd_ctx *ctx, size_t *bytes);

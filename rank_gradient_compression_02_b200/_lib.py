@@ -69,6 +69,7 @@ _SIGS = {
     "psgd_dist_finish": (ctypes.c_int, [_P, _P, _P]),
     "psgd_set_svd_refresh": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int]),
     "psgd_set_svd_oversampling": (ctypes.c_int, [_P, ctypes.c_int]),
+    "psgd_test_stall_products": (ctypes.c_int, [_P, ctypes.c_int]),
     "psgd_profile_enable": (ctypes.c_int, [_P, ctypes.c_int]),
     "psgd_profile_read": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]),
 }
@@ -408,6 +409,11 @@ class PowerSGD:
 
     def status(self):
         self._check(self.lib.psgd_status(self._h))
+
+    def test_stall_products(self, on: bool) -> None:
+        """Testing the bounded waits: the tensor-core second pass of later
+        steps issues no products, so its waits run out (psgd.h)."""
+        self._check(self.lib.psgd_test_stall_products(self._h, 1 if on else 0))
 
     @property
     def workspace_bytes(self) -> int:

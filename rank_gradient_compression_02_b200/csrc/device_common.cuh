@@ -115,6 +115,9 @@ struct Params {
     // (lambda_{r'} / lambda_{r_conv})^(iter - 1) <= conv_eps
     int iter, track_conv, r_conv;
     double conv_eps;
+    // testing the bounded waits: the tensor-core second pass issues no
+    // products (and commits none), so its waits run out
+    int stall_products;
 };
 
 enum : int {

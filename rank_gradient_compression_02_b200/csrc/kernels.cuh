@@ -1756,7 +1756,7 @@ __device__ __forceinline__ void pass_b_tc(const Params& p, const LayerDesc& d, c
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        if (warp == 0) {
+        if (warp == 0 && !p.stall_products) {
             // warp-uniform loop; one elected lane issues
             const bool leader = elect_one();
             const uint32_t acc0 = (w % kTcGroup) ? 1u : 0u;

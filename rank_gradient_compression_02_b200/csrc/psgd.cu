@@ -195,6 +195,7 @@ struct psgd_ctx {
     size_t prof_used = 0;
 
     int iters = 1;          // power iterations per step
+    int stall_products = 0; // psgd_test_stall_products
     int w_global = 0;       // workers over all ranks (distributed step); 0 = W
     int dist_phase = 0;     // distributed step: 0 idle, 1 after P, 2 after Q
     bool tab_l_has_recon = false;
@@ -326,6 +327,7 @@ psgd::Params base_params(psgd_ctx* ctx) {
     p.inv_w = 1.0f / static_cast<float>(ctx->W);
     p.drop_tol = kDropTol;
     p.inv_w_global = 1.0 / static_cast<double>(ctx->w_global > 0 ? ctx->w_global : ctx->W);
+    p.stall_products = ctx->stall_products;
     return p;
 }
 
@@ -1470,6 +1472,12 @@ int psgd_set_svd_oversampling(psgd_ctx* ctx, int extra) {
     return configure_refresh(ctx);
 }
 
+int psgd_test_stall_products(psgd_ctx* ctx, int on) {
+    if (!ctx) return PSGD_ERR_ARG;
+    ctx->stall_products = on != 0;
+    return PSGD_OK;
+}
+
 int psgd_profile_enable(psgd_ctx* ctx, int enable) {
     if (!ctx) return PSGD_ERR_ARG;
     ctx->profiling = enable != 0;
@@ -1506,7 +1514,12 @@ int psgd_status(psgd_ctx* ctx) {
     int st = 0;
     e = cudaMemcpy(&st, ctx->work.status, sizeof(int), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "status read");
-    if (st) return fail(ctx, PSGD_ERR_DEVICE, "device status word 0x%x", st);
+    if (st) {
+        // reported once: the word is cleared for the steps that follow
+        e = cudaMemset(ctx->work.status, 0, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "status clear");
+        return fail(ctx, PSGD_ERR_DEVICE, "device status word 0x%x", st);
+    }
     return PSGD_OK;
 }
 
