@@ -77,7 +77,8 @@ enum {
     PSGD_ERR_CUDA = 3,   /* a CUDA runtime call failed */
     PSGD_ERR_OOM = 4,    /* workspace allocation failed */
     PSGD_ERR_STATE = 5,  /* call not valid in this context's mode */
-    PSGD_ERR_DEVICE = 6  /* the device status word is set (psgd_status) */
+    PSGD_ERR_DEVICE = 6, /* a kernel found a reduction counter inconsistent (psgd_status) */
+    PSGD_ERR_TIMEOUT = 7 /* a bounded wait in a kernel ran out (psgd_status) */
 };
 
 typedef enum { PSGD_F32 = 0, PSGD_BF16 = 1 } psgd_dtype; /* dtype of G only */
@@ -190,20 +191,22 @@ PSGD_API int psgd_vec_mean(psgd_ctx *ctx, const float *const *vecs, float *const
 
 /* Service calls (no counterpart in the pages).
  * Synchronise the last stream used and read the device status word:
- * PSGD_OK, or PSGD_ERR_DEVICE if a kernel flagged an inconsistency (bit 0x1:
- * a reduction counter held an impossible value, e.g. overlapping steps on
- * one context; bit 0x2: a bounded wait of a tensor-core pass ran out, about
- * one second, and that tile wrote nothing), or PSGD_ERR_CUDA if a launch
- * failed.  A set word is reported once and then cleared, so the steps that
- * follow report their own state (the context's counters stay consistent
- * either way). */
+ * PSGD_OK; PSGD_ERR_TIMEOUT if a bounded wait of a tensor-core pass ran out
+ * (about one second; that tile wrote nothing; bit 0x2 of the word);
+ * PSGD_ERR_DEVICE if a reduction counter held an impossible value (bit 0x1,
+ * e.g. steps overlapping on one context); or PSGD_ERR_CUDA if a launch
+ * failed.  psgd_last_error gives the word.  A set word is reported once and
+ * then cleared, so the steps that follow report their own state (the
+ * context's counters stay consistent either way).  Either error means the
+ * results of the step(s) since the last clean report are not valid. */
 PSGD_API int psgd_status(psgd_ctx *ctx);
 
 /* For testing the bounded waits (no counterpart in the pages): with on != 0
  * the tensor-core second pass (ranks 16 and 32, 16-byte rows) of later
  * steps issues no products and commits none, so each of its tiles waits
- * out its one-second limit, sets bit 0x2 of the status word, releases its
- * tensor memory and writes no partial; that step's results are not valid.
+ * out its one-second limit, sets bit 0x2 of the status word (psgd_status:
+ * PSGD_ERR_TIMEOUT), releases its tensor memory and writes no partial; that
+ * step's results are not valid.
  * on = 0 (the default) restores normal steps. */
 PSGD_API int psgd_test_stall_products(psgd_ctx *ctx, int on);
 
@@ -257,10 +260,11 @@ PSGD_API int psgd_step_static(int64_t m, int64_t n, int rank, int workers, int g
 
 /* Status of the last psgd_step_static call on the current device (no
  * counterpart in the pages): synchronises `stream`, then reads the status
- * word at the head of the static array.  PSGD_OK, or PSGD_ERR_DEVICE when a
- * kernel of that call found a reduction counter inconsistent (what calls
- * that overlap on the GPU produce: their results are then wrong), or
- * PSGD_ERR_CUDA.  Allocates nothing. */
+ * word at the head of the static array.  PSGD_OK, PSGD_ERR_TIMEOUT when a
+ * bounded wait of a kernel of that call ran out, PSGD_ERR_DEVICE when one
+ * found a reduction counter inconsistent (what calls that overlap on the
+ * GPU produce: their results are then wrong), or PSGD_ERR_CUDA.  Allocates
+ * nothing. */
 PSGD_API int psgd_step_static_status(void *stream);
 
 /* Distributed step.  On a real data-parallel job every rank (GPU) holds

@@ -19,14 +19,15 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpsgd.so")
 
-PSGD_OK, PSGD_ERR_ARG, PSGD_ERR_ALIGN, PSGD_ERR_CUDA, PSGD_ERR_OOM, PSGD_ERR_STATE, PSGD_ERR_DEVICE = range(7)
+(PSGD_OK, PSGD_ERR_ARG, PSGD_ERR_ALIGN, PSGD_ERR_CUDA, PSGD_ERR_OOM, PSGD_ERR_STATE, PSGD_ERR_DEVICE,
+ PSGD_ERR_TIMEOUT) = range(8)
 PSGD_F32, PSGD_BF16 = 0, 1
 FLAG_LAZY_ERRORS = 1
 FLAG_SUM_FIRST = 2
 FLAG_NO_WARM_START = 4
 
 _ERR_NAMES = {1: "PSGD_ERR_ARG", 2: "PSGD_ERR_ALIGN", 3: "PSGD_ERR_CUDA", 4: "PSGD_ERR_OOM",
-              5: "PSGD_ERR_STATE", 6: "PSGD_ERR_DEVICE"}
+              5: "PSGD_ERR_STATE", 6: "PSGD_ERR_DEVICE", 7: "PSGD_ERR_TIMEOUT"}
 
 
 class PsgdError(RuntimeError):

@@ -1241,6 +1241,8 @@ int psgd_step_static_status(void* stream) {
         e = cudaMemcpy(&word, static_cast<unsigned char*>(base_v) + kStaticStatusOffset, sizeof(int),
                        cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return fail(nullptr, PSGD_ERR_CUDA, "static status: %s", cudaGetErrorString(e));
+    if (word & psgd::kStatusTimeout)
+        return fail(nullptr, PSGD_ERR_TIMEOUT, "device status word 0x%x: a bounded wait ran out", word);
     if (word != 0)
         return fail(nullptr, PSGD_ERR_DEVICE, "device status word 0x%x: a reduction counter was inconsistent "
                     "(calls overlapping on the GPU)", word);
@@ -1518,7 +1520,9 @@ int psgd_status(psgd_ctx* ctx) {
         // reported once: the word is cleared for the steps that follow
         e = cudaMemset(ctx->work.status, 0, sizeof(int));
         if (e != cudaSuccess) return cuda_fail(ctx, e, "status clear");
-        return fail(ctx, PSGD_ERR_DEVICE, "device status word 0x%x", st);
+        if (st & psgd::kStatusTimeout)
+            return fail(ctx, PSGD_ERR_TIMEOUT, "device status word 0x%x: a bounded wait ran out", st);
+        return fail(ctx, PSGD_ERR_DEVICE, "device status word 0x%x: a reduction counter was inconsistent", st);
     }
     return PSGD_OK;
 }

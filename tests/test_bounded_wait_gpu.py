@@ -1,7 +1,7 @@
 """The bounded waits of the tensor-core second pass (ranks 16 and 32,
 16-byte rows).  With the test hook on, its tiles issue no products, so every
 wait on them runs out after about a second: the status word reports it once
-(bit 0x2), the tensor memory is released, and the same context then runs
+(PSGD_ERR_TIMEOUT, bit 0x2), the tensor memory is released, and the same context then runs
 correct steps again.  No GPU fault and no hang is involved: the wait ends
 by its own limit."""
 import time
@@ -15,7 +15,7 @@ from . import _harness as H
 
 pytestmark = pytest.mark.gpu
 
-PSGD_ERR_DEVICE = 6
+PSGD_ERR_TIMEOUT = 7
 
 
 def test_bounded_wait_runs_out_and_the_context_recovers():
@@ -36,7 +36,7 @@ def test_bounded_wait_runs_out_and_the_context_recovers():
     waited = time.monotonic() - t0
     with pytest.raises(PsgdError) as err:
         run.lib.status()
-    assert err.value.code == PSGD_ERR_DEVICE
+    assert err.value.code == PSGD_ERR_TIMEOUT
     assert "0x2" in str(err.value)
     assert 0.5 < waited < 60.0            # about one second per wait, bounded
     run.lib.status()                      # reported once, then cleared
