@@ -39,6 +39,17 @@ def test_eight_byte_rows_odd_row_counts(rank):
         H.assert_close(e, H.TOL["f32"], f"step {t}")
 
 
+@pytest.mark.parametrize("rank", [4, 32])
+def test_tall_layer(rank):
+    # 40000 x 64: m R up to 1.28 M elements of P_hat, past the P_hat
+    # kernel's 4096 x 256 threads (its grid-stride loop), and 625 row blocks
+    # (20 super-blocks) in the second pass's two-level reduction
+    wl = H.small_workload([(40000, 64)], rank, 2)
+    _, _, hist = H.run_free(wl, steps=2)
+    for t, e in enumerate(hist):
+        H.assert_close(e, H.TOL["f32"], f"step {t}")
+
+
 @pytest.mark.parametrize("rank", [1, 4, 16, 32])
 def test_mixed_shapes_bf16(rank):
     wl = H.small_workload(MIXED, rank, 4, dtype="bf16")
