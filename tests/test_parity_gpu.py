@@ -39,6 +39,30 @@ def test_eight_byte_rows_odd_row_counts(rank):
         H.assert_close(e, H.TOL["f32"], f"step {t}")
 
 
+# n % 4 == 2 with even row counts: 8-byte lanes, from one or three slots
+# per row (n = 2, 6) to the LSTM's 650 columns
+PAIRS = [(4, 6), (16, 14), (6, 10), (40, 130), (300, 650), (1000, 650)]
+
+
+@pytest.mark.parametrize("rank,workers", [(1, 1), (2, 5), (3, 16), (4, 3), (4, 6)])
+def test_eight_byte_rows_worker_counts(rank, workers):
+    # every worker remainder of the first pass's load groups
+    layers = PAIRS + ([(50, 2), (2, 6)] if rank <= 2 else [])
+    wl = H.small_workload(layers, rank, workers)
+    _, _, hist = H.run_free(wl, steps=3)
+    for t, e in enumerate(hist):
+        H.assert_close(e, H.TOL["f32"], f"step {t}")
+
+
+@pytest.mark.parametrize("lazy,sum_first,dtype", [(True, False, "f32"), (False, True, "f32"),
+                                                  (False, False, "bf16"), (True, True, "bf16")])
+def test_eight_byte_rows_modes(lazy, sum_first, dtype):
+    wl = H.small_workload(PAIRS, 4, 3, dtype=dtype)
+    _, _, hist = H.run_free(wl, steps=3, lazy=lazy, sum_first=sum_first)
+    for t, e in enumerate(hist):
+        H.assert_close(e, 1e-4, f"step {t}")
+
+
 @pytest.mark.parametrize("rank", [4, 32])
 def test_tall_layer(rank):
     # 40000 x 64: m R up to 1.28 M elements of P_hat, past the P_hat
