@@ -149,19 +149,28 @@ PSGD_API int psgd_step(psgd_ctx *ctx, const void *const *grads, float *const *er
  * library copies them into a device staging area it owns (allocated on
  * first use), runs psgd_step, and copies P_hat and Q_bar back to
  * p_hat_host[l] (m x rank) and q_host[l] (n x rank) if those are non-NULL.
- * errors and q stay device pointers (they are state). */
+ * errors and q stay device pointers (they are state).
+ * Upload and step overlap: the layers are split into at most 8 contiguous
+ * groups of about equal size; the copies run on a stream of the context's
+ * own, which starts after everything already queued on `stream`, and
+ * group g's passes start on `stream` as soon as group g's copies are done
+ * (one launch of each pass per group).  Steps with power iterations, an SVD
+ * refresh or profiling on wait for the whole upload and launch as
+ * psgd_step does.  Everything the call enqueues is ordered before later
+ * work on `stream`, as for psgd_step. */
 PSGD_API int psgd_step_host(psgd_ctx *ctx, const void *const *grads_host, float *const *errors, float *const *q,
                    float *const *p_hat_host, float *const *q_host, void *stream);
 
 /* psgd_step_host for gradients packed into one host buffer per worker (a
  * flat gradient bucket): layer l of worker w starts at element
- * layer_offset[l] of grads_host[w] (grad dtype).  The library uploads each
- * worker's buffer with ONE copy of elements [0, max_l(layer_offset[l] +
- * m_l * n_l)), so the caller guarantees that span is one allocation
- * (pinned for asynchronous copies); bytes between layers are copied and
- * ignored.  layer_offset[l] * sizeof(grad dtype) must be a multiple of 16
- * (PSGD_ERR_ALIGN otherwise), offsets must be >= 0.  Otherwise as
- * psgd_step_host. */
+ * layer_offset[l] of grads_host[w] (grad dtype).  Per layer group (see
+ * psgd_step_host) the library uploads each worker's layers with one copy
+ * per run of layers that follow one another in the buffer (gaps holding no
+ * layer's elements are copied and ignored), so the caller guarantees that
+ * elements [0, max_l(layer_offset[l] + m_l * n_l)) of each worker are one
+ * allocation (pinned for asynchronous copies).  layer_offset[l] *
+ * sizeof(grad dtype) must be a multiple of 16 (PSGD_ERR_ALIGN otherwise),
+ * offsets must be >= 0.  Otherwise as psgd_step_host. */
 PSGD_API int psgd_step_host_flat(psgd_ctx *ctx, const void *const *grads_host, const int64_t *layer_offset,
                                  float *const *errors, float *const *q, float *const *p_hat_host,
                                  float *const *q_host, void *stream);
@@ -217,7 +226,8 @@ PSGD_API int psgd_workspace_bytes(const psgd_ctx *ctx, size_t *bytes);
  * (for launch accounting): per power iteration the first pass, the P_hat
  * kernel and the second pass, + 1 for the third pass in eager mode, + 1
  * with PSGD_FLAG_NO_WARM_START.  An SVD-refresh step makes the launches
- * stated at psgd_set_svd_refresh. */
+ * stated at psgd_set_svd_refresh.  The host-buffer steps launch each pass
+ * once per layer group (psgd_step_host). */
 PSGD_API int psgd_step_launches(const psgd_ctx *ctx);
 
 /* Allocation-free step for one layer.  No counterpart in the pages: this

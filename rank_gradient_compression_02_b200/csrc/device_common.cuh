@@ -118,6 +118,10 @@ struct Params {
     // testing the bounded waits: the tensor-core second pass issues no
     // products (and commits none), so its waits run out
     int stall_products;
+    // a launch over a range of layers (host-buffer steps overlap the upload
+    // of later layers with the passes of earlier ones): the first tile of
+    // the grouped passes' grids and the first layer of the P_hat grid
+    int tile_base, layer_base;
 };
 
 enum : int {

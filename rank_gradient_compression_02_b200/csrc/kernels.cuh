@@ -1008,7 +1008,7 @@ __device__ void pass_a_epilogue(const Params& p, const LayerDesc& d, const TileC
 template <int R, typename GT, bool LAZY, bool SF, bool READM>
 __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_a(Params p) {
     extern __shared__ __align__(16) unsigned char smem[];
-    const int t = tile_index<false>();
+    const int t = p.tile_base + tile_index<false>();
     const int l = p.t.tile_layer[t];
     if (p.track_conv && p.iter > p.ws.conv_iter[l]) return;   // converged refresh layer
     const LayerDesc d = p.t.layers[l];
@@ -1899,7 +1899,7 @@ __device__ void pass_b_epilogue(const Params& p, const LayerDesc& d, const TileC
 template <int R, bool SF>
 __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_b(Params p) {
     extern __shared__ __align__(16) unsigned char smem[];
-    const int t = tile_index<true>();
+    const int t = p.tile_base + tile_index<true>();
     const int l = p.t.tile_layer[t];
     if (p.track_conv && p.iter > p.ws.conv_iter[l]) return;   // converged refresh layer
     const LayerDesc d = p.t.layers[l];
@@ -1939,13 +1939,13 @@ __global__ void __launch_bounds__(kThreads, (R <= 8 ? 3 : 2)) k_pass_b(Params p)
 // P_hat = P_bar T (T = R^-1 from the orthogonalisation) for every layer,
 // once per layer: float64 sums in column order over the upper-triangular T,
 // rounded to float32, into the workspace (read by the second and third
-// passes) and the caller's P_hat.  Grid (x, L): layer blockIdx.y, its m R
-// elements strided over blockIdx.x; a thread's loads of its row are all in
-// flight together.
+// passes) and the caller's P_hat.  Grid (x, layers): layer layer_base +
+// blockIdx.y, its m R elements strided over blockIdx.x; a thread's loads
+// of its row are all in flight together.
 template <int R>
 __global__ void __launch_bounds__(kThreads) k_phat(Params p) {
     __shared__ double T_s[R * R];
-    const int l = blockIdx.y;
+    const int l = p.layer_base + static_cast<int>(blockIdx.y);
     if (p.track_conv && p.iter > p.ws.conv_iter[l]) return;   // converged refresh layer
     const LayerDesc d = p.t.layers[l];
     const double* T = p.ws.T + d.t_off;
@@ -2203,7 +2203,7 @@ __device__ __forceinline__ void pass_c_rows(const Params& p, const LayerDesc& d,
 template <int R>
 __global__ void __launch_bounds__(kThreads, 2) k_pass_c(Params p) {
     extern __shared__ __align__(16) unsigned char smem[];
-    const int t = tile_index<false>();
+    const int t = p.tile_base + tile_index<false>();
     const int l = p.t.tile_layer[t];
     const LayerDesc d = p.t.layers[l];
     const TileCoord tc = decode_tile(d, t, l);

@@ -188,6 +188,11 @@ struct psgd_ctx {
 
     void* stage = nullptr;  // device staging of host gradients
     size_t stage_bytes = 0;
+    // host-buffer steps: the uploads run on their own stream, one event per
+    // layer group, so that a group's passes start once its bytes are in
+    cudaStream_t up_stream = nullptr;
+    cudaEvent_t up_start = nullptr;
+    std::vector<cudaEvent_t> up_ev;
 
     // optional per-kernel timing (psgd_profile_*)
     bool profiling = false;
@@ -358,6 +363,74 @@ int launch(psgd_ctx* ctx, int which, bool lazy, const psgd::Params& p, size_t sm
     cudaError_t e = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(ctx->ntiles)), dim3(psgd::kThreads), args, smem,
                                      stream);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "kernel launch");
+    return PSGD_OK;
+}
+
+// launch() over the layers [l0, l1) only: their tiles are one contiguous
+// range of the grouped grid, and the P_hat grid covers just those layers.
+int launch_layers(psgd_ctx* ctx, int which, bool lazy, const psgd::Params& p0, size_t smem, cudaStream_t stream,
+                  int l0, int l1) {
+    const LayerDesc& last = ctx->desc[l1 - 1];
+    const int64_t t0 = ctx->desc[l0].tile_begin;
+    const int64_t t1 = last.tile_begin + static_cast<int64_t>(last.nrb) * last.nchunk;
+    if (t1 <= t0) return PSGD_OK;
+    void* fn = kernel_ptr(which, ctx->R, ctx->dtype, lazy, (ctx->flags & PSGD_FLAG_SUM_FIRST) != 0);
+    if (!fn) return fail(ctx, PSGD_ERR_ARG, "no kernel for rank %d", ctx->r);
+    psgd::Params p = p0;
+    p.tile_base = static_cast<int>(t0);
+    p.layer_base = l0;
+    void* args[] = {&p};
+    if (which == 1) {
+        int64_t maxm = 1;
+        for (int l = l0; l < l1; ++l) maxm = std::max(maxm, ctx->desc[l].m);
+        cudaError_t e = cudaLaunchKernel(kernel_ptr(7, ctx->R, ctx->dtype, false, false),
+                                         phat_grid(maxm, static_cast<size_t>(l1 - l0), ctx->R), dim3(psgd::kThreads),
+                                         args, 0, stream);
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "P_hat launch");
+    }
+    cudaError_t e = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(t1 - t0)), dim3(psgd::kThreads), args, smem, stream);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "kernel launch");
+    return PSGD_OK;
+}
+
+// Layer groups of a host-buffer step: contiguous layer ranges of about
+// equal size, at most kUploadGroups of them.  Group g's passes wait only
+// for group g's upload, so the later groups' copies overlap them.
+constexpr int kUploadGroups = 8;
+using LayerGroups = std::vector<std::pair<int, int>>;
+LayerGroups upload_groups(const psgd_ctx* ctx) {
+    LayerGroups g;
+    double total = 0.0;
+    for (auto& d : ctx->desc) total += static_cast<double>(d.m) * static_cast<double>(d.n);
+    const int K = std::min(ctx->L, kUploadGroups);
+    double acc = 0.0;
+    int start = 0;
+    for (int l = 0; l < ctx->L; ++l) {
+        acc += static_cast<double>(ctx->desc[l].m) * static_cast<double>(ctx->desc[l].n);
+        const bool cut = static_cast<int>(g.size()) < K - 1 && acc >= total * static_cast<double>(g.size() + 1) / K;
+        if (cut || l == ctx->L - 1) {
+            g.emplace_back(start, l + 1);
+            start = l + 1;
+        }
+    }
+    return g;
+}
+
+// The upload stream and one event per group; the uploads start after
+// everything already queued on the caller's stream (the previous step's
+// passes may still read the staging).
+int begin_upload(psgd_ctx* ctx, size_t groups, cudaStream_t s) {
+    cudaError_t e = cudaSuccess;
+    if (!ctx->up_stream) e = cudaStreamCreateWithFlags(&ctx->up_stream, cudaStreamNonBlocking);
+    if (e == cudaSuccess && !ctx->up_start) e = cudaEventCreateWithFlags(&ctx->up_start, cudaEventDisableTiming);
+    while (e == cudaSuccess && ctx->up_ev.size() < groups) {
+        cudaEvent_t x = nullptr;
+        e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+        if (e == cudaSuccess) ctx->up_ev.push_back(x);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(ctx->up_start, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ctx->up_stream, ctx->up_start, 0);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "upload stream");
     return PSGD_OK;
 }
 
@@ -544,6 +617,9 @@ void psgd_destroy(psgd_ctx* ctx) {
     ctx->tab_sub.release();
     if (ctx->ws) cudaFree(ctx->ws);
     if (ctx->stage) cudaFree(ctx->stage);
+    for (auto& x : ctx->up_ev) cudaEventDestroy(x);
+    if (ctx->up_start) cudaEventDestroy(ctx->up_start);
+    if (ctx->up_stream) cudaStreamDestroy(ctx->up_stream);
     ctx->tab_w.release();
     ctx->tab_l.release();
     ctx->tab_m.release();
@@ -671,8 +747,11 @@ static int refresh_oversampled(psgd_ctx* ctx, const psgd::Params& p, bool lazy, 
     return PSGD_OK;
 }
 
+// With `groups` (host-buffer steps), the gradients of group g are ready
+// once ctx->up_ev[g] has fired; a step that cannot run group by group
+// (power iterations, refresh, profiling) waits for the whole upload.
 static int step_impl(psgd_ctx* ctx, const void* const* grads, float* const* errors, float* const* q,
-                     float* const* p_hat, float* const* recon, cudaStream_t s) {
+                     float* const* p_hat, float* const* recon, cudaStream_t s, const LayerGroups* groups = nullptr) {
     const size_t WL = static_cast<size_t>(ctx->W) * ctx->L;
     std::vector<uint64_t> tw(2 * WL);
     for (size_t i = 0; i < WL; ++i) {
@@ -716,7 +795,26 @@ static int step_impl(psgd_ctx* ctx, const void* const* grads, float* const* erro
         if (e != cudaSuccess) return cuda_fail(ctx, e, "fresh Q launch");
     }
     const bool refresh = ctx->svd_every > 0 && (ctx->steps_done + 1) % ctx->svd_every == 0;
-    if (refresh && ctx->sub) {
+    const bool grouped = groups && !groups->empty() && !refresh && ctx->iters == 1 && !ev;
+    if (groups && !groups->empty() && !grouped) {
+        e = cudaStreamWaitEvent(s, ctx->up_ev[groups->size() - 1], 0);
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "upload wait");
+    }
+    if (grouped) {
+        for (size_t g = 0; g < groups->size() && !rc; ++g) {
+            const int l0 = (*groups)[g].first, l1 = (*groups)[g].second;
+            e = cudaStreamWaitEvent(s, ctx->up_ev[g], 0);
+            if (e != cudaSuccess) return cuda_fail(ctx, e, "upload wait");
+            rc = launch_layers(ctx, 0, lazy, p, ctx->smem_a, s, l0, l1);
+            if (!rc) rc = launch_layers(ctx, 1, lazy, p, ctx->smem_b, s, l0, l1);
+            if (!rc && (!lazy || recon)) {
+                psgd::Params pc = p;
+                pc.do_resid = lazy ? 0 : 1;
+                pc.do_recon = recon ? 1 : 0;
+                rc = launch_layers(ctx, 2, lazy, pc, ctx->smem_c, s, l0, l1);
+            }
+        }
+    } else if (refresh && ctx->sub) {
         rc = refresh_oversampled(ctx, p, lazy, s, ev);
     } else {
         rc = launch(ctx, 0, lazy, p, ctx->smem_a, s);
@@ -745,7 +843,7 @@ static int step_impl(psgd_ctx* ctx, const void* const* grads, float* const* erro
             cudaEventRecord(ev[4], s);
         }
     }
-    if (!rc && (!lazy || recon)) {
+    if (!rc && !grouped && (!lazy || recon)) {
         psgd::Params pc = p;
         pc.do_resid = lazy ? 0 : 1;
         pc.do_recon = recon ? 1 : 0;
@@ -791,8 +889,9 @@ static int ensure_stage(psgd_ctx* ctx, size_t need) {
 
 // The step on staged gradients, then P_hat and Q_bar copied to the host.
 static int step_and_download(psgd_ctx* ctx, const void* const* dev_grads, float* const* errors, float* const* q,
-                             float* const* p_hat_host, float* const* q_host, cudaStream_t s) {
-    int rc = step_impl(ctx, dev_grads, errors, q, nullptr, nullptr, s);
+                             float* const* p_hat_host, float* const* q_host, cudaStream_t s,
+                             const LayerGroups* groups) {
+    int rc = step_impl(ctx, dev_grads, errors, q, nullptr, nullptr, s, groups);
     if (rc) return rc;
     for (int l = 0; l < ctx->L; ++l) {
         const LayerDesc& d = ctx->desc[l];
@@ -836,16 +935,25 @@ int psgd_step_host(psgd_ctx* ctx, const void* const* grads_host, float* const* e
     }
     rc = ensure_stage(ctx, per_worker * ctx->W);
     if (rc) return rc;
+    const LayerGroups groups = upload_groups(ctx);
+    rc = begin_upload(ctx, groups.size(), s);
+    if (rc) return rc;
     std::vector<const void*> dev_grads(WL);
-    for (int w = 0; w < ctx->W; ++w)
-        for (int l = 0; l < ctx->L; ++l) {
-            unsigned char* dst = static_cast<unsigned char*>(ctx->stage) + per_worker * w + offs[l];
-            const size_t bytes = static_cast<size_t>(ctx->desc[l].m * ctx->desc[l].n) * esz;
-            cudaError_t e = cudaMemcpyAsync(dst, grads_host[w * ctx->L + l], bytes, cudaMemcpyHostToDevice, s);
-            if (e != cudaSuccess) return cuda_fail(ctx, e, "gradient upload");
-            dev_grads[w * ctx->L + l] = dst;
-        }
-    return step_and_download(ctx, dev_grads.data(), errors, q, p_hat_host, q_host, s);
+    for (size_t g = 0; g < groups.size(); ++g) {
+        for (int w = 0; w < ctx->W; ++w)
+            for (int l = groups[g].first; l < groups[g].second; ++l) {
+                unsigned char* dst = static_cast<unsigned char*>(ctx->stage) + per_worker * w + offs[l];
+                const size_t bytes = static_cast<size_t>(ctx->desc[l].m * ctx->desc[l].n) * esz;
+                cudaError_t e = bytes ? cudaMemcpyAsync(dst, grads_host[w * ctx->L + l], bytes, cudaMemcpyHostToDevice,
+                                                        ctx->up_stream)
+                                      : cudaSuccess;
+                if (e != cudaSuccess) return cuda_fail(ctx, e, "gradient upload");
+                dev_grads[w * ctx->L + l] = dst;
+            }
+        cudaError_t e = cudaEventRecord(ctx->up_ev[g], ctx->up_stream);
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "upload event");
+    }
+    return step_and_download(ctx, dev_grads.data(), errors, q, p_hat_host, q_host, s, &groups);
 }
 
 int psgd_step_host_flat(psgd_ctx* ctx, const void* const* grads_host, const int64_t* layer_offset,
@@ -879,11 +987,41 @@ int psgd_step_host_flat(psgd_ctx* ctx, const void* const* grads_host, const int6
     std::vector<const void*> dev_grads(WL);
     for (int w = 0; w < ctx->W; ++w) {
         unsigned char* dst = static_cast<unsigned char*>(ctx->stage) + per_worker * w;
-        cudaError_t e = cudaMemcpyAsync(dst, grads_host[w], span * esz, cudaMemcpyHostToDevice, s);
-        if (e != cudaSuccess) return cuda_fail(ctx, e, "gradient upload");
         for (int l = 0; l < ctx->L; ++l) dev_grads[w * ctx->L + l] = dst + static_cast<size_t>(layer_offset[l]) * esz;
     }
-    return step_and_download(ctx, dev_grads.data(), errors, q, p_hat_host, q_host, s);
+    // per group: runs of layers whose element ranges follow one another in
+    // the host buffer (gaps that hold no layer's elements included), one
+    // copy per run and worker
+    auto lend = [&](int l) { return layer_offset[l] + ctx->desc[l].m * ctx->desc[l].n; };
+    auto gap_free = [&](int64_t a, int64_t b) {
+        for (int k = 0; k < ctx->L; ++k)
+            if (ctx->desc[k].m * ctx->desc[k].n > 0 && layer_offset[k] < b && lend(k) > a) return false;
+        return true;
+    };
+    const LayerGroups groups = upload_groups(ctx);
+    rc = begin_upload(ctx, groups.size(), s);
+    if (rc) return rc;
+    for (size_t g = 0; g < groups.size(); ++g) {
+        for (int l = groups[g].first; l < groups[g].second;) {
+            const int64_t a = layer_offset[l];
+            int64_t b = lend(l);
+            int k = l + 1;
+            while (k < groups[g].second && layer_offset[k] >= b && gap_free(b, layer_offset[k])) b = std::max(b, lend(k++));
+            if (b > a)
+                for (int w = 0; w < ctx->W; ++w) {
+                    const size_t off = static_cast<size_t>(a) * esz;
+                    cudaError_t e = cudaMemcpyAsync(static_cast<unsigned char*>(ctx->stage) + per_worker * w + off,
+                                                    static_cast<const unsigned char*>(grads_host[w]) + off,
+                                                    static_cast<size_t>(b - a) * esz, cudaMemcpyHostToDevice,
+                                                    ctx->up_stream);
+                    if (e != cudaSuccess) return cuda_fail(ctx, e, "gradient upload");
+                }
+            l = k;
+        }
+        cudaError_t e = cudaEventRecord(ctx->up_ev[g], ctx->up_stream);
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "upload event");
+    }
+    return step_and_download(ctx, dev_grads.data(), errors, q, p_hat_host, q_host, s, &groups);
 }
 
 int psgd_materialize_errors(psgd_ctx* ctx, float* const* errors, void* stream) {

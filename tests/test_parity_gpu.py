@@ -444,6 +444,48 @@ def test_step_host_flat_matches_device_step(dtype):
         b.lib.step_host_flat(flat, bad, b.E, b.Q)
 
 
+@pytest.mark.parametrize("case", ["reversed", "many_layers", "lazy", "power2", "bf16"])
+def test_step_host_flat_grouped_uploads(case):
+    # the host-buffer step uploads contiguous layer groups on a stream of
+    # its own and starts each group's passes once its copies have landed:
+    # bit for bit the device step.  Layers packed in order (one copy per
+    # group and worker) or in reverse order (one copy per layer); 14 layers
+    # for 8 groups of one or two; lazy errors; two power iterations (the
+    # step waits for the whole upload); bf16 gradients.
+    layers = MIXED * 2 if case == "many_layers" else MIXED
+    wl = H.small_workload(layers, 4, 3, dtype="bf16" if case == "bf16" else "f32")
+    kw = {"lazy": case == "lazy", "iters": 2 if case == "power2" else 1}
+    a = H.LibRun(wl, **kw)
+    b = H.LibRun(wl, **kw)
+    L = len(wl.layers)
+    esz = 2 if case == "bf16" else 4
+    per16 = 16 // esz
+    order = list(range(L))[::-1] if case == "reversed" else list(range(L))
+    offs, o = [0] * L, 0
+    for l in order:
+        m, n = wl.layers[l]
+        offs[l] = o
+        o = -(-(o + m * n) // per16) * per16
+    hdt = torch.bfloat16 if case == "bf16" else torch.float32
+    flat = [torch.full((o,), float("nan"), dtype=hdt).pin_memory() for _ in range(wl.workers)]
+    for t in range(3):
+        host = a.fill_grads_host(t)
+        a.run_step()
+        for w in range(wl.workers):
+            for l, (m, n) in enumerate(wl.layers):
+                flat[w][offs[l]:offs[l] + m * n].copy_(host[w][l].reshape(-1))
+        ph = [torch.empty(m, wl.rank).pin_memory() for (m, _) in wl.layers]
+        qh = [torch.empty(n, wl.rank).pin_memory() for (_, n) in wl.layers]
+        b.lib.step_host_flat(flat, offs, b.E, b.Q, ph, qh)
+        torch.cuda.synchronize()
+        for l in range(L):
+            assert torch.equal(a.Q[l].cpu(), qh[l]), (t, l)
+            assert torch.equal(a.P[l].cpu(), ph[l]), (t, l)
+            for w in range(wl.workers):
+                assert torch.equal(a.E[w][l], b.E[w][l]), (t, l, w)
+    b.lib.status()
+
+
 def test_bad_arguments_rejected():
     from rank_gradient_compression_02_b200 import PowerSGD, PsgdError
     wl = H.small_workload([(64, 48)], 2, 2)
