@@ -19,6 +19,11 @@ int main() {
     cs.push_back({2600, 650, 4, 16});
     cs.push_back({33280, 650, 4, 16});
     int64_t tf[][2] = {{4096,12288},{4096,4096},{16384,4096},{4096,16384}};
+    const auto& tf4 = tf;
+    // the ResNet-18 set's 20 matrices in list order
+    const int64_t resnet20[][2] = {{64,576},{64,576},{64,576},{64,576},{128,576},{128,1152},{128,1152},{128,1152},
+                                   {256,1152},{256,2304},{256,2304},{256,2304},{512,2304},{512,4608},{512,4608},
+                                   {512,4608},{128,64},{256,128},{512,256},{10,512}};
     for (auto& s : tf) cs.push_back({s[0], s[1], 4, 4});
     for (int r : {1,2,3,4,8,16,32}) {
         cs.push_back({8192, 8192, r, 8});
@@ -61,6 +66,73 @@ int main() {
             }
         }
         if (sz.tiles != (int64_t)d.nrb * d.nchunk) fail("tile count");
+    }
+    // layer groups of the host-buffer steps (upload of later groups
+    // overlapping the passes of earlier ones): 1..min(L, 8) groups, each a
+    // non-empty contiguous layer range, every layer once, each group within
+    // one layer of an equal share of the elements, and the groups' tile
+    // ranges (the grids of their launches) following one another over the
+    // whole grouped grid
+    auto check_groups = [&](const char* name, const std::vector<std::pair<int64_t, int64_t>>& shapes, int r, int W) {
+        psgd_ctx ctx;
+        ctx.L = static_cast<int>(shapes.size());
+        const int R = pad_rank(r);
+        int64_t tiles = 0;
+        double total = 0.0, biggest = 0.0;
+        for (auto& sh : shapes) {
+            LayerSizes sz{};
+            LayerDesc d = layer_geometry(sh.first, sh.second, R, W, &sz);
+            d.tile_begin = tiles;
+            tiles += sz.tiles;
+            ctx.desc.push_back(d);
+            total += double(sh.first) * double(sh.second);
+            biggest = std::max(biggest, double(sh.first) * double(sh.second));
+        }
+        const LayerGroups g = upload_groups(&ctx);
+        ++n;
+        auto gfail = [&](const char* what) {
+            ++bad;
+            std::printf("FAIL groups %s: %s (%zu groups)\n", name, what, g.size());
+        };
+        if (g.empty() || static_cast<int>(g.size()) > std::min(ctx.L, kUploadGroups)) gfail("1..min(L, 8) groups");
+        int next = 0;
+        int64_t tnext = 0;
+        for (auto& lr : g) {
+            const int l0 = lr.first, l1 = lr.second;
+            if (l0 != next || l1 <= l0 || l1 > ctx.L) {
+                gfail("contiguous, none empty");
+                break;
+            }
+            double size = 0.0;
+            for (int l = l0; l < l1; ++l) size += double(ctx.desc[l].m) * double(ctx.desc[l].n);
+            if (size > total / double(g.size()) + biggest) gfail("within one layer of an equal share");
+            const LayerDesc& last = ctx.desc[l1 - 1];
+            const int64_t t0 = ctx.desc[l0].tile_begin, t1 = last.tile_begin + int64_t(last.nrb) * last.nchunk;
+            if (t0 != tnext || t1 < t0) gfail("tile ranges follow one another");
+            tnext = t1;
+            next = l1;
+        }
+        if (next != ctx.L || tnext != tiles) gfail("every layer and tile once");
+    };
+    {
+        std::vector<std::pair<int64_t, int64_t>> tf, rn, ls, mx, mx2;
+        for (int b = 0; b < 24; ++b)
+            for (auto& s2 : tf4) tf.push_back({s2[0], s2[1]});
+        for (auto& s2 : resnet20) rn.push_back({s2[0], s2[1]});
+        for (int k = 0; k < 6; ++k) ls.push_back({2600, 650});
+        ls.push_back({33280, 650});
+        ls.push_back({33280, 650});
+        for (auto& s2 : mixed) mx.push_back({s2[0], s2[1]});
+        mx2 = mx;
+        mx2.insert(mx2.end(), mx.begin(), mx.end());
+        check_groups("transformer set", tf, 4, 4);
+        check_groups("ResNet-18 set", rn, 2, 16);
+        check_groups("LSTM set", ls, 4, 16);
+        check_groups("mixed shapes", mx, 4, 3);
+        check_groups("mixed shapes twice", mx2, 4, 3);
+        check_groups("one layer", {{300, 650}}, 4, 3);
+        check_groups("small layers, one large last", {{8, 8}, {8, 8}, {8, 8}, {4096, 4096}}, 2, 2);
+        check_groups("large first", {{4096, 4096}, {8, 8}, {8, 8}, {8, 8}, {8, 8}, {8, 8}, {8, 8}, {8, 8}, {8, 8}}, 2, 2);
     }
     std::printf("%d cases, %d failures\n", n, bad);
     return bad != 0;

@@ -5,7 +5,10 @@ workloads use, that the lane
 width divides the row, chunks and row blocks cover the matrix with none
 empty, the tensor-core tiles are whole 16-row groups, the rows buffer and
 the widest chunk fit, and each pass's shared memory fits in 227 KB and
-leaves room for the CTAs per SM its launch bounds aim at."""
+leaves room for the CTAs per SM its launch bounds aim at; and that the
+layer groups of the host-buffer steps are contiguous, cover every layer and
+tile once, number at most min(L, 8), and stay within one layer of an equal
+share."""
 import os
 import shutil
 import subprocess
