@@ -814,9 +814,10 @@ def main():
 def run_e2e(lib, B, wl, r, args, world, device, DB=None):
     """The same metric through the public API with host buffers: pinned
     host gradients, one flat buffer per worker, copied in every step
-    (psgd_step_host_flat on one GPU; one copy per worker into the device
-    buffers before the distributed step on several), P_hat and Q_bar (and
-    the 1-D means) read back.  When the library's device staging of the
+    (psgd_step_host_flat on one GPU, which uploads layer groups on a stream
+    of its own and starts each group's passes once its copies have landed;
+    one copy per worker into the device buffers before the distributed step
+    on several), P_hat and Q_bar (and the 1-D means) read back.  When the library's device staging of the
     host gradients would not fit beside the resident buffers (the
     transformer set: 38.7 GB of bf16 gradients beside 77 GB of error
     memory), the device gradient buffers are released first: the staging
@@ -830,7 +831,7 @@ def run_e2e(lib, B, wl, r, args, world, device, DB=None):
         return {"value": None, "unit": UNIT,
                 "skipped": f"host RAM too small for {host_bytes / 1e9:.1f} GB of pinned gradients"}
     # one pinned host buffer per worker holding every layer (a flat gradient
-    # bucket), uploaded with one copy per worker
+    # bucket); the library uploads it in layer groups
     Gh = [_pinned_empty(B.offs[-1], B.G_flat[0].dtype) for _ in range(W)]
     for w in range(W):
         Gh[w].copy_(B.G_flat[w])
