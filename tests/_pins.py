@@ -313,11 +313,55 @@ def check_subspace_sin_max(ora):
         assert abs(got - want) <= 1e-12 + 1e-6 * want, (angles, got, want)
 
 
+def check_orthogonal_equivariance(ora):
+    """Rotating the problem rotates the answer: for orthogonal U (m x m) and
+    V (n x n), the step on U G_w V, U E_w V with warm start V^T Q gives
+    U P_hat, V^T Q_bar and U E'_w V.  P = (U M V)(V^T Q) = U M Q keeps its
+    Gram matrix, so the orthogonalisation is the same ([N152] "Method":
+    P = M Q, orthogonalise, Q = M^T P_hat, E' = M - P_hat Q^T).  A product
+    taken on the wrong side or with a transposed operand breaks it."""
+    rng = _rng(12)
+    m, n, r, W = 30, 22, 3, 3
+    G = [rng.standard_normal((m, n)) for _ in range(W)]
+    E = [0.5 * rng.standard_normal((m, n)) for _ in range(W)]
+    Q = rng.standard_normal((n, r))
+    U, _ = np.linalg.qr(rng.standard_normal((m, m)))
+    V, _ = np.linalg.qr(rng.standard_normal((n, n)))
+    o = ora.step(G, E, Q)
+    o2 = ora.step([U @ g @ V for g in G], [U @ e @ V for e in E], V.T @ Q)
+    np.testing.assert_allclose(o2["P_hat"], U @ o["P_hat"], atol=1e-10)
+    np.testing.assert_allclose(o2["Q_bar"], V.T @ o["Q_bar"], atol=1e-10)
+    for w in range(W):
+        np.testing.assert_allclose(o2["E_new"][w], U @ o["E_new"][w] @ V, atol=1e-10)
+
+
+def check_scale_homogeneity(ora):
+    """Scaling G and E by c: P = c M Q has Gram matrix c^2 P^T P, so the
+    normalised P_hat becomes sign(c) P_hat, Q_bar = (c M)^T P_hat becomes
+    |c| Q_bar, and E'_w and G_hat become c times theirs ([N152] "Method":
+    the orthogonalisation normalises the columns).  A missing or repeated
+    normalisation, or a sign lost in it, breaks it."""
+    rng = _rng(13)
+    m, n, r, W = 26, 19, 4, 2
+    G = [rng.standard_normal((m, n)) for _ in range(W)]
+    E = [0.5 * rng.standard_normal((m, n)) for _ in range(W)]
+    Q = rng.standard_normal((n, r))
+    o = ora.step(G, E, Q)
+    for c in (8.0, -0.5, 3.0e-3):
+        oc = ora.step([c * g for g in G], [c * e for e in E], Q)
+        scale = max(1.0, abs(c))
+        np.testing.assert_allclose(oc["P_hat"], math.copysign(1.0, c) * o["P_hat"], atol=1e-12)
+        np.testing.assert_allclose(oc["Q_bar"], abs(c) * o["Q_bar"], atol=1e-12 * scale)
+        np.testing.assert_allclose(oc["G_hat"], c * o["G_hat"], atol=1e-12 * scale)
+        for w in range(W):
+            np.testing.assert_allclose(oc["E_new"][w], c * o["E_new"][w], atol=1e-12 * scale)
+
+
 ALL_CHECKS = [
     check_hand_cases, check_gram_schmidt_vs_householder, check_gram_schmidt_rank_deficient,
     check_full_rank_is_lossless,
     check_rank1_closed_form, check_exact_low_rank, check_identities, check_linearity,
     check_jacobi_svd, check_warm_start_convergence, check_error_feedback_telescopes,
     check_momentum_closed_form, check_vec_mean, check_power_iterations, check_svd_refresh,
-    check_subspace_sin_max,
+    check_subspace_sin_max, check_orthogonal_equivariance, check_scale_homogeneity,
 ]
